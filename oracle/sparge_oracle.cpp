@@ -1,0 +1,396 @@
+// CPU oracle for pooled block-sparse attention with a hybrid Top-k / Top-p
+// block mask, and for its sparse + linear mix.
+//
+// TEST INFRASTRUCTURE ONLY. This file is the plain, slow, single-threaded
+// restatement of what the method computes. Only the test suite, the smoke
+// check and the benchmark's CPU-baseline leg may load it. It shares no code,
+// header, table or constant with the CUDA library, and the CUDA library never
+// calls it.
+//
+// Sources (the articles print no formula; each step restates their prose):
+//   [SA2 s1]  SpargeAttention2 article ("Tsinghua invents an AI
+//             attention-slimming technique", arXiv:2602.13515), section 1:
+//             Top-k keeps a fixed number of the most important items; Top-p
+//             keeps items until their summed importance reaches a threshold;
+//             the hybrid runs both and merges (unions) the two selections.
+//   [SA2 s4]  same article, section 4: a pre-filter pools neighbouring tokens
+//             to score blocks cheaply, a selection stage applies the hybrid
+//             rule, and attention runs block by block, each block either fully
+//             computed or fully skipped, under a block-level mask.
+//   [SLA2 s1] SLA2 article (arXiv:2602.12675), section 1: important regions get
+//             sparse (softmax) attention, the rest get linear attention.
+//   [SLA2 s2] same article, section 2: the sparse branch is renormalised over
+//             the kept region only; the output is alpha * sparse output plus
+//             (1 - alpha) * linear output, alpha a learnt ratio.
+//
+// Readings where the articles are silent (each one is listed with its reason
+// in the design notes of the repository):
+//   * pooling is the mean over a block's valid rows (a ragged last block
+//     averages only the rows it has);
+//   * block importance is softmax_J(qbar_I . kbar_J / sqrt(d)) along each
+//     query-block row;
+//   * Top-k keeps ceil(k * Nkb) blocks (computed as ceil(k*Nkb - 1e-9) to
+//     absorb representation error), k = 0 disables it;
+//   * Top-p keeps the shortest prefix of the (P descending, index ascending)
+//     order whose running sum is >= p, p = 0 disables it;
+//   * both selections are prefixes of the same order, so their union is the
+//     longer prefix; every row keeps at least one block;
+//   * the linear branch uses phi(x) = elu(x) + 1 on the keys outside the kept
+//     blocks, normalised: O_l = sum_j (phi(q).phi(k_j)) v_j / sum_j phi(q).phi(k_j);
+//     an empty complement gives O_l = 0;
+//   * no causal masking (bidirectional video attention).
+//
+// Precision: attention outputs are computed in double from the exactly widened
+// bf16 inputs. The block selection is an integer decision taken from floating
+// point, so it is offered in two precisions: the double-precision definition,
+// and the single-precision decision with a fixed operation order that the GPU
+// kernel also follows (pool: sequential float sum over rows, then divide by the
+// row count; score: sequential fused multiply-add over channels, then multiply
+// by (float)(1/sqrt(d)); softmax: expf(z - max) / sum).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+namespace {
+
+double widen(uint16_t h) {
+  uint32_t u = static_cast<uint32_t>(h) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return static_cast<double>(f);
+}
+
+float widen_f(uint16_t h) {
+  uint32_t u = static_cast<uint32_t>(h) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+// phi(x) = elu(x) + 1: x + 1 for x > 0, exp(x) otherwise [SLA2 s1, reading].
+double phi(double x) { return x > 0.0 ? x + 1.0 : std::exp(x); }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+enum { OK = 0, ERR_ARG = 1 };
+
+bool shape_ok(int64_t BH, int64_t N, int d, int blk) {
+  return BH > 0 && N > 0 && d > 0 && blk > 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+// ---------------------------------------------------------------------------
+// Pooling [SA2 s4]: mean of each block's valid rows.
+// X: bf16 bits, [BH, N, d] contiguous. out: [BH, ceil(N/blk), d].
+// ---------------------------------------------------------------------------
+int oracle_pool_f64(const uint16_t* X, int64_t BH, int64_t N, int d, int blk, double* out) {
+  if (!X || !out || !shape_ok(BH, N, d, blk)) return ERR_ARG;
+  const int64_t nb = ceil_div(N, blk);
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t I = 0; I < nb; ++I) {
+      const int64_t r0 = I * blk, r1 = std::min<int64_t>(N, r0 + blk);
+      for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int64_t r = r0; r < r1; ++r) acc += widen(X[(bh * N + r) * d + c]);
+        out[(bh * nb + I) * d + c] = acc / static_cast<double>(r1 - r0);
+      }
+    }
+  return OK;
+}
+
+// Single-precision pooling with the GPU kernel's operation order.
+int oracle_pool_f32(const uint16_t* X, int64_t BH, int64_t N, int d, int blk, float* out) {
+  if (!X || !out || !shape_ok(BH, N, d, blk)) return ERR_ARG;
+  const int64_t nb = ceil_div(N, blk);
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t I = 0; I < nb; ++I) {
+      const int64_t r0 = I * blk, r1 = std::min<int64_t>(N, r0 + blk);
+      for (int c = 0; c < d; ++c) {
+        float acc = 0.0f;
+        for (int64_t r = r0; r < r1; ++r) acc = acc + widen_f(X[(bh * N + r) * d + c]);
+        out[(bh * nb + I) * d + c] = acc / static_cast<float>(r1 - r0);
+      }
+    }
+  return OK;
+}
+
+// ---------------------------------------------------------------------------
+// Pooled block importance [SA2 s4]: P[I, J] = softmax_J(qbar_I . kbar_J / sqrt d).
+// qbar [BH, Nqb, d], kbar [BH, Nkb, d], P [BH, Nqb, Nkb].
+// ---------------------------------------------------------------------------
+int oracle_block_probs_f64(const double* qbar, const double* kbar, int64_t BH, int64_t Nqb,
+                           int64_t Nkb, int d, double* P) {
+  if (!qbar || !kbar || !P || BH <= 0 || Nqb <= 0 || Nkb <= 0 || d <= 0) return ERR_ARG;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(d));
+  std::vector<double> s(Nkb);
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t I = 0; I < Nqb; ++I) {
+      const double* q = qbar + (bh * Nqb + I) * d;
+      double mx = -std::numeric_limits<double>::infinity();
+      for (int64_t J = 0; J < Nkb; ++J) {
+        const double* k = kbar + (bh * Nkb + J) * d;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += q[c] * k[c];
+        s[J] = dot * scale;
+        mx = std::max(mx, s[J]);
+      }
+      double sum = 0.0;
+      for (int64_t J = 0; J < Nkb; ++J) {
+        s[J] = std::exp(s[J] - mx);
+        sum += s[J];
+      }
+      double* row = P + (bh * Nqb + I) * Nkb;
+      for (int64_t J = 0; J < Nkb; ++J) row[J] = s[J] / sum;
+    }
+  return OK;
+}
+
+// Single precision with the GPU kernel's operation order: sequential fmaf over
+// channels, times (float)(1/sqrt(d)); expf(z - max); divide by the row sum.
+int oracle_block_probs_f32(const float* qbar, const float* kbar, int64_t BH, int64_t Nqb,
+                           int64_t Nkb, int d, float* P) {
+  if (!qbar || !kbar || !P || BH <= 0 || Nqb <= 0 || Nkb <= 0 || d <= 0) return ERR_ARG;
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  std::vector<float> z(Nkb);
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t I = 0; I < Nqb; ++I) {
+      const float* q = qbar + (bh * Nqb + I) * d;
+      float mx = -std::numeric_limits<float>::infinity();
+      for (int64_t J = 0; J < Nkb; ++J) {
+        const float* k = kbar + (bh * Nkb + J) * d;
+        float dot = 0.0f;
+        for (int c = 0; c < d; ++c) dot = std::fmaf(q[c], k[c], dot);
+        z[J] = dot * scale;
+        mx = std::max(mx, z[J]);
+      }
+      float sum = 0.0f;
+      for (int64_t J = 0; J < Nkb; ++J) {
+        z[J] = std::exp(z[J] - mx);
+        sum = sum + z[J];
+      }
+      float* row = P + (bh * Nqb + I) * Nkb;
+      for (int64_t J = 0; J < Nkb; ++J) row[J] = z[J] / sum;
+    }
+  return OK;
+}
+
+// ---------------------------------------------------------------------------
+// Hybrid Top-k / Top-p selection on one row of block probabilities [SA2 s1].
+//
+// P: Nkb probabilities. kept: receives the kept block indices in ascending
+// order (capacity Nkb). Optional outputs: m (kept count), kc and pc (the Top-k
+// and Top-p counts), order (the full (P desc, index asc) order), cum (cum[m] =
+// running sum of the first m sorted probabilities, m = 0..Nkb, in double).
+// ---------------------------------------------------------------------------
+int oracle_select_row(const double* P, int64_t Nkb, double topk, double topp, int32_t* kept,
+                      int64_t* m_out, int64_t* kc_out, int64_t* pc_out, int32_t* order_out,
+                      double* cum_out) {
+  if (!P || !kept || Nkb <= 0) return ERR_ARG;
+  if (!(topk >= 0.0 && topk <= 1.0) || !(topp >= 0.0 && topp <= 1.0)) return ERR_ARG;
+  // Order: most important first; equal importance goes to the lower index.
+  std::vector<int32_t> order(Nkb);
+  for (int64_t j = 0; j < Nkb; ++j) order[j] = static_cast<int32_t>(j);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return P[a] > P[b]; });
+
+  // Top-k: a fixed count regardless of how importance is spread.
+  int64_t kc = 0;
+  if (topk > 0.0) {
+    kc = static_cast<int64_t>(std::ceil(topk * static_cast<double>(Nkb) - 1e-9));
+    kc = std::min<int64_t>(std::max<int64_t>(kc, 0), Nkb);
+  }
+  // Top-p: the shortest prefix whose summed importance reaches p.
+  std::vector<double> cum(Nkb + 1, 0.0);
+  for (int64_t m = 1; m <= Nkb; ++m) cum[m] = cum[m - 1] + P[order[m - 1]];
+  int64_t pc = 0;
+  if (topp > 0.0) {
+    pc = Nkb;
+    for (int64_t m = 1; m <= Nkb; ++m)
+      if (cum[m] >= topp) {
+        pc = m;
+        break;
+      }
+  }
+  // Union of two prefixes of one order = the longer prefix; keep >= 1 block.
+  const int64_t m = std::max<int64_t>(std::max(kc, pc), 1);
+  std::vector<int32_t> sel(order.begin(), order.begin() + m);
+  std::sort(sel.begin(), sel.end());
+  for (int64_t i = 0; i < m; ++i) kept[i] = sel[i];
+  if (m_out) *m_out = m;
+  if (kc_out) *kc_out = kc;
+  if (pc_out) *pc_out = pc;
+  if (order_out)
+    for (int64_t j = 0; j < Nkb; ++j) order_out[j] = order[j];
+  if (cum_out)
+    for (int64_t j = 0; j <= Nkb; ++j) cum_out[j] = cum[j];
+  return OK;
+}
+
+// ---------------------------------------------------------------------------
+// Full mask [SA2 s1, s4]: pool, score, select, for every query-block row.
+// Q, K: bf16 bits [B*H, N, d]. kv_idx [B*H, Nqb, Nkb] (first kv_cnt entries
+// valid, ascending), kv_cnt [B*H, Nqb]. precision: 32 (the kernel's decision
+// precision) or 64 (the double definition). P_out: optional [B*H, Nqb, Nkb].
+// ---------------------------------------------------------------------------
+int oracle_mask(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int d, int bq,
+                int bk, double topk, double topp, int precision, int32_t* kv_idx,
+                int32_t* kv_cnt, double* P_out) {
+  if (!Q || !K || !kv_idx || !kv_cnt || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
+  if (precision != 32 && precision != 64) return ERR_ARG;
+  const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
+  std::vector<double> P(static_cast<size_t>(BH * Nqb * Nkb));
+  if (precision == 64) {
+    std::vector<double> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
+    oracle_pool_f64(Q, BH, N, d, bq, qb.data());
+    oracle_pool_f64(K, BH, N, d, bk, kb.data());
+    oracle_block_probs_f64(qb.data(), kb.data(), BH, Nqb, Nkb, d, P.data());
+  } else {
+    std::vector<float> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
+    std::vector<float> Pf(P.size());
+    oracle_pool_f32(Q, BH, N, d, bq, qb.data());
+    oracle_pool_f32(K, BH, N, d, bk, kb.data());
+    oracle_block_probs_f32(qb.data(), kb.data(), BH, Nqb, Nkb, d, Pf.data());
+    for (size_t i = 0; i < P.size(); ++i) P[i] = static_cast<double>(Pf[i]);
+  }
+  for (int64_t row = 0; row < BH * Nqb; ++row) {
+    int64_t m = 0;
+    int rc = oracle_select_row(P.data() + row * Nkb, Nkb, topk, topp, kv_idx + row * Nkb, &m,
+                               nullptr, nullptr, nullptr, nullptr);
+    if (rc != OK) return rc;
+    for (int64_t j = m; j < Nkb; ++j) kv_idx[row * Nkb + j] = 0;
+    kv_cnt[row] = static_cast<int32_t>(m);
+  }
+  if (P_out) std::memcpy(P_out, P.data(), P.size() * sizeof(double));
+  return OK;
+}
+
+// ---------------------------------------------------------------------------
+// Attention outputs for a list of rows, in double.
+//
+// mode 0: sparse branch [SA2 s4, SLA2 s2] - softmax over the keys of the kept
+//         blocks only (renormalised over that region), scale 1/sqrt(d).
+// mode 1: linear branch [SLA2 s1] - phi-feature attention over the keys of
+//         the blocks NOT kept, normalised; 0 when that set is empty.
+// mode 2: the mix [SLA2 s2] - alpha_h * sparse + (1 - alpha_h) * linear.
+// mode 3: dense softmax attention over all keys (all blocks kept).
+//
+// rows: flat row ids r = bh*N + i. O: [nrows, d]. lse (optional, modes 0 and
+// 3): natural-log sum of exp of the scaled scores, -inf for an empty set.
+// kv_idx / kv_cnt as produced by oracle_mask; entries must lie in [0, Nkb).
+// ---------------------------------------------------------------------------
+int oracle_attention_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t BH,
+                          int64_t N, int d, int bq, int bk, const int32_t* kv_idx,
+                          const int32_t* kv_cnt, const float* alpha, int64_t H, int mode,
+                          const int64_t* rows, int64_t nrows, double* O, double* lse) {
+  if (!Q || !K || !V || !rows || !O || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
+  if (mode < 0 || mode > 3) return ERR_ARG;
+  if (mode != 3 && (!kv_idx || !kv_cnt)) return ERR_ARG;
+  if (mode == 2 && (!alpha || H <= 0 || BH % H != 0)) return ERR_ARG;
+  const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
+  const double scale = 1.0 / std::sqrt(static_cast<double>(d));
+
+  // Rows are grouped by head so each head's widened K, V and phi(K) are built once.
+  std::vector<int64_t> idx(nrows);
+  for (int64_t i = 0; i < nrows; ++i) {
+    if (rows[i] < 0 || rows[i] >= BH * N) return ERR_ARG;
+    idx[i] = i;
+  }
+  std::stable_sort(idx.begin(), idx.end(), [&](int64_t a, int64_t b) { return rows[a] / N < rows[b] / N; });
+
+  std::vector<double> Kd, Vd, phiK, q(d), phiq(d), s, acc(d), acc_s(d), acc_l(d);
+  std::vector<char> kept(Nkb);
+  int64_t cur_bh = -1;
+  for (int64_t t = 0; t < nrows; ++t) {
+    const int64_t ri = idx[t];
+    const int64_t bh = rows[ri] / N, i = rows[ri] % N, I = i / bq;
+    if (bh != cur_bh) {
+      cur_bh = bh;
+      Kd.assign(static_cast<size_t>(N * d), 0.0);
+      Vd.assign(static_cast<size_t>(N * d), 0.0);
+      for (int64_t e = 0; e < N * d; ++e) {
+        Kd[e] = widen(K[bh * N * d + e]);
+        Vd[e] = widen(V[bh * N * d + e]);
+      }
+      if (mode == 1 || mode == 2) {
+        phiK.assign(static_cast<size_t>(N * d), 0.0);
+        for (int64_t e = 0; e < N * d; ++e) phiK[e] = phi(Kd[e]);
+      }
+    }
+    for (int c = 0; c < d; ++c) {
+      q[c] = widen(Q[(bh * N + i) * d + c]);
+      phiq[c] = phi(q[c]);
+    }
+    // Block membership of this row's query block.
+    if (mode == 3) {
+      std::fill(kept.begin(), kept.end(), 1);
+    } else {
+      std::fill(kept.begin(), kept.end(), 0);
+      const int64_t cnt = kv_cnt[bh * Nqb + I];
+      if (cnt < 0 || cnt > Nkb) return ERR_ARG;
+      for (int64_t e = 0; e < cnt; ++e) {
+        const int32_t J = kv_idx[(bh * Nqb + I) * Nkb + e];
+        if (J < 0 || J >= Nkb) return ERR_ARG;
+        kept[J] = 1;
+      }
+    }
+
+    // Softmax branch over the kept keys (two passes: max, then exp-weighted sums).
+    double lse_row = -std::numeric_limits<double>::infinity();
+    std::fill(acc_s.begin(), acc_s.end(), 0.0);
+    if (mode != 1) {
+      double mx = -std::numeric_limits<double>::infinity();
+      s.assign(static_cast<size_t>(N), 0.0);
+      for (int64_t j = 0; j < N; ++j) {
+        if (!kept[j / bk]) continue;
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += q[c] * Kd[j * d + c];
+        s[j] = dot * scale;
+        mx = std::max(mx, s[j]);
+      }
+      if (mx > -std::numeric_limits<double>::infinity()) {
+        double l = 0.0;
+        for (int64_t j = 0; j < N; ++j) {
+          if (!kept[j / bk]) continue;
+          const double e = std::exp(s[j] - mx);
+          l += e;
+          for (int c = 0; c < d; ++c) acc_s[c] += e * Vd[j * d + c];
+        }
+        for (int c = 0; c < d; ++c) acc_s[c] /= l;
+        lse_row = mx + std::log(l);
+      }
+    }
+    // Linear branch over the complement.
+    std::fill(acc_l.begin(), acc_l.end(), 0.0);
+    if (mode == 1 || mode == 2) {
+      double den = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        if (kept[j / bk]) continue;
+        double w = 0.0;
+        for (int c = 0; c < d; ++c) w += phiq[c] * phiK[j * d + c];
+        den += w;
+        for (int c = 0; c < d; ++c) acc_l[c] += w * Vd[j * d + c];
+      }
+      if (den > 0.0)
+        for (int c = 0; c < d; ++c) acc_l[c] /= den;
+    }
+    double a = 1.0;
+    if (mode == 2) a = static_cast<double>(alpha[bh % H]);
+    for (int c = 0; c < d; ++c) {
+      double v;
+      if (mode == 0 || mode == 3) v = acc_s[c];
+      else if (mode == 1) v = acc_l[c];
+      else v = a * acc_s[c] + (1.0 - a) * acc_l[c];
+      O[ri * d + c] = v;
+    }
+    if (lse) lse[ri] = lse_row;
+  }
+  return OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,360 @@
+"""Pins for the CPU oracle against facts that do not come from the oracle itself.
+
+Each test ties one oracle function to a library routine it does not call, a
+closed form, an invariant, hand-derived golden values or exact brute force.
+Sources of the rules: SpargeAttention2 article (arXiv:2602.13515) sections 1
+and 4; SLA2 article (arXiv:2602.12675) sections 1 and 2.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from block_sparse_attention_pooled_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "select_rows.json")
+
+
+def _bf16(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _rand_qkv(B, H, N, d, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    q = _bf16(torch.randn(B, H, N, d, generator=g) * scale)
+    k = _bf16(torch.randn(B, H, N, d, generator=g) * scale)
+    v = _bf16(torch.randn(B, H, N, d, generator=g))
+    return q, k, v
+
+
+def _block_bool_mask(kv_idx, kv_cnt, N, bq, bk):
+    """[B,H,N,N] boolean key mask expanded from block lists (test-side helper)."""
+    B, H, nqb, nkb = kv_idx.shape
+    m = np.zeros((B, H, N, N), bool)
+    for b in range(B):
+        for h in range(H):
+            for I in range(nqb):
+                for e in range(int(kv_cnt[b, h, I])):
+                    J = int(kv_idx[b, h, I, e])
+                    m[b, h, I * bq:(I + 1) * bq, J * bk:(J + 1) * bk] = True
+    return m
+
+
+def _phi_torch(x):
+    return F.elu(x) + 1.0
+
+
+# ----------------------------------------------------------------------------- pooling
+def test_pool_full_blocks_match_avg_pool(oracle_mod):
+    q, _, _ = _rand_qkv(1, 2, 256, 16, 1)
+    got = oracle_mod.pool(q, 64, precision=64)
+    x = q.double().reshape(2, 256, 16).transpose(1, 2)  # (BH, d, N)
+    ref = F.avg_pool1d(x, kernel_size=64, stride=64).transpose(1, 2).reshape(1, 2, 4, 16)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_pool_ragged_block_averages_valid_rows_only(oracle_mod):
+    # N = 70 with blocks of 64: the last block holds rows 64..69 only.
+    x = torch.zeros(1, 1, 70, 4)
+    x[0, 0, :64] = 3.0
+    x[0, 0, 64:] = torch.arange(6, dtype=torch.float32)[:, None]  # rows 0..5 -> mean 2.5
+    got = oracle_mod.pool(_bf16(x), 64, precision=64)
+    assert got.shape == (1, 1, 2, 4)
+    np.testing.assert_array_equal(got[0, 0, 0], 3.0)
+    np.testing.assert_array_equal(got[0, 0, 1], 2.5)
+    got32 = oracle_mod.pool(_bf16(x), 64, precision=32)
+    np.testing.assert_array_equal(got32[0, 0, 1], np.float32(2.5))
+
+
+def test_pool_single_precision_close_to_double(oracle_mod):
+    q, _, _ = _rand_qkv(1, 2, 300, 32, 2, scale=3.0)
+    a = oracle_mod.pool(q, 128, 64)
+    b = oracle_mod.pool(q, 128, 32).astype(np.float64)
+    np.testing.assert_allclose(b, a, rtol=0, atol=1e-5)
+
+
+# ----------------------------------------------------------------------------- block scores
+def test_block_probs_match_torch_softmax(oracle_mod):
+    g = torch.Generator().manual_seed(3)
+    qb = torch.randn(1, 2, 5, 16, generator=g, dtype=torch.float64) * 2
+    kb = torch.randn(1, 2, 9, 16, generator=g, dtype=torch.float64) * 2
+    got = oracle_mod.block_probs(qb.numpy(), kb.numpy())
+    ref = torch.softmax(qb @ kb.transpose(-1, -2) / math.sqrt(16), dim=-1)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-12)
+    got32 = oracle_mod.block_probs(qb.numpy().astype(np.float32), kb.numpy().astype(np.float32))
+    np.testing.assert_allclose(got32, ref.numpy(), rtol=1e-4, atol=1e-6)
+    np.testing.assert_allclose(got32.sum(-1, dtype=np.float64), 1.0, atol=1e-5)
+
+
+# ----------------------------------------------------------------------------- selection
+def _golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_select_golden_rows(oracle_mod, case):
+    P = np.array([float(Fraction(p)) for p in case["P"]])
+    r = oracle_mod.select_row(P, case["topk"], case["topp"])
+    assert r["kc"] == case["kc"]
+    assert r["pc"] == case["pc"]
+    assert r["kept"].tolist() == case["kept"]
+
+
+def _brute_select(P_frac, topk, topp):
+    """Exact selection by brute force: ranks from pairwise comparison, running
+    sums in exact rational arithmetic."""
+    n = len(P_frac)
+    rank = [sum(1 for i in range(n) if P_frac[i] > P_frac[j] or (P_frac[i] == P_frac[j] and i < j))
+            for j in range(n)]
+    order = sorted(range(n), key=lambda j: rank[j])
+    kc = min(n, math.ceil(Fraction(topk).limit_denominator(10**9) * n)) if topk > 0 else 0
+    pc = 0
+    if topp > 0:
+        pc = n
+        run = Fraction(0)
+        for m in range(1, n + 1):
+            run += P_frac[order[m - 1]]
+            if run >= Fraction(topp):
+                pc = m
+                break
+    m = max(kc, pc, 1)
+    return sorted(order[:m]), kc, pc
+
+
+def test_select_matches_exact_brute_force():
+    import oracle
+
+    rng = np.random.default_rng(7)
+    for trial in range(400):
+        n = int(rng.integers(1, 9))
+        # Dyadic weights with frequent ties, normalised exactly.
+        w = rng.integers(0, 5, size=n)
+        if w.sum() == 0:
+            w[0] = 1
+        tot = int(w.sum())
+        # Scale to a power-of-two denominator so doubles hold the values exactly.
+        den = 1 << 12
+        num = [int(x) * den // tot for x in w]
+        P_frac = [Fraction(x, den) for x in num]
+        P = np.array([float(x) for x in P_frac])
+        topk = float(rng.choice([0.0, 0.125, 0.25, 0.5, 1.0]))
+        topp = float(rng.choice([0.0, 0.25, 0.5, 0.75, 0.875, 1.0]))
+        kept, kc, pc = _brute_select(P_frac, topk, topp)
+        r = oracle.select_row(P, topk, topp)
+        assert (r["kc"], r["pc"]) == (kc, pc), (P_frac, topk, topp)
+        assert r["kept"].tolist() == kept, (P_frac, topk, topp)
+
+
+def test_select_invariants_random_rows(oracle_mod):
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        n = int(rng.integers(1, 300))
+        P = rng.dirichlet(np.full(n, float(rng.choice([0.05, 1.0, 20.0]))))
+        topk, topp = float(rng.uniform(0, 0.3)), float(rng.uniform(0, 1))
+        r = oracle_mod.select_row(P, topk, topp)
+        kept = set(r["kept"].tolist())
+        order = r["order"].tolist()
+        assert r["kept"].tolist() == sorted(kept)  # ascending, unique
+        assert set(order[: r["kc"]]) <= kept  # mask contains the Top-k set
+        assert set(order[: r["pc"]]) <= kept  # mask contains the Top-p set
+        assert len(kept) == max(r["kc"], r["pc"], 1)
+        if r["pc"] > 0 and r["pc"] < n:
+            assert r["cum"][r["pc"]] >= topp > r["cum"][r["pc"] - 1]
+
+
+def test_mask_single_precision_agrees_with_double(oracle_mod):
+    Q, K, _ = synth.make_qkv(1, 2, 2000, 64, grid=(2, 25, 40), s=1.5, seed=5)
+    i32, c32, P32 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=32)
+    i64, c64, P64 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=64)
+    np.testing.assert_allclose(P32, P64, rtol=1e-3, atol=1e-7)
+    same = (c32 == c64) & np.all(i32 == i64, axis=-1)
+    assert same.mean() > 0.95
+    np.testing.assert_allclose(P64.sum(-1), 1.0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- attention
+def test_dense_matches_sdpa(oracle_mod):
+    q, k, v = _rand_qkv(1, 2, 200, 16, 21, scale=1.5)
+    O, lse = oracle_mod.attention_rows(q, k, v, 64, 32, mode="dense")
+    ref = F.scaled_dot_product_attention(q.double(), k.double(), v.double())
+    np.testing.assert_allclose(O.reshape(1, 2, 200, 16), ref.numpy(), rtol=0, atol=1e-12)
+    s = (q.double() @ k.double().transpose(-1, -2)) / math.sqrt(16)
+    np.testing.assert_allclose(lse.reshape(1, 2, 200), torch.logsumexp(s, -1).numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("N,bq,bk", [(200, 64, 32), (256, 128, 64), (130, 128, 64)])
+def test_sparse_matches_masked_sdpa(oracle_mod, N, bq, bk):
+    q, k, v = _rand_qkv(1, 2, N, 16, 22, scale=1.5)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx, kv_cnt = synth.random_mask(1, 2, nqb, nkb, nkb, seed=N)
+    # masked SDPA needs at least one key per row: give empty rows block 0
+    empty = kv_cnt == 0
+    kv_cnt[empty] = 1
+    kv_idx[..., 0][empty] = 0
+    O, lse = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    m = torch.from_numpy(_block_bool_mask(kv_idx.numpy(), kv_cnt.numpy(), N, bq, bk))
+    ref = F.scaled_dot_product_attention(q.double(), k.double(), v.double(), attn_mask=m)
+    np.testing.assert_allclose(O.reshape(1, 2, N, 16), ref.numpy(), rtol=0, atol=1e-12)
+    s = (q.double() @ k.double().transpose(-1, -2)) / math.sqrt(16)
+    s = s.masked_fill(~m, -math.inf)
+    np.testing.assert_allclose(lse.reshape(1, 2, N), torch.logsumexp(s, -1).numpy(), atol=1e-12)
+
+
+def test_all_blocks_kept_equals_dense(oracle_mod):
+    N, bq, bk = 200, 64, 32
+    q, k, v = _rand_qkv(1, 1, N, 8, 23, scale=2.0)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx = np.tile(np.arange(nkb, dtype=np.int32), (1, 1, nqb, 1))
+    kv_cnt = np.full((1, 1, nqb), nkb, np.int32)
+    Os, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    Od, _ = oracle_mod.attention_rows(q, k, v, bq, bk, mode="dense")
+    np.testing.assert_allclose(Os, Od, rtol=0, atol=1e-12)
+    # and the mask itself keeps all blocks when k = 1
+    idx, cnt, _ = oracle_mod.mask(q, k, bq, bk, 1.0, 0.0)
+    assert (cnt == nkb).all()
+    idx, cnt, _ = oracle_mod.mask(q, k, bq, bk, 0.0, 1.0, precision=64)
+    assert (cnt >= 1).all()
+
+
+def test_constant_v_and_zero_q_closed_forms(oracle_mod):
+    N, bq, bk, d = 150, 64, 32, 8
+    q, k, _ = _rand_qkv(1, 1, N, d, 24, scale=2.0)
+    v = _bf16(torch.full((1, 1, N, d), 0.75))
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx, kv_cnt = synth.random_mask(1, 1, nqb, nkb, 2, seed=3)
+    alpha = np.array([0.3], np.float32)
+    for mode in ("sparse", "linear", "sla2", "dense"):
+        O, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, alpha, mode=mode)
+        rows_nonempty = []
+        for i in range(N):
+            c = int(kv_cnt[0, 0, i // bq])
+            kept_keys = sum(min(bk, N - int(J) * bk) for J in kv_idx[0, 0, i // bq, :c])
+            sparse_ok = kept_keys > 0
+            linear_ok = kept_keys < N
+            expect = 0.75
+            if mode == "sparse" and not sparse_ok:
+                expect = 0.0
+            if mode == "linear" and not linear_ok:
+                expect = 0.0
+            if mode == "sla2":
+                expect = 0.3 * (0.75 if sparse_ok else 0.0) + 0.7 * (0.75 if linear_ok else 0.0)
+            np.testing.assert_allclose(O[i], expect, atol=1e-12)
+    # Q = 0: uniform weights, the mean of V over the kept valid keys.
+    q0 = _bf16(torch.zeros(1, 1, N, d))
+    _, _, v = _rand_qkv(1, 1, N, d, 25)
+    O, _ = oracle_mod.attention_rows(q0, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    vd = v.double().numpy()[0, 0]
+    for i in range(N):
+        c = int(kv_cnt[0, 0, i // bq])
+        keys = [j for J in kv_idx[0, 0, i // bq, :c] for j in range(int(J) * bk, min(N, int(J) * bk + bk))]
+        expect = vd[keys].mean(0) if keys else np.zeros(d)
+        np.testing.assert_allclose(O[i], expect, atol=1e-12)
+
+
+def test_empty_row_gives_zero_and_neg_inf_lse(oracle_mod):
+    q, k, v = _rand_qkv(1, 1, 64, 8, 26)
+    kv_idx = np.zeros((1, 1, 1, 1), np.int32)
+    kv_cnt = np.zeros((1, 1, 1), np.int32)
+    O, lse = oracle_mod.attention_rows(q, k, v, 64, 64, kv_idx, kv_cnt, mode="sparse")
+    assert np.all(O == 0) and np.all(np.isneginf(lse))
+
+
+def test_linear_branch_matches_associative_form(oracle_mod):
+    # Empty mask: the complement is every key, and the normalised linear
+    # attention equals phi(Q) (phi(K)^T V) / (phi(Q) . sum_j phi(k_j)).
+    N, d = 130, 16
+    q, k, v = _rand_qkv(1, 2, N, d, 27, scale=1.5)
+    kv_idx = np.zeros((1, 2, 2, 3), np.int32)
+    kv_cnt = np.zeros((1, 2, 2), np.int32)
+    O, _ = oracle_mod.attention_rows(q, k, v, 128, 64, kv_idx, kv_cnt, mode="linear")
+    pq, pk = _phi_torch(q.double()), _phi_torch(k.double())
+    num = pq @ (pk.transpose(-1, -2) @ v.double())
+    den = pq @ pk.sum(-2, keepdim=True).transpose(-1, -2)
+    np.testing.assert_allclose(O.reshape(1, 2, N, d), (num / den).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_branch_matches_masked_quadratic_form(oracle_mod):
+    N, bq, bk, d = 200, 64, 32, 8
+    q, k, v = _rand_qkv(1, 2, N, d, 28, scale=1.2)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx, kv_cnt = synth.random_mask(1, 2, nqb, nkb, nkb - 1, seed=9)
+    O, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="linear")
+    keep = torch.from_numpy(_block_bool_mask(kv_idx.numpy(), kv_cnt.numpy(), N, bq, bk))
+    W = (_phi_torch(q.double()) @ _phi_torch(k.double()).transpose(-1, -2)) * (~keep)
+    ref = (W @ v.double()) / W.sum(-1, keepdim=True)
+    np.testing.assert_allclose(O.reshape(1, 2, N, d), ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_phi_is_elu_plus_one(oracle_mod):
+    # With one key outside the kept set, O_l = v of that key regardless of phi,
+    # so use two keys and a scalar feature: weights phi(q) phi(k_j).
+    xs = [-3.0, -0.5, 0.0, 0.25, 2.0]
+    for x in xs:
+        q = _bf16(torch.tensor([x]).reshape(1, 1, 1, 1).expand(1, 1, 2, 1).contiguous())
+        k = _bf16(torch.tensor([x, 1.0]).reshape(1, 1, 2, 1))
+        v = _bf16(torch.tensor([1.0, 0.0]).reshape(1, 1, 2, 1))
+        kv_idx = np.zeros((1, 1, 1, 2), np.int32)
+        kv_cnt = np.zeros((1, 1, 1), np.int32)
+        O, _ = oracle_mod.attention_rows(q, k, v, 2, 1, kv_idx, kv_cnt, mode="linear")
+        ph = float(F.elu(torch.tensor(float(q[0, 0, 0, 0]), dtype=torch.float64)) + 1)
+        pk0 = float(F.elu(torch.tensor(float(k[0, 0, 0, 0]), dtype=torch.float64)) + 1)
+        pk1 = float(F.elu(torch.tensor(1.0, dtype=torch.float64)) + 1)
+        expect = ph * pk0 / (ph * pk0 + ph * pk1)
+        np.testing.assert_allclose(O[0, 0], expect, atol=1e-14)
+
+
+def test_sla2_mix_endpoints_and_linearity(oracle_mod):
+    N, bq, bk, d = 192, 64, 32, 8
+    q, k, v = _rand_qkv(1, 3, N, d, 29, scale=1.3)
+    nqb, nkb = N // bq, N // bk
+    kv_idx, kv_cnt = synth.random_mask(1, 3, nqb, nkb, 3, seed=4)
+    Os, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    Ol, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="linear")
+    a1, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, np.ones(3, np.float32), mode="sla2")
+    a0, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, np.zeros(3, np.float32), mode="sla2")
+    np.testing.assert_array_equal(a1, Os)
+    np.testing.assert_array_equal(a0, Ol)
+    al = np.array([0.6, 0.75, 1.0], np.float32)
+    am, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, al, mode="sla2")
+    w = np.repeat(al.astype(np.float64), N)[:, None]
+    np.testing.assert_allclose(am, w * Os + (1 - w) * Ol, atol=1e-14)
+
+
+def test_key_permutation_within_block_is_invisible(oracle_mod):
+    N, bq, bk, d = 128, 64, 32, 8
+    q, k, v = _rand_qkv(1, 1, N, d, 30, scale=1.5)
+    kv_idx, kv_cnt = synth.random_mask(1, 1, 2, 4, 3, seed=6)
+    perm = torch.cat([torch.randperm(bk, generator=torch.Generator().manual_seed(J)) + J * bk for J in range(4)])
+    kp, vp = k[:, :, perm].contiguous(), v[:, :, perm].contiguous()
+    for mode in ("sparse", "linear"):
+        a, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode=mode)
+        b, _ = oracle_mod.attention_rows(q, kp, vp, bq, bk, kv_idx, kv_cnt, mode=mode)
+        np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+def test_sampled_rows_equal_full_rows(oracle_mod):
+    q, k, v = _rand_qkv(1, 2, 160, 8, 31)
+    kv_idx, kv_cnt = synth.random_mask(1, 2, 3, 5, 3, seed=8)
+    full, lse = oracle_mod.attention_rows(q, k, v, 64, 32, kv_idx, kv_cnt, mode="sparse")
+    rows = np.array([319, 0, 200, 17, 160], np.int64)
+    part, lse_p = oracle_mod.attention_rows(q, k, v, 64, 32, kv_idx, kv_cnt, mode="sparse", rows=rows)
+    np.testing.assert_array_equal(part, full[rows])
+    np.testing.assert_array_equal(lse_p, lse[rows])
+
+
+def test_invalid_arguments_are_rejected(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.select_row(np.array([0.5, 0.5]), 1.5, 0.5)
+    q, k, v = _rand_qkv(1, 1, 64, 8, 32)
+    kv_idx = np.full((1, 1, 1, 1), 5, np.int32)  # block index out of range
+    kv_cnt = np.ones((1, 1, 1), np.int32)
+    with pytest.raises(ValueError):
+        oracle_mod.attention_rows(q, k, v, 64, 64, kv_idx, kv_cnt, mode="sparse")
