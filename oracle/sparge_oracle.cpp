@@ -46,7 +46,8 @@
 // and the single-precision decision with a fixed operation order that the GPU
 // kernel also follows (pool: sequential float sum over rows, then divide by the
 // row count; score: sequential fused multiply-add over channels, then multiply
-// by (float)(1/sqrt(d)); softmax: expf(z - max) / sum).
+// by (float)(1/sqrt(d)); softmax: expf(z - max) / sum, the row sum taken as
+// 32 interleaved partial sums combined pairwise).
 
 #include <algorithm>
 #include <cmath>
@@ -153,7 +154,8 @@ int oracle_block_probs_f64(const double* qbar, const double* kbar, int64_t BH, i
 }
 
 // Single precision with the GPU kernel's operation order: sequential fmaf over
-// channels, times (float)(1/sqrt(d)); expf(z - max); divide by the row sum.
+// channels, times (float)(1/sqrt(d)); expf(z - max); divide by the row sum
+// (32 interleaved partial sums combined pairwise).
 int oracle_block_probs_f32(const float* qbar, const float* kbar, int64_t BH, int64_t Nqb,
                            int64_t Nkb, int d, float* P) {
   if (!qbar || !kbar || !P || BH <= 0 || Nqb <= 0 || Nkb <= 0 || d <= 0) return ERR_ARG;
@@ -170,11 +172,21 @@ int oracle_block_probs_f32(const float* qbar, const float* kbar, int64_t BH, int
         z[J] = dot * scale;
         mx = std::max(mx, z[J]);
       }
-      float sum = 0.0f;
+      // Row sum in the kernel's order: 32 interleaved partial sums (partial
+      // l adds the terms l, l+32, l+64, ... in turn), then combined pairwise
+      // at distances 16, 8, 4, 2, 1.
+      float part[32];
+      for (int l = 0; l < 32; ++l) part[l] = 0.0f;
       for (int64_t J = 0; J < Nkb; ++J) {
         z[J] = std::exp(z[J] - mx);
-        sum = sum + z[J];
+        part[J % 32] = part[J % 32] + z[J];
       }
+      for (int o = 16; o > 0; o >>= 1) {
+        float nxt[32];
+        for (int l = 0; l < 32; ++l) nxt[l] = part[l] + part[l ^ o];
+        for (int l = 0; l < 32; ++l) part[l] = nxt[l];
+      }
+      const float sum = part[0];
       float* row = P + (bh * Nqb + I) * Nkb;
       for (int64_t J = 0; J < Nkb; ++J) row[J] = z[J] / sum;
     }
