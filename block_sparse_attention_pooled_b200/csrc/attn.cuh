@@ -1,0 +1,345 @@
+// Block-sparse attention forward on the 5th-generation tensor cores.
+//
+// What it computes (SpargeAttention2 article, arXiv:2602.13515, section 4:
+// attention runs block by block and each block is either fully computed or
+// fully skipped; SLA2 article, arXiv:2602.12675, section 2: the sparse branch
+// is renormalised over the kept region only):
+//   O[i] = sum_{j in kept keys of block(i)} softmax_j(q_i . k_j / sqrt(d)) v_j
+//
+// One CTA owns one 128-row query tile of one (batch, head) and walks only the
+// key tiles (64 keys each) of that tile's kept blocks:
+//   warp 0      TMA producer: Q once, then K and V tiles into two 2-slot rings;
+//   warp 1      MMA issuer and TMEM owner: S = Q K^T into a double-buffered
+//               TMEM S, then O += P V with P read back from TMEM;
+//   warps 2..5  softmax: one query row per thread (TMEM lane), fp32 online
+//               softmax with lazy rescaling, P written to TMEM as bf16 over
+//               its own S columns; then the epilogue (O / l -> bf16 -> TMA
+//               store, optional log-sum-exp).
+// TMEM columns: S0 [0,64), S1 [64,128), O [128,128+D).
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace sparge {
+
+constexpr int kAttnThreads = 192;
+constexpr int kTileQ = 128;   // query rows per MMA tile
+constexpr int kTileK = 64;    // keys per MMA tile
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+
+// Error site codes recorded in g_device_error by the attention kernel.
+enum : unsigned int {
+  kErrAttnQ = 0x100, kErrAttnKFull, kErrAttnVFull, kErrAttnKEmpty, kErrAttnVEmpty, kErrAttnSFull,
+  kErrAttnPFull, kErrAttnODone, kErrAttnOFinal, kErrAttnDrain
+};
+
+struct AttnParams {
+  const int32_t* kv_idx;  // [BH, nqb, nkb]
+  const int32_t* kv_cnt;  // [BH, nqb]
+  float* lse;             // [BH, N] or null
+  int N;
+  int nqb;
+  int nkb;
+  int bq;                 // 64 or 128: rows of the query block that share a mask row
+  int bk;                 // 64 or 128: keys per mask block (bk / 64 key tiles each)
+  float scale_log2;       // log2(e) / sqrt(d)
+};
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kQBytes = kTileQ * D * 2;
+  static constexpr int kKBytes = kTileK * D * 2;
+  static constexpr int kVBytes = kTileK * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + 2 * kKBytes;
+  static constexpr int kOffBar = kOffV + 2 * kVBytes;
+  static constexpr int kNumBars = 16;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kUsed = kOffTmem + 16;
+  // Pad so that at most two CTAs fit on an SM: two CTAs x 256 TMEM columns
+  // use the SM's 512 columns exactly, and a third would block in alloc.
+  static constexpr int kBytes = (kUsed + 1024 > 80 * 1024 ? kUsed + 1024 : 80 * 1024);
+};
+
+// Barrier slots.
+enum { kBarQ = 0, kBarKFull = 1, kBarVFull = 3, kBarKEmpty = 5, kBarVEmpty = 7, kBarSFull = 9,
+       kBarPFull = 11, kBarODone = 13, kBarOFinal = 14, kBarDrain = 15 };
+
+// Waits on an mbarrier unless another role already gave up; gives up itself
+// (and tells the others through *abort) after the global time limit.
+__device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, unsigned int site,
+                                          volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(site);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// First key of key tile t of a query tile whose kept-block list is `lst`.
+__device__ __forceinline__ int tile_key0(const int32_t* lst, int t, int tiles_per_block, int bk) {
+  const int e = t / tiles_per_block;
+  return __ldg(lst + e) * bk + (t % tiles_per_block) * kTileK;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const AttnParams p) {
+  using L = AttnSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const uint32_t sQ = sbase + L::kOffQ, sK = sbase + L::kOffK, sV = sbase + L::kOffV;
+  const uint32_t bar0 = sbase + L::kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tile = blockIdx.x;                 // (bh, query block), head-major
+  const int bh = tile / p.nqb;
+  const int qb = tile % p.nqb;
+  const int q0 = qb * p.bq;                    // first query row of the tile
+  const int tiles_per_block = p.bk / kTileK;
+  const int cnt = min(max(__ldg(p.kv_cnt + tile), 0), p.nkb);  // a bad count cannot walk past the list
+  const int T = cnt * tiles_per_block;         // key tiles to visit
+  const int32_t* lst = p.kv_idx + (int64_t)tile * p.nkb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQ), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+      mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarPFull + s), 128);
+    }
+    mbar_init(bar(kBarODone), 1);
+    mbar_init(bar(kBarOFinal), 1);
+    mbar_init(bar(kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::kOffTmem, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && T > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar(kBarQ), L::kQBytes);
+      for (int b = 0; b < D / 64; ++b) tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(kBarQ), b * 64, q0, bh);
+      int nk = 0, nv = 0;  // K and V tiles issued
+      for (int t = 0; t < T; ++t) {
+        const int slot = t & 1;
+        const int key0 = tile_key0(lst, t, tiles_per_block, p.bk);
+        if (t >= 2 && !role_wait(bar(kBarKEmpty + slot), ((t >> 1) - 1) & 1, kErrAttnKEmpty, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(kBarKFull + slot), L::kKBytes);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(sK + slot * L::kKBytes + b * (kTileK * 128), &tmK, bar(kBarKFull + slot), b * 64, key0, bh);
+        ++nk;
+        if (t >= 2 && !role_wait(bar(kBarVEmpty + slot), ((t >> 1) - 1) & 1, kErrAttnVEmpty, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(kBarVFull + slot), L::kVBytes);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(sV + slot * L::kVBytes + b * (kTileK * 128), &tmV, bar(kBarVFull + slot), b * 64, key0, bh);
+        ++nv;
+      }
+      // Never leave with copies in flight: wait for the last loads issued to
+      // land (they normally have; this only matters when a role gave up).
+      mbar_wait(bar(kBarQ), 0, kErrAttnQ);
+      for (int t = (nk > 2 ? nk - 2 : 0); t < nk; ++t) mbar_wait(bar(kBarKFull + (t & 1)), (t >> 1) & 1, kErrAttnKFull);
+      for (int t = (nv > 2 ? nv - 2 : 0); t < nv; ++t) mbar_wait(bar(kBarVFull + (t & 1)), (t >> 1) & 1, kErrAttnVFull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kTileQ, kTileK, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kTileQ, D, false, true);
+      bool ok = role_wait(bar(kBarQ), 0, kErrAttnQ, abort_flag);
+      tc_fence_after();
+      for (int t = 0; ok && t <= T; ++t) {
+        if (t < T) {
+          const int slot = t & 1;
+          if (!role_wait(bar(kBarKFull + slot), (t >> 1) & 1, kErrAttnKFull, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t kbase = sK + slot * L::kKBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32u;  // 16 bf16 = 32 bytes along K inside the swizzle row
+            const uint64_t a = sdesc_sw128(sQ + (kk >> 2) * (kTileQ * 128) + off, 16, 1024);
+            const uint64_t b = sdesc_sw128(kbase + (kk >> 2) * (kTileK * 128) + off, 16, 1024);
+            mma_ss(tS + slot * 64, a, b, idS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(kBarSFull + slot));
+          mma_commit(bar(kBarKEmpty + slot));
+        }
+        if (t >= 1) {
+          const int u = t - 1, slot = u & 1;
+          if (!role_wait(bar(kBarPFull + slot), (u >> 1) & 1, kErrAttnPFull, abort_flag)) break;
+          if (!role_wait(bar(kBarVFull + slot), (u >> 1) & 1, kErrAttnVFull, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t vbase = sV + slot * L::kVBytes;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            const uint64_t b = sdesc_sw128(vbase + kk * (16 * 128), kTileK * 128, 1024);
+            mma_ts(tO, tS + slot * 64 + kk * 8, b, idPV, (u > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(kBarVEmpty + slot));
+          mma_commit(bar(kBarODone));
+          if (u == T - 1) mma_commit(bar(kBarOFinal));
+        }
+      }
+      // Drain: every MMA this thread issued has completed before TMEM is freed.
+      mma_commit(bar(kBarDrain));
+      mbar_wait(bar(kBarDrain), 0, kErrAttnDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int r = q * 32 + lane;             // row of the query tile
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int slot = t & 1;
+      ok = __all_sync(0xffffffffu, role_wait(bar(kBarSFull + slot), (t >> 1) & 1, kErrAttnSFull, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kTileK];
+      {
+        uint32_t v[4][16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld16(tS + lane_off + slot * 64 + 16 * c, v[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(v[c][j]);
+      }
+      const int key0 = tile_key0(lst, t, tiles_per_block, p.bk);
+      if (key0 + kTileK > p.N) {
+#pragma unroll
+        for (int j = 0; j < kTileK; ++j)
+          if (key0 + j >= p.N) s[j] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kTileK; ++j) mx = fmaxf(mx, s[j]);
+      const float m_new = fmaxf(m_run, mx * p.scale_log2);
+      if (t == 0) {
+        m_run = m_new;
+      } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold)) {
+        // O holds sum_j 2^(s_j - m_run) v_j; move it to the new reference.
+        // The decision is warp-wide (TMEM loads and stores are warp
+        // collectives); each row scales by its own factor (1 if its max held).
+        ok = __all_sync(0xffffffffu, role_wait(bar(kBarODone), (t - 1) & 1, kErrAttnODone, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const float f = ex2_approx(m_run - m_new);
+        uint32_t v[16];
+#pragma unroll 1
+        for (int c = 0; c < D; c += 16) {
+          tmem_ld16(tO + lane_off + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+          tmem_st16(tO + lane_off + c, v);
+        }
+        tmem_st_wait();
+        l_run *= f;
+        m_run = m_new;
+      }
+      const float neg_m = -m_run;
+      float psum = 0.0f;
+      uint32_t pk[kTileK / 2];
+#pragma unroll
+      for (int j = 0; j < kTileK; j += 2) {
+        const float a = ex2_approx(fmaf(s[j], p.scale_log2, neg_m));
+        const float b = ex2_approx(fmaf(s[j + 1], p.scale_log2, neg_m));
+        psum += a + b;
+        pk[j / 2] = pack_bf16x2(a, b);
+      }
+      l_run += psum;
+      // P (bf16) overwrites the first 32 columns of this S buffer.
+      tmem_st16(tS + lane_off + slot * 64, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      tmem_st16(tS + lane_off + slot * 64 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + slot));
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, role_wait(bar(kBarOFinal), 0, kErrAttnOFinal, abort_flag));
+      tc_fence_after();
+    }
+    // Epilogue: O / l -> bf16 rows into the (now idle) Q buffer, laid out the
+    // way the 128-byte-swizzled O tensor map expects, then TMA stores.
+    const float inv_l = (T > 0 && l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < D; c += 16) {
+      uint32_t v[16];
+      if (T > 0 && ok) {
+        tmem_ld16(tO + lane_off + c, v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0u;
+      }
+      uint32_t w[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        w[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
+      const int box = c / 64, cc = c % 64;             // column within the 64-wide box
+      const uint32_t row_addr = sQ + box * (kTileQ * 128) + r * 128;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int chunk = (cc / 8 + h) ^ (r & 7);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
+                     "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
+                     : "memory");
+      }
+    }
+    if (p.lse != nullptr && r < p.bq && q0 + r < p.N) {
+      const float lse = (T > 0 && l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      p.lse[(int64_t)bh * p.N + q0 + r] = lse;
+    }
+    fence_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0) {
+      for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmO, sQ + b * (kTileQ * 128), b * 64, q0, bh);
+      tma_store_commit();
+      tma_store_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace sparge

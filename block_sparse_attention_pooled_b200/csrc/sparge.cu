@@ -1,0 +1,256 @@
+// Host side of the C ABI declared in include/sparge.h: argument checks,
+// workspace carving, TMA descriptors and kernel launches. All kernels of the
+// library are compiled in this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sparge.h"
+#include "ptx.cuh"
+#include "mask.cuh"
+#include "attn.cuh"
+
+namespace {
+
+using namespace sparge;
+
+constexpr int kMaxNkb = 4096;
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Dims {
+  int64_t BH, nqb, nkb;
+};
+
+// Shape checks shared by every entry point. Returns OK / INVALID / UNSUPPORTED.
+sparge_status check_shape(const sparge_shape* s, Dims* out) {
+  if (s == nullptr) return SPARGE_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->H <= 0 || s->N <= 0 || s->d <= 0 || s->bq <= 0 || s->bk <= 0) return SPARGE_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return SPARGE_ERR_UNSUPPORTED;
+  if (s->bq != 64 && s->bq != 128) return SPARGE_ERR_UNSUPPORTED;
+  if (s->bk != 64 && s->bk != 128) return SPARGE_ERR_UNSUPPORTED;
+  out->BH = (int64_t)s->B * s->H;
+  out->nqb = ceil_div(s->N, s->bq);
+  out->nkb = ceil_div(s->N, s->bk);
+  if (out->nkb > kMaxNkb) return SPARGE_ERR_UNSUPPORTED;
+  if (out->BH * out->nqb > INT32_MAX || out->BH > INT32_MAX) return SPARGE_ERR_UNSUPPORTED;
+  return SPARGE_OK;
+}
+
+sparge_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SPARGE_OK;
+  (void)cudaGetLastError();  // clear the sticky-free launch error
+  return SPARGE_ERR_CUDA;
+}
+
+struct MaskWs {
+  size_t qbar, kbar, probs, total;
+};
+
+MaskWs mask_ws(const sparge_shape* s, const Dims& d) {
+  MaskWs w;
+  w.qbar = 0;
+  w.kbar = w.qbar + align256((size_t)d.BH * d.nqb * s->d * 4);
+  w.probs = w.kbar + align256((size_t)d.BH * d.nkb * s->d * 4);
+  w.total = w.probs + align256((size_t)d.BH * d.nqb * d.nkb * 4);
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link-time libcuda).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over [BH][N][d] with a (64 columns x rows x 1) box, 128-byte
+// swizzle, zero fill outside the tensor.
+bool make_map_bhnd(CUtensorMap* m, const void* base, int64_t BH, int N, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Raises a kernel's dynamic shared memory limit once per device.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes, int slot) {
+  static int done[64][8];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && done[dev][slot] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev < 64) done[dev][slot] = bytes;
+  return e;
+}
+
+template <int D>
+sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, const Dims& dm, int kc, double topp,
+                          int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs, uint8_t* ws,
+                          cudaStream_t st) {
+  const MaskWs w = mask_ws(s, dm);
+  float* qbar = reinterpret_cast<float*>(ws + w.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + w.kbar);
+  float* P = probs ? probs : reinterpret_cast<float*>(ws + w.probs);
+  constexpr int per_cta = 128 / (D / 8);
+  const int64_t gq = ceil_div(dm.BH * dm.nqb, per_cta), gk = ceil_div(dm.BH * dm.nkb, per_cta);
+  pool_kernel<D><<<(unsigned)gq, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), dm.BH, s->N, s->bq, qbar);
+  pool_kernel<D><<<(unsigned)gk, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(K), dm.BH, s->N, s->bk, kbar);
+  const float scale = (float)(1.0 / std::sqrt((double)D));
+  const int ssm = score_smem_bytes<D>();
+  cudaError_t e = ensure_smem(score_softmax_kernel<D>, ssm, D == 64 ? 0 : 1);
+  if (e != cudaSuccess) return cuda_status(e);
+  const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows);
+  score_softmax_kernel<D><<<(unsigned)tiles, 128, ssm, st>>>(qbar, kbar, dm.BH, (int)dm.nqb, (int)dm.nkb, scale, P);
+  const int sel_sm = select_smem_bytes((int)dm.nkb);
+  e = ensure_smem(select_kernel, sel_sm, 2);
+  if (e != cudaSuccess) return cuda_status(e);
+  select_kernel<<<(unsigned)(dm.BH * dm.nqb), kSelectThreads, sel_sm, st>>>(P, dm.BH * dm.nqb, (int)dm.nkb, kc, topp,
+                                                                           kv_idx, kv_cnt, row_thresh);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+sparge_status launch_attn(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
+                          const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, D, s->bq))
+    return SPARGE_ERR_CUDA;
+  AttnParams p;
+  p.kv_idx = kv_idx;
+  p.kv_cnt = kv_cnt;
+  p.lse = lse;
+  p.N = s->N;
+  p.nqb = (int)dm.nqb;
+  p.nkb = (int)dm.nkb;
+  p.bq = s->bq;
+  p.bk = s->bk;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  const int smem = AttnSmem<D>::kBytes;
+  cudaError_t e = ensure_smem(attn_fwd_kernel<D>, smem, D == 64 ? 3 : 4);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_fwd_kernel<D><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st>>>(mq, mk, mv, mo, p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
+  Dims dm;
+  if (check_shape(shape, &dm) != SPARGE_OK) return 0;
+  switch (op) {
+    case SPARGE_OP_MASK:
+      return mask_ws(shape, dm).total;
+    case SPARGE_OP_ATTN:
+      return 0;
+    case SPARGE_OP_SLA2:
+      return 0;
+    default:
+      return 0;
+  }
+}
+
+sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shape, double topk_frac, double topp,
+                          int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || (probs && !aligned16(probs))) return SPARGE_ERR_INVALID_ARG;
+  if (!(topk_frac >= 0.0 && topk_frac <= 1.0) || !(topp >= 0.0 && topp <= 1.0)) return SPARGE_ERR_INVALID_ARG;
+  const size_t need = mask_ws(shape, dm).total;
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
+  int kc = 0;
+  if (topk_frac > 0.0) {
+    const double c = std::ceil(topk_frac * (double)dm.nkb - 1e-9);
+    kc = (int)std::min<double>(std::max<double>(c, 0.0), (double)dm.nkb);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (shape->d == 64) return launch_mask<64>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
+  return launch_mask<128>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
+}
+
+sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !V || !O || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARGE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (shape->d == 64) return launch_attn<64>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, s);
+  return launch_attn<128>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, s);
+}
+
+sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                            const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, void* O,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  (void)Q; (void)K; (void)V; (void)kv_idx; (void)kv_cnt; (void)alpha; (void)O;
+  (void)workspace; (void)workspace_bytes; (void)stream;
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  return SPARGE_ERR_UNSUPPORTED;
+}
+
+sparge_status sparge_device_status(void* stream, int32_t* code) {
+  if (code == nullptr) return SPARGE_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_status(e);
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, sparge::g_device_error, sizeof v);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = cudaMemcpyToSymbol(sparge::g_device_error, &zero, sizeof zero);
+  if (e != cudaSuccess) return cuda_status(e);
+  *code = (int32_t)v;
+  return v ? SPARGE_ERR_DEVICE_TIMEOUT : SPARGE_OK;
+}
+
+const char* sparge_status_string(sparge_status status) {
+  switch (status) {
+    case SPARGE_OK: return "ok";
+    case SPARGE_ERR_INVALID_ARG: return "invalid argument";
+    case SPARGE_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case SPARGE_ERR_WORKSPACE: return "workspace missing or too small";
+    case SPARGE_ERR_CUDA: return "CUDA error";
+    case SPARGE_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

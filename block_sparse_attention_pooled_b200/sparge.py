@@ -1,0 +1,155 @@
+"""Python binding of the C ABI in include/sparge.h (argument marshalling only).
+
+Importing this module loads ``libsparge.so`` from the package directory and
+raises ImportError when it is missing: there is no fallback implementation.
+Tensors are torch CUDA tensors; every call is enqueued on the current torch
+stream (or the stream given) and returns without synchronising.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsparge.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m block_sparse_attention_pooled_b200.build`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
+OP_MASK, OP_ATTN, OP_SLA2 = 0, 1, 2
+
+# Every symbol the header declares.
+EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
+           "sparge_device_status", "sparge_status_string")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "d", "bq", "bk")]
+
+
+_vp, _sz, _dbl = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_double
+_lib.sparge_workspace_bytes.argtypes = [ctypes.c_int, ctypes.POINTER(Shape)]
+_lib.sparge_workspace_bytes.restype = _sz
+_lib.sparge_mask.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _dbl, _dbl, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sparge_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sla2_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
+_lib.sparge_status_string.argtypes = [ctypes.c_int]
+_lib.sparge_status_string.restype = ctypes.c_char_p
+for _f in ("sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status"):
+    getattr(_lib, _f).restype = ctypes.c_int
+
+
+class SpargeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {_lib.sparge_status_string(code).decode()} (status {code})")
+        self.code = code
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def raw() -> ctypes.CDLL:
+    """The loaded library (for callers that marshal pointers themselves)."""
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise SpargeError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_shape(Q: torch.Tensor, bq: int, bk: int) -> Shape:
+    B, H, N, d = Q.shape
+    return Shape(B, H, N, d, bq, bk)
+
+
+def workspace_bytes(op: int, shape: Shape) -> int:
+    return int(_lib.sparge_workspace_bytes(op, ctypes.byref(shape)))
+
+
+def _workspace(op: int, shape: Shape, device) -> Tuple[Optional[torch.Tensor], int]:
+    n = workspace_bytes(op, shape)
+    if n == 0:
+        return None, 0
+    return torch.empty(n, dtype=torch.uint8, device=device), n
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("Q/K/V/O must be contiguous bf16 CUDA tensors of shape [B,H,N,d]")
+
+
+def sparge_mask(Q, K, bq: int, bk: int, topk: float, topp: float, kv_idx=None, kv_cnt=None,
+                row_thresh=None, probs=None, workspace=None, stream=None):
+    """Hybrid Top-k / Top-p block mask. Returns (kv_idx, kv_cnt)."""
+    _check_qkv(Q, K)
+    shape = make_shape(Q, bq, bk)
+    B, H, N, _ = Q.shape
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, H, nqb, nkb), dtype=torch.int32, device=Q.device)
+    if kv_cnt is None:
+        kv_cnt = torch.empty((B, H, nqb), dtype=torch.int32, device=Q.device)
+    if workspace is None:
+        workspace, nws = _workspace(OP_MASK, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sparge_mask(_ptr(Q), _ptr(K), ctypes.byref(shape), float(topk), float(topp), _ptr(kv_idx),
+                            _ptr(kv_cnt), _ptr(row_thresh), _ptr(probs), _ptr(workspace), nws, _stream(stream)),
+           "sparge_mask")
+    return kv_idx, kv_cnt
+
+
+def sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, bq: int, bk: int, O=None, lse=None, workspace=None, stream=None):
+    """Block-sparse attention over the kept blocks. Returns O (and fills lse if given)."""
+    _check_qkv(Q, K, V)
+    shape = make_shape(Q, bq, bk)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace, nws = _workspace(OP_ATTN, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sparge_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt), _ptr(O),
+                                _ptr(lse), _ptr(workspace), nws, _stream(stream)), "sparge_attn_fwd")
+    return O
+
+
+def sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, bq: int, bk: int, O=None, workspace=None, stream=None):
+    """alpha * sparse + (1 - alpha) * linear (phi = elu + 1 over the blocks not kept). Returns O."""
+    _check_qkv(Q, K, V)
+    shape = make_shape(Q, bq, bk)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace, nws = _workspace(OP_SLA2, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sla2_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt),
+                              _ptr(alpha), _ptr(O), _ptr(workspace), nws, _stream(stream)), "sla2_attn_fwd")
+    return O
+
+
+def device_status(stream=None) -> int:
+    """Synchronises the stream, returns and clears the device error word (0 = none)."""
+    code = ctypes.c_int32(0)
+    rc = _lib.sparge_device_status(_stream(stream), ctypes.byref(code))
+    if rc not in (OK, ERR_DEVICE_TIMEOUT):
+        raise SpargeError(rc, "sparge_device_status")
+    return int(code.value)

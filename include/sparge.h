@@ -1,0 +1,136 @@
+/*
+ * sparge.h - C ABI of the pooled block-sparse attention library (sm_100a).
+ *
+ * Three operations, each one stream-ordered launch sequence on the caller's
+ * CUDA stream:
+ *
+ *   sparge_mask      block mask: mean-pool Q and K per block, score the
+ *                    pooled blocks with softmax(qbar . kbar / sqrt(d)) along
+ *                    each query-block row, keep the union of the Top-k and
+ *                    Top-p selections. SpargeAttention2 article ("Tsinghua
+ *                    invents an AI attention-slimming technique",
+ *                    arXiv:2602.13515), section 1 (Top-k, Top-p and their
+ *                    merge) and section 4 (pooling pre-filter, block-level
+ *                    mask, blocks computed whole or skipped whole).
+ *   sparge_attn_fwd  block-sparse attention over the kept blocks only, softmax
+ *                    renormalised over the kept keys. Same article, section 4;
+ *                    SLA2 article (arXiv:2602.12675), section 2 (the sparse
+ *                    branch is renormalised over the kept region).
+ *   sla2_attn_fwd    O = alpha_h * O_sparse + (1 - alpha_h) * O_linear, the
+ *                    linear branch being phi-feature attention,
+ *                    phi(x) = elu(x) + 1, over the keys of the blocks NOT kept.
+ *                    SLA2 article, section 1 (sparse attention for important
+ *                    regions, linear attention for the rest) and section 2
+ *                    (learnable mixing ratio alpha).
+ *
+ * Conventions shared by every entry point
+ *   - Q, K, V, O: bf16, [B, H, N, d] contiguous (d fastest), device memory,
+ *     16-byte aligned. d is 64 or 128 (sla2_attn_fwd: 128).
+ *   - Blocks: bq query rows and bk keys per block, each 64 or 128.
+ *     Nqb = ceil(N / bq), Nkb = ceil(N / bk); a ragged last block holds the
+ *     remaining rows only. No causal masking.
+ *   - Block mask: kv_idx int32 [B, H, Nqb, Nkb] and kv_cnt int32 [B, H, Nqb].
+ *     Row (b, h, I) keeps the kv_cnt[b,h,I] blocks kv_idx[b,h,I,0..cnt), which
+ *     are strictly ascending and lie in [0, Nkb). Entries past cnt are not
+ *     read and not written. The attention entry points trust these lists
+ *     (they are not validated on the device).
+ *   - Ownership: the caller owns every buffer. The library allocates no
+ *     memory and keeps no state between calls, except the device error word
+ *     read by sparge_device_status.
+ *   - Workspace: scratch device memory of at least
+ *     sparge_workspace_bytes(op, shape) bytes, 256-byte aligned, owned by the
+ *     caller, not used across calls. May be NULL when that size is 0.
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued on it; the calls return without synchronising.
+ *   - Errors: arguments are checked on the host before anything is launched;
+ *     a failed check returns a status and launches nothing. A failed launch
+ *     returns SPARGE_ERR_CUDA. Device-side waits are bounded: a kernel that
+ *     gives up records a code that sparge_device_status returns. Nothing
+ *     crosses the ABI as an exception.
+ *   - Determinism: identical inputs give bit-identical outputs.
+ */
+#ifndef SPARGE_H_
+#define SPARGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPARGE_OK = 0,
+  SPARGE_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, bad fraction, misaligned buffer */
+  SPARGE_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement (d, bq, bk, Nkb) */
+  SPARGE_ERR_WORKSPACE = 3,    /* workspace missing or smaller than sparge_workspace_bytes */
+  SPARGE_ERR_CUDA = 4,         /* a CUDA call or launch failed */
+  SPARGE_ERR_DEVICE_TIMEOUT = 5 /* a kernel gave up a bounded wait (from sparge_device_status) */
+} sparge_status;
+
+typedef struct {
+  int32_t B, H, N, d; /* batch, heads, tokens, head dim */
+  int32_t bq, bk;     /* query rows per block, keys per block */
+} sparge_shape;
+
+enum { SPARGE_OP_MASK = 0, SPARGE_OP_ATTN = 1, SPARGE_OP_SLA2 = 2 };
+
+/* Workspace bytes the operation needs for this shape (0 if none, or if the
+ * shape is invalid). */
+size_t sparge_workspace_bytes(int op, const sparge_shape* shape);
+
+/* Block mask (SpargeAttention2 article, sections 1 and 4).
+ *   Q, K        bf16 [B,H,N,d], device.
+ *   topk_frac   in [0,1]: Top-k keeps kc = ceil(topk_frac * Nkb) blocks
+ *               (computed as ceil(topk_frac*Nkb - 1e-9)); 0 disables Top-k.
+ *   topp        in [0,1]: Top-p keeps the shortest prefix of the blocks
+ *               ordered by probability (descending; ties to the lower index)
+ *               whose summed probability is >= topp; 0 disables Top-p.
+ *   kv_idx, kv_cnt  outputs (see conventions). Each row keeps
+ *               max(kc, pc, 1) blocks: the union of two prefixes of one order.
+ *   row_thresh  optional output, float [B,H,Nqb]: probability of the last
+ *               kept block of each row (NULL to skip).
+ *   probs       optional output, float [B,H,Nqb,Nkb]: the pooled block
+ *               probabilities (NULL to skip; the workspace holds them then).
+ * Precision of the decision: fp32 pooling (row-order sums), fp32 scores
+ * (channel-order fused multiply-adds), fp32 softmax, double running sums.
+ * Limits: Nkb <= 4096. */
+sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shape, double topk_frac,
+                          double topp, int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention forward (SpargeAttention2 article, section 4).
+ *   O[b,h,i] = sum over the keys j of the kept blocks of i's query block of
+ *              softmax_j(q_i . k_j / sqrt(d)) v_j, in fp32, stored as bf16.
+ *   lse         optional output, float [B,H,N]: natural-log log-sum-exp of the
+ *               scaled scores over the kept keys; -inf where nothing is kept.
+ * A row whose block keeps nothing gets O = 0. Workspace: none (0 bytes). */
+sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Sparse + linear mix (SLA2 article, sections 1 and 2).
+ *   O = alpha[h] * O_sparse + (1 - alpha[h]) * O_linear, with O_sparse as in
+ *   sparge_attn_fwd and, over the keys j of the blocks NOT kept,
+ *   O_linear[i] = sum_j (phi(q_i) . phi(k_j)) v_j / sum_j phi(q_i) . phi(k_j),
+ *   phi(x) = elu(x) + 1; O_linear = 0 when every block is kept.
+ *   alpha       float [H], device.
+ * d must be 128. Workspace: sparge_workspace_bytes(SPARGE_OP_SLA2, shape). */
+sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                            const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, void* O,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device error word after synchronising the stream.
+ * *code receives 0 if no kernel gave up a wait since the last call, else the
+ * site code of the first one. Returns SPARGE_ERR_DEVICE_TIMEOUT in that
+ * case, SPARGE_ERR_CUDA if the synchronisation or the read fails. */
+sparge_status sparge_device_status(void* stream, int32_t* code);
+
+/* Static, human-readable name of a status. */
+const char* sparge_status_string(sparge_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARGE_H_ */

@@ -1,0 +1,84 @@
+"""Comparison helpers shared by the GPU parity tests.
+
+The bars: masks bit-exact except blocks whose probability lies within 1e-6
+(relative) of the row's selection threshold, or rows whose Top-p running sum
+lies within 1e-6 of p at the boundary; outputs within max-abs 2e-2 and mean
+relative L1 5e-3 of the double-precision oracle on the same mask.
+"""
+import numpy as np
+
+import oracle
+
+MAX_ABS = 2e-2
+MEAN_REL_L1 = 5e-3
+AMBIG_REL = 1e-6
+
+
+def compare_masks(g_idx, g_cnt, o_idx, o_cnt, P, topk, topp):
+    """Returns (n_rows, n_mismatched_rows, n_ambiguous_rows); raises on a
+    mismatch outside the ambiguity rule. Arrays are numpy; P is the oracle's
+    probability array in the decision precision."""
+    g_idx = np.asarray(g_idx).reshape(-1, g_idx.shape[-1])
+    o_idx = np.asarray(o_idx).reshape(-1, o_idx.shape[-1])
+    g_cnt = np.asarray(g_cnt).reshape(-1)
+    o_cnt = np.asarray(o_cnt).reshape(-1)
+    P = np.asarray(P).reshape(-1, P.shape[-1])
+    nkb = P.shape[1]
+    cols = np.arange(nkb)[None, :]
+    valid_g = cols < g_cnt[:, None]
+    valid_o = cols < o_cnt[:, None]
+    same = (g_cnt == o_cnt) & np.all(np.where(valid_o, g_idx == o_idx, True), axis=1)
+    bad_rows = np.nonzero(~same)[0]
+    n_amb = 0
+    for r in bad_rows:
+        gs = set(g_idx[r, : g_cnt[r]].tolist())
+        os_ = set(o_idx[r, : o_cnt[r]].tolist())
+        sel = oracle.select_row(P[r], topk, topp)
+        m = sel["m"]
+        order = sel["order"]
+        t = P[r, order[m - 1]]
+        allowed = set(np.nonzero(np.abs(P[r] - t) <= AMBIG_REL * t)[0].tolist())
+        cum = sel["cum"]
+        if topp > 0:
+            # Every Top-p count whose boundary lies within the tolerance of p
+            # is a correct answer for some rounding of the running sums.
+            ok_pc = [c for c in range(1, nkb + 1)
+                     if cum[c] >= topp - AMBIG_REL and cum[c - 1] < topp + AMBIG_REL]
+            if cum[nkb] < topp + AMBIG_REL:
+                ok_pc.append(nkb)
+            ms = [max(sel["kc"], c, 1) for c in ok_pc] + [m]
+            allowed |= set(int(j) for j in order[min(ms):max(ms)])
+        diff = gs ^ os_
+        if not diff <= allowed:
+            raise AssertionError(
+                f"mask row {r}: GPU keeps {sorted(gs)[:20]}... ({len(gs)}), oracle {sorted(os_)[:20]}... "
+                f"({len(os_)}); unexplained blocks {sorted(diff - allowed)[:10]}, threshold {t}")
+        n_amb += 1
+    return len(g_cnt), len(bad_rows), n_amb
+
+
+def output_errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    denom = float(np.abs(ref).sum())
+    mean_rel = float(err.sum() / denom) if denom > 0 else float(err.sum())
+    return max_abs, mean_rel
+
+
+def assert_outputs(got, ref, what=""):
+    max_abs, mean_rel = output_errors(got, ref)
+    assert max_abs <= MAX_ABS and mean_rel <= MEAN_REL_L1, f"{what}: max-abs {max_abs:.3e}, mean-rel-L1 {mean_rel:.3e}"
+    return max_abs, mean_rel
+
+
+def sample_rows(B, H, N, bq, n, seed):
+    """Flat row ids: n random rows plus the first and last rows of the first
+    and last query blocks of a few heads (the ragged tail included)."""
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(0, B * H * N, size=n).tolist())
+    for bh in {0, B * H - 1, (B * H) // 2}:
+        for i in (0, bq - 1, N - 1, max(0, N - 2), (N - 1) // bq * bq):
+            rows.add(bh * N + i)
+    return np.array(sorted(rows), np.int64)

@@ -1,0 +1,92 @@
+"""The C ABI loads, exports every declared symbol and rejects bad arguments
+on the host (no GPU needed: nothing here reaches a CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparge.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparge_\w+|sla2_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_pooled_b200 import build
+
+    build.build()
+    from block_sparse_attention_pooled_b200 import sparge
+
+    return sparge
+
+
+def test_header_declares_the_three_operations():
+    names = _declared_functions()
+    for n in ("sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_workspace_bytes",
+              "sparge_device_status", "sparge_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = lib.raw()
+    for name in _declared_functions():
+        assert hasattr(raw, name), name
+    assert set(_declared_functions()) == set(lib.EXPORTS)
+
+
+def test_status_strings(lib):
+    raw = lib.raw()
+    for code in range(6):
+        assert raw.sparge_status_string(code)
+    assert raw.sparge_status_string(0) == b"ok"
+
+
+def test_workspace_bytes_host_arithmetic(lib):
+    s = lib.Shape(1, 40, 75600, 128, 128, 64)
+    nqb, nkb = 591, 1182
+    need = lib.workspace_bytes(lib.OP_MASK, s)
+    assert need >= 40 * (nqb + nkb) * 128 * 4 + 40 * nqb * nkb * 4
+    assert lib.workspace_bytes(lib.OP_ATTN, s) == 0
+    bad = lib.Shape(1, 1, 100, 96, 64, 64)  # unsupported head dim
+    assert lib.workspace_bytes(lib.OP_MASK, bad) == 0
+
+
+def test_invalid_arguments_rejected_before_any_launch(lib):
+    raw = lib.raw()
+    s = lib.Shape(1, 2, 4096, 64, 64, 64)
+    P = ctypes.c_void_p(16 * 1024)  # never dereferenced: checks fail first
+    # null shape, null inputs
+    assert raw.sparge_mask(P, P, None, 0.1, 0.9, P, P, None, None, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_mask(None, P, ctypes.byref(s), 0.1, 0.9, P, P, None, None, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    # fractions out of range
+    assert raw.sparge_mask(P, P, ctypes.byref(s), 1.5, 0.9, P, P, None, None, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_mask(P, P, ctypes.byref(s), 0.1, -0.1, P, P, None, None, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_mask(P, P, ctypes.byref(s), float("nan"), 0.9, P, P, None, None, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    # workspace missing / too small
+    assert raw.sparge_mask(P, P, ctypes.byref(s), 0.1, 0.9, P, P, None, None, None, 0, None) == lib.ERR_WORKSPACE
+    assert raw.sparge_mask(P, P, ctypes.byref(s), 0.1, 0.9, P, P, None, None, P, 16, None) == lib.ERR_WORKSPACE
+    # misaligned input
+    assert raw.sparge_mask(ctypes.c_void_p(16 * 1024 + 2), P, ctypes.byref(s), 0.1, 0.9, P, P, None, None, P,
+                           1 << 30, None) == lib.ERR_INVALID_ARG
+    # unsupported shapes
+    for bad in (lib.Shape(1, 1, 100, 96, 64, 64), lib.Shape(1, 1, 100, 64, 32, 64), lib.Shape(1, 1, 100, 64, 64, 256),
+                lib.Shape(1, 1, 64 * 5000, 64, 64, 64)):
+        assert raw.sparge_attn_fwd(P, P, P, ctypes.byref(bad), P, P, P, None, None, 0, None) == lib.ERR_UNSUPPORTED
+    for bad in (lib.Shape(0, 1, 100, 64, 64, 64), lib.Shape(1, 1, -5, 64, 64, 64)):
+        assert raw.sparge_attn_fwd(P, P, P, ctypes.byref(bad), P, P, P, None, None, 0, None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_attn_fwd(P, P, None, ctypes.byref(s), P, P, P, None, None, 0, None) == lib.ERR_INVALID_ARG
+    assert raw.sla2_attn_fwd(P, P, P, None, P, P, P, P, None, 0, None) == lib.ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lib.sparge_mask(q, q, 64, 64, 0.1, 0.9)

@@ -1,0 +1,84 @@
+"""GPU block mask vs the CPU oracle (decision taken in single precision on
+both sides, same operation order; see the oracle's header)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_pooled_b200 import synth
+from parity import compare_masks
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(Q, K, bq, bk, topk, topp):
+    from block_sparse_attention_pooled_b200 import sparge
+
+    dev = torch.device("cuda")
+    Qd, Kd = Q.to(dev), K.to(dev)
+    B, H, N, d = Q.shape
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    probs = torch.empty((B, H, nqb, nkb), dtype=torch.float32, device=dev)
+    thr = torch.empty((B, H, nqb), dtype=torch.float32, device=dev)
+    idx, cnt = sparge.sparge_mask(Qd, Kd, bq, bk, topk, topp, row_thresh=thr, probs=probs)
+    torch.cuda.synchronize()
+    assert sparge.device_status() == 0
+    return idx.cpu().numpy(), cnt.cpu().numpy(), probs.cpu().numpy(), thr.cpu().numpy()
+
+
+def _check(Q, K, bq, bk, topk, topp):
+    g_idx, g_cnt, g_P, g_thr = _run(Q, K, bq, bk, topk, topp)
+    o_idx, o_cnt, o_P = oracle.mask(Q, K, bq, bk, topk, topp, precision=32)
+    # probabilities: same operation order except the row sum and expf rounding
+    np.testing.assert_allclose(g_P, o_P, rtol=1e-6, atol=1e-37)
+    n, bad, amb = compare_masks(g_idx, g_cnt, o_idx, o_cnt, o_P, topk, topp)
+    # threshold output: probability of the last kept block (rows that agree)
+    rows = g_cnt.reshape(-1) == o_cnt.reshape(-1)
+    assert np.all(g_thr.reshape(-1) > 0)
+    return n, bad, amb
+
+
+@pytest.mark.parametrize("N,d,bq,bk", [(4096, 64, 64, 64), (1000, 64, 64, 64), (1000, 128, 128, 64),
+                                        (777, 128, 64, 128), (130, 64, 128, 128), (64, 128, 64, 64)])
+@pytest.mark.parametrize("topk,topp", [(0.1, 0.9), (0.0, 0.9), (0.2, 0.0), (0.0, 0.0), (1.0, 0.5), (0.05, 1.0)])
+def test_mask_small(N, d, bq, bk, topk, topp):
+    Q, K, _ = synth.make_qkv(1, 2, N, d, grid=None, s=1.5, seed=N + d)
+    _check(Q, K, bq, bk, topk, topp)
+
+
+@pytest.mark.parametrize("name", ["tiny", "480p", "sla2_480p", "sweep_flat", "sweep_peaked"])
+def test_mask_workloads(name):
+    w = synth.WORKLOADS[name]
+    Q, K, _, _ = synth.make_workload(w)
+    n, bad, amb = _check(Q, K, w.bq, w.bk, w.topk, w.topp)
+    print(f"{name}: rows {n}, mismatched rows {bad} (all within the ambiguity rule)")
+
+
+def test_mask_720p_all_heads():
+    w = synth.WORKLOADS["720p"]
+    Q, K, _, _ = synth.make_workload(w)
+    n, bad, amb = _check(Q, K, w.bq, w.bk, w.topk, w.topp)
+    print(f"720p: rows {n}, mismatched rows {bad} (all within the ambiguity rule)")
+
+
+@pytest.mark.parametrize("topk,topp", [(t, p) for t in synth.SWEEP_TOPK for p in synth.SWEEP_TOPP]
+                         + [(0.05, 0.0), (0.0, 0.9)])
+def test_mask_sweep_regimes(topk, topp):
+    w = synth.WORKLOADS["sweep_peaked"]
+    Q, K, _ = synth.make_qkv(1, 4, w.N, w.d, w.grid, w.s, w.seed)
+    _check(Q, K, w.bq, w.bk, topk, topp)
+
+
+def test_mask_is_deterministic():
+    from block_sparse_attention_pooled_b200 import sparge
+
+    w = synth.WORKLOADS["480p"]
+    Q, K, _ = synth.make_qkv(1, 3, w.N, w.d, w.grid, w.s, w.seed)
+    Qd, Kd = Q.cuda(), K.cuda()
+    a = [t.clone() for t in sparge.sparge_mask(Qd, Kd, w.bq, w.bk, w.topk, w.topp)]
+    b = sparge.sparge_mask(Qd, Kd, w.bq, w.bk, w.topk, w.topp)
+    cnt = a[1]
+    assert torch.equal(a[1], b[1])
+    cols = torch.arange(a[0].shape[-1], device=cnt.device)
+    valid = cols[None, None, None, :] < cnt[..., None]
+    assert torch.equal(a[0][valid], b[0][valid])
