@@ -1,0 +1,367 @@
+"""Benchmark of the pooled block-sparse attention hot path on B200.
+
+One step = the whole path for one batch of synthetic video-shaped input:
+the block mask (pool, score + softmax, hybrid Top-k/Top-p select) followed by
+block-sparse attention; for the SLA2 workloads also the per-head linear
+summaries and the sparse + linear mix.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). Under torchrun every rank runs its own copy of
+the workload (independent problems, no collective on the data path: weak
+scaling); only the timing uses the process group.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_pooled_b200 import synth  # noqa: E402
+
+METRIC = "ms/call, effective TFLOPS & tensor-pipe % of bf16 peak at 32K/75K-token shapes"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="480p", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- work accounting
+def kept_flops(kv_idx: torch.Tensor, kv_cnt: torch.Tensor, N: int, d: int, bq: int, bk: int) -> float:
+    """4*d * sum over kept (query block, key block) pairs of valid rows x valid keys."""
+    B, H, nqb, nkb = kv_idx.shape
+    rows = torch.clamp(N - torch.arange(nqb, device=kv_idx.device) * bq, max=bq).to(torch.float64)
+    keys_of_block = torch.clamp(N - torch.arange(nkb, device=kv_idx.device) * bk, max=bk).to(torch.float64)
+    valid = torch.arange(nkb, device=kv_idx.device)[None, None, None, :] < kv_cnt[..., None]
+    keys = torch.where(valid, keys_of_block[kv_idx.long().clamp(0, nkb - 1)], torch.zeros((), dtype=torch.float64,
+                                                                                          device=kv_idx.device))
+    per_row = keys.sum(-1) * rows[None, None, :]
+    return float(4.0 * d * per_row.sum().item())
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clocks and throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _smi_id(dev) -> str:
+    """nvidia-smi --id for a torch device: its UUID when torch exposes it."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        cvd = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [x for x in cvd.split(",") if x.strip()]
+        return ids[dev.index].strip() if dev.index < len(ids) else str(dev.index)
+
+
+def kernel_source_sha() -> str:
+    """Digest of the CUDA sources, to tell whether stored counters still apply."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_pooled_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    capture, or None when there is none or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entry = json.load(f).get(workload)
+    if not entry or entry.get("kernel") != kernel or entry.get("csrc_sha") != kernel_source_sha():
+        return None
+    return entry["dram_bytes_per_launch"]
+
+
+# ----------------------------------------------------------------------------- peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1):
+    """Times the oracle on a bounded sample: the mask of `heads` head(s) and the
+    attention of `n_qblocks` query blocks of the first head, and returns
+    (effective FLOP/s, description, threads)."""
+    import oracle
+
+    oracle.build()
+    Qh, Kh, Vh = Q[:1, :heads].contiguous(), K[:1, :heads].contiguous(), V[:1, :heads].contiguous()
+    t0 = time.perf_counter()
+    idx, cnt, _ = oracle.mask(Qh, Kh, w.bq, w.bk, w.topk, w.topp, precision=32)
+    t_mask = time.perf_counter() - t0
+    qbs = np.linspace(0, w.nqb - 1, n_qblocks).astype(np.int64)
+    rows = np.concatenate([np.arange(qb * w.bq, min(w.N, qb * w.bq + w.bq)) for qb in qbs]).astype(np.int64)
+    mode = "sla2" if w.sla2 else "sparse"
+    t0 = time.perf_counter()
+    oracle.attention_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, alpha[:heads].numpy(), mode=mode, rows=rows)
+    t_attn = time.perf_counter() - t0
+    flops = 0.0
+    for qb in qbs:
+        nrows = min(w.bq, w.N - qb * w.bq)
+        keys = sum(min(w.bk, w.N - int(J) * w.bk) for J in idx[0, 0, qb, : cnt[0, 0, qb]])
+        flops += 4.0 * w.d * nrows * keys
+    # the mask's time is charged pro rata to the sampled query blocks
+    t = t_attn + t_mask * (len(qbs) / (w.nqb * heads))
+    desc = (f"oracle mask of {heads} head(s) ({t_mask:.2f} s, charged pro rata) + {mode} attention of "
+            f"{len(qbs)} query blocks x {w.bq} rows ({t_attn:.2f} s); {w.name} workload")
+    return flops / t, desc, 1
+
+
+# ----------------------------------------------------------------------------- runs
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    Q, K, V, alpha = synth.make_workload(w, heads=[(0, 0)])
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
+                   "topk": w.topk, "topp": w.topp},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    from block_sparse_attention_pooled_b200 import sparge
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    seedw = synth.Workload(**{**w.__dict__, "seed": w.seed + rank})
+    Qh, Kh, Vh, alpha_h = synth.make_workload(seedw)
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    Qh, Kh, Vh = pin(Qh), pin(Kh), pin(Vh)
+    Q, K, V, alpha = Qh.to(dev), Kh.to(dev), Vh.to(dev), alpha_h.to(dev)
+    B, H, N, d = Q.shape
+    shape = sparge.make_shape(Q, w.bq, w.bk)
+    ws_mask = torch.empty(max(1, sparge.workspace_bytes(sparge.OP_MASK, shape)), dtype=torch.uint8, device=dev)
+    n_sla2 = sparge.workspace_bytes(sparge.OP_SLA2, shape) if w.sla2 else 0
+    ws_sla2 = torch.empty(max(1, n_sla2), dtype=torch.uint8, device=dev)
+    kv_idx = torch.empty((B, H, w.nqb, w.nkb), dtype=torch.int32, device=dev)
+    kv_cnt = torch.empty((B, H, w.nqb), dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    stream = torch.cuda.current_stream()
+
+    def step(ev_a=None, ev_b=None):
+        sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
+        if ev_a is not None:
+            ev_a.record(stream)
+        if w.sla2:
+            sparge.sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, w.bq, w.bk, O=O, workspace=ws_sla2)
+        else:
+            sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    launches_per_step = 4 + (sparge.SLA2_LAUNCHES if w.sla2 else 1)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
+    flops = kept_flops(kv_idx, kv_cnt, N, d, w.bq, w.bk)
+    dense_flops = 4.0 * B * H * N * N * d
+
+    # ---- device-timed region (inputs resident in HBM, larger than L2)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(_smi_id(dev)) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(*evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    attn_avg = sum(attn_ms) / len(attn_ms)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        for _ in range(2):
+            Q.copy_(Qh, non_blocking=True); K.copy_(Kh, non_blocking=True); V.copy_(Vh, non_blocking=True)
+            step()
+            Oh.copy_(O, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ksteps = max(3, args.steps // 4)
+        e0.record(stream)
+        for _ in range(ksteps):
+            Q.copy_(Qh, non_blocking=True); K.copy_(Kh, non_blocking=True); V.copy_(Vh, non_blocking=True)
+            step()
+            Oh.copy_(O, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / ksteps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        h2d = 3 * Q.numel() * Q.element_size()
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": O.numel() * O.element_size(), "ms_per_step": e2e_ms}
+    assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
+
+    if rank != 0:
+        return
+    peaks, peak_kind = measured_peaks()
+    clocks = clk.summary()
+    # Burst peak when the clocks held their maximum through the timed region,
+    # the sustained (power-capped) one otherwise.
+    burst = clocks["sm_mhz"] is not None and clocks["sm_max_mhz"] and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+    peak = float(peaks["bf16_tflops"] if burst else peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak_desc = f"{peak_kind} bf16 {'burst (SM clock at max during the timed region)' if burst else 'sustained'}"
+    achieved = flops / (attn_avg * 1e-3) / 1e12
+    kernel_name = "sla2_attn_fwd_kernel" if w.sla2 else "attn_fwd_kernel"
+    traffic = dram_traffic(w.name, kernel_name)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h)
+        cpu = {"value": v / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-shaped Q/K/V, see synth.py)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
+                   "topk": w.topk, "topp": w.topp, "alpha": "U[0.6,1] per head" if w.sla2 else 1.0,
+                   "l2": f"inputs larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V per rank)",
+                   "parallelism": f"independent replicas x{world}"},
+        "kept_fraction": flops / dense_flops,
+        "dense_equiv_tflops": dense_flops * world / (ms_step * 1e-3) / 1e12,
+        "attn_ms": attn_avg,
+        "mask_ms": ms_step - attn_avg,
+        "roofline": {"kernel": kernel_name, "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_desc, "traffic": traffic},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, rank, world)
+        else:
+            run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

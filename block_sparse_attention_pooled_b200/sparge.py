@@ -22,6 +22,9 @@ _lib = ctypes.CDLL(_LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
 OP_MASK, OP_ATTN, OP_SLA2 = 0, 1, 2
 
+# Kernel launches per call of each entry point (for launch accounting).
+MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES = 4, 1, 2
+
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
            "sparge_device_status", "sparge_status_string")
