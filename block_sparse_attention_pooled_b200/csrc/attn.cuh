@@ -16,6 +16,19 @@
 //               its own S columns; then the epilogue (O / l -> bf16 -> TMA
 //               store, optional log-sum-exp).
 // TMEM columns: S0 [0,64), S1 [64,128), O [128,128+D).
+//
+// With LIN = true the same kernel also produces the sparse + linear mix of
+// the SLA2 article (arXiv:2602.12675, sections 1 and 2):
+//   O = alpha_h * O_sparse + (1 - alpha_h) * O_linear,
+//   O_linear[i] = phi(q_i)^T S_c / phi(q_i) . z_c  over the blocks NOT kept,
+// where S_c = S_all - S_kept and z_c = z_all - z_kept. S_all / z_all come from
+// linear_summary_kernel; S_kept = sum over the kept key tiles of
+// phi(K_t)^T [V_t | 1] is accumulated here with one more MMA per tile (A =
+// the phi(K) tile, B = the V tile followed by a ones block, both already in
+// shared memory), into TMEM columns [256, 400). The epilogue writes
+// [S_c | z_c] as bf16 into shared memory, turns the Q tile into phi(Q) in
+// place and runs one more MMA, phi(Q) [S_c | z_c], whose column 128 is the
+// denominator.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -33,13 +46,17 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max
 // Error site codes recorded in g_device_error by the attention kernel.
 enum : unsigned int {
   kErrAttnQ = 0x100, kErrAttnKFull, kErrAttnVFull, kErrAttnKEmpty, kErrAttnVEmpty, kErrAttnSFull,
-  kErrAttnPFull, kErrAttnODone, kErrAttnOFinal, kErrAttnDrain
+  kErrAttnPFull, kErrAttnODone, kErrAttnOFinal, kErrAttnDrain, kErrAttnLin
 };
 
 struct AttnParams {
   const int32_t* kv_idx;  // [BH, nqb, nkb]
   const int32_t* kv_cnt;  // [BH, nqb]
   float* lse;             // [BH, N] or null
+  const float* s_all;     // LIN: [BH, 128, 128] fp32
+  const float* z_all;     // LIN: [BH, 128] fp32
+  const float* alpha;     // LIN: [H]
+  int H;
   int N;
   int nqb;
   int nkb;
@@ -48,26 +65,34 @@ struct AttnParams {
   float scale_log2;       // log2(e) / sqrt(d)
 };
 
-template <int D>
+template <int D, bool LIN>
 struct AttnSmem {
   static constexpr int kQBytes = kTileQ * D * 2;
   static constexpr int kKBytes = kTileK * D * 2;
-  static constexpr int kVBytes = kTileK * D * 2;
+  static constexpr int kVData = kTileK * D * 2;
+  static constexpr int kVBytes = kVData + (LIN ? 8192 : 0);   // LIN: ones block after V
+  static constexpr int kPBytes = LIN ? kTileK * D * 2 : 0;     // phi(K) tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + 2 * kKBytes;
-  static constexpr int kOffBar = kOffV + 2 * kVBytes;
-  static constexpr int kNumBars = 16;
+  static constexpr int kOffP = kOffV + 2 * kVBytes;
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kNumBars = 18;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kUsed = kOffTmem + 16;
   // Pad so that at most two CTAs fit on an SM: two CTAs x 256 TMEM columns
   // use the SM's 512 columns exactly, and a third would block in alloc.
+  // LIN needs all 512 columns and is one CTA per SM by its size.
   static constexpr int kBytes = (kUsed + 1024 > 80 * 1024 ? kUsed + 1024 : 80 * 1024);
+  static constexpr int kTmemCols = LIN ? 512 : 256;
+  // LIN epilogue: [S_c | z_c] staged over the (then idle) K and V rings.
+  static constexpr int kOffStage = kOffK;
+  static_assert(!LIN || kOffStage + 3 * 128 * 128 <= kOffV + kVData, "stage must not reach the ones block");
 };
 
 // Barrier slots.
 enum { kBarQ = 0, kBarKFull = 1, kBarVFull = 3, kBarKEmpty = 5, kBarVEmpty = 7, kBarSFull = 9,
-       kBarPFull = 11, kBarODone = 13, kBarOFinal = 14, kBarDrain = 15 };
+       kBarPFull = 11, kBarODone = 13, kBarOFinal = 14, kBarDrain = 15, kBarLin = 16 };
 
 // Waits on an mbarrier unless another role already gave up; gives up itself
 // (and tells the others through *abort) after the global time limit.
@@ -92,17 +117,20 @@ __device__ __forceinline__ int tile_key0(const int32_t* lst, int t, int tiles_pe
   return __ldg(lst + e) * bk + (t % tiles_per_block) * kTileK;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__device__ __forceinline__ float phi_attn(float x) { return x > 0.0f ? x + 1.0f : __expf(x); }
+
+template <int D, bool LIN>
+__global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                    const AttnParams p) {
-  using L = AttnSmem<D>;
+                    const __grid_constant__ CUtensorMap tmPhiK, const AttnParams p) {
+  static_assert(!LIN || D == 128, "the linear branch is built for d = 128");
+  using L = AttnSmem<D, LIN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw);
-  const uint32_t sQ = sbase + L::kOffQ, sK = sbase + L::kOffK, sV = sbase + L::kOffV;
+  const uint32_t sQ = sbase + L::kOffQ, sK = sbase + L::kOffK, sV = sbase + L::kOffV, sP = sbase + L::kOffP;
   const uint32_t bar0 = sbase + L::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
@@ -131,22 +159,32 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     mbar_init(bar(kBarODone), 1);
     mbar_init(bar(kBarOFinal), 1);
     mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarLin), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (LIN) {
+    // Ones block after each V slot: the 16 extra B columns that yield z.
+    for (int sl = 0; sl < 2; ++sl) {
+      uint4* ones = reinterpret_cast<uint4*>(sgen + L::kOffV + sl * L::kVBytes + L::kVData);
+      for (int u = threadIdx.x; u < 8192 / 16; u += kAttnThreads)
+        ones[u] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    }
+    fence_async_smem();
+  }
   if (warp == 1) {
-    tmem_alloc(sbase + L::kOffTmem, 256);
+    tmem_alloc(sbase + L::kOffTmem, L::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tS = tmem, tO = tmem + 128, tL = tmem + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && T > 0) {
+    if (lane == 0 && (T > 0 || LIN)) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -162,9 +200,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           tma_load_3d(sK + slot * L::kKBytes + b * (kTileK * 128), &tmK, bar(kBarKFull + slot), b * 64, key0, bh);
         ++nk;
         if (t >= 2 && !role_wait(bar(kBarVEmpty + slot), ((t >> 1) - 1) & 1, kErrAttnVEmpty, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(kBarVFull + slot), L::kVBytes);
+        mbar_arrive_expect_tx(bar(kBarVFull + slot), L::kVData + L::kPBytes);
         for (int b = 0; b < D / 64; ++b)
           tma_load_3d(sV + slot * L::kVBytes + b * (kTileK * 128), &tmV, bar(kBarVFull + slot), b * 64, key0, bh);
+        if (LIN)
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_3d(sP + slot * L::kPBytes + b * (kTileK * 128), &tmPhiK, bar(kBarVFull + slot), b * 64, key0, bh);
         ++nv;
       }
       // Never leave with copies in flight: wait for the last loads issued to
@@ -207,6 +248,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             const uint64_t b = sdesc_sw128(vbase + kk * (16 * 128), kTileK * 128, 1024);
             mma_ts(tO, tS + slot * 64 + kk * 8, b, idPV, (u > 0 || kk > 0) ? 1u : 0u);
           }
+          if (LIN) {
+            // S_kept[feature, 0..143] += phi(K_u)^T [V_u | 1]
+            constexpr uint32_t idL = idesc_bf16_f32(128, 144, true, true);
+            const uint32_t pbase = sP + slot * L::kPBytes;
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              const uint64_t a = sdesc_sw128(pbase + kk * (16 * 128), kTileK * 128, 1024);
+              const uint64_t b = sdesc_sw128(vbase + kk * (16 * 128), kTileK * 128, 1024);
+              mma_ss(tL, a, b, idL, (u > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
           mma_commit(bar(kBarVEmpty + slot));
           mma_commit(bar(kBarODone));
           if (u == T - 1) mma_commit(bar(kBarOFinal));
@@ -222,6 +274,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int r = q * 32 + lane;             // row of the query tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     float m_run = -INFINITY, l_run = 0.0f;
+    int kept_keys = 0;  // valid keys in the kept tiles (LIN: the complement is empty when this is N)
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int slot = t & 1;
@@ -240,6 +293,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(v[c][j]);
       }
       const int key0 = tile_key0(lst, t, tiles_per_block, p.bk);
+      kept_keys += max(0, min(kTileK, p.N - key0));
       if (key0 + kTileK > p.N) {
 #pragma unroll
         for (int j = 0; j < kTileK; ++j)
@@ -294,24 +348,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       ok = __all_sync(0xffffffffu, role_wait(bar(kBarOFinal), 0, kErrAttnOFinal, abort_flag));
       tc_fence_after();
     }
-    // Epilogue: O / l -> bf16 rows into the (now idle) Q buffer, laid out the
-    // way the 128-byte-swizzled O tensor map expects, then TMA stores.
     const float inv_l = (T > 0 && l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-#pragma unroll 1
-    for (int c = 0; c < D; c += 16) {
-      uint32_t v[16];
-      if (T > 0 && ok) {
-        tmem_ld16(tO + lane_off + c, v);
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0u;
-      }
+    // Writes 16 output values of row r (columns c..c+15) as bf16 into the
+    // Q buffer, laid out the way the 128-byte-swizzled O tensor map expects.
+    auto stage_out16 = [&](int c, const float (&o)[16]) {
       uint32_t w[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        w[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
-      const int box = c / 64, cc = c % 64;             // column within the 64-wide box
+      for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
+      const int box = c / 64, cc = c % 64;
       const uint32_t row_addr = sQ + box * (kTileQ * 128) + r * 128;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -319,6 +363,133 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
                      "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
                      : "memory");
+      }
+    };
+    if constexpr (!LIN) {
+      // Epilogue: O / l -> bf16 -> Q buffer -> TMA store.
+#pragma unroll 1
+      for (int c = 0; c < D; c += 16) {
+        uint32_t v[16];
+        if (T > 0 && ok) {
+          tmem_ld16(tO + lane_off + c, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0u;
+        }
+        float o[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v[j]) * inv_l;
+        stage_out16(c, o);
+      }
+    } else {
+      // 1. Q is needed as phi(Q): wait for it when no key tile was visited.
+      if (ok && T == 0) ok = __all_sync(0xffffffffu, role_wait(bar(kBarQ), 0, kErrAttnQ, abort_flag));
+      // 2. [S_c | z_c] for feature a = r: S_all - S_kept, z_all - z_kept, as
+      //    bf16 into the stage, MN-major with 128-byte swizzle (row a, three
+      //    64-column boxes; column 128 = z_c, the rest of box 2 zero).
+      const uint32_t sStage = sbase + L::kOffStage;
+      const float* srow = p.s_all + ((int64_t)bh * 128 + r) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 144; c += 16) {
+        uint32_t v[16];
+        if (T > 0 && ok) {
+          tmem_ld16(tL + lane_off + c, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0u;
+        }
+        float sc[16];
+        if (c < 128) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sc[j] = __ldg(srow + c + j) - __uint_as_float(v[j]);
+        } else {
+          sc[0] = __ldg(p.z_all + (int64_t)bh * 128 + r) - __uint_as_float(v[0]);
+#pragma unroll
+          for (int j = 1; j < 16; ++j) sc[j] = 0.0f;
+        }
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(sc[2 * j], sc[2 * j + 1]);
+        const int box = c / 64, cc = c % 64;
+        const uint32_t row_addr = sStage + box * (128 * 128) + r * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int chunk = (cc / 8 + h) ^ (r & 7);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
+                       "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
+                       : "memory");
+        }
+      }
+      {  // zero the rest of box 2 (columns 144..191), which the MMA does not read but keep defined
+        const uint32_t row_addr = sStage + 2 * (128 * 128) + r * 128;
+#pragma unroll
+        for (int ch = 2; ch < 8; ++ch)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(row_addr + ((ch ^ (r & 7)) * 16)), "r"(0u)
+                       : "memory");
+      }
+      // 3. phi(Q) in place over this thread's row of the Q tile (elementwise,
+      //    so the swizzle does not matter).
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b) {
+        uint4* row = reinterpret_cast<uint4*>(sgen + L::kOffQ + b * (kTileQ * 128) + r * 128);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 x = row[ch];
+          __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&x);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float2 f = __bfloat1622float2(hx[j]);
+            hx[j] = __floats2bfloat162_rn(phi_attn(f.x), phi_attn(f.y));
+          }
+          row[ch] = x;
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // 4. O_lin numerator and denominator: phi(Q) [S_c | z_c] -> TMEM [256, 400).
+      if (warp == 2 && lane == 0 && ok) {
+        tc_fence_after();
+        constexpr uint32_t idF = idesc_bf16_f32(kTileQ, 144, false, true);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sdesc_sw128(sQ + (kk >> 2) * (kTileQ * 128) + (kk & 3) * 32u, 16, 1024);
+          const uint64_t b = sdesc_sw128(sStage + kk * (16 * 128), 128 * 128, 1024);
+          mma_ss(tL, a, b, idF, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kBarLin));
+      }
+      if (ok) ok = __all_sync(0xffffffffu, role_wait(bar(kBarLin), 0, kErrAttnLin, abort_flag));
+      tc_fence_after();
+      // 5. Mix and stage the output row.
+      const float a_h = __ldg(p.alpha + (bh % p.H));
+      float inv_den = 0.0f;
+      if (ok) {
+        uint32_t v[16];
+        tmem_ld16(tL + lane_off + 128, v);
+        tmem_ld_wait();
+        const float den = __uint_as_float(v[0]);
+        inv_den = (kept_keys < p.N && den > 0.0f) ? 1.0f / den : 0.0f;
+      }
+      const float ws = a_h * inv_l, wl = (1.0f - a_h) * inv_den;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 16) {
+        uint32_t vo[16], vl[16];
+        if (ok) {
+          if (T > 0) tmem_ld16(tO + lane_off + c, vo);
+          tmem_ld16(tL + lane_off + c, vl);
+          tmem_ld_wait();
+        }
+        float o[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float os = (ok && T > 0) ? __uint_as_float(vo[j]) : 0.0f;
+          const float ol = ok ? __uint_as_float(vl[j]) : 0.0f;
+          o[j] = ws * os + wl * ol;
+        }
+        stage_out16(c, o);
       }
     }
     if (p.lse != nullptr && r < p.bq && q0 + r < p.N) {
@@ -338,7 +509,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 

@@ -13,6 +13,7 @@
 #include "ptx.cuh"
 #include "mask.cuh"
 #include "attn.cuh"
+#include "linear.cuh"
 
 namespace {
 
@@ -136,14 +137,36 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
   return cuda_status(cudaGetLastError());
 }
 
-template <int D>
+struct Sla2Ws {
+  size_t phik, s_all, z_all, partial, total;
+};
+
+inline int lin_ctas_per_head(int N) { return (int)ceil_div(ceil_div(N, 64), kLinTilesPerCta); }
+
+Sla2Ws sla2_ws(const sparge_shape* s, const Dims& d) {
+  Sla2Ws w;
+  w.phik = 0;
+  w.s_all = w.phik + align256((size_t)d.BH * s->N * s->d * 2);
+  w.z_all = w.s_all + align256((size_t)d.BH * s->d * s->d * 4);
+  w.partial = w.z_all + align256((size_t)d.BH * s->d * 4);
+  w.total = w.partial + align256((size_t)d.BH * lin_ctas_per_head(s->N) * kLinPartial * 4);
+  return w;
+}
+
+template <int D, bool LIN>
 sparge_status launch_attn(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
-                          const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo;
+                          const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, const void* phik,
+                          const float* s_all, const float* z_all, const float* alpha, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo, mp;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
-      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, D, s->bq))
+      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, D, s->bq) ||
+      !make_map_bhnd(&mp, LIN ? phik : K, dm.BH, s->N, D, kTileK))
     return SPARGE_ERR_CUDA;
   AttnParams p;
+  p.s_all = s_all;
+  p.z_all = z_all;
+  p.alpha = alpha;
+  p.H = s->H;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
   p.lse = lse;
@@ -153,10 +176,29 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
   p.bq = s->bq;
   p.bk = s->bk;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const int smem = AttnSmem<D>::kBytes;
-  cudaError_t e = ensure_smem(attn_fwd_kernel<D>, smem, D == 64 ? 3 : 4);
+  const int smem = AttnSmem<D, LIN>::kBytes;
+  cudaError_t e = ensure_smem(attn_fwd_kernel<D, LIN>, smem, LIN ? 5 : (D == 64 ? 3 : 4));
   if (e != cudaSuccess) return cuda_status(e);
-  attn_fwd_kernel<D><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st>>>(mq, mk, mv, mo, p);
+  attn_fwd_kernel<D, LIN><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st>>>(mq, mk, mv, mo, mp, p);
+  return cuda_status(cudaGetLastError());
+}
+
+sparge_status launch_summaries(const void* K, const void* V, const sparge_shape* s, const Dims& dm, void* phik,
+                               float* partial, float* s_all, float* z_all, cudaStream_t st) {
+  CUtensorMap mk, mv, mp;
+  if (!make_map_bhnd(&mk, K, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
+      !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64))
+    return SPARGE_ERR_CUDA;
+  LinParams p;
+  p.partial = partial;
+  p.N = s->N;
+  p.ntiles = (int)ceil_div(s->N, 64);
+  p.ctas_per_head = lin_ctas_per_head(s->N);
+  cudaError_t e = ensure_smem(linear_summary_kernel, LinSmem::kBytes, 6);
+  if (e != cudaSuccess) return cuda_status(e);
+  linear_summary_kernel<<<(unsigned)(dm.BH * p.ctas_per_head), kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+  dim3 grid((unsigned)ceil_div(kLinPartial, 256), (unsigned)dm.BH);
+  linear_reduce_kernel<<<grid, 256, 0, st>>>(partial, p.ctas_per_head, s_all, z_all);
   return cuda_status(cudaGetLastError());
 }
 
@@ -173,7 +215,7 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
     case SPARGE_OP_ATTN:
       return 0;
     case SPARGE_OP_SLA2:
-      return 0;
+      return shape->d == 128 ? sla2_ws(shape, dm).total : 0;
     default:
       return 0;
   }
@@ -213,19 +255,32 @@ sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const
   if (!Q || !K || !V || !O || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARGE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (shape->d == 64) return launch_attn<64>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, s);
-  return launch_attn<128>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, s);
+  if (shape->d == 64)
+    return launch_attn<64, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, nullptr, nullptr, nullptr, s);
+  return launch_attn<128, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                             const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, void* O,
                             void* workspace, size_t workspace_bytes, void* stream) {
-  (void)Q; (void)K; (void)V; (void)kv_idx; (void)kv_cnt; (void)alpha; (void)O;
-  (void)workspace; (void)workspace_bytes; (void)stream;
   Dims dm;
   sparge_status st = check_shape(shape, &dm);
   if (st != SPARGE_OK) return st;
-  return SPARGE_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !O || !kv_idx || !kv_cnt || !alpha) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARGE_ERR_INVALID_ARG;
+  if (shape->d != 128 || dm.BH > 65535) return SPARGE_ERR_UNSUPPORTED;
+  const Sla2Ws w = sla2_ws(shape, dm);
+  if (workspace == nullptr || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* phik = ws + w.phik;
+  float* s_all = reinterpret_cast<float*>(ws + w.s_all);
+  float* z_all = reinterpret_cast<float*>(ws + w.z_all);
+  float* partial = reinterpret_cast<float*>(ws + w.partial);
+  st = launch_summaries(K, V, shape, dm, phik, partial, s_all, z_all, s);
+  if (st != SPARGE_OK) return st;
+  return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, phik, s_all, z_all, alpha, s);
 }
 
 sparge_status sparge_device_status(void* stream, int32_t* code) {

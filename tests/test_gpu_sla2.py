@@ -1,0 +1,101 @@
+"""GPU sparse + linear mix (sla2_attn_fwd) vs the double-precision oracle on
+the same (oracle-computed or seeded) block mask."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_pooled_b200 import synth
+from parity import assert_outputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_sla2(Q, K, V, idx, cnt, alpha, bq, bk):
+    from block_sparse_attention_pooled_b200 import sparge
+
+    dev = torch.device("cuda")
+    O = sparge.sla2_attn_fwd(Q.to(dev), K.to(dev), V.to(dev), torch.as_tensor(idx, dtype=torch.int32).to(dev),
+                             torch.as_tensor(cnt, dtype=torch.int32).to(dev),
+                             torch.as_tensor(alpha, dtype=torch.float32).to(dev), bq, bk)
+    torch.cuda.synchronize()
+    assert sparge.device_status() == 0
+    return O.float().cpu().numpy()
+
+
+def _check(Q, K, V, idx, cnt, alpha, bq, bk, rows=None):
+    B, H, N, d = Q.shape
+    O = _gpu_sla2(Q, K, V, idx, cnt, alpha, bq, bk)
+    ref, _ = oracle.attention_rows(Q, K, V, bq, bk, idx, cnt, np.asarray(alpha, np.float32), mode="sla2", rows=rows)
+    got = O.reshape(-1, d) if rows is None else O.reshape(-1, d)[rows]
+    return assert_outputs(got, ref, "sla2")
+
+
+@pytest.mark.parametrize("N,bq,bk,max_keep", [(1000, 128, 64, 6), (777, 64, 64, 5), (2000, 128, 128, 4),
+                                               (130, 128, 64, 3), (64, 64, 64, 1), (4100, 128, 64, 20)])
+def test_sla2_random_masks(N, bq, bk, max_keep):
+    Q, K, V = synth.make_qkv(1, 3, N, 128, grid=None, s=1.5, seed=N + bq)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    idx, cnt = synth.random_mask(1, 3, nqb, nkb, min(nkb, max_keep), seed=N)
+    alpha = np.array([0.6, 0.85, 1.0], np.float32)
+    _check(Q, K, V, idx.numpy(), cnt.numpy(), alpha, bq, bk)
+
+
+def test_sla2_alpha_endpoints():
+    from block_sparse_attention_pooled_b200 import sparge
+
+    N, bq, bk = 1500, 128, 64
+    Q, K, V = synth.make_qkv(1, 2, N, 128, grid=None, s=1.5, seed=3)
+    idx, cnt = synth.random_mask(1, 2, -(-N // bq), -(-N // bk), 7, seed=5)
+    cnt = torch.clamp(cnt, min=1)
+    for h in range(2):
+        for I in range(cnt.shape[-1]):
+            c = int(cnt[0, h, I])
+            if len(set(idx[0, h, I, :c].tolist())) != c:
+                idx[0, h, I, :c] = torch.arange(c)
+    # alpha = 1: exactly the pure sparse kernel's output
+    O1 = _gpu_sla2(Q, K, V, idx, cnt, np.ones(2, np.float32), bq, bk)
+    dev = torch.device("cuda")
+    Os = sparge.sparge_attn_fwd(Q.to(dev), K.to(dev), V.to(dev), idx.to(dev), cnt.to(dev), bq, bk)
+    assert np.array_equal(O1, Os.float().cpu().numpy())
+    # alpha = 0: pure linear branch over the complement
+    O0 = _gpu_sla2(Q, K, V, idx, cnt, np.zeros(2, np.float32), bq, bk)
+    ref, _ = oracle.attention_rows(Q, K, V, bq, bk, idx, cnt, mode="linear")
+    assert_outputs(O0.reshape(-1, 128), ref, "linear branch")
+
+
+def test_sla2_empty_and_full_rows():
+    N, bq, bk = 512, 128, 64
+    Q, K, V = synth.make_qkv(1, 1, N, 128, grid=None, s=1.0, seed=11)
+    idx = np.zeros((1, 1, 4, 8), np.int32)
+    cnt = np.array([[[0, 3, 8, 1]]], np.int32)
+    idx[0, 0, 1, :3] = [0, 4, 7]
+    idx[0, 0, 2, :] = np.arange(8)  # every block kept: linear part is 0
+    idx[0, 0, 3, 0] = 7             # the ragged-free last block only
+    _check(Q, K, V, idx, cnt, np.array([0.7], np.float32), bq, bk)
+
+
+@pytest.mark.parametrize("name", ["sla2_480p", "720p"])
+def test_sla2_workload_oracle_mask(name):
+    w = synth.WORKLOADS[name]
+    if name == "720p":
+        heads = [(0, 0), (0, 17), (0, 39)]
+        Q, K, V, _ = synth.make_workload(w, heads=heads)
+        alpha = synth.make_alpha(w.H, w.seed, True).numpy()[[h for _, h in heads]]
+    else:
+        Q, K, V, alpha = synth.make_workload(w)
+        alpha = alpha.numpy()
+    idx, cnt, _ = oracle.mask(Q, K, w.bq, w.bk, w.topk, w.topp, precision=32)
+    B, H = Q.shape[:2]
+    rows = sample_rows(B, H, w.N, w.bq, 48, seed=2)
+    max_abs, mean_rel = _check(Q, K, V, idx, cnt, alpha, w.bq, w.bk, rows=rows)
+    print(f"{name}: max-abs {max_abs:.2e} mean-rel-L1 {mean_rel:.2e}")
+
+
+def test_sla2_is_deterministic():
+    N = 3000
+    Q, K, V = synth.make_qkv(1, 2, N, 128, grid=None, s=2.0, seed=12)
+    idx, cnt = synth.random_mask(1, 2, -(-N // 128), -(-N // 64), 10, seed=7)
+    a = _gpu_sla2(Q, K, V, idx, cnt, np.array([0.7, 0.9], np.float32), 128, 64)
+    b = _gpu_sla2(Q, K, V, idx, cnt, np.array([0.7, 0.9], np.float32), 128, 64)
+    assert np.array_equal(a, b)
