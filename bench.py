@@ -47,6 +47,16 @@ def parse():
     return ap.parse_args()
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The maximum of a per-rank scalar over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- work accounting
 def kept_flops(kv_idx: torch.Tensor, kv_cnt: torch.Tensor, N: int, d: int, bq: int, bk: int) -> float:
     """4*d * sum over kept (query block, key block) pairs of valid rows x valid keys."""
@@ -264,12 +274,8 @@ def run_ours(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     attn_ms = [a.elapsed_time(b) for a, b in evs]
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(tt.item())
     ms_step = ms_total / args.steps
     value = flops * world / (ms_step * 1e-3) / 1e12
     attn_avg = sum(attn_ms) / len(attn_ms)
@@ -292,11 +298,7 @@ def run_ours(args, w, rank, world, local_rank):
             Oh.copy_(O, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / ksteps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / ksteps, world, dev)
         h2d = 3 * Q.numel() * Q.element_size()
         e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": O.numel() * O.element_size(), "ms_per_step": e2e_ms}
