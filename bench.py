@@ -252,7 +252,7 @@ def run_ours(args, w, rank, world, local_rank):
         if ev_b is not None:
             ev_b.record(stream)
 
-    launches_per_step = 4 + (sparge.SLA2_LAUNCHES if w.sla2 else 1)
+    launches_per_step = sparge.MASK_LAUNCHES + (sparge.SLA2_LAUNCHES if w.sla2 else sparge.ATTN_LAUNCHES)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()

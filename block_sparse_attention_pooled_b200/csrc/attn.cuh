@@ -8,7 +8,8 @@
 //
 // One CTA owns one 128-row query tile of one (batch, head) and walks only the
 // key tiles (64 keys each) of that tile's kept blocks:
-//   warp 0      TMA producer: Q once, then K and V tiles into two 2-slot rings;
+//   warp 0      TMA producer: Q once, then K and V tiles into two rings (2 slots;
+//               3 for the LIN variant, which runs one CTA per SM);
 //   warp 1      MMA issuer and TMEM owner: S = Q K^T into a double-buffered
 //               TMEM S, then O += P V with P read back from TMEM;
 //   warps 2..5  softmax: one query row per thread (TMEM lane), fp32 online
@@ -67,6 +68,9 @@ struct AttnParams {
 
 template <int D, bool LIN>
 struct AttnSmem {
+  // K / V (/ phi(K)) ring depth. Two slots keep the plain kernel small enough
+  // for two CTAs per SM; the LIN kernel runs one CTA per SM and uses three.
+  static constexpr int NS = LIN ? 3 : 2;
   static constexpr int kQBytes = kTileQ * D * 2;
   static constexpr int kKBytes = kTileK * D * 2;
   static constexpr int kVData = kTileK * D * 2;
@@ -74,10 +78,16 @@ struct AttnSmem {
   static constexpr int kPBytes = LIN ? kTileK * D * 2 : 0;     // phi(K) tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + 2 * kKBytes;
-  static constexpr int kOffP = kOffV + 2 * kVBytes;
-  static constexpr int kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kNumBars = 18;
+  static constexpr int kOffV = kOffK + NS * kKBytes;
+  static constexpr int kOffP = kOffV + NS * kVBytes;
+  static constexpr int kOffBar = kOffP + NS * kPBytes;
+  // Barrier slots: K full / V full / K empty / V empty rings, S full and
+  // P full pairs, then single barriers.
+  static constexpr int kBarQ = 0, kBarKFull = 1, kBarVFull = 1 + NS, kBarKEmpty = 1 + 2 * NS,
+                       kBarVEmpty = 1 + 3 * NS, kBarSFull = 1 + 4 * NS, kBarPFull = 3 + 4 * NS,
+                       kBarODone = 5 + 4 * NS, kBarOFinal = 6 + 4 * NS, kBarDrain = 7 + 4 * NS,
+                       kBarLin = 8 + 4 * NS;
+  static constexpr int kNumBars = 9 + 4 * NS;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kUsed = kOffTmem + 16;
   // Pad so that at most two CTAs fit on an SM: two CTAs x 256 TMEM columns
@@ -90,9 +100,6 @@ struct AttnSmem {
   static_assert(!LIN || kOffStage + 3 * 128 * 128 <= kOffV + kVData, "stage must not reach the ones block");
 };
 
-// Barrier slots.
-enum { kBarQ = 0, kBarKFull = 1, kBarVFull = 3, kBarKEmpty = 5, kBarVEmpty = 7, kBarSFull = 9,
-       kBarPFull = 11, kBarODone = 13, kBarOFinal = 14, kBarDrain = 15, kBarLin = 16 };
 
 // Waits on an mbarrier unless another role already gave up; gives up itself
 // (and tells the others through *abort) after the global time limit.
@@ -126,6 +133,10 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
                     const __grid_constant__ CUtensorMap tmPhiK, const AttnParams p) {
   static_assert(!LIN || D == 128, "the linear branch is built for d = 128");
   using L = AttnSmem<D, LIN>;
+  constexpr int NS = L::NS;
+  constexpr int kBarQ = L::kBarQ, kBarKFull = L::kBarKFull, kBarVFull = L::kBarVFull, kBarKEmpty = L::kBarKEmpty,
+                kBarVEmpty = L::kBarVEmpty, kBarSFull = L::kBarSFull, kBarPFull = L::kBarPFull,
+                kBarODone = L::kBarODone, kBarOFinal = L::kBarOFinal, kBarDrain = L::kBarDrain, kBarLin = L::kBarLin;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -148,11 +159,13 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarPFull + s), 128);
     }
@@ -165,7 +178,7 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
   }
   if (LIN) {
     // Ones block after each V slot: the 16 extra B columns that yield z.
-    for (int sl = 0; sl < 2; ++sl) {
+    for (int sl = 0; sl < NS; ++sl) {
       uint4* ones = reinterpret_cast<uint4*>(sgen + L::kOffV + sl * L::kVBytes + L::kVData);
       for (int u = threadIdx.x; u < 8192 / 16; u += kAttnThreads)
         ones[u] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
@@ -192,14 +205,14 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
       for (int b = 0; b < D / 64; ++b) tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(kBarQ), b * 64, q0, bh);
       int nk = 0, nv = 0;  // K and V tiles issued
       for (int t = 0; t < T; ++t) {
-        const int slot = t & 1;
+        const int slot = t % NS, round = t / NS;
         const int key0 = tile_key0(lst, t, tiles_per_block, p.bk);
-        if (t >= 2 && !role_wait(bar(kBarKEmpty + slot), ((t >> 1) - 1) & 1, kErrAttnKEmpty, abort_flag)) break;
+        if (t >= NS && !role_wait(bar(kBarKEmpty + slot), (round - 1) & 1, kErrAttnKEmpty, abort_flag)) break;
         mbar_arrive_expect_tx(bar(kBarKFull + slot), L::kKBytes);
         for (int b = 0; b < D / 64; ++b)
           tma_load_3d(sK + slot * L::kKBytes + b * (kTileK * 128), &tmK, bar(kBarKFull + slot), b * 64, key0, bh);
         ++nk;
-        if (t >= 2 && !role_wait(bar(kBarVEmpty + slot), ((t >> 1) - 1) & 1, kErrAttnVEmpty, abort_flag)) break;
+        if (t >= NS && !role_wait(bar(kBarVEmpty + slot), (round - 1) & 1, kErrAttnVEmpty, abort_flag)) break;
         mbar_arrive_expect_tx(bar(kBarVFull + slot), L::kVData + L::kPBytes);
         for (int b = 0; b < D / 64; ++b)
           tma_load_3d(sV + slot * L::kVBytes + b * (kTileK * 128), &tmV, bar(kBarVFull + slot), b * 64, key0, bh);
@@ -211,8 +224,10 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
       // Never leave with copies in flight: wait for the last loads issued to
       // land (they normally have; this only matters when a role gave up).
       mbar_wait(bar(kBarQ), 0, kErrAttnQ);
-      for (int t = (nk > 2 ? nk - 2 : 0); t < nk; ++t) mbar_wait(bar(kBarKFull + (t & 1)), (t >> 1) & 1, kErrAttnKFull);
-      for (int t = (nv > 2 ? nv - 2 : 0); t < nv; ++t) mbar_wait(bar(kBarVFull + (t & 1)), (t >> 1) & 1, kErrAttnVFull);
+      for (int t = (nk > NS ? nk - NS : 0); t < nk; ++t)
+        mbar_wait(bar(kBarKFull + t % NS), (t / NS) & 1, kErrAttnKFull);
+      for (int t = (nv > NS ? nv - NS : 0); t < nv; ++t)
+        mbar_wait(bar(kBarVFull + t % NS), (t / NS) & 1, kErrAttnVFull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -223,8 +238,8 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
       tc_fence_after();
       for (int t = 0; ok && t <= T; ++t) {
         if (t < T) {
-          const int slot = t & 1;
-          if (!role_wait(bar(kBarKFull + slot), (t >> 1) & 1, kErrAttnKFull, abort_flag)) break;
+          const int slot = t % NS;
+          if (!role_wait(bar(kBarKFull + slot), (t / NS) & 1, kErrAttnKFull, abort_flag)) break;
           tc_fence_after();
           const uint32_t kbase = sK + slot * L::kKBytes;
 #pragma unroll
@@ -232,26 +247,21 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
             const uint32_t off = (kk & 3) * 32u;  // 16 bf16 = 32 bytes along K inside the swizzle row
             const uint64_t a = sdesc_sw128(sQ + (kk >> 2) * (kTileQ * 128) + off, 16, 1024);
             const uint64_t b = sdesc_sw128(kbase + (kk >> 2) * (kTileK * 128) + off, 16, 1024);
-            mma_ss(tS + slot * 64, a, b, idS, kk > 0 ? 1u : 0u);
+            mma_ss(tS + (t & 1) * 64, a, b, idS, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(kBarSFull + slot));
+          mma_commit(bar(kBarSFull + (t & 1)));
           mma_commit(bar(kBarKEmpty + slot));
         }
         if (t >= 1) {
-          const int u = t - 1, slot = u & 1;
-          if (!role_wait(bar(kBarPFull + slot), (u >> 1) & 1, kErrAttnPFull, abort_flag)) break;
-          if (!role_wait(bar(kBarVFull + slot), (u >> 1) & 1, kErrAttnVFull, abort_flag)) break;
+          const int u = t - 1, vs = u % NS;
+          if (!role_wait(bar(kBarVFull + vs), (u / NS) & 1, kErrAttnVFull, abort_flag)) break;
           tc_fence_after();
-          const uint32_t vbase = sV + slot * L::kVBytes;
-#pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk) {
-            const uint64_t b = sdesc_sw128(vbase + kk * (16 * 128), kTileK * 128, 1024);
-            mma_ts(tO, tS + slot * 64 + kk * 8, b, idPV, (u > 0 || kk > 0) ? 1u : 0u);
-          }
+          const uint32_t vbase = sV + vs * L::kVBytes;
           if (LIN) {
-            // S_kept[feature, 0..143] += phi(K_u)^T [V_u | 1]
+            // S_kept[feature, 0..143] += phi(K_u)^T [V_u | 1]; independent of
+            // the softmax, so it is queued before waiting for P_u.
             constexpr uint32_t idL = idesc_bf16_f32(128, 144, true, true);
-            const uint32_t pbase = sP + slot * L::kPBytes;
+            const uint32_t pbase = sP + vs * L::kPBytes;
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               const uint64_t a = sdesc_sw128(pbase + kk * (16 * 128), kTileK * 128, 1024);
@@ -259,7 +269,14 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
               mma_ss(tL, a, b, idL, (u > 0 || kk > 0) ? 1u : 0u);
             }
           }
-          mma_commit(bar(kBarVEmpty + slot));
+          if (!role_wait(bar(kBarPFull + (u & 1)), (u >> 1) & 1, kErrAttnPFull, abort_flag)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            const uint64_t b = sdesc_sw128(vbase + kk * (16 * 128), kTileK * 128, 1024);
+            mma_ts(tO, tS + (u & 1) * 64 + kk * 8, b, idPV, (u > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(kBarVEmpty + vs));
           mma_commit(bar(kBarODone));
           if (u == T - 1) mma_commit(bar(kBarOFinal));
         }

@@ -27,12 +27,20 @@ namespace sparge {
 // walks its rows in order (16-byte loads, 8 fp32 accumulators).
 // ----------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ X, int64_t BH, int N,
-                                                   int blk, float* __restrict__ out) {
+__global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                   const __nv_bfloat16* __restrict__ K, int64_t BH, int N, int bq,
+                                                   int bk, int64_t q_ctas, float* __restrict__ qbar,
+                                                   float* __restrict__ kbar) {
   constexpr int TPB = D / 8;            // threads per block-row
   constexpr int BLOCKS_PER_CTA = 128 / TPB;
+  // CTAs [0, q_ctas) pool Q blocks, the rest pool K blocks.
+  const bool is_q = blockIdx.x < q_ctas;
+  const __nv_bfloat16* X = is_q ? Q : K;
+  float* out = is_q ? qbar : kbar;
+  const int blk = is_q ? bq : bk;
+  const int64_t cta = is_q ? blockIdx.x : blockIdx.x - q_ctas;
   const int nb = (N + blk - 1) / blk;
-  const int64_t g = (int64_t)blockIdx.x * BLOCKS_PER_CTA + threadIdx.x / TPB;  // flat (bh, block)
+  const int64_t g = cta * BLOCKS_PER_CTA + threadIdx.x / TPB;  // flat (bh, block)
   if (g >= BH * nb) return;
   const int c8 = (threadIdx.x % TPB) * 8;
   const int64_t bh = g / nb;
@@ -44,24 +52,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
   const int rows = r1 - r0;
-  int r = 0;
-  for (; r + 4 <= rows; r += 4) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = __ldg(src + (int64_t)(r + u) * (D / 8));
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float2 f = __bfloat1622float2(h[j]);
-        acc[2 * j] = __fadd_rn(acc[2 * j], f.x);
-        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], f.y);
-      }
-    }
-  }
-  for (; r < rows; ++r) {
-    uint4 v = __ldg(src + (int64_t)r * (D / 8));
+  auto add_row = [&](uint4 v) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -69,7 +60,16 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
       acc[2 * j] = __fadd_rn(acc[2 * j], f.x);
       acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], f.y);
     }
+  };
+  int r = 0;
+  for (; r + 8 <= rows; r += 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + (int64_t)(r + u) * (D / 8));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) add_row(v[u]);  // rows in order
   }
+  for (; r < rows; ++r) add_row(__ldg(src + (int64_t)r * (D / 8)));
   const float cnt = (float)rows;
   float4* dst = reinterpret_cast<float4*>(out + g * D + c8);
   dst[0] = make_float4(__fdiv_rn(acc[0], cnt), __fdiv_rn(acc[1], cnt), __fdiv_rn(acc[2], cnt),
@@ -79,13 +79,12 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ----------------------------------------------------------------------------
-// Scores + row softmax. One CTA = 16 query-block rows of one (b,h) against all
-// Nkb key blocks. Pooled K is staged through shared memory 64 blocks at a time
-// (rows padded by 4 floats so that 16-byte loads of different rows fall in
-// different banks); each thread owns 2 rows x 4 key blocks and runs their
-// fused multiply-add chains over channels in order. The scaled scores are
-// written to the output rows, which the same CTA then turns into
-// probabilities in place (the rows stay in L2 between the two passes).
+// Scaled scores z[I, J] = (q̄_I . k̄_J) * (float)(1/sqrt(d)). One CTA = 16
+// query-block rows x 64 key blocks of one (b,h); each thread owns 2 rows x 4
+// key blocks and runs their fused multiply-add chains over channels in order.
+// Pooled K rows are padded by 4 floats in shared memory so that the 16-byte
+// loads of different rows fall in different banks. The row softmax happens
+// in the selection kernel, which reads the whole row anyway.
 // ----------------------------------------------------------------------------
 constexpr int kScoreRows = 16;
 constexpr int kScoreTileJ = 64;
@@ -96,90 +95,73 @@ __host__ __device__ constexpr int score_smem_bytes() {
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) score_softmax_kernel(const float* __restrict__ qbar,
-                                                            const float* __restrict__ kbar, int64_t BH,
-                                                            int nqb, int nkb, float scale,
-                                                            float* __restrict__ P) {
+__global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+                                                    int nqb, int nkb, float scale, float* __restrict__ Z) {
   extern __shared__ __align__(16) float sm[];
   float* sq = sm;                                   // [16][D]
   float* sk = sq + kScoreRows * D;                  // [64][D+4]
-  const int tiles_per_bh = (nqb + kScoreRows - 1) / kScoreRows;
-  const int64_t bh = blockIdx.x / tiles_per_bh;
-  const int I0 = (blockIdx.x % tiles_per_bh) * kScoreRows;
+  const int tiles_q = (nqb + kScoreRows - 1) / kScoreRows;
+  const int tiles_j = (nkb + kScoreTileJ - 1) / kScoreTileJ;
+  const int64_t cta = blockIdx.x;
+  const int64_t bh = cta / ((int64_t)tiles_q * tiles_j);
+  const int rem = (int)(cta % ((int64_t)tiles_q * tiles_j));
+  const int I0 = (rem / tiles_j) * kScoreRows;
+  const int J0 = (rem % tiles_j) * kScoreTileJ;
   const int nrows = min(kScoreRows, nqb - I0);
+  const int nj = min(kScoreTileJ, nkb - J0);
   const int tid = threadIdx.x;
-
-  for (int e = tid; e < kScoreRows * D; e += 128) {
-    const int i = e / D;
-    sq[e] = (i < nrows) ? qbar[(bh * nqb + I0 + i) * D + (e % D)] : 0.0f;
+  for (int e = tid; e < kScoreRows * (D / 4); e += 128) {
+    const int i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < nrows) v = *reinterpret_cast<const float4*>(qbar + (bh * nqb + I0 + i) * D + c4);
+    *reinterpret_cast<float4*>(sq + i * D + c4) = v;
   }
+  for (int e = tid; e < kScoreTileJ * (D / 4); e += 128) {
+    const int j = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < nj) v = *reinterpret_cast<const float4*>(kbar + (bh * nkb + J0 + j) * D + c4);
+    *reinterpret_cast<float4*>(sk + j * (D + 4) + c4) = v;
+  }
+  __syncthreads();
   const int jl = tid % 16;   // key blocks jl, jl+16, jl+32, jl+48 of the tile
   const int ig = tid / 16;   // query rows 2*ig, 2*ig+1
-  const float* kb_head = kbar + bh * (int64_t)nkb * D;
-  for (int J0 = 0; J0 < nkb; J0 += kScoreTileJ) {
-    __syncthreads();
-    const int nj = min(kScoreTileJ, nkb - J0);
-    for (int e = tid; e < kScoreTileJ * (D / 4); e += 128) {
-      const int j = e / (D / 4), c4 = (e % (D / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < nj) v = *reinterpret_cast<const float4*>(kb_head + (int64_t)(J0 + j) * D + c4);
-      *reinterpret_cast<float4*>(sk + j * (D + 4) + c4) = v;
-    }
-    __syncthreads();
-    float acc[2][4];
+  float acc[2][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 2; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
 #pragma unroll 4
-    for (int c = 0; c < D; c += 4) {
-      float4 q[2], k[4];
+  for (int c = 0; c < D; c += 4) {
+    float4 q[2], k[4];
 #pragma unroll
-      for (int a = 0; a < 2; ++a) q[a] = *reinterpret_cast<const float4*>(sq + (2 * ig + a) * D + c);
+    for (int a = 0; a < 2; ++a) q[a] = *reinterpret_cast<const float4*>(sq + (2 * ig + a) * D + c);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) k[b] = *reinterpret_cast<const float4*>(sk + (jl + 16 * b) * (D + 4) + c);
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          acc[a][b] = __fmaf_rn(q[a].x, k[b].x, acc[a][b]);
-          acc[a][b] = __fmaf_rn(q[a].y, k[b].y, acc[a][b]);
-          acc[a][b] = __fmaf_rn(q[a].z, k[b].z, acc[a][b]);
-          acc[a][b] = __fmaf_rn(q[a].w, k[b].w, acc[a][b]);
-        }
-    }
+    for (int b = 0; b < 4; ++b) k[b] = *reinterpret_cast<const float4*>(sk + (jl + 16 * b) * (D + 4) + c);
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int j = jl + 16 * b;
-        if (j < nj && 2 * ig + a < nrows)
-          P[(bh * nqb + I0 + 2 * ig + a) * (int64_t)nkb + J0 + j] = __fmul_rn(acc[a][b], scale);
+        acc[a][b] = __fmaf_rn(q[a].x, k[b].x, acc[a][b]);
+        acc[a][b] = __fmaf_rn(q[a].y, k[b].y, acc[a][b]);
+        acc[a][b] = __fmaf_rn(q[a].z, k[b].z, acc[a][b]);
+        acc[a][b] = __fmaf_rn(q[a].w, k[b].w, acc[a][b]);
       }
   }
-  __syncthreads();
-  // Softmax: warp w handles rows w, w+4, w+8, w+12.
-  const int warp = tid / 32, lane = tid % 32;
-  for (int i = warp; i < nrows; i += 4) {
-    float* z = P + (bh * nqb + I0 + i) * (int64_t)nkb;
-    float mx = -INFINITY;
-    for (int j = lane; j < nkb; j += 32) mx = fmaxf(mx, z[j]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.0f;
-    for (int j = lane; j < nkb; j += 32) {
-      const float e = expf(__fsub_rn(z[j], mx));
-      z[j] = e;
-      sum = __fadd_rn(sum, e);
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = jl + 16 * b;
+      if (j < nj && 2 * ig + a < nrows)
+        Z[(bh * nqb + I0 + 2 * ig + a) * (int64_t)nkb + J0 + j] = __fmul_rn(acc[a][b], scale);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
-    for (int j = lane; j < nkb; j += 32) z[j] = __fdiv_rn(z[j], sum);
-  }
 }
 
 // ----------------------------------------------------------------------------
-// Selection. One CTA of 256 threads per query-block row:
+// Softmax + selection. One CTA of 256 threads per query-block row:
+//   0. P = expf(z - rowmax) / rowsum, the row sum taken as 32 interleaved
+//      partial sums (partial l adds z-terms l, l+32, ... in turn) combined
+//      pairwise at distances 16, 8, 4, 2, 1; P is written back over z;
 //   1. keys (~bits(P) << 32 | J): ascending order = P descending, J ascending;
 //   2. bitonic sort in shared memory (padded to a power of two);
 //   3. running sums of the sorted P in double -> pc = first prefix >= topp;
@@ -199,7 +181,7 @@ __host__ __device__ constexpr int select_smem_bytes(int nkb) {
   return select_pad(nkb) * 8 + select_pad(nkb) * 4 + kSelectThreads * 8 + 64;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_kernel(const float* __restrict__ P, int64_t rows,
+__global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restrict__ P, int64_t rows,
                                                                  int nkb, int kc, double topp,
                                                                  int32_t* __restrict__ kv_idx,
                                                                  int32_t* __restrict__ kv_cnt,
@@ -213,13 +195,41 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const float* __r
   const int64_t row = blockIdx.x;
   if (row >= rows) return;
   const int tid = threadIdx.x;
-  const float* prow = P + row * (int64_t)nkb;
+  float* prow = P + row * (int64_t)nkb;
+  float* ev = reinterpret_cast<float*>(flag);  // e-values, before the flags need the space
+  float* red = reinterpret_cast<float*>(tsum);
 
+  // 0. Row softmax.
+  float mx = -INFINITY;
+  for (int j = tid; j < nkb; j += kSelectThreads) {
+    const float z = prow[j];
+    ev[j] = z;
+    mx = fmaxf(mx, z);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int w = 1; w < kSelectThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+  for (int j = tid; j < nkb; j += kSelectThreads) ev[j] = expf(__fsub_rn(ev[j], mx));
+  __syncthreads();
+  if (tid < 32) {
+    float part = 0.0f;
+    for (int j = tid; j < nkb; j += 32) part = __fadd_rn(part, ev[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+    if (tid == 0) red[16] = part;
+  }
+  __syncthreads();
+  const float rsum = red[16];
   for (int j = tid; j < n; j += kSelectThreads) {
     unsigned long long k = ~0ull;
     if (j < nkb) {
-      const unsigned int bits = __float_as_uint(prow[j]);
-      k = ((unsigned long long)(0xFFFFFFFFu - bits) << 32) | (unsigned int)j;
+      const float pj = __fdiv_rn(ev[j], rsum);
+      prow[j] = pj;
+      k = ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(pj)) << 32) | (unsigned int)j;
     }
     key[j] = k;
   }

@@ -121,14 +121,16 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
   float* P = probs ? probs : reinterpret_cast<float*>(ws + w.probs);
   constexpr int per_cta = 128 / (D / 8);
   const int64_t gq = ceil_div(dm.BH * dm.nqb, per_cta), gk = ceil_div(dm.BH * dm.nkb, per_cta);
-  pool_kernel<D><<<(unsigned)gq, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(Q), dm.BH, s->N, s->bq, qbar);
-  pool_kernel<D><<<(unsigned)gk, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(K), dm.BH, s->N, s->bk, kbar);
+  pool_kernel<D><<<(unsigned)(gq + gk), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(Q),
+                                                     static_cast<const __nv_bfloat16*>(K), dm.BH, s->N, s->bq,
+                                                     s->bk, gq, qbar, kbar);
   const float scale = (float)(1.0 / std::sqrt((double)D));
   const int ssm = score_smem_bytes<D>();
-  cudaError_t e = ensure_smem(score_softmax_kernel<D>, ssm, D == 64 ? 0 : 1);
+  cudaError_t e = ensure_smem(score_kernel<D>, ssm, D == 64 ? 0 : 1);
   if (e != cudaSuccess) return cuda_status(e);
-  const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows);
-  score_softmax_kernel<D><<<(unsigned)tiles, 128, ssm, st>>>(qbar, kbar, dm.BH, (int)dm.nqb, (int)dm.nkb, scale, P);
+  const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows) * ceil_div(dm.nkb, kScoreTileJ);
+  if (tiles > INT32_MAX) return SPARGE_ERR_UNSUPPORTED;
+  score_kernel<D><<<(unsigned)tiles, 128, ssm, st>>>(qbar, kbar, (int)dm.nqb, (int)dm.nkb, scale, P);
   const int sel_sm = select_smem_bytes((int)dm.nkb);
   e = ensure_smem(select_kernel, sel_sm, 2);
   if (e != cudaSuccess) return cuda_status(e);
