@@ -160,44 +160,153 @@ __global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qb
 // ----------------------------------------------------------------------------
 // Softmax + selection. One CTA of 256 threads per query-block row:
 //   0. P = expf(z - rowmax) / rowsum, the row sum taken as 32 interleaved
-//      partial sums (partial l adds z-terms l, l+32, ... in turn) combined
-//      pairwise at distances 16, 8, 4, 2, 1; P is written back over z;
-//   1. keys (~bits(P) << 32 | J): ascending order = P descending, J ascending;
-//   2. bitonic sort in shared memory (padded to a power of two);
-//   3. running sums of the sorted P in double -> pc = first prefix >= topp;
-//   4. m = max(kc, pc, 1); flag the first m blocks; compact the flags in block
-//      order to emit the kept list ascending.
+//      partial sums (partial l adds the terms l, l+32, ... in turn) combined
+//      pairwise at distances 16, 8, 4, 2, 1; P is written back over z.
+//   1. Key of block j = the bit pattern of P_j (ordered like P for P >= 0);
+//      weight of block j = P_j in 64-bit fixed point (2^62 = 1), exact for
+//      P >= 2^-39 and truncated below, so running sums are exact integers
+//      whatever the summation order.
+//   2. Top-p: radix select (four 8-bit digits, most significant first) of the
+//      key at which the descending running weight first reaches p; ties at
+//      that key all weigh the same, so the count needed follows by division.
+//   3. m = max(kc, pc, 1); a second radix select (counting) finds the key of
+//      the m-th largest block; blocks above it are kept, and of the blocks at
+//      it the lowest indices fill the remaining places.
+//   4. Kept flags are compacted in block order (block-wide scans) into the
+//      ascending kept list.
 // ----------------------------------------------------------------------------
 constexpr int kSelectThreads = 256;
-
-__host__ __device__ constexpr int select_pad(int nkb) {
-  int n = 32;
-  while (n < nkb) n <<= 1;
-  return n;
-}
+constexpr int kSelectMaxPer = 16;  // blocks per thread: Nkb <= 4096
 
 __host__ __device__ constexpr int select_smem_bytes(int nkb) {
-  // keys (8 B each) + flags/scan (4 B each) + per-thread sums (8 B each)
-  return select_pad(nkb) * 8 + select_pad(nkb) * 4 + kSelectThreads * 8 + 64;
+  // z / P row (4 B per block) + keys (4 B per block) + histograms + scratch
+  return ((nkb + 3) / 4 * 4) * 8 + 256 * 12 + 1024;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restrict__ P, int64_t rows,
-                                                                 int nkb, int kc, double topp,
-                                                                 int32_t* __restrict__ kv_idx,
+__device__ __forceinline__ unsigned long long p_fixed62(unsigned int bits) {
+  const int e = (int)((bits >> 23) & 0xFFu);
+  if (e == 0) return 0ull;  // zero or subnormal: below 2^-126
+  const unsigned long long mant = (unsigned long long)((bits & 0x7FFFFFu) | 0x800000u);
+  const int sh = e - 88;    // value = mant * 2^(e - 150); times 2^62
+  if (sh >= 0) return mant << sh;
+  return (-sh >= 64) ? 0ull : (mant >> (-sh));
+}
+
+// Block-wide exclusive scan of one int per thread (256 threads).
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[wid] = x;
+  __syncthreads();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kSelectThreads / 32; ++w) {
+    const int s = scratch[w];
+    if (w < wid) base += s;
+    tot += s;
+  }
+  __syncthreads();
+  *total = tot;
+  return base + x - v;
+}
+
+// One radix-select pass. Candidates are keys whose bits above `shift + 8`
+// equal `prefix`. Buckets are digits (key >> shift) & 255 taken from the top
+// (largest key) down. With weights (by_weight) it finds the bucket where the
+// running weight, starting from *above_w, first reaches `target`; otherwise
+// the bucket where the running count, starting from *above_c, first reaches
+// it. Updates prefix / above_w / above_c. Called by all 256 threads.
+__device__ void radix_pass(const unsigned int* keys, int nkb, int shift, unsigned int hi_mask, bool by_weight,
+                           unsigned long long target, unsigned int* prefix, unsigned long long* above_w,
+                           int* above_c, unsigned int* hcnt, unsigned long long* hsum, unsigned int* bc) {
+  const int tid = threadIdx.x;
+  hcnt[tid] = 0u;
+  hsum[tid] = 0ull;
+  __syncthreads();
+  const unsigned int pre = *prefix;
+  for (int j = tid; j < nkb; j += kSelectThreads) {
+    const unsigned int k = keys[j];
+    if ((k & hi_mask) == pre) {
+      const unsigned int d = (k >> shift) & 255u;
+      atomicAdd(&hcnt[d], 1u);
+      if (by_weight) atomicAdd(&hsum[d], p_fixed62(k));
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // Lane l owns buckets 255-8l ... 248-8l (descending).
+    unsigned long long lw = 0ull;
+    unsigned int lc = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = 255 - 8 * tid - i;
+      lw += hsum[b];
+      lc += hcnt[b];
+    }
+    unsigned long long xw = lw;
+    unsigned int xc = lc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long yw = __shfl_up_sync(0xffffffffu, xw, o);
+      const unsigned int yc = __shfl_up_sync(0xffffffffu, xc, o);
+      if (tid >= o) {
+        xw += yw;
+        xc += yc;
+      }
+    }
+    const unsigned long long aw = *above_w + xw - lw;  // running value before this lane's buckets
+    const unsigned int ac = (unsigned int)*above_c + xc - lc;
+    const bool reach = by_weight ? (aw + lw >= target) : ((unsigned long long)(ac + lc) >= target);
+    const unsigned int ballot = __ballot_sync(0xffffffffu, reach);
+    const int first = __ffs(ballot) - 1;  // first lane (from the top) whose buckets reach the target
+    if (tid == first) {
+      unsigned long long w = aw;
+      unsigned int c = ac;
+      int bsel = 255 - 8 * tid - 7;
+      for (int i = 0; i < 8; ++i) {
+        const int b = 255 - 8 * tid - i;
+        const bool hit = by_weight ? (w + hsum[b] >= target) : ((unsigned long long)(c + hcnt[b]) >= target);
+        if (hit) {
+          bsel = b;
+          break;
+        }
+        w += hsum[b];
+        c += hcnt[b];
+      }
+      bc[0] = (unsigned int)bsel;
+      bc[1] = c;
+      *reinterpret_cast<unsigned long long*>(bc + 2) = w;
+    }
+  }
+  __syncthreads();
+  *prefix = pre | (bc[0] << shift);
+  *above_c = (int)bc[1];
+  *above_w = *reinterpret_cast<unsigned long long*>(bc + 2);
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restrict__ P, int64_t rows, int nkb,
+                                                                 int kc, double topp, int32_t* __restrict__ kv_idx,
                                                                  int32_t* __restrict__ kv_cnt,
                                                                  float* __restrict__ row_thresh) {
   extern __shared__ __align__(16) unsigned char smraw[];
-  const int n = select_pad(nkb);
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(smraw);
-  int* flag = reinterpret_cast<int*>(smraw + (size_t)n * 8);
-  double* tsum = reinterpret_cast<double*>(smraw + (size_t)n * 12);
-  int* s_misc = reinterpret_cast<int*>(smraw + (size_t)n * 12 + kSelectThreads * 8);
+  const int npad = (nkb + 3) / 4 * 4;
+  float* ev = reinterpret_cast<float*>(smraw);                                  // [npad]
+  unsigned int* keys = reinterpret_cast<unsigned int*>(smraw + npad * 4);        // [npad]
+  unsigned long long* hsum = reinterpret_cast<unsigned long long*>(smraw + npad * 8);  // [256]
+  unsigned int* hcnt = reinterpret_cast<unsigned int*>(smraw + npad * 8 + 2048);       // [256]
+  unsigned int* bc = hcnt + 256;                                                  // [4]
+  float* red = reinterpret_cast<float*>(bc + 4);                                  // [16]
+  int* scratch = reinterpret_cast<int*>(red + 16);                                // [8]
   const int64_t row = blockIdx.x;
   if (row >= rows) return;
   const int tid = threadIdx.x;
   float* prow = P + row * (int64_t)nkb;
-  float* ev = reinterpret_cast<float*>(flag);  // e-values, before the flags need the space
-  float* red = reinterpret_cast<float*>(tsum);
 
   // 0. Row softmax.
   float mx = -INFINITY;
@@ -220,97 +329,95 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restric
     for (int j = tid; j < nkb; j += 32) part = __fadd_rn(part, ev[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
-    if (tid == 0) red[16] = part;
+    if (tid == 0) red[8] = part;
   }
   __syncthreads();
-  const float rsum = red[16];
-  for (int j = tid; j < n; j += kSelectThreads) {
-    unsigned long long k = ~0ull;
-    if (j < nkb) {
-      const float pj = __fdiv_rn(ev[j], rsum);
-      prow[j] = pj;
-      k = ((unsigned long long)(0xFFFFFFFFu - __float_as_uint(pj)) << 32) | (unsigned int)j;
-    }
-    key[j] = k;
+  const float rsum = red[8];
+  for (int j = tid; j < nkb; j += kSelectThreads) {
+    const float pj = __fdiv_rn(ev[j], rsum);
+    prow[j] = pj;
+    keys[j] = __float_as_uint(pj);
   }
-  if (tid == 0) s_misc[0] = nkb;  // pc candidate (min), starts at "never reached"
   __syncthreads();
 
-  // Bitonic sort, ascending.
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = tid; t < n / 2; t += kSelectThreads) {
-        const int lo = 2 * t - (t & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const unsigned long long a = key[lo], b = key[hi];
-        if ((a > b) == up) {
-          key[lo] = b;
-          key[hi] = a;
-        }
-      }
-      __syncthreads();
-    }
-  }
-
-  // Top-p: each thread sums a contiguous chunk of the sorted order in double,
-  // an exclusive scan over the chunk sums gives each chunk's start, then each
-  // thread finds the first crossing inside its chunk.
+  // 2. Top-p count.
   int pc = 0;
   if (topp > 0.0) {
-    const int chunk = (nkb + kSelectThreads - 1) / kSelectThreads;
-    const int s0 = min(nkb, tid * chunk), s1 = min(nkb, s0 + chunk);
-    double local = 0.0;
-    for (int s = s0; s < s1; ++s)
-      local += (double)__uint_as_float(0xFFFFFFFFu - (unsigned int)(key[s] >> 32));
-    tsum[tid] = local;
+    const unsigned long long target = (unsigned long long)ceil(topp * 4611686018427387904.0);  // p * 2^62
+    unsigned long long tot = 0ull;  // total weight (exact integer sum)
+    for (int j = tid; j < nkb; j += kSelectThreads) tot += p_fixed62(keys[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    if ((tid & 31) == 0) hsum[tid >> 5] = tot;
     __syncthreads();
-    // Hillis-Steele inclusive scan over 256 doubles.
-    for (int off = 1; off < kSelectThreads; off <<= 1) {
-      const double v = (tid >= off) ? tsum[tid - off] : 0.0;
-      __syncthreads();
-      tsum[tid] += v;
-      __syncthreads();
-    }
-    double run = tsum[tid] - local;  // exclusive prefix
-    for (int s = s0; s < s1; ++s) {
-      run += (double)__uint_as_float(0xFFFFFFFFu - (unsigned int)(key[s] >> 32));
-      if (run >= topp) {
-        atomicMin(&s_misc[0], s + 1);
-        break;
+    tot = 0ull;
+#pragma unroll
+    for (int w = 0; w < kSelectThreads / 32; ++w) tot += hsum[w];
+    __syncthreads();
+    if (tot < target) {
+      pc = nkb;  // never reached
+    } else {
+      unsigned int prefix = 0u;
+      unsigned long long above_w = 0ull;
+      int above_c = 0;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        const unsigned int hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        radix_pass(keys, nkb, shift, hi_mask, true, target, &prefix, &above_w, &above_c, hcnt, hsum, bc);
       }
+      // All blocks with key == prefix weigh the same.
+      const unsigned long long wt = p_fixed62(prefix);
+      const unsigned long long need = target - above_w;  // > 0 by construction
+      const unsigned long long c = wt ? (need + wt - 1) / wt : 0ull;
+      pc = above_c + (int)c;
     }
-    __syncthreads();
-    pc = s_misc[0];
   }
-  const int m = max(max(kc, pc), 1);
+  const int m = min(nkb, max(max(kc, pc), 1));
 
-  // Flag kept blocks, then compact in block-index order.
-  for (int j = tid; j < n; j += kSelectThreads) flag[j] = 0;
-  __syncthreads();
-  for (int s = tid; s < m; s += kSelectThreads) flag[(int)(key[s] & 0xFFFFFFFFu)] = 1;
-  __syncthreads();
-  // Block-wide exclusive scan of flags, each thread owning a contiguous chunk.
-  const int chunk = n / kSelectThreads > 0 ? n / kSelectThreads : 1;
-  const int c0 = tid * chunk, c1 = min(n, c0 + chunk);
-  int cnt = 0;
-  for (int j = c0; j < c1; ++j) cnt += flag[j];
-  int* tcnt = reinterpret_cast<int*>(tsum);
-  tcnt[tid] = cnt;
-  __syncthreads();
-  for (int off = 1; off < kSelectThreads; off <<= 1) {
-    const int v = (tid >= off) ? tcnt[tid - off] : 0;
-    __syncthreads();
-    tcnt[tid] += v;
-    __syncthreads();
+  // 3. Key of the m-th largest block, and how many of its ties are kept.
+  unsigned int tkey = 0u;
+  int above_m = 0;
+  {
+    unsigned int prefix = 0u;
+    unsigned long long above_w = 0ull;
+    int above_c = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      const unsigned int hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+      radix_pass(keys, nkb, shift, hi_mask, false, (unsigned long long)m, &prefix, &above_w, &above_c, hcnt, hsum,
+                 bc);
+    }
+    tkey = prefix;
+    above_m = above_c;
   }
-  int pos = tcnt[tid] - cnt;
+  const int ties_kept = m - above_m;
+
+  // 4. Compaction in block order: each thread owns a contiguous chunk.
+  const int per = (nkb + kSelectThreads - 1) / kSelectThreads;
+  const int j0 = min(nkb, tid * per), j1 = min(nkb, j0 + per);
+  int nt = 0;
+  for (int j = j0; j < j1; ++j) nt += keys[j] == tkey;
+  int tie_tot;
+  int tie_rank = block_excl_scan(nt, scratch, &tie_tot);
+  int nk = 0;
+  {
+    int tr = tie_rank;
+    for (int j = j0; j < j1; ++j) {
+      const unsigned int k = keys[j];
+      if (k > tkey || (k == tkey && tr++ < ties_kept)) ++nk;
+    }
+  }
+  int kept_tot;
+  int pos = block_excl_scan(nk, scratch, &kept_tot);
   int32_t* out = kv_idx + row * (int64_t)nkb;
-  for (int j = c0; j < c1; ++j)
-    if (flag[j]) out[pos++] = j;
+  {
+    int tr = tie_rank;
+    for (int j = j0; j < j1; ++j) {
+      const unsigned int k = keys[j];
+      if (k > tkey || (k == tkey && tr++ < ties_kept)) out[pos++] = j;
+    }
+  }
   if (tid == 0) {
     kv_cnt[row] = m;
-    if (row_thresh) row_thresh[row] = __uint_as_float(0xFFFFFFFFu - (unsigned int)(key[m - 1] >> 32));
+    if (row_thresh) row_thresh[row] = __uint_as_float(tkey);
   }
 }
 
