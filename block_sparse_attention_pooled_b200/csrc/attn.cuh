@@ -43,6 +43,9 @@ constexpr int kAttnThreads = 192;
 constexpr int kTileQ = 128;   // query rows per MMA tile
 constexpr int kTileK = 64;    // keys per MMA tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+// Of the 64 exponentials per row and tile, this many run on the FMA pipe
+// (exp2_poly) and the rest on the MUFU (ex2.approx).
+constexpr int kPolyExp = 0;
 
 // Error site codes recorded in g_device_error by the attention kernel.
 enum : unsigned int {
@@ -204,9 +207,11 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
       mbar_arrive_expect_tx(bar(kBarQ), L::kQBytes);
       for (int b = 0; b < D / 64; ++b) tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(kBarQ), b * 64, q0, bh);
       int nk = 0, nv = 0;  // K and V tiles issued
+      int key_next = tile_key0(lst, 0, tiles_per_block, p.bk);
       for (int t = 0; t < T; ++t) {
         const int slot = t % NS, round = t / NS;
-        const int key0 = tile_key0(lst, t, tiles_per_block, p.bk);
+        const int key0 = key_next;
+        if (t + 1 < T) key_next = tile_key0(lst, t + 1, tiles_per_block, p.bk);  // latency hidden by the waits
         if (t >= NS && !role_wait(bar(kBarKEmpty + slot), (round - 1) & 1, kErrAttnKEmpty, abort_flag)) break;
         mbar_arrive_expect_tx(bar(kBarKFull + slot), L::kKBytes);
         for (int b = 0; b < D / 64; ++b)
@@ -293,8 +298,13 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
     float m_run = -INFINITY, l_run = 0.0f;
     int kept_keys = 0;  // valid keys in the kept tiles (LIN: the complement is empty when this is N)
     bool ok = true;
+    // The block index of tile t+1 is requested while tile t is processed, so
+    // its global-load latency stays off the softmax's critical path.
+    int key_next = T > 0 ? tile_key0(lst, 0, tiles_per_block, p.bk) : 0;
     for (int t = 0; t < T; ++t) {
       const int slot = t & 1;
+      const int key0 = key_next;
+      if (t + 1 < T) key_next = tile_key0(lst, t + 1, tiles_per_block, p.bk);
       ok = __all_sync(0xffffffffu, role_wait(bar(kBarSFull + slot), (t >> 1) & 1, kErrAttnSFull, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -309,16 +319,21 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
 #pragma unroll
           for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(v[c][j]);
       }
-      const int key0 = tile_key0(lst, t, tiles_per_block, p.bk);
       kept_keys += max(0, min(kTileK, p.N - key0));
       if (key0 + kTileK > p.N) {
 #pragma unroll
         for (int j = 0; j < kTileK; ++j)
           if (key0 + j >= p.N) s[j] = -INFINITY;
       }
-      float mx = -INFINITY;
+      float mx;  // tree reduction: depth 6 instead of a 64-long chain
+      {
+        float m8[8];
 #pragma unroll
-      for (int j = 0; j < kTileK; ++j) mx = fmaxf(mx, s[j]);
+        for (int j = 0; j < 8; ++j)
+          m8[j] = fmaxf(fmaxf(fmaxf(s[j], s[8 + j]), fmaxf(s[16 + j], s[24 + j])),
+                        fmaxf(fmaxf(s[32 + j], s[40 + j]), fmaxf(s[48 + j], s[56 + j])));
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       if (t == 0) {
         m_run = m_new;
@@ -344,16 +359,17 @@ __global__ void __launch_bounds__(kAttnThreads, LIN ? 1 : 2)
         m_run = m_new;
       }
       const float neg_m = -m_run;
-      float psum = 0.0f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: short dependency chains
       uint32_t pk[kTileK / 2];
 #pragma unroll
       for (int j = 0; j < kTileK; j += 2) {
-        const float a = ex2_approx(fmaf(s[j], p.scale_log2, neg_m));
-        const float b = ex2_approx(fmaf(s[j + 1], p.scale_log2, neg_m));
-        psum += a + b;
+        const float xa = fmaf(s[j], p.scale_log2, neg_m), xb = fmaf(s[j + 1], p.scale_log2, neg_m);
+        const float a = (j < kPolyExp) ? exp2_poly(xa) : ex2_approx(xa);
+        const float b = (j < kPolyExp) ? exp2_poly(xb) : ex2_approx(xb);
+        ps[(j >> 1) & 3] += a + b;
         pk[j / 2] = pack_bf16x2(a, b);
       }
-      l_run += psum;
+      l_run += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       // P (bf16) overwrites the first 32 columns of this S buffer.
       tmem_st16(tS + lane_off + slot * 64, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
       tmem_st16(tS + lane_off + slot * 64 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
