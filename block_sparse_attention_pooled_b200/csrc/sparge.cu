@@ -204,6 +204,33 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
   return cuda_status(cudaGetLastError());
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for sparge_mask_noalloc: a fixed array in device memory, part of
+// the loaded module, so that entry point needs no allocation at all. Every
+// device that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device. Host code may
+// not use the array's name as an address; cudaGetSymbolAddress is called once
+// per device (with that device current) and the result is cached.
+sparge_status noalloc_scratch(uint8_t** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cuda_status(cudaErrorInvalidDevice);
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return cuda_status(e == cudaSuccess ? cudaErrorInvalidSymbol : e);
+    addr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(addr[dev]);
+  return SPARGE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -242,6 +269,33 @@ sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shap
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (shape->d == 64) return launch_mask<64>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
+  return launch_mask<128>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
+}
+
+sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_shape* shape, double topk_frac,
+                                  double topp, int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs,
+                                  void* stream) {
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || (probs && !aligned16(probs))) return SPARGE_ERR_INVALID_ARG;
+  if (!(topk_frac >= 0.0 && topk_frac <= 1.0) || !(topp >= 0.0 && topp <= 1.0)) return SPARGE_ERR_INVALID_ARG;
+  // Pooled Q and K always live in the scratch; the probability rows too
+  // unless the caller supplies `probs`.
+  const MaskWs w = mask_ws(shape, dm);
+  const size_t need = probs ? w.probs : w.total;
+  if (need > kNoAllocScratchBytes) return SPARGE_ERR_WORKSPACE;
+  uint8_t* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != SPARGE_OK) return st;
+  int kc = 0;
+  if (topk_frac > 0.0) {
+    const double c = std::ceil(topk_frac * (double)dm.nkb - 1e-9);
+    kc = (int)std::min<double>(std::max<double>(c, 0.0), (double)dm.nkb);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (shape->d == 64) return launch_mask<64>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
   return launch_mask<128>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
 }

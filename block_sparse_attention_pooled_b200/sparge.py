@@ -27,7 +27,7 @@ MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES = 3, 1, 3
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
-           "sparge_device_status", "sparge_status_string")
+           "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc")
 
 
 class Shape(ctypes.Structure):
@@ -38,6 +38,8 @@ _vp, _sz, _dbl = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_double
 _lib.sparge_workspace_bytes.argtypes = [ctypes.c_int, ctypes.POINTER(Shape)]
 _lib.sparge_workspace_bytes.restype = _sz
 _lib.sparge_mask.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _dbl, _dbl, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sparge_mask_noalloc.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _dbl, _dbl, _vp, _vp, _vp, _vp, _vp]
+_lib.sparge_mask_noalloc.restype = ctypes.c_int
 _lib.sparge_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sla2_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]

@@ -99,6 +99,34 @@ sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shap
                           double topp, int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* The same block mask as sparge_mask, for callers that cannot allocate
+ * device memory: code hosted inside a framework or runtime that owns every
+ * device allocation (a plug-in may not call cudaMalloc behind its host's
+ * allocator), or code that must not risk an allocation failure or pay
+ * allocation latency in the middle of its work. The articles have no
+ * counterpart; this is an interface convenience, not part of the method.
+ *
+ * Arguments and results are those of sparge_mask; the caller still passes
+ * Q, K and every output. The scratch (pooled Q and K, and the probability
+ * rows when `probs` is NULL) is a fixed 16 MiB array inside the library's
+ * device code, so nothing is allocated: not by this call, not by the
+ * library, not through any allocating library routine.
+ *   - Limit: pooled Q + pooled K (+ probability rows when probs is NULL)
+ *     must fit in 16 MiB: 4*B*H*d*(Nqb + Nkb) (+ 4*B*H*Nqb*Nkb) bytes, each
+ *     part rounded up to 256. Larger shapes return SPARGE_ERR_WORKSPACE
+ *     before anything is launched.
+ *   - The first call on a device looks up the array's device address on
+ *     that device (cudaGetSymbolAddress, with the device current) and
+ *     caches it; make that first call before any stream capture.
+ *   - Every call, on any stream, uses the same array, and it keeps the last
+ *     call's contents. Calls whose kernels overlap on the GPU race on it;
+ *     order them (one stream, or events). Nothing in it needs to start at
+ *     zero: each call overwrites what it reads.
+ *   - Every device that loads the library holds the 16 MiB until exit. */
+sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_shape* shape, double topk_frac,
+                                  double topp, int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs,
+                                  void* stream);
+
 /* Block-sparse attention forward (SpargeAttention2 article, section 4).
  *   O[b,h,i] = sum over the keys j of the kept blocks of i's query block of
  *              softmax_j(q_i . k_j / sqrt(d)) v_j, in fp32, stored as bf16.
