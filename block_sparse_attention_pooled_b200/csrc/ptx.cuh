@@ -175,6 +175,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// One lane of a converged warp: true in exactly one lane.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0u;
+}
+
 // Arrives once on the mbarrier when every previously issued tcgen05.mma of
 // this thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -239,20 +250,78 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// 2^x on the FMA pipe, for x <= 127 (x < -126 gives 0): Cody-Waite split
-// x = n + f with n = floor(x), f in [0, 1), then a cubic for 2^f whose
-// coefficients were fitted to 2^f on [0, 1] by relative-error minimax
-// (Lawson's iteration on weighted least squares); max relative error 8.4e-5.
-// The exponent n is added straight into the result's exponent field.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -126.0f);
-  const float n = floorf(xc);
-  const float f = xc - n;
-  float p = fmaf(0.07808296382427216f, f, 0.22612518072128296f);
-  p = fmaf(p, f, 0.695733368396759f);
-  p = fmaf(p, f, 0.9999415278434753f);
-  const float r = __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
-  return x < -126.0f ? 0.0f : r;
+// Waits on an mbarrier unless another role already gave up; gives up itself
+// (and tells the others through *abort) after the global time limit.
+__device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, unsigned int site,
+                                          volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(site);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------- fp32 pairs
+// sm_100 runs add / sub / fma on two fp32 lanes held in one 64-bit register
+// pair, one instruction for both, and max on three operands.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for two lanes on the FMA and integer pipes (x finite, x <= 127):
+// x = j + f with j = rint(x), found by adding 1.5 * 2^23 (the sum's low
+// mantissa bits are then j), and f = x - j in [-0.5, 0.5]; a cubic gives 2^f
+// and j goes straight into the exponent field. The cubic's coefficients were
+// fitted to 2^f on [-0.5, 0.5] by relative-error minimax (Lawson's iteration
+// on weighted least squares): maximum relative error 7.5e-5, far below a
+// bf16 probability's 2^-9. j is clamped to >= -125, so results below 2^-125
+// come out as about 2^-125 (< 3e-38) instead of 0: no bf16 P, no fp32 row
+// sum of values >= 1 can tell the difference.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  const uint64_t magic = f2(12582912.0f, 12582912.0f);
+  const uint64_t t = add2(x, magic);
+  const uint64_t f = sub2(x, sub2(t, magic));
+  uint64_t p = fma2(f2(0.0551715046f, 0.0551715046f), f, f2(0.242610946f, 0.242610946f));
+  p = fma2(p, f, f2(0.693260968f, 0.693260968f));
+  p = fma2(p, f, f2(0.999928057f, 0.999928057f));
+  const float2 tv = f2_split(t), pv = f2_split(p);
+  constexpr int kMinBits = 0x4B400000 - 125;  // bits of 1.5 * 2^23 + (-125)
+  const uint32_t lo = __float_as_uint(pv.x) + ((uint32_t)max(__float_as_int(tv.x), kMinBits) << 23);
+  const uint32_t hi = __float_as_uint(pv.y) + ((uint32_t)max(__float_as_int(tv.y), kMinBits) << 23);
+  return f2(__uint_as_float(lo), __uint_as_float(hi));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -14,6 +14,7 @@
 #include "mask.cuh"
 #include "attn.cuh"
 #include "linear.cuh"
+#include "lin_out.cuh"
 
 namespace {
 
@@ -155,18 +156,15 @@ Sla2Ws sla2_ws(const sparge_shape* s, const Dims& d) {
   return w;
 }
 
-template <int D, bool LIN>
+template <int D, bool MIX>
 sparge_status launch_attn(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
-                          const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, const void* phik,
-                          const float* s_all, const float* z_all, const float* alpha, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo, mp;
+                          const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, const float* alpha,
+                          cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
-      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, D, s->bq) ||
-      !make_map_bhnd(&mp, LIN ? phik : K, dm.BH, s->N, D, kTileK))
+      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, D, s->bq))
     return SPARGE_ERR_CUDA;
   AttnParams p;
-  p.s_all = s_all;
-  p.z_all = z_all;
   p.alpha = alpha;
   p.H = s->H;
   p.kv_idx = kv_idx;
@@ -178,10 +176,36 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
   p.bq = s->bq;
   p.bk = s->bk;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const int smem = AttnSmem<D, LIN>::kBytes;
-  cudaError_t e = ensure_smem(attn_fwd_kernel<D, LIN>, smem, LIN ? 5 : (D == 64 ? 3 : 4));
+  const int smem = AttnSmem<D, MIX>::kBytes;
+  cudaError_t e = ensure_smem(attn_fwd_kernel<D, MIX>, smem, MIX ? 5 : (D == 64 ? 3 : 4));
   if (e != cudaSuccess) return cuda_status(e);
-  attn_fwd_kernel<D, LIN><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st>>>(mq, mk, mv, mo, mp, p);
+  attn_fwd_kernel<D, MIX><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st>>>(mq, mk, mv, mo, p);
+  return cuda_status(cudaGetLastError());
+}
+
+// (1 - alpha_h) O_linear into O, one CTA per query block (d = 128).
+sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape* s, const Dims& dm,
+                                const int32_t* kv_idx, const int32_t* kv_cnt, const void* phik, const float* s_all,
+                                const float* z_all, const float* alpha, void* O, cudaStream_t st) {
+  CUtensorMap mq, mv, mp, mo;
+  if (!make_map_bhnd(&mq, Q, dm.BH, s->N, 128, 128) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
+      !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
+    return SPARGE_ERR_CUDA;
+  LoParams p;
+  p.kv_idx = kv_idx;
+  p.kv_cnt = kv_cnt;
+  p.s_all = s_all;
+  p.z_all = z_all;
+  p.alpha = alpha;
+  p.H = s->H;
+  p.N = s->N;
+  p.nqb = (int)dm.nqb;
+  p.nkb = (int)dm.nkb;
+  p.bq = s->bq;
+  p.bk = s->bk;
+  cudaError_t e = ensure_smem(linear_out_kernel, LoSmem::kBytes, 7);
+  if (e != cudaSuccess) return cuda_status(e);
+  linear_out_kernel<<<(unsigned)(dm.BH * dm.nqb), kLoThreads, LoSmem::kBytes, st>>>(mq, mv, mp, mo, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -312,8 +336,8 @@ sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARGE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (shape->d == 64)
-    return launch_attn<64, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, nullptr, nullptr, nullptr, s);
-  return launch_attn<128, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, nullptr, nullptr, nullptr, s);
+    return launch_attn<64, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s);
+  return launch_attn<128, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s);
 }
 
 sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
@@ -336,7 +360,9 @@ sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const s
   float* partial = reinterpret_cast<float*>(ws + w.partial);
   st = launch_summaries(K, V, shape, dm, phik, partial, s_all, z_all, s);
   if (st != SPARGE_OK) return st;
-  return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, phik, s_all, z_all, alpha, s);
+  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, alpha, O, s);
+  if (st != SPARGE_OK) return st;
+  return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, alpha, s);
 }
 
 sparge_status sparge_device_status(void* stream, int32_t* code) {

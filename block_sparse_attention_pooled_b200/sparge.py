@@ -23,7 +23,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOU
 OP_MASK, OP_ATTN, OP_SLA2 = 0, 1, 2
 
 # Kernel launches per call of each entry point (for launch accounting).
-MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES = 3, 1, 3
+MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES = 3, 1, 4
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",

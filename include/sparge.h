@@ -143,7 +143,12 @@ sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const
  *   O_linear[i] = sum_j (phi(q_i) . phi(k_j)) v_j / sum_j phi(q_i) . phi(k_j),
  *   phi(x) = elu(x) + 1; O_linear = 0 when every block is kept.
  *   alpha       float [H], device.
- * d must be 128. Workspace: sparge_workspace_bytes(SPARGE_OP_SLA2, shape). */
+ * d must be 128. Workspace: sparge_workspace_bytes(SPARGE_OP_SLA2, shape).
+ * Four launches: phi(K) and per-CTA partial sums of phi(K)^T [V | 1]; their
+ * fixed-order reduction to the per-head totals; the linear branch of every
+ * query block, written into O as (1 - alpha[h]) O_linear (bf16); the sparse
+ * branch, which reads that tile back and adds alpha[h] O_sparse. O is
+ * therefore also scratch between the last two launches. */
 sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                             const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, void* O,
                             void* workspace, size_t workspace_bytes, void* stream);

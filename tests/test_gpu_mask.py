@@ -82,3 +82,20 @@ def test_mask_is_deterministic():
     cols = torch.arange(a[0].shape[-1], device=cnt.device)
     valid = cols[None, None, None, :] < cnt[..., None]
     assert torch.equal(a[0][valid], b[0][valid])
+
+
+@pytest.mark.parametrize("topk,topp", [(0.1, 0.0), (0.0, 0.3), (0.05, 0.5), (0.0, 1.0)])
+def test_mask_exact_ties_take_lower_indices(topk, topp):
+    # Every key block holds the same rows, so every pooled score of a row is
+    # the same number on both sides: all probabilities tie exactly and the
+    # kept blocks must be the lowest indices, in the counts the oracle gives.
+    B, H, N, d, bq, bk = 1, 2, 4096, 64, 64, 64
+    Q, K, _ = synth.make_qkv(B, H, N, d, grid=None, s=1.5, seed=77)
+    K = K[:, :, :bk].repeat(1, 1, N // bk, 1).contiguous()
+    g_idx, g_cnt, g_P, _ = _run(Q, K, bq, bk, topk, topp)
+    o_idx, o_cnt, o_P = oracle.mask(Q, K, bq, bk, topk, topp, precision=32)
+    np.testing.assert_array_equal(g_P, o_P)
+    np.testing.assert_array_equal(g_cnt, o_cnt)
+    for r, c in enumerate(g_cnt.reshape(-1)):
+        np.testing.assert_array_equal(g_idx.reshape(-1, g_idx.shape[-1])[r, :c], np.arange(c))
+        np.testing.assert_array_equal(o_idx.reshape(-1, o_idx.shape[-1])[r, :c], np.arange(c))
