@@ -28,7 +28,6 @@
 #include <cuda.h>
 #include <cstdint>
 #include <cuda_bf16.h>
-#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -95,6 +94,124 @@ struct AttnSmem {
   static constexpr int kBytes = (kUsed + 1024 > 80 * 1024 ? kUsed + 1024 : 80 * 1024);
   static constexpr int kTmemCols = 256;
 };
+
+// ---------------------------------------------------------------- softmax tile
+// One thread = one query row (its TMEM lane); a tile = 64 keys.
+
+// The row's 64 scores of S from TMEM (taddr includes the warp's lane offset).
+__device__ __forceinline__ void load_scores(uint32_t taddr, float (&s)[kTileK]) {
+  uint32_t v[4][16];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld16(taddr + 16 * c, v[c]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(v[c][j]);
+}
+
+// Keys at or past N score -inf.
+__device__ __forceinline__ void mask_tail(float (&s)[kTileK], int key0, int N) {
+  if (key0 + kTileK > N) {
+#pragma unroll
+    for (int j = 0; j < kTileK; ++j)
+      if (key0 + j >= N) s[j] = -INFINITY;
+  }
+}
+
+// Three-operand max tree: 36 instructions, depth 4.
+__device__ __forceinline__ float row_max64(const float (&s)[kTileK]) {
+  float m8[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    m8[j] = fmax3(fmax3(s[j], s[8 + j], s[16 + j]), fmax3(s[24 + j], s[32 + j], s[40 + j]), fmaxf(s[48 + j], s[56 + j]));
+  return fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+}
+
+// Multiplies the row's D accumulator columns at taddr by f.
+template <int D>
+__device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
+  uint32_t v[16];
+#pragma unroll 1
+  for (int c = 0; c < D; c += 16) {
+    tmem_ld16(taddr + c, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+    tmem_st16(taddr + c, v);
+  }
+  tmem_st_wait();
+}
+
+// p_j = 2^(s_j * scale_log2 - m) packed as bf16 pairs into pk; returns the
+// sum of the p_j in fp32. Pair instructions throughout but the MUFU; the
+// first 2 * NPOLY values take the polynomial exp2 instead.
+template <int NPOLY>
+__device__ __forceinline__ float exp_pack(const float (&s)[kTileK], float scale_log2, float m,
+                                          uint32_t (&pk)[kTileK / 2]) {
+  const uint64_t scale2 = f2(scale_log2, scale_log2), negm2 = f2(-m, -m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // four pair sums: short dependency chains
+#pragma unroll
+  for (int k = 0; k < kTileK / 2; ++k) {
+    const uint64_t x = fma2(f2(s[2 * k], s[2 * k + 1]), scale2, negm2);
+    uint64_t e;
+    if (k < NPOLY) {
+      e = exp2_poly2(x);
+    } else {
+      const float2 xv = f2_split(x);
+      e = f2(ex2_approx(xv.x), ex2_approx(xv.y));
+    }
+    acc[k & 3] = add2(acc[k & 3], e);
+    const float2 ev = f2_split(e);
+    pk[k] = pack_bf16x2(ev.x, ev.y);
+  }
+  const float2 a = f2_split(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])));
+  return a.x + a.y;
+}
+
+// P (bf16 pairs) into the first 32 columns of its S buffer.
+__device__ __forceinline__ void store_p(uint32_t taddr, const uint32_t (&pk)[kTileK / 2]) {
+  tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+  tmem_st16(taddr + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+  tmem_st_wait();
+}
+
+// Writes 16 values of row r (columns c..c+15) as bf16 into a tile of
+// 128-row, 64-column boxes with the 128-byte swizzle (the TMA layout).
+__device__ __forceinline__ void stage_row16(uint32_t tile, int r, int c, const float (&o)[16]) {
+  uint32_t w[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
+  const int box = c / 64, cc = c % 64;
+  const uint32_t row_addr = tile + box * (kTileQ * 128) + r * 128;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int chunk = (cc / 8 + h) ^ (r & 7);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
+                 "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
+                 : "memory");
+  }
+}
+
+// Reads 16 bf16 values of row r (columns c..c+15) from such a tile.
+__device__ __forceinline__ void read_row16(uint32_t tile, int r, int c, float (&o)[16]) {
+  const int box = c / 64, cc = c % 64;
+  const uint32_t row_addr = tile + box * (kTileQ * 128) + r * 128;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t x[4];
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3])
+                 : "r"(row_addr + (((cc / 8 + h) ^ (r & 7)) * 16))
+                 : "memory");
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&x[k]));
+      o[8 * h + 2 * k] = f.x;
+      o[8 * h + 2 * k + 1] = f.y;
+    }
+  }
+}
 
 // First key of key tile t of a query tile whose kept-block list is `lst`.
 __device__ __forceinline__ int tile_key0(const int32_t* lst, int t, int tiles_per_block, int bk) {
@@ -299,31 +416,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       if (!ok) break;
       tc_fence_after();
       float s[kTileK];
-      {
-        uint32_t v[4][16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld16(tS + lane_off + pb * 64 + 16 * c, v[c]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int j = 0; j < 16; ++j) s[16 * c + j] = __uint_as_float(v[c][j]);
-      }
-      if (key0 + kTileK > p.N) {
-#pragma unroll
-        for (int j = 0; j < kTileK; ++j)
-          if (key0 + j >= p.N) s[j] = -INFINITY;
-      }
-      float mx;  // three-operand max tree: 36 instructions, depth 4
-      {
-        float m8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          m8[j] = fmax3(fmax3(s[j], s[8 + j], s[16 + j]), fmax3(s[24 + j], s[32 + j], s[40 + j]),
-                        fmaxf(s[48 + j], s[56 + j]));
-        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      }
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
+      load_scores(tS + lane_off + pb * 64, s);
+      mask_tail(s, key0, p.N);
+      const float m_new = fmaxf(m_run, row_max64(s) * p.scale_log2);
       if (t == 0) {
         m_run = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m_run + kRescaleThreshold)) {
@@ -334,54 +429,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (!ok) break;
         tc_fence_after();
         const float f = ex2_approx(m_run - m_new);
-        uint32_t v[16];
-#pragma unroll 1
-        for (int c = 0; c < D; c += 16) {
-          tmem_ld16(tO + lane_off + c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-          tmem_st16(tO + lane_off + c, v);
-        }
-        tmem_st_wait();
+        rescale_row<D>(tO + lane_off, f);
         l_run *= f;
         m_run = m_new;
       }
-      // x = s * scale_log2 - m_run, p = 2^x, row sum and bf16 packing, on
-      // fp32 pairs: one instruction per two scores for each step but the MUFU.
-      const uint64_t scale2 = f2(p.scale_log2, p.scale_log2), negm2 = f2(-m_run, -m_run);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // four pair sums: short dependency chains
       uint32_t pk[kTileK / 2];
-      const bool full_tile = key0 + kTileK <= p.N;  // the same for every row of the tile
-      auto exp_pairs = [&](auto poly_pairs) {
-        constexpr int kPoly = decltype(poly_pairs)::value;
-#pragma unroll
-        for (int k = 0; k < kTileK / 2; ++k) {
-          const uint64_t x = fma2(f2(s[2 * k], s[2 * k + 1]), scale2, negm2);
-          uint64_t e;
-          if (k < kPoly) {
-            e = exp2_poly2(x);
-          } else {
-            const float2 xv = f2_split(x);
-            e = f2(ex2_approx(xv.x), ex2_approx(xv.y));
-          }
-          acc[k & 3] = add2(acc[k & 3], e);
-          const float2 ev = f2_split(e);
-          pk[k] = pack_bf16x2(ev.x, ev.y);
-        }
-      };
-      if (full_tile)
-        exp_pairs(std::integral_constant<int, kPolyPairs>{});
+      if (key0 + kTileK <= p.N)  // the same for every row of the tile
+        l_run += exp_pack<kPolyPairs>(s, p.scale_log2, m_run, pk);
       else
-        exp_pairs(std::integral_constant<int, 0>{});
-      {
-        const float2 a = f2_split(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])));
-        l_run += a.x + a.y;
-      }
-      // P (bf16) overwrites the first 32 columns of this S buffer.
-      tmem_st16(tS + lane_off + pb * 64, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(tS + lane_off + pb * 64 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-      tmem_st_wait();
+        l_run += exp_pack<0>(s, p.scale_log2, m_run, pk);
+      store_p(tS + lane_off + pb * 64, pk);
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + pb));
     }
@@ -390,22 +447,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tc_fence_after();
     }
     const float inv_l = (T > 0 && l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-    // Writes 16 output values of row r (columns c..c+15) as bf16 into the
-    // Q buffer, laid out the way the 128-byte-swizzled O tensor map expects.
-    auto stage_out16 = [&](int c, const float (&o)[16]) {
-      uint32_t w[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
-      const int box = c / 64, cc = c % 64;
-      const uint32_t row_addr = sQ + box * (kTileQ * 128) + r * 128;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int chunk = (cc / 8 + h) ^ (r & 7);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
-                     "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
-                     : "memory");
-      }
-    };
     // MIX: the Q buffer holds (1 - alpha_h) O_linear for this tile.
     if (MIX && ok) ok = __all_sync(0xffffffffu, role_wait(bar(kBarOl), 0, kErrAttnOl, abort_flag));
     const float w_s = (MIX ? __ldg(p.alpha + (bh % p.H)) : 1.0f) * inv_l;
@@ -424,24 +465,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v[j]) * w_s;
       if (MIX && ok) {
-        const int box = c / 64, cc = c % 64;
-        const uint32_t row_addr = sQ + box * (kTileQ * 128) + r * 128;
+        float ol[16];
+        read_row16(sQ, r, c, ol);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t x[4];
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3])
-                       : "r"(row_addr + (((cc / 8 + h) ^ (r & 7)) * 16))
-                       : "memory");
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&x[k]));
-            o[8 * h + 2 * k] += f.x;
-            o[8 * h + 2 * k + 1] += f.y;
-          }
-        }
+        for (int j = 0; j < 16; ++j) o[j] += ol[j];
       }
-      stage_out16(c, o);
+      stage_row16(sQ, r, c, o);
     }
     if (p.lse != nullptr && r < p.bq && q0 + r < p.N) {
       const float lse = (T > 0 && l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;

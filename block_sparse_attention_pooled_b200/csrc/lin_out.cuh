@@ -3,7 +3,8 @@
 // attention; section 2: O = alpha * O_sparse + (1 - alpha) * O_linear).
 //
 // Per query tile (bq rows of one (batch, head), computed as a 128-row tile):
-//   S_kept      = sum over the tile's kept key tiles t of phi(K_t)^T [V_t | 1]
+//   S_kept      = sum over the tile's kept key tiles t of phi(K_t)^T V_t
+//   z_kept      = sum over the same tiles of z_tile[t]
 //   [S_c | z_c] = [S_all - S_kept | z_all - z_kept]      (the blocks NOT kept)
 //   O_linear[i] = phi(q_i)^T S_c / phi(q_i) . z_c
 // and the tile of O is written as (1 - alpha_h) O_linear in bf16. The
@@ -12,30 +13,34 @@
 // O_sparse never before the mix.
 //
 // phi(x) = elu(x) + 1. phi(K) comes precomputed in bf16 from
-// linear_summary_kernel, the same values S_all and z_all were built from, so
-// the complement S_all - S_kept is exactly the sum over the blocks not kept
-// up to fp32 rounding.
+// linear_summary_kernel, the same values S_all, z_all and z_tile were built
+// from, so the complements are the sums over the blocks not kept up to fp32
+// rounding.
 //
 // 192 threads:
-//   warp 0      TMA producer: phi(K) and V tiles of the kept blocks into a
-//               two-slot ring; then the Q tile, once the ring is idle;
+//   warp 0      TMA producer (whole warp, one elected lane issues): phi(K)
+//               and V tiles of the kept blocks into a three-slot ring, then
+//               the Q tile once the ring is idle;
 //   warp 1      MMA issuer (whole warp, one elected lane issues) and TMEM
-//               owner: S_kept[feature, 0..143] += phi(K_t)^T [V_t | 1]
-//               (M 128, N 144, K 64 per tile; both operands MN-major; the
-//               ones block after each V slot yields z_kept in column 128);
-//               then phi(Q) [S_c | z_c] into the same TMEM columns;
-//   warps 2..5  epilogue: TMEM lane r is feature r for [S_c | z_c] (bf16,
-//               staged in shared memory as the MN-major B operand) and query
-//               row r for the output.
-// Shared memory: ring slot s = [phi(K) 16 KB | V 16 KB | ones 8 KB]; after the
-// last MMA of the ring the same bytes hold [S_c | z_c] (three 128-row boxes,
-// 48 KB) and the Q tile (32 KB), which becomes phi(Q) and then the output.
+//               owner: S_kept[feature, 0..127] += phi(K_t)^T V_t (M 128,
+//               N 128, K 64 per tile, both operands MN-major), then
+//               phi(Q) S_c into the same TMEM columns;
+//   warps 2..5  while the MMAs run: z_kept (thread r adds z_tile[t][r] over
+//               the kept tiles); then the epilogue: TMEM lane r is feature r
+//               for S_c (bf16, staged in shared memory as the MN-major B
+//               operand) and query row r for the output, whose denominator
+//               phi(q_r) . z_c they take in fp32.
+// Shared memory: ring slot s = [phi(K) 16 KB | V 16 KB]; after the last MMA
+// of the ring the same bytes hold S_c (two 128-row boxes, 32 KB) and the Q
+// tile (32 KB), which becomes phi(Q) and then the output. Three slots keep two
+// CTAs per SM, six tiles in flight per SM.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "attn.cuh"
 
 namespace sparge {
 
@@ -45,21 +50,24 @@ enum : unsigned int {
   kErrLoFull = 0x300, kErrLoEmpty, kErrLoKept, kErrLoQ, kErrLoStage, kErrLoOut, kErrLoDrain
 };
 
+#ifndef SPARGE_LO_SLOTS
+#define SPARGE_LO_SLOTS 3
+#endif
+
 struct LoSmem {
-  static constexpr int NS = 2;
-  static constexpr int kPhiK = 64 * 128 * 2;        // phi(K) tile: two 64-column boxes of 64 keys
-  static constexpr int kV = 64 * 128 * 2;           // V tile, same layout
-  static constexpr int kOnes = 8192;                // B columns 128..191 of the tile (16 used)
-  static constexpr int kSlot = kPhiK + kV + kOnes;  // 40 KB
-  static constexpr int kOffStage = 0;               // epilogue: [S_c | z_c], three boxes of 128 rows
-  static constexpr int kOffQ = 3 * 128 * 128;       // epilogue: Q tile -> phi(Q) -> output
-  static constexpr int kOffBar = NS * kSlot;
+  static constexpr int NS = SPARGE_LO_SLOTS;
+  static constexpr int kTile = 64 * 128 * 2;         // phi(K) or V tile: two 64-column boxes of 64 keys
+  static constexpr int kSlot = 2 * kTile;            // 32 KB
+  static constexpr int kOffStage = 0;                // epilogue: S_c, two boxes of 128 rows
+  static constexpr int kOffQ = 2 * 128 * 128;        // epilogue: Q tile -> phi(Q) -> output
+  static constexpr int kOffX = NS * kSlot;           // zc[128] (fp32)
+  static constexpr int kOffBar = kOffX + 128 * 4;
   static constexpr int kBarFull = 0, kBarEmpty = NS, kBarKept = 2 * NS, kBarQ = 2 * NS + 1,
                        kBarStage = 2 * NS + 2, kBarOut = 2 * NS + 3, kBarDrain = 2 * NS + 4;
   static constexpr int kNumBars = 2 * NS + 5;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;  // + alignment slack: two CTAs per SM
-  static_assert(kOffQ + 2 * 128 * 128 <= kOffBar, "epilogue tiles must fit in the ring");
+  static_assert(kOffQ + 2 * 128 * 128 <= kOffX, "epilogue tiles must fit in the ring");
 };
 
 struct LoParams {
@@ -67,9 +75,11 @@ struct LoParams {
   const int32_t* kv_cnt;  // [BH, nqb]
   const float* s_all;     // [BH, 128, 128] fp32, row = feature
   const float* z_all;     // [BH, 128] fp32
+  const float* z_tile;    // [BH, ntiles, 128] fp32
   const float* alpha;     // [H]
   int H;
   int N;
+  int ntiles;             // ceil(N / 64)
   int nqb;
   int nkb;
   int bq;
@@ -77,6 +87,7 @@ struct LoParams {
 };
 
 __device__ __forceinline__ float phi_lin(float x) { return x > 0.0f ? x + 1.0f : __expf(x); }
+
 
 __global__ void __launch_bounds__(kLoThreads, 2)
     linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmV,
@@ -89,6 +100,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw);
   const uint32_t sStage = sbase + L::kOffStage, sQ = sbase + L::kOffQ;
+  float* zc = reinterpret_cast<float*>(sgen + L::kOffX);  // [128] z_c
   const uint32_t bar0 = sbase + L::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
@@ -117,12 +129,6 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int s = 0; s < NS; ++s) {
-    uint4* ones = reinterpret_cast<uint4*>(sgen + s * L::kSlot + L::kPhiK + L::kV);
-    for (int u = threadIdx.x; u < L::kOnes / 16; u += kLoThreads)
-      ones[u] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-  }
-  fence_async_smem();
   if (warp == 1) {
     tmem_alloc(sbase + L::kOffTmem, 256);
     tmem_relinquish();
@@ -131,38 +137,57 @@ __global__ void __launch_bounds__(kLoThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
+    return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tmPhiK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmQ);
-      int issued = 0;
-      bool ok = true;
-      for (int t = 0; t < T; ++t) {
-        const int slot = t % NS;
-        const int key0 = __ldg(lst + t / tiles_per_block) * p.bk + (t % tiles_per_block) * 64;
-        if (t >= NS && !role_wait(bar(L::kBarEmpty + slot), (t / NS - 1) & 1, kErrLoEmpty, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sp = sbase + slot * L::kSlot, sv = sp + L::kPhiK;
-        mbar_arrive_expect_tx(bar(L::kBarFull + slot), L::kPhiK + L::kV);
+    }
+    // Kept-block indices, 32 at a time, one per lane, a chunk ahead of use.
+    int idx_cur = lane < cnt ? __ldg(lst + lane) : 0;
+    int idx_nxt = 32 + lane < cnt ? __ldg(lst + 32 + lane) : 0;
+    int issued = 0;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int slot = t % NS;
+      const int e = t / tiles_per_block, sub = t % tiles_per_block;
+      if (e > 0 && (e & 31) == 0 && sub == 0) {
+        idx_cur = idx_nxt;
+        idx_nxt = e + 32 + lane < cnt ? __ldg(lst + e + 32 + lane) : 0;
+      }
+      const int key0 = __shfl_sync(0xffffffffu, idx_cur, e & 31) * p.bk + sub * 64;
+      if (t >= NS && !warp_wait(L::kBarEmpty + slot, (t / NS - 1) & 1, kErrLoEmpty)) {
+        ok = false;
+        break;
+      }
+      if (leader) {
+        const uint32_t sp = sbase + slot * L::kSlot, sv = sp + L::kTile;
+        mbar_arrive_expect_tx(bar(L::kBarFull + slot), L::kSlot);
         for (int b = 0; b < 2; ++b) {
           tma_load_3d(sp + b * 8192, &tmPhiK, bar(L::kBarFull + slot), b * 64, key0, bh);
           tma_load_3d(sv + b * 8192, &tmV, bar(L::kBarFull + slot), b * 64, key0, bh);
         }
-        ++issued;
       }
-      // Q goes where the ring was, once every MMA that reads the ring is done.
-      bool q_issued = false;
-      if (ok && role_wait(bar(L::kBarKept), 0, kErrLoKept, abort_flag)) {
+      __syncwarp();
+      ++issued;
+    }
+    // Q goes where the ring was, once every MMA that reads the ring is done.
+    bool q_issued = false;
+    if (ok && warp_wait(L::kBarKept, 0, kErrLoKept)) {
+      if (leader) {
         mbar_arrive_expect_tx(bar(L::kBarQ), 2 * 128 * 128);
         for (int b = 0; b < 2; ++b) tma_load_3d(sQ + b * (128 * 128), &tmQ, bar(L::kBarQ), b * 64, q0, bh);
-        q_issued = true;
       }
-      // Never leave with copies in flight.
+      q_issued = true;
+    }
+    // Never leave with copies in flight.
+    if (leader) {
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
         mbar_wait(bar(L::kBarFull + t % NS), (t / NS) & 1, kErrLoFull);
       if (q_issued) mbar_wait(bar(L::kBarQ), 0, kErrLoQ);
@@ -170,14 +195,11 @@ __global__ void __launch_bounds__(kLoThreads, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const bool leader = elect_one();
-    constexpr uint32_t idKept = idesc_bf16_f32(128, 144, true, true);
-    constexpr uint32_t idOut = idesc_bf16_f32(128, 144, false, true);
-    const uint64_t dRing = sdesc_sw128(sbase, 64 * 128, 1024);        // MN-major, 64-row boxes
-    const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);                    // K-major, 128-row boxes
-    const uint64_t dStage = sdesc_sw128(sStage, 128 * 128, 1024);     // MN-major, 128-row boxes
-    auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
-      return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
-    };
+    constexpr uint32_t idKept = idesc_bf16_f32(128, 128, true, true);
+    constexpr uint32_t idOut = idesc_bf16_f32(128, 128, false, true);
+    const uint64_t dRing = sdesc_sw128(sbase, 64 * 128, 1024);     // MN-major, 64-row boxes
+    const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);                 // K-major, 128-row boxes
+    const uint64_t dStage = sdesc_sw128(sStage, 128 * 128, 1024);  // MN-major, 128-row boxes
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       const int slot = t % NS;
@@ -188,7 +210,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       tc_fence_after();
       if (leader) {
         const uint64_t dP = dRing + (uint64_t)((slot * L::kSlot) >> 4);
-        const uint64_t dV = dP + (uint64_t)(L::kPhiK >> 4);
+        const uint64_t dV = dP + (uint64_t)(L::kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 16 keys = 2048 bytes of each operand
           mma_ss(tmem, dP + kk * 128, dV + kk * 128, idKept, (t > 0 || kk > 0) ? 1u : 0u);
@@ -216,18 +238,33 @@ __global__ void __launch_bounds__(kLoThreads, 2)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // TMEM lane quadrant of this warp
-    const int r = q * 32 + lane;       // feature (phase 1) / query row (phase 2)
+    const int r = q * 32 + lane;       // feature (S_c, z_c) / query row (output)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
-      return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
-    };
+    // z_kept[r] over the kept tiles, four loads in flight at a time.
+    float zk = 0.0f;
+    {
+      const float* zt = p.z_tile + (int64_t)bh * p.ntiles * 128 + r;
+      int t = 0;
+      for (; t + 4 <= T; t += 4) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int tt = t + u;
+          const int tile64 = (__ldg(lst + tt / tiles_per_block) * p.bk + (tt % tiles_per_block) * 64) / 64;
+          v[u] = __ldg(zt + (int64_t)tile64 * 128);
+        }
+        zk += (v[0] + v[1]) + (v[2] + v[3]);
+      }
+      for (; t < T; ++t)
+        zk += __ldg(zt + (int64_t)((__ldg(lst + t / tiles_per_block) * p.bk + (t % tiles_per_block) * 64) / 64) * 128);
+    }
     bool ok = warp_wait(L::kBarKept, 0, kErrLoKept);
     tc_fence_after();
-    // 1. [S_c | z_c] row r as bf16, MN-major with the 128-byte swizzle
-    //    (three 64-column boxes; column 128 = z_c, the rest of box 2 zero).
+    // 1. S_c row a = r: S_all - S_kept as bf16, MN-major for the last MMA
+    //    (two 64-column boxes of 128 rows, 128-byte swizzle).
     const float* srow = p.s_all + ((int64_t)bh * 128 + r) * 128;
 #pragma unroll 1
-    for (int c = 0; c < 144; c += 16) {
+    for (int c = 0; c < 128; c += 16) {
       uint32_t v[16];
       if (ok && T > 0) {
         tmem_ld16(tmem + lane_off + c, v);
@@ -237,35 +274,12 @@ __global__ void __launch_bounds__(kLoThreads, 2)
         for (int j = 0; j < 16; ++j) v[j] = 0u;
       }
       float sc[16];
-      if (c < 128) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) sc[j] = __ldg(srow + c + j) - __uint_as_float(v[j]);
-      } else {
-        sc[0] = __ldg(p.z_all + (int64_t)bh * 128 + r) - __uint_as_float(v[0]);
-#pragma unroll
-        for (int j = 1; j < 16; ++j) sc[j] = 0.0f;
-      }
-      uint32_t w[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = pack_bf16x2(sc[2 * j], sc[2 * j + 1]);
-      const int box = c / 64, cc = c % 64;
-      const uint32_t row_addr = sStage + box * (128 * 128) + r * 128;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int chunk = (cc / 8 + h) ^ (r & 7);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
-                     "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
-                     : "memory");
-      }
+      for (int j = 0; j < 16; ++j) sc[j] = __ldg(srow + c + j) - __uint_as_float(v[j]);
+      stage_row16(sStage, r, c, sc);
     }
-    {  // columns 144..191 of box 2: not read by the MMA (N = 144), kept defined
-      const uint32_t row_addr = sStage + 2 * (128 * 128) + r * 128;
-#pragma unroll
-      for (int ch = 2; ch < 8; ++ch)
-        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(row_addr + ((ch ^ (r & 7)) * 16)), "r"(0u)
-                     : "memory");
-    }
-    // 2. phi(Q) in place over query row r (elementwise: the swizzle does not matter).
+    // 2. z_c, then phi(Q) in place over query row r (elementwise: the swizzle does not matter).
+    zc[r] = __ldg(p.z_all + (int64_t)bh * 128 + r) - zk;
     if (ok) ok = warp_wait(L::kBarQ, 0, kErrLoQ);
     if (ok) {
 #pragma unroll
@@ -287,19 +301,22 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     fence_async_smem();
     tc_fence_before();
     mbar_arrive(bar(L::kBarStage));
-    // 3. O tile = (1 - alpha_h) * numerator / denominator, bf16, TMA store.
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // z_c complete
+    // 3. Denominator phi(q_r) . z_c in fp32; every block kept: the
+    //    complement is empty and the linear branch is 0.
+    float den = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 16) {
+      float qv[16];
+      read_row16(sQ, r, c, qv);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) den = fmaf(qv[j], zc[c + j], den);
+    }
+    const float a_h = __ldg(p.alpha + (bh % p.H));
+    const float wl = (cnt < p.nkb && den > 0.0f) ? (1.0f - a_h) / den : 0.0f;
     if (ok) ok = warp_wait(L::kBarOut, 0, kErrLoOut);
     tc_fence_after();
-    const float a_h = __ldg(p.alpha + (bh % p.H));
-    float wl = 0.0f;
-    if (ok) {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_off + 128, v);
-      tmem_ld_wait();
-      const float den = __uint_as_float(v[0]);
-      // Every block kept: the complement is empty and the linear branch is 0.
-      wl = (cnt < p.nkb && den > 0.0f) ? (1.0f - a_h) / den : 0.0f;
-    }
+    // 4. O tile = (1 - alpha_h) numerator / denominator, bf16, TMA store.
 #pragma unroll 1
     for (int c = 0; c < 128; c += 16) {
       uint32_t v[16];
@@ -310,19 +327,10 @@ __global__ void __launch_bounds__(kLoThreads, 2)
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0u;
       }
-      uint32_t w[8];
+      float o[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        w[j] = pack_bf16x2(wl * __uint_as_float(v[2 * j]), wl * __uint_as_float(v[2 * j + 1]));
-      const int box = c / 64, cc = c % 64;
-      const uint32_t row_addr = sQ + box * (128 * 128) + r * 128;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int chunk = (cc / 8 + h) ^ (r & 7);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + chunk * 16), "r"(w[4 * h]),
-                     "r"(w[4 * h + 1]), "r"(w[4 * h + 2]), "r"(w[4 * h + 3])
-                     : "memory");
-      }
+      for (int j = 0; j < 16; ++j) o[j] = wl * __uint_as_float(v[j]);
+      stage_row16(sQ, r, c, o);
     }
     fence_async_smem();
     asm volatile("bar.sync 1, 128;" ::: "memory");

@@ -6,6 +6,8 @@
 //   phiK  = phi(K)                         bf16 [N, d]   (kept for the attention kernel)
 //   S_all = sum_j phi(k_j) v_j^T           fp32 [d, d]   (row = feature, column = value dim)
 //   z_all = sum_j phi(k_j)                 fp32 [d]
+//   z_tile[t] = sum of phi(k_j) over the 64 keys of tile t, from the bf16
+//               phi(K) values (fp32 [ceil(N / 64), d])
 // The attention kernel subtracts the kept blocks' share of S_all and z_all to
 // get the complement's summaries.
 //
@@ -45,6 +47,7 @@ constexpr int kLinPartial = 128 * 129;  // per CTA: [feature][128 value columns 
 
 struct LinParams {
   float* partial;  // [BH, ctas_per_head, 128, 129]
+  float* z_tile;   // [BH, ntiles, 128]
   int N;
   int ntiles;         // ceil(N / 64)
   int ctas_per_head;
@@ -153,7 +156,22 @@ __global__ void __launch_bounds__(kLinThreads)
         mma_ss(tmem, a, b, idesc, (i > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(bar_mma(slot));
-      if (i + 2 < n) {
+    }
+    {
+      // z_tile: thread = feature; column sum over the tile's 64 rows of the
+      // swizzled phi(K) tile (a warp reads 64 contiguous bytes per row).
+      const int a = tid, col = a & 63;
+      const uint8_t* tb = sgen + slot * L::kSlot + (a >> 6) * 8192;
+      float zs = 0.0f;
+#pragma unroll 8
+      for (int row = 0; row < 64; ++row)
+        zs += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+            tb + row * 128 + ((((col >> 3) ^ (row & 7)) << 4) | ((col & 7) << 1))));
+      p.z_tile[((int64_t)bh * p.ntiles + t0 + i) * 128 + a] = zs;
+    }
+    if (i + 2 < n) {
+      __syncthreads();  // every thread has finished reading the slot
+      if (tid == 0) {
         // The slot is reused once its MMAs and its phi(K) store have read it.
         stalled = !mbar_wait(bar_mma(slot), (i >> 1) & 1, kErrLinMma);
         tma_store_wait_read0();

@@ -102,7 +102,7 @@ bool make_map_bhnd(CUtensorMap* m, const void* base, int64_t BH, int N, int d, i
 // Raises a kernel's dynamic shared memory limit once per device.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int bytes, int slot) {
-  static int done[64][8];
+  static int done[64][16];  // [device][slot]: one slot per kernel
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -141,7 +141,7 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
 }
 
 struct Sla2Ws {
-  size_t phik, s_all, z_all, partial, total;
+  size_t phik, s_all, z_all, z_tile, partial, total;
 };
 
 inline int lin_ctas_per_head(int N) { return (int)ceil_div(ceil_div(N, 64), kLinTilesPerCta); }
@@ -151,7 +151,8 @@ Sla2Ws sla2_ws(const sparge_shape* s, const Dims& d) {
   w.phik = 0;
   w.s_all = w.phik + align256((size_t)d.BH * s->N * s->d * 2);
   w.z_all = w.s_all + align256((size_t)d.BH * s->d * s->d * 4);
-  w.partial = w.z_all + align256((size_t)d.BH * s->d * 4);
+  w.z_tile = w.z_all + align256((size_t)d.BH * s->d * 4);
+  w.partial = w.z_tile + align256((size_t)d.BH * ceil_div(s->N, 64) * s->d * 4);
   w.total = w.partial + align256((size_t)d.BH * lin_ctas_per_head(s->N) * kLinPartial * 4);
   return w;
 }
@@ -186,7 +187,8 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
 // (1 - alpha_h) O_linear into O, one CTA per query block (d = 128).
 sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape* s, const Dims& dm,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, const void* phik, const float* s_all,
-                                const float* z_all, const float* alpha, void* O, cudaStream_t st) {
+                                const float* z_all, const float* z_tile, const float* alpha, void* O,
+                                cudaStream_t st) {
   CUtensorMap mq, mv, mp, mo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, 128, 128) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
@@ -196,9 +198,11 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   p.kv_cnt = kv_cnt;
   p.s_all = s_all;
   p.z_all = z_all;
+  p.z_tile = z_tile;
   p.alpha = alpha;
   p.H = s->H;
   p.N = s->N;
+  p.ntiles = (int)ceil_div(s->N, 64);
   p.nqb = (int)dm.nqb;
   p.nkb = (int)dm.nkb;
   p.bq = s->bq;
@@ -210,13 +214,14 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
 }
 
 sparge_status launch_summaries(const void* K, const void* V, const sparge_shape* s, const Dims& dm, void* phik,
-                               float* partial, float* s_all, float* z_all, cudaStream_t st) {
+                               float* partial, float* s_all, float* z_all, float* z_tile, cudaStream_t st) {
   CUtensorMap mk, mv, mp;
   if (!make_map_bhnd(&mk, K, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64))
     return SPARGE_ERR_CUDA;
   LinParams p;
   p.partial = partial;
+  p.z_tile = z_tile;
   p.N = s->N;
   p.ntiles = (int)ceil_div(s->N, 64);
   p.ctas_per_head = lin_ctas_per_head(s->N);
@@ -357,10 +362,11 @@ sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const s
   void* phik = ws + w.phik;
   float* s_all = reinterpret_cast<float*>(ws + w.s_all);
   float* z_all = reinterpret_cast<float*>(ws + w.z_all);
+  float* z_tile = reinterpret_cast<float*>(ws + w.z_tile);
   float* partial = reinterpret_cast<float*>(ws + w.partial);
-  st = launch_summaries(K, V, shape, dm, phik, partial, s_all, z_all, s);
+  st = launch_summaries(K, V, shape, dm, phik, partial, s_all, z_all, z_tile, s);
   if (st != SPARGE_OK) return st;
-  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, alpha, O, s);
+  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, z_tile, alpha, O, s);
   if (st != SPARGE_OK) return st;
   return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, alpha, s);
 }
