@@ -22,14 +22,15 @@
 //               and V tiles of the kept blocks into a three-slot ring, then
 //               the Q tile once the ring is idle;
 //   warp 1      MMA issuer (whole warp, one elected lane issues) and TMEM
-//               owner: S_kept[feature, 0..127] += phi(K_t)^T V_t (M 128,
-//               N 128, K 64 per tile, both operands MN-major), then
-//               phi(Q) S_c into the same TMEM columns;
-//   warps 2..5  while the MMAs run: z_kept (thread r adds z_tile[t][r] over
-//               the kept tiles); then the epilogue: TMEM lane r is feature r
-//               for S_c (bf16, staged in shared memory as the MN-major B
-//               operand) and query row r for the output, whose denominator
-//               phi(q_r) . z_c they take in fp32.
+//               owner: D[feature, 0..127] += phi(K_t)^T V_t (M 128, N 128,
+//               K 64 per tile, both operands MN-major) on top of D = -S_all,
+//               which leaves D = -S_c; then phi(Q) S_c into the same columns;
+//   warps 2..5  first D = -S_all (thread r writes feature row r), then, while
+//               the MMAs run, z_kept (thread r adds z_tile[t][r] over the kept
+//               tiles); then the epilogue: TMEM lane r is feature r for S_c
+//               (bf16, staged in shared memory as the MN-major B operand) and
+//               query row r for the output, whose denominator phi(q_r) . z_c
+//               they take in fp32.
 // Shared memory: ring slot s = [phi(K) 16 KB | V 16 KB]; after the last MMA
 // of the ring the same bytes hold S_c (two 128-row boxes, 32 KB) and the Q
 // tile (32 KB), which becomes phi(Q) and then the output. Three slots keep two
@@ -47,7 +48,7 @@ namespace sparge {
 constexpr int kLoThreads = 192;
 
 enum : unsigned int {
-  kErrLoFull = 0x300, kErrLoEmpty, kErrLoKept, kErrLoQ, kErrLoStage, kErrLoOut, kErrLoDrain
+  kErrLoFull = 0x300, kErrLoEmpty, kErrLoKept, kErrLoQ, kErrLoStage, kErrLoOut, kErrLoDrain, kErrLoInit
 };
 
 #ifndef SPARGE_LO_SLOTS
@@ -63,8 +64,8 @@ struct LoSmem {
   static constexpr int kOffX = NS * kSlot;           // zc[128] (fp32)
   static constexpr int kOffBar = kOffX + 128 * 4;
   static constexpr int kBarFull = 0, kBarEmpty = NS, kBarKept = 2 * NS, kBarQ = 2 * NS + 1,
-                       kBarStage = 2 * NS + 2, kBarOut = 2 * NS + 3, kBarDrain = 2 * NS + 4;
-  static constexpr int kNumBars = 2 * NS + 5;
+                       kBarStage = 2 * NS + 2, kBarOut = 2 * NS + 3, kBarDrain = 2 * NS + 4, kBarInit = 2 * NS + 5;
+  static constexpr int kNumBars = 2 * NS + 6;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;  // + alignment slack: two CTAs per SM
   static_assert(kOffQ + 2 * 128 * 128 <= kOffX, "epilogue tiles must fit in the ring");
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     mbar_init(bar(L::kBarStage), 128);
     mbar_init(bar(L::kBarOut), 1);
     mbar_init(bar(L::kBarDrain), 1);
+    mbar_init(bar(L::kBarInit), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -200,8 +202,8 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     const uint64_t dRing = sdesc_sw128(sbase, 64 * 128, 1024);     // MN-major, 64-row boxes
     const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);                 // K-major, 128-row boxes
     const uint64_t dStage = sdesc_sw128(sStage, 128 * 128, 1024);  // MN-major, 128-row boxes
-    bool ok = true;
-    for (int t = 0; t < T; ++t) {
+    bool ok = warp_wait(L::kBarInit, 0, kErrLoInit);  // D = -S_all
+    for (int t = 0; ok && t < T; ++t) {
       const int slot = t % NS;
       if (!warp_wait(L::kBarFull + slot, (t / NS) & 1, kErrLoFull)) {
         ok = false;
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
         const uint64_t dV = dP + (uint64_t)(L::kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 16 keys = 2048 bytes of each operand
-          mma_ss(tmem, dP + kk * 128, dV + kk * 128, idKept, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tmem, dP + kk * 128, dV + kk * 128, idKept, 1u);
         mma_commit(bar(L::kBarEmpty + slot));
       }
       __syncwarp();
@@ -240,6 +242,29 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     const int q = warp & 3;            // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;       // feature (S_c, z_c) / query row (output)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    // D = -S_all, row r (feature r): all 32 loads in flight at once, so
+    // the MMAs wait for one round trip only.
+    {
+      const float4* srow = reinterpret_cast<const float4*>(p.s_all + ((int64_t)bh * 128 + r) * 128);
+      float4 v4[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) v4[k] = __ldg(srow + k);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[4 * j] = __float_as_uint(-v4[4 * k + j].x);
+          v[4 * j + 1] = __float_as_uint(-v4[4 * k + j].y);
+          v[4 * j + 2] = __float_as_uint(-v4[4 * k + j].z);
+          v[4 * j + 3] = __float_as_uint(-v4[4 * k + j].w);
+        }
+        tmem_st16(tmem + lane_off + 16 * k, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarInit));
+    }
     // z_kept[r] over the kept tiles, four loads in flight at a time.
     float zk = 0.0f;
     {
@@ -260,13 +285,12 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     }
     bool ok = warp_wait(L::kBarKept, 0, kErrLoKept);
     tc_fence_after();
-    // 1. S_c row a = r: S_all - S_kept as bf16, MN-major for the last MMA
-    //    (two 64-column boxes of 128 rows, 128-byte swizzle).
-    const float* srow = p.s_all + ((int64_t)bh * 128 + r) * 128;
+    // 1. S_c row a = r (= -D) as bf16, MN-major for the last MMA (two
+    //    64-column boxes of 128 rows, 128-byte swizzle).
 #pragma unroll 1
     for (int c = 0; c < 128; c += 16) {
       uint32_t v[16];
-      if (ok && T > 0) {
+      if (ok) {
         tmem_ld16(tmem + lane_off + c, v);
         tmem_ld_wait();
       } else {
@@ -275,27 +299,26 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       }
       float sc[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) sc[j] = __ldg(srow + c + j) - __uint_as_float(v[j]);
+      for (int j = 0; j < 16; ++j) sc[j] = -__uint_as_float(v[j]);
       stage_row16(sStage, r, c, sc);
     }
-    // 2. z_c, then phi(Q) in place over query row r (elementwise: the swizzle does not matter).
+    // 2. z_c, then phi(Q) in place. phi is elementwise, so the tile is
+    //    walked as a flat array of 16-byte units, consecutive threads on
+    //    consecutive units (no bank conflicts).
     zc[r] = __ldg(p.z_all + (int64_t)bh * 128 + r) - zk;
     if (ok) ok = warp_wait(L::kBarQ, 0, kErrLoQ);
     if (ok) {
+      uint4* qt = reinterpret_cast<uint4*>(sgen + L::kOffQ);
+#pragma unroll 4
+      for (int k = 0; k < (2 * 128 * 128) / 16 / 128; ++k) {
+        uint4 x = qt[r + 128 * k];
+        __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&x);
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        uint4* row = reinterpret_cast<uint4*>(sgen + L::kOffQ + b * (128 * 128) + r * 128);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 x = row[ch];
-          __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&x);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(hx[j]);
-            hx[j] = __floats2bfloat162_rn(phi_lin(f.x), phi_lin(f.y));
-          }
-          row[ch] = x;
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(hx[j]);
+          hx[j] = __floats2bfloat162_rn(phi_lin(f.x), phi_lin(f.y));
         }
+        qt[r + 128 * k] = x;
       }
     }
     fence_async_smem();
