@@ -79,14 +79,15 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ----------------------------------------------------------------------------
-// Scaled scores z[I, J] = (q̄_I . k̄_J) * (float)(1/sqrt(d)). One CTA = 16
-// query-block rows x 64 key blocks of one (b,h); each thread owns 2 rows x 4
-// key blocks and runs their fused multiply-add chains over channels in order.
+// Scaled scores z[I, J] = (q̄_I . k̄_J) * (float)(1/sqrt(d)). One CTA = 32
+// query-block rows x 64 key blocks of one (b,h); each thread owns 4 rows x 4
+// key blocks (8 shared-memory vector loads per 64 fused multiply-adds) and
+// runs their fused multiply-add chains over channels in order.
 // Pooled K rows are padded by 4 floats in shared memory so that the 16-byte
 // loads of different rows fall in different banks. The row softmax happens
 // in the selection kernel, which reads the whole row anyway.
 // ----------------------------------------------------------------------------
-constexpr int kScoreRows = 16;
+constexpr int kScoreRows = 32;
 constexpr int kScoreTileJ = 64;
 
 template <int D>
@@ -98,7 +99,7 @@ template <int D>
 __global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                                                     int nqb, int nkb, float scale, float* __restrict__ Z) {
   extern __shared__ __align__(16) float sm[];
-  float* sq = sm;                                   // [16][D]
+  float* sq = sm;                                   // [32][D]
   float* sk = sq + kScoreRows * D;                  // [64][D+4]
   const int tiles_q = (nqb + kScoreRows - 1) / kScoreRows;
   const int tiles_j = (nkb + kScoreTileJ - 1) / kScoreTileJ;
@@ -124,21 +125,21 @@ __global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qb
   }
   __syncthreads();
   const int jl = tid % 16;   // key blocks jl, jl+16, jl+32, jl+48 of the tile
-  const int ig = tid / 16;   // query rows 2*ig, 2*ig+1
-  float acc[2][4];
+  const int ig = tid / 16;   // query rows 4*ig .. 4*ig+3
+  float acc[4][4];
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-#pragma unroll 4
+#pragma unroll 2
   for (int c = 0; c < D; c += 4) {
-    float4 q[2], k[4];
+    float4 q[4], k[4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a) q[a] = *reinterpret_cast<const float4*>(sq + (2 * ig + a) * D + c);
+    for (int a = 0; a < 4; ++a) q[a] = *reinterpret_cast<const float4*>(sq + (4 * ig + a) * D + c);
 #pragma unroll
     for (int b = 0; b < 4; ++b) k[b] = *reinterpret_cast<const float4*>(sk + (jl + 16 * b) * (D + 4) + c);
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
         acc[a][b] = __fmaf_rn(q[a].x, k[b].x, acc[a][b]);
@@ -148,12 +149,12 @@ __global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qb
       }
   }
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int j = jl + 16 * b;
-      if (j < nj && 2 * ig + a < nrows)
-        Z[(bh * nqb + I0 + 2 * ig + a) * (int64_t)nkb + J0 + j] = __fmul_rn(acc[a][b], scale);
+      if (j < nj && 4 * ig + a < nrows)
+        Z[(bh * nqb + I0 + 4 * ig + a) * (int64_t)nkb + J0 + j] = __fmul_rn(acc[a][b], scale);
     }
 }
 
@@ -169,9 +170,10 @@ __global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qb
 //   2. Top-p: radix select (four 8-bit digits, most significant first) of the
 //      key at which the descending running weight first reaches p; ties at
 //      that key all weigh the same, so the count needed follows by division.
-//   3. m = max(kc, pc, 1); a second radix select (counting) finds the key of
-//      the m-th largest block; blocks above it are kept, and of the blocks at
-//      it the lowest indices fill the remaining places.
+//   3. m = max(kc, pc, 1). When m = pc the m-th largest key is the Top-p key
+//      just found; otherwise a second radix select (counting) finds it.
+//      Blocks above it are kept, and of the blocks at it the lowest indices
+//      fill the remaining places.
 //   4. Kept flags are compacted in block order (block-wide scans) into the
 //      ascending kept list.
 // ----------------------------------------------------------------------------
@@ -342,6 +344,9 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restric
 
   // 2. Top-p count.
   int pc = 0;
+  unsigned int p_key = 0u;  // key of the pc-th largest block, when the Top-p select ran
+  int p_above = 0;          // blocks above that key
+  bool have_p = false;
   if (topp > 0.0) {
     const unsigned long long target = (unsigned long long)ceil(topp * 4611686018427387904.0);  // p * 2^62
     unsigned long long tot = 0ull;  // total weight (exact integer sum)
@@ -369,14 +374,17 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restric
       const unsigned long long need = target - above_w;  // > 0 by construction
       const unsigned long long c = wt ? (need + wt - 1) / wt : 0ull;
       pc = above_c + (int)c;
+      p_key = prefix;
+      p_above = above_c;
+      have_p = true;
     }
   }
   const int m = min(nkb, max(max(kc, pc), 1));
 
   // 3. Key of the m-th largest block, and how many of its ties are kept.
-  unsigned int tkey = 0u;
-  int above_m = 0;
-  {
+  unsigned int tkey = p_key;
+  int above_m = p_above;
+  if (!(have_p && m == pc)) {
     unsigned int prefix = 0u;
     unsigned long long above_w = 0ull;
     int above_c = 0;
