@@ -50,9 +50,13 @@ def _load():
         lib.oracle_mask.argtypes = [p, p, i64, i64, i32, i32, i32, dbl, dbl, i32, p, p, p]
         lib.oracle_attention_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, i32,
                                               p, i64, p, p]
+        lib.oracle_quant_q8.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
+        lib.oracle_e4m3.argtypes = [p, i64, p]
+        lib.oracle_attention_q8_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, p]
         for f in (lib.oracle_pool_f64, lib.oracle_pool_f32, lib.oracle_block_probs_f64,
                   lib.oracle_block_probs_f32, lib.oracle_select_row, lib.oracle_mask,
-                  lib.oracle_attention_rows):
+                  lib.oracle_attention_rows, lib.oracle_quant_q8, lib.oracle_e4m3,
+                  lib.oracle_attention_q8_rows):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -166,3 +170,47 @@ def attention_rows(Q, K, V, bq: int, bk: int, kv_idx=None, kv_cnt=None, alpha=No
                                          _ptr(cnt), _ptr(al), H, MODES[mode], _ptr(rows),
                                          rows.shape[0], _ptr(O), _ptr(lse)), "attention_rows")
     return O, lse
+
+
+def e4m3(x) -> np.ndarray:
+    """Nearest fp8 e4m3 value of each element (ties to even, saturating at 448), as float64."""
+    a = np.ascontiguousarray(np.asarray(x, np.float64))
+    out = np.empty_like(a)
+    _check(_load().oracle_e4m3(_ptr(a), a.size, _ptr(out)), "e4m3")
+    return out
+
+
+def quant_q8(Q, K, V, bq: int, bk: int):
+    """Quantised operands of the low-bit sparse branch.
+
+    Returns (q8 int8 [B,H,N,d], sq float32 [B,H,Nqb], k8 int8 [B,H,N,d],
+    sk float32 [B,H,Nkb], v8 float64 [B,H,N,d] (e4m3 values), sv float32 [B,H,d])."""
+    q, k, v = _bits(Q), _bits(K), _bits(V)
+    B, H, N, d = q.shape
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    q8 = np.empty((B, H, N, d), np.int8)
+    k8 = np.empty((B, H, N, d), np.int8)
+    v8 = np.empty((B, H, N, d), np.float64)
+    sq = np.empty((B, H, nqb), np.float32)
+    sk = np.empty((B, H, nkb), np.float32)
+    sv = np.empty((B, H, d), np.float32)
+    _check(_load().oracle_quant_q8(_ptr(q), _ptr(k), _ptr(v), B * H, N, d, bq, bk, _ptr(q8), _ptr(sq),
+                                   _ptr(k8), _ptr(sk), _ptr(v8), _ptr(sv)), "quant_q8")
+    return q8, sq, k8, sk, v8, sv
+
+
+def attention_q8_rows(Q, K, V, bq: int, bk: int, kv_idx, kv_cnt, rows=None) -> np.ndarray:
+    """Low-bit sparse branch outputs (float64 [nrows, d]) for selected rows
+    (flat ids b*H*N + h*N + i; default every row)."""
+    q, k, v = _bits(Q), _bits(K), _bits(V)
+    B, H, N, d = q.shape
+    if rows is None:
+        rows = np.arange(B * H * N, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, np.int64)
+    idx = np.ascontiguousarray(np.asarray(kv_idx), np.int32)
+    cnt = np.ascontiguousarray(np.asarray(kv_cnt), np.int32)
+    O = np.zeros((rows.shape[0], d), np.float64)
+    _check(_load().oracle_attention_q8_rows(_ptr(q), _ptr(k), _ptr(v), B * H, N, d, bq, bk, _ptr(idx),
+                                            _ptr(cnt), _ptr(rows), rows.shape[0], _ptr(O)),
+           "attention_q8_rows")
+    return O

@@ -406,3 +406,175 @@ int oracle_attention_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* 
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Low-bit sparse branch [SLA2 s3]: the article quantises the sparse branch's
+// queries, keys, attention probabilities and values to a low-bit format
+// ("for example 8-bit integers"), scaling into the low-bit range before the
+// products and back after. It fixes neither the formats nor the scale
+// granularity; the readings taken here:
+//   * Q and K: int8, symmetric, one scale per (batch, head, block): the
+//     block's max |x| maps to 127; q8 = rint(x * s) (ties to even), clamped
+//     to [-127, 127]; s = 127 / amax in float (1 when amax = 0), the product
+//     x * s in float. S = q8 . k8 is an exact integer.
+//   * V: fp8 e4m3, one scale per (batch, head, channel) over all keys: the
+//     channel's max |v| maps to 448; v8 = e4m3(v * s_v), the product in float.
+//   * P: e4m3 relative to a running integer log2 maximum, in the order the
+//     kept key tiles (64 keys, ascending blocks) are visited:
+//       x_j   = float(S_j) * c, c = float(log2(e)/sqrt(d)) / (s_q * s_k) in float;
+//       m     = max(m, ceil(max_j x_j)) per tile, the accumulators scaled by
+//               2^(m_old - m_new) (exact) when m grows;
+//       e_j   = 2^(x_j - m), x_j - m in float; p_j = e4m3(e_j);
+//       l += e_j (the normaliser is not quantised: only the operands of the
+//       two products are); acc += p_j v8_j;
+//     O = acc / (l * s_v). Because m is an integer and e4m3 rounding commutes
+//     with powers of two (above its subnormal range), the result does not
+//     depend on where in the walk m settled.
+// e4m3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; largest finite 448,
+// subnormals down to 2^-9; rounding to nearest, ties to even; magnitudes
+// above 448 saturate to 448.
+// ===========================================================================
+
+namespace {
+
+double e4m3_rne(double x) {
+  if (x == 0.0 || std::isnan(x)) return x;
+  const double a = std::fabs(x);
+  if (a >= 448.0) return std::copysign(448.0, x);
+  int k;
+  std::frexp(a, &k);                    // a = f * 2^k, f in [0.5, 1): binade exponent k - 1
+  const int e = std::max(k - 1, -6);    // below 2^-6 the spacing stays 2^-9 (subnormals)
+  const double q = std::ldexp(1.0, e - 3);
+  const double r = std::nearbyint(a / q) * q;  // default rounding mode: to nearest, ties to even
+  return std::copysign(std::min(r, 448.0), x);
+}
+
+float quant_scale(float amax, float top) { return amax > 0.0f ? top / amax : 1.0f; }
+
+int8_t quant_i8(float x, float s) {
+  float v = x * s;
+  float r = std::nearbyint(v);
+  if (r > 127.0f) r = 127.0f;
+  if (r < -127.0f) r = -127.0f;
+  return static_cast<int8_t>(r);
+}
+
+}  // namespace
+
+extern "C" {
+
+// ---------------------------------------------------------------------------
+// Quantised operands of the low-bit sparse branch (readings above).
+// Q, K, V: bf16 bits [BH, N, d]. q8 / k8: int8 [BH, N, d]; sq: [BH, ceil(N/bq)];
+// sk: [BH, ceil(N/bk)]; v8: the e4m3 values as double [BH, N, d]; sv: [BH, d].
+// ---------------------------------------------------------------------------
+int oracle_quant_q8(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t BH, int64_t N, int d, int bq,
+                    int bk, int8_t* q8, float* sq, int8_t* k8, float* sk, double* v8, float* sv) {
+  if (!Q || !K || !V || !q8 || !sq || !k8 || !sk || !v8 || !sv || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
+  const int64_t nqb = ceil_div(N, bq), nkb = ceil_div(N, bk);
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    for (int pass = 0; pass < 2; ++pass) {
+      const uint16_t* X = pass == 0 ? Q : K;
+      int8_t* out = pass == 0 ? q8 : k8;
+      float* sc = pass == 0 ? sq : sk;
+      const int blk = pass == 0 ? bq : bk;
+      const int64_t nb = pass == 0 ? nqb : nkb;
+      for (int64_t I = 0; I < nb; ++I) {
+        const int64_t r0 = I * blk, r1 = std::min<int64_t>(N, r0 + blk);
+        float amax = 0.0f;
+        for (int64_t r = r0; r < r1; ++r)
+          for (int c = 0; c < d; ++c) amax = std::max(amax, std::fabs(widen_f(X[(bh * N + r) * d + c])));
+        const float s = quant_scale(amax, 127.0f);
+        sc[bh * nb + I] = s;
+        for (int64_t r = r0; r < r1; ++r)
+          for (int c = 0; c < d; ++c) out[(bh * N + r) * d + c] = quant_i8(widen_f(X[(bh * N + r) * d + c]), s);
+      }
+    }
+    for (int c = 0; c < d; ++c) {
+      float amax = 0.0f;
+      for (int64_t r = 0; r < N; ++r) amax = std::max(amax, std::fabs(widen_f(V[(bh * N + r) * d + c])));
+      const float s = quant_scale(amax, 448.0f);
+      sv[bh * d + c] = s;
+      for (int64_t r = 0; r < N; ++r) {
+        const float v = widen_f(V[(bh * N + r) * d + c]) * s;
+        v8[(bh * N + r) * d + c] = e4m3_rne(static_cast<double>(v));
+      }
+    }
+  }
+  return OK;
+}
+
+// Nearest e4m3 value of each x (ties to even, saturating at 448).
+int oracle_e4m3(const double* x, int64_t n, double* out) {
+  if (!x || !out || n < 0) return ERR_ARG;
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_rne(x[i]);
+  return OK;
+}
+
+// ---------------------------------------------------------------------------
+// Low-bit sparse branch outputs for selected rows (readings above).
+// rows: flat row ids bh*N + i. O: [nrows, d] double.
+// ---------------------------------------------------------------------------
+int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t BH, int64_t N,
+                             int d, int bq, int bk, const int32_t* kv_idx, const int32_t* kv_cnt,
+                             const int64_t* rows, int64_t nrows, double* O) {
+  if (!Q || !K || !V || !rows || !O || !kv_idx || !kv_cnt || !shape_ok(BH, N, d, bq) || bk <= 0 || bk % 64 != 0)
+    return ERR_ARG;
+  const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
+  std::vector<int8_t> q8(static_cast<size_t>(BH * N * d)), k8(static_cast<size_t>(BH * N * d));
+  std::vector<float> sq(static_cast<size_t>(BH * Nqb)), sk(static_cast<size_t>(BH * Nkb)), sv(static_cast<size_t>(BH * d));
+  std::vector<double> v8(static_cast<size_t>(BH * N * d));
+  const int rc = oracle_quant_q8(Q, K, V, BH, N, d, bq, bk, q8.data(), sq.data(), k8.data(), sk.data(), v8.data(),
+                                 sv.data());
+  if (rc != OK) return rc;
+  const float c0 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  std::vector<double> acc(d);
+  std::vector<float> x(64);
+  for (int64_t t = 0; t < nrows; ++t) {
+    const int64_t r = rows[t];
+    if (r < 0 || r >= BH * N) return ERR_ARG;
+    const int64_t bh = r / N, i = r % N, I = i / bq;
+    const int64_t cnt = kv_cnt[bh * Nqb + I];
+    if (cnt < 0 || cnt > Nkb) return ERR_ARG;
+    const int8_t* qi = &q8[static_cast<size_t>((bh * N + i) * d)];
+    float m = -std::numeric_limits<float>::infinity();
+    double l = 0.0;
+    std::fill(acc.begin(), acc.end(), 0.0);
+    for (int64_t e = 0; e < cnt; ++e) {
+      const int64_t J = kv_idx[(bh * Nqb + I) * Nkb + e];
+      if (J < 0 || J >= Nkb) return ERR_ARG;
+      const float c = c0 / (sq[bh * Nqb + I] * sk[bh * Nkb + J]);
+      for (int64_t key0 = J * bk; key0 < std::min<int64_t>(N, (J + 1) * bk); key0 += 64) {
+        const int64_t key1 = std::min<int64_t>(N, key0 + 64);
+        float mt = -std::numeric_limits<float>::infinity();
+        for (int64_t j = key0; j < key1; ++j) {
+          const int8_t* kj = &k8[static_cast<size_t>((bh * N + j) * d)];
+          int64_t S = 0;
+          for (int cc = 0; cc < d; ++cc) S += static_cast<int64_t>(qi[cc]) * kj[cc];
+          x[j - key0] = static_cast<float>(S) * c;
+          mt = std::max(mt, x[j - key0]);
+        }
+        const float m_new = std::max(m, std::ceil(mt));
+        if (m_new > m && l > 0.0) {
+          const double f = std::exp2(static_cast<double>(m - m_new));
+          l *= f;
+          for (int cc = 0; cc < d; ++cc) acc[cc] *= f;
+        }
+        m = m_new;
+        for (int64_t j = key0; j < key1; ++j) {
+          const float y = x[j - key0] - m;
+          const double ej = std::exp2(static_cast<double>(y));
+          const double pj = e4m3_rne(ej);
+          l += ej;
+          for (int cc = 0; cc < d; ++cc) acc[cc] += pj * v8[static_cast<size_t>((bh * N + j) * d + cc)];
+        }
+      }
+    }
+    for (int cc = 0; cc < d; ++cc)
+      O[t * d + cc] = l > 0.0 ? acc[cc] / (l * static_cast<double>(sv[bh * d + cc])) : 0.0;
+  }
+  return OK;
+}
+
+}  // extern "C"
+

@@ -358,3 +358,99 @@ def test_invalid_arguments_are_rejected(oracle_mod):
     kv_cnt = np.ones((1, 1, 1), np.int32)
     with pytest.raises(ValueError):
         oracle_mod.attention_rows(q, k, v, 64, 64, kv_idx, kv_cnt, mode="sparse")
+
+
+# ----------------------------------------------------------------------------- low-bit sparse branch
+def _e4m3_torch(x):
+    """fp8 e4m3 rounding through torch's own cast (values already in fp32, |x| <= 448)."""
+    t = torch.as_tensor(np.asarray(x), dtype=torch.float64).to(torch.float32).clamp(-448, 448)
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_rounding_matches_torch_float8(oracle_mod):
+    x = np.concatenate([np.linspace(-448, 448, 40001), np.exp2(np.linspace(-12, 8.8, 5001)),
+                        -np.exp2(np.linspace(-12, 8.8, 5001)), [0.0, 2.0 ** -10, 3 * 2.0 ** -11, 1.0625, 1.1875]])
+    x = x.astype(np.float32).astype(np.float64)  # the GPU rounds fp32 values
+    np.testing.assert_array_equal(oracle_mod.e4m3(x), _e4m3_torch(x))
+    # saturation instead of overflow
+    np.testing.assert_array_equal(oracle_mod.e4m3(np.array([500.0, -1e6, 449.0])), [448.0, -448.0, 448.0])
+
+
+def test_q8_quantisation_closed_forms(oracle_mod):
+    # A block whose max |x| is 127 * 2^-3 and whose values are multiples of 2^-3:
+    # the scale is exactly 2^3 and every code is the integer x * 8.
+    d, N = 8, 64
+    vals = (torch.arange(N * d, dtype=torch.float32).reshape(N, d) % 255 - 127) / 8.0
+    Q = _bf16(vals.reshape(1, 1, N, d))
+    K = _bf16(-vals.reshape(1, 1, N, d))
+    V = _bf16(torch.ones(1, 1, N, d))
+    q8, sq, k8, sk, v8, sv = oracle_mod.quant_q8(Q, K, V, 64, 64)
+    assert sq[0, 0, 0] == 8.0 and sk[0, 0, 0] == 8.0
+    np.testing.assert_array_equal(q8[0, 0], (vals * 8).numpy().astype(np.int8))
+    np.testing.assert_array_equal(k8[0, 0], (-vals * 8).numpy().astype(np.int8))
+    # V all ones: the channel max maps to 448 exactly.
+    np.testing.assert_array_equal(v8, 448.0)
+    np.testing.assert_allclose(sv, 448.0)
+    # Ties go to even: x * s = k + 1/2 with amax fixing s = 127 / 2.
+    Qt = _bf16(torch.tensor([2.0, 5.0 / 127.0, 3.0 / 127.0, 1.0 / 127.0]).reshape(1, 1, 1, 4))
+    q8t, sqt, *_ = oracle_mod.quant_q8(Qt, Qt, Qt, 64, 64)
+    expect = np.rint(Qt.float().numpy() * np.float32(127.0 / 2.0))
+    np.testing.assert_array_equal(q8t.reshape(-1), expect.reshape(-1).astype(np.int8))
+
+
+def test_q8_constant_v_and_identical_keys(oracle_mod):
+    B, H, N, d, bq, bk = 1, 2, 256, 16, 64, 64
+    q, k, v = _rand_qkv(B, H, N, d, 40, scale=1.5)
+    kv_idx, kv_cnt = (np.asarray(a) for a in synth.random_mask(B, H, N // bq, N // bk, 3, seed=12))
+    # V constant per channel: the output is that constant times sum(p)/sum(e),
+    # the e4m3-rounded weights over the unrounded normaliser, so within the
+    # format's relative rounding of 2^-4 (and the same factor in every channel).
+    c = torch.linspace(-2.0, 3.0, d)
+    vc = _bf16(c.expand(B, H, N, d).clone())
+    out = oracle_mod.attention_q8_rows(q, k, vc, bq, bk, kv_idx, kv_cnt)
+    nonempty = np.repeat(kv_cnt.reshape(-1) > 0, bq)  # rows of empty blocks keep nothing: 0
+    assert nonempty.any() and not nonempty.all()
+    const = vc[0, 0, 0].float().numpy().astype(np.float64)
+    ratio = out[nonempty] / const
+    np.testing.assert_allclose(ratio, ratio[:, :1].repeat(d, axis=1), rtol=1e-6)  # fp32 channel scales
+    assert np.all(np.abs(ratio - 1.0) <= 2.0 ** -4)
+    np.testing.assert_array_equal(out[~nonempty], 0.0)
+    # All keys identical: every kept key gets probability e4m3(1) = 1, so the
+    # output is the mean of the e4m3-coded values over the kept keys.
+    kc = _bf16(k[:, :, :1].expand(B, H, N, d).clone())
+    out = oracle_mod.attention_q8_rows(q, kc, v, bq, bk, kv_idx, kv_cnt)
+    sv = np.float32(448.0) / np.abs(v.float().numpy()).max(axis=2)  # [B,H,d], fp32
+    v8 = _e4m3_torch((v.float().numpy() * sv[:, :, None, :]).astype(np.float64)) / sv[:, :, None, :]
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                I = i // bq
+                row = out[(b * H + h) * N + i]
+                if kv_cnt[b, h, I] == 0:
+                    np.testing.assert_array_equal(row, 0.0)
+                    continue
+                keys = np.concatenate([np.arange(J * bk, (J + 1) * bk) for J in kv_idx[b, h, I, :kv_cnt[b, h, I]]])
+                np.testing.assert_allclose(row, v8[b, h, keys].mean(axis=0), rtol=1e-9, atol=1e-12)
+
+
+def test_q8_scaling_v_by_two_scales_output_exactly(oracle_mod):
+    q, k, v = _rand_qkv(1, 1, 192, 16, 41, scale=2.0)
+    kv_idx, kv_cnt = synth.random_mask(1, 1, 3, 3, 2, seed=13)
+    a = oracle_mod.attention_q8_rows(q, k, v, 64, 64, kv_idx, kv_cnt)
+    b = oracle_mod.attention_q8_rows(q, k, _bf16(v.float() * 2.0), 64, 64, kv_idx, kv_cnt)
+    np.testing.assert_array_equal(b, 2.0 * a)
+
+
+def test_q8_close_to_exact_sparse_attention(oracle_mod):
+    # Within the error that 8-bit Q/K codes and e4m3 P/V allow: each e4m3
+    # value carries up to 2^-4 relative error and each int8 code half a step
+    # of the block's max / 127; on these inputs the outputs stay within a few
+    # percent of the exact sparse branch (mean relative L1).
+    q, k, v = _rand_qkv(1, 2, 512, 64, 42, scale=1.0)
+    kv_idx, kv_cnt, _ = oracle_mod.mask(q, k, 64, 64, 0.25, 0.9)
+    rows = np.arange(0, 1024, 7)
+    a = oracle_mod.attention_q8_rows(q, k, v, 64, 64, kv_idx, kv_cnt, rows)
+    e, _ = oracle_mod.attention_rows(q, k, v, 64, 64, kv_idx, kv_cnt, mode="sparse", rows=rows)
+    rel = np.abs(a - e).sum() / np.abs(e).sum()
+    assert rel < 0.06, rel
+    assert rel > 1e-4  # the quantisation is really applied
