@@ -415,8 +415,9 @@ def test_q8_constant_v_and_identical_keys(oracle_mod):
     np.testing.assert_allclose(ratio, ratio[:, :1].repeat(d, axis=1), rtol=1e-6)  # fp32 channel scales
     assert np.all(np.abs(ratio - 1.0) <= 2.0 ** -4)
     np.testing.assert_array_equal(out[~nonempty], 0.0)
-    # All keys identical: every kept key gets probability e4m3(1) = 1, so the
-    # output is the mean of the e4m3-coded values over the kept keys.
+    # All keys identical: every kept key gets the same weight e4m3(e) over the
+    # normaliser's e, so the output is the mean of the e4m3-coded values over
+    # the kept keys times one factor within 2^-4 of 1, the same in every channel.
     kc = _bf16(k[:, :, :1].expand(B, H, N, d).clone())
     out = oracle_mod.attention_q8_rows(q, kc, v, bq, bk, kv_idx, kv_cnt)
     sv = np.float32(448.0) / np.abs(v.float().numpy()).max(axis=2)  # [B,H,d], fp32
@@ -430,7 +431,11 @@ def test_q8_constant_v_and_identical_keys(oracle_mod):
                     np.testing.assert_array_equal(row, 0.0)
                     continue
                 keys = np.concatenate([np.arange(J * bk, (J + 1) * bk) for J in kv_idx[b, h, I, :kv_cnt[b, h, I]]])
-                np.testing.assert_allclose(row, v8[b, h, keys].mean(axis=0), rtol=1e-9, atol=1e-12)
+                mean = v8[b, h, keys].mean(axis=0)
+                big = np.abs(mean) > 1e-3
+                ratio = row[big] / mean[big]
+                np.testing.assert_allclose(ratio, ratio[0], rtol=1e-9)
+                assert abs(ratio[0] - 1.0) <= 2.0 ** -4
 
 
 def test_q8_scaling_v_by_two_scales_output_exactly(oracle_mod):
