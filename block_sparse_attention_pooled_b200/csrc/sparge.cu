@@ -15,6 +15,8 @@
 #include "attn.cuh"
 #include "linear.cuh"
 #include "lin_out.cuh"
+#include "quant.cuh"
+#include "attn_q8.cuh"
 
 namespace {
 
@@ -137,6 +139,82 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
   if (e != cudaSuccess) return cuda_status(e);
   select_kernel<<<(unsigned)(dm.BH * dm.nqb), kSelectThreads, sel_sm, st>>>(P, dm.BH * dm.nqb, (int)dm.nkb, kc, topp,
                                                                            kv_idx, kv_cnt, row_thresh);
+  return cuda_status(cudaGetLastError());
+}
+
+// 3-D map over one-byte codes [BH][N][128] with a (128 x rows x 1) box,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map_u8(CUtensorMap* m, const void* base, int64_t BH, int N, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {128, (cuuint64_t)N * 128};
+  cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Workspace of the low-bit sparse branch: codes and scales of Q, K, V.
+struct Q8Ws {
+  size_t q8, k8, v8, sq, sk, sv, vpart, total;
+};
+
+Q8Ws q8_ws(const sparge_shape* s, const Dims& d) {
+  Q8Ws w;
+  const size_t codes = align256((size_t)d.BH * s->N * s->d);
+  const int64_t nch = ceil_div(s->N, kVChunk);
+  w.q8 = 0;
+  w.k8 = w.q8 + codes;
+  w.v8 = w.k8 + codes;
+  w.sq = w.v8 + codes;
+  w.sk = w.sq + align256((size_t)d.BH * d.nqb * 4);
+  w.sv = w.sk + align256((size_t)d.BH * d.nkb * 4);
+  w.vpart = w.sv + align256((size_t)d.BH * s->d * 4);
+  w.total = w.vpart + align256((size_t)d.BH * nch * s->d * 4);
+  return w;
+}
+
+sparge_status launch_q8(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
+                        const int32_t* kv_idx, const int32_t* kv_cnt, void* O, uint8_t* ws, cudaStream_t st) {
+  const Q8Ws w = q8_ws(s, dm);
+  int8_t* q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  int8_t* k8 = reinterpret_cast<int8_t*>(ws + w.k8);
+  uint8_t* v8 = ws + w.v8;
+  float* sq = reinterpret_cast<float*>(ws + w.sq);
+  float* sk = reinterpret_cast<float*>(ws + w.sk);
+  float* sv = reinterpret_cast<float*>(ws + w.sv);
+  float* vpart = reinterpret_cast<float*>(ws + w.vpart);
+  const int64_t q_ctas = dm.BH * dm.nqb, k_ctas = dm.BH * dm.nkb, nch = ceil_div(s->N, kVChunk);
+  const int64_t total = q_ctas + k_ctas + dm.BH * nch;
+  if (total > INT32_MAX) return SPARGE_ERR_UNSUPPORTED;
+  const __nv_bfloat16* Qb = static_cast<const __nv_bfloat16*>(Q);
+  const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(K);
+  const __nv_bfloat16* Vb = static_cast<const __nv_bfloat16*>(V);
+  quant_qk_vmax_kernel<128><<<(unsigned)total, kQuantThreads, 0, st>>>(Qb, Kb, Vb, dm.BH, s->N, s->bq, s->bk, q_ctas,
+                                                                       k_ctas, q8, sq, k8, sk, vpart);
+  quant_v_kernel<128><<<(unsigned)(dm.BH * nch), kQuantThreads, 0, st>>>(Vb, s->N, vpart, v8, sv);
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map_u8(&mq, q8, dm.BH, s->N, kTileQ) || !make_map_u8(&mk, k8, dm.BH, s->N, kTileK) ||
+      !make_map_u8(&mv, v8, dm.BH, s->N, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
+    return SPARGE_ERR_CUDA;
+  Q8Params p;
+  p.kv_idx = kv_idx;
+  p.kv_cnt = kv_cnt;
+  p.sq = sq;
+  p.sk = sk;
+  p.sv = sv;
+  p.N = s->N;
+  p.nqb = (int)dm.nqb;
+  p.nkb = (int)dm.nkb;
+  p.bq = s->bq;
+  p.bk = s->bk;
+  p.c0 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  cudaError_t e = ensure_smem(attn_q8_kernel, Q8Smem::kBytes, 9);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_q8_kernel<<<(unsigned)(dm.BH * dm.nqb), kQ8Threads, Q8Smem::kBytes, st>>>(mq, mk, mv, mo, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -274,6 +352,8 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
       return 0;
     case SPARGE_OP_SLA2:
       return shape->d == 128 ? sla2_ws(shape, dm).total : 0;
+    case SPARGE_OP_ATTN_Q8:
+      return shape->d == 128 ? q8_ws(shape, dm).total : 0;
     default:
       return 0;
   }
@@ -343,6 +423,22 @@ sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const
   if (shape->d == 64)
     return launch_attn<64, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s);
   return launch_attn<128, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s);
+}
+
+sparge_status sparge_attn_fwd_q8(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                                 const int32_t* kv_idx, const int32_t* kv_cnt, void* O, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !V || !O || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARGE_ERR_INVALID_ARG;
+  if (shape->d != 128 || dm.BH > 65535) return SPARGE_ERR_UNSUPPORTED;
+  const Q8Ws w = q8_ws(shape, dm);
+  if (workspace == nullptr || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
+  return launch_q8(Q, K, V, shape, dm, kv_idx, kv_cnt, O, static_cast<uint8_t*>(workspace),
+                   static_cast<cudaStream_t>(stream));
 }
 
 sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,

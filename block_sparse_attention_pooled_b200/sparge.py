@@ -20,14 +20,14 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
-OP_MASK, OP_ATTN, OP_SLA2 = 0, 1, 2
+OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8 = 0, 1, 2, 3
 
 # Kernel launches per call of each entry point (for launch accounting).
-MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES = 3, 1, 4
+MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES = 3, 1, 4, 3
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
-           "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc")
+           "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8")
 
 
 class Shape(ctypes.Structure):
@@ -42,10 +42,11 @@ _lib.sparge_mask_noalloc.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _dbl, _dbl
 _lib.sparge_mask_noalloc.restype = ctypes.c_int
 _lib.sparge_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sla2_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sparge_attn_fwd_q8.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 _lib.sparge_status_string.argtypes = [ctypes.c_int]
 _lib.sparge_status_string.restype = ctypes.c_char_p
-for _f in ("sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status"):
+for _f in ("sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -134,6 +135,42 @@ def sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, bq: int, bk: int, O=None, lse=None,
     _check(_lib.sparge_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt), _ptr(O),
                                 _ptr(lse), _ptr(workspace), nws, _stream(stream)), "sparge_attn_fwd")
     return O
+
+
+def sparge_attn_fwd_q8(Q, K, V, kv_idx, kv_cnt, bq: int, bk: int, O=None, workspace=None, stream=None):
+    """Low-bit block-sparse attention (int8 Q/K codes, e4m3 P and V codes). Returns O."""
+    _check_qkv(Q, K, V)
+    shape = make_shape(Q, bq, bk)
+    if O is None:
+        O = torch.empty_like(Q)
+    if workspace is None:
+        workspace, nws = _workspace(OP_ATTN_Q8, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sparge_attn_fwd_q8(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt),
+                                   _ptr(O), _ptr(workspace), nws, _stream(stream)), "sparge_attn_fwd_q8")
+    return O
+
+
+def quant_q8_workspace_views(workspace, shape):
+    """(q8, k8, v8, sq, sk, sv) views into a sparge_attn_fwd_q8 workspace, in the
+    library's layout (codes [B,H,N,128] int8 / e4m3 bytes; scales fp32)."""
+    B, H, N, d, bq, bk = shape.B, shape.H, shape.N, shape.d, shape.bq, shape.bk
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    codes = a256(B * H * N * d)
+    off_q8, off_k8, off_v8 = 0, codes, 2 * codes
+    off_sq = 3 * codes
+    off_sk = off_sq + a256(B * H * nqb * 4)
+    off_sv = off_sk + a256(B * H * nkb * 4)
+    w = workspace.view(torch.uint8)
+    q8 = w[off_q8:off_q8 + B * H * N * d].view(torch.int8).view(B, H, N, d)
+    k8 = w[off_k8:off_k8 + B * H * N * d].view(torch.int8).view(B, H, N, d)
+    v8 = w[off_v8:off_v8 + B * H * N * d].view(B, H, N, d)
+    sq = w[off_sq:off_sq + B * H * nqb * 4].view(torch.float32).view(B, H, nqb)
+    sk = w[off_sk:off_sk + B * H * nkb * 4].view(torch.float32).view(B, H, nkb)
+    sv = w[off_sv:off_sv + B * H * d * 4].view(torch.float32).view(B, H, d)
+    return q8, k8, v8, sq, sk, sv
 
 
 def sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, bq: int, bk: int, O=None, workspace=None, stream=None):

@@ -73,7 +73,7 @@ typedef struct {
   int32_t bq, bk;     /* query rows per block, keys per block */
 } sparge_shape;
 
-enum { SPARGE_OP_MASK = 0, SPARGE_OP_ATTN = 1, SPARGE_OP_SLA2 = 2 };
+enum { SPARGE_OP_MASK = 0, SPARGE_OP_ATTN = 1, SPARGE_OP_SLA2 = 2, SPARGE_OP_ATTN_Q8 = 3 };
 
 /* Workspace bytes the operation needs for this shape (0 if none, or if the
  * shape is invalid). */
@@ -136,6 +136,25 @@ sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_sha
 sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                               const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Low-bit block-sparse attention forward (SLA2 article, section 3: the
+ * sparse branch computes with Q, K, the attention probabilities P and V in
+ * a low-bit format, scaled into its range and back). Same mask and output
+ * conventions as sparge_attn_fwd; d must be 128.
+ * Formats and scales (the article fixes neither; these are this library's):
+ *   Q, K  int8 codes, symmetric, one scale per (batch, head, block of bq / bk
+ *         rows): s = 127 / max|x| (fp32), code = rint(x * s) clamped to +-127.
+ *   V     fp8 e4m3 codes, one scale per (batch, head, channel): s = 448 / max|v|.
+ *   S     exact int32 products of the codes; x = float(S) * c with
+ *         c = (log2(e)/sqrt(d)) / (s_q * s_k) in fp32.
+ *   P     e4m3 codes of e = 2^(x - m), m a running integer maximum of x over
+ *         the kept key tiles (64 keys, ascending); the normaliser sums e.
+ *   O     = sum(P * v_codes) / (sum(e) * s_v), stored as bf16.
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN_Q8, shape) (codes and
+ * scales). Three launches: Q/K codes with V channel maxima, V codes, attention. */
+sparge_status sparge_attn_fwd_q8(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                                 const int32_t* kv_idx, const int32_t* kv_cnt, void* O, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* Sparse + linear mix (SLA2 article, sections 1 and 2).
  *   O = alpha[h] * O_sparse + (1 - alpha[h]) * O_linear, with O_sparse as in

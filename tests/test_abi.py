@@ -55,6 +55,10 @@ def test_workspace_bytes_host_arithmetic(lib):
     assert lib.workspace_bytes(lib.OP_ATTN, s) == 0
     bad = lib.Shape(1, 1, 100, 96, 64, 64)  # unsupported head dim
     assert lib.workspace_bytes(lib.OP_MASK, bad) == 0
+    # Low-bit branch: three code tensors of one byte per element plus the scales.
+    need_q8 = lib.workspace_bytes(lib.OP_ATTN_Q8, s)
+    assert need_q8 >= 3 * 40 * 75600 * 128 + 4 * 40 * (nqb + nkb + 128)
+    assert lib.workspace_bytes(lib.OP_ATTN_Q8, lib.Shape(1, 1, 4096, 64, 64, 64)) == 0  # d = 128 only
 
 
 def test_invalid_arguments_rejected_before_any_launch(lib):
@@ -82,6 +86,12 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
         assert raw.sparge_attn_fwd(P, P, P, ctypes.byref(bad), P, P, P, None, None, 0, None) == lib.ERR_INVALID_ARG
     assert raw.sparge_attn_fwd(P, P, None, ctypes.byref(s), P, P, P, None, None, 0, None) == lib.ERR_INVALID_ARG
     assert raw.sla2_attn_fwd(P, P, P, None, P, P, P, P, None, 0, None) == lib.ERR_INVALID_ARG
+    # Low-bit branch: d = 128 only, workspace required.
+    assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s), P, P, P, P, 1 << 30, None) == lib.ERR_UNSUPPORTED
+    s128 = lib.Shape(1, 2, 4096, 128, 128, 64)
+    assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s128), P, P, P, None, 0, None) == lib.ERR_WORKSPACE
+    assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s128), P, P, P, P, 64, None) == lib.ERR_WORKSPACE
+    assert raw.sparge_attn_fwd_q8(P, None, P, ctypes.byref(s128), P, P, P, P, 1 << 30, None) == lib.ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors(lib):
