@@ -9,8 +9,10 @@
 //   S_j = q8_i . k8_j                     exact int32, tcgen05 kind::i8
 //   x_j = float(S_j) * c_IJ,              c_IJ = c0 / (s_q[I] * s_k[J]) in fp32,
 //                                         c0 = log2(e) / sqrt(d)
-//   m   = max(m, ceil(max_j x_j))         an integer, per tile; O and l are
-//                                         scaled by 2^(m_old - m_new) (exact)
+//   m   = ceil(max_j x_j) of the first     an integer; later it moves up to a
+//         tile                            tile's ceil(max_j x_j) only when that
+//                                         exceeds m + 8 (so e_j <= 2^8 < 448),
+//                                         O and l then scaled by 2^(m_old - m_new)
 //   e_j = 2^(x_j - m),  l += e_j,  p_j = e4m3(e_j)
 //   O  += p_j v8_j                        fp32 in TMEM, tcgen05 kind::f8f6f4
 // and O_i = O / (l * s_v) per channel. Because m only takes integer values
@@ -113,7 +115,17 @@ __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint
 // int32 -> float, exact for |v| < 2^22: the integer is placed in the mantissa
 // of 1.5 * 2^23 and the offset taken off again (integer add, float subtract).
 __device__ __forceinline__ float i2f_small(int v) {
-  return __fsub_rn(__int_as_float(v + 0x4B400000), 12582912.0f);
+  return __fsub_rn(__uint_as_float((uint32_t)v + 0x4B400000u), 12582912.0f);
+}
+
+// Largest of the row's 64 scores: eight independent chains, then a tree.
+__device__ __forceinline__ int row_max64_i(const int (&s)[kTileK]) {
+  int m8[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    m8[j] = max(max(max(s[j], s[8 + j]), max(s[16 + j], s[24 + j])),
+                max(max(s[32 + j], s[40 + j]), max(s[48 + j], s[56 + j])));
+  return max(max(max(m8[0], m8[1]), max(m8[2], m8[3])), max(max(m8[4], m8[5]), max(m8[6], m8[7])));
 }
 
 __global__ void __launch_bounds__(kQ8Threads, 2)
@@ -258,21 +270,24 @@ __global__ void __launch_bounds__(kQ8Threads, 2)
     bool ok = true;
     const float sqv = __ldg(p.sq + tile);
     const float* skh = p.sk + (int64_t)bh * p.nkb;
-    // Kept-block indices and their key scales, 32 at a time, one per lane, a chunk ahead.
+    // Kept-block indices and their score factors c = c0 / (s_q * s_k), 32
+    // at a time, one per lane, a chunk ahead (the division runs once per
+    // entry, in parallel across the lanes).
+    auto factor = [&](int J) { return __fdiv_rn(p.c0, __fmul_rn(sqv, __ldg(skh + J))); };
     int idx_cur = lane < cnt ? __ldg(lst + lane) : 0;
     int idx_nxt = 32 + lane < cnt ? __ldg(lst + 32 + lane) : 0;
-    float sk_cur = __ldg(skh + idx_cur), sk_nxt = __ldg(skh + idx_nxt);
+    float c_cur = factor(idx_cur), c_nxt = factor(idx_nxt);
     for (int t = 0; t < T; ++t) {
       const int pb = t & 1;
       const int e = t / tiles_per_block, sub = t % tiles_per_block;
       if (e > 0 && (e & 31) == 0 && sub == 0) {
         idx_cur = idx_nxt;
-        sk_cur = sk_nxt;
+        c_cur = c_nxt;
         idx_nxt = e + 32 + lane < cnt ? __ldg(lst + e + 32 + lane) : 0;
-        sk_nxt = __ldg(skh + idx_nxt);
+        c_nxt = factor(idx_nxt);
       }
       const int key0 = __shfl_sync(0xffffffffu, idx_cur, e & 31) * p.bk + sub * kTileK;
-      const float c = __fdiv_rn(p.c0, __fmul_rn(sqv, __shfl_sync(0xffffffffu, sk_cur, e & 31)));
+      const float c = __shfl_sync(0xffffffffu, c_cur, e & 31);
       ok = warp_wait(L::kBarSFull + pb, (t >> 1) & 1, kErrQ8SFull);
       if (!ok) break;
       tc_fence_after();
@@ -289,18 +304,23 @@ __global__ void __launch_bounds__(kQ8Threads, 2)
       }
       const bool full_tile = key0 + kTileK <= p.N;  // the same for every row of the tile
       const int nvalid = full_tile ? kTileK : p.N - key0;
-      int smax = INT_MIN;
+      if (!full_tile) {  // keys past N (zero-filled K rows) must not win the max
 #pragma unroll
-      for (int j = 0; j < kTileK; ++j)
-        if (full_tile || j < nvalid) smax = max(smax, s[j]);
+        for (int j = 0; j < kTileK; ++j)
+          if (j >= nvalid) s[j] = INT_MIN;
+      }
+      const int smax = row_max64_i(s);
       // A tile wholly past N (the second tile of a ragged 128-key block) has
       // no valid key: it leaves m as it is and contributes nothing.
-      const float m_new = nvalid > 0 ? fmaxf(m_run, ceilf(__fmul_rn(i2f_small(smax), c))) : m_run;
+      const float cm = nvalid > 0 ? ceilf(__fmul_rn(i2f_small(smax), c)) : m_run;
+      // Each row moves its reference only past a margin of 2^8 (its own
+      // decision, so the result does not depend on the other rows of the warp).
+      const float m_new = (t == 0 || cm > m_run + 8.0f) ? cm : m_run;
       if (t == 0) {
         m_run = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m_run)) {
         // Exact rescale by 2^(m_run - m_new), an integer power of two; rows
-        // whose maximum held scale by 1.
+        // whose reference held scale by 1.
         ok = warp_wait(L::kBarODone, (t - 1) & 1, kErrQ8ODone);
         if (!ok) break;
         tc_fence_after();
@@ -316,7 +336,8 @@ __global__ void __launch_bounds__(kQ8Threads, 2)
       uint32_t pw[kTileK / 4];
 #pragma unroll
       for (int k = 0; k < kTileK / 2; ++k) {
-        const uint64_t sf = sub2(f2(__int_as_float(s[2 * k] + 0x4B400000), __int_as_float(s[2 * k + 1] + 0x4B400000)),
+        const uint64_t sf = sub2(f2(__uint_as_float((uint32_t)s[2 * k] + 0x4B400000u),
+                                    __uint_as_float((uint32_t)s[2 * k + 1] + 0x4B400000u)),
                                  magic2);
         const uint64_t y = add2(fma2(sf, c2, 0ull), negm2);
         const float2 yv = f2_split(y);

@@ -100,16 +100,33 @@ __global__ void __launch_bounds__(kQuantThreads)
     }
     return;
   }
-  // Channel maxima of V over one chunk of rows: thread t owns channels
-  // t, t + 128, ... (D <= 128: one channel per thread) and walks the rows.
+  // Channel maxima of V over one chunk of rows: each thread takes 8
+  // channels of every RPP-th row (16-byte loads), then the row groups are
+  // combined through shared memory.
+  __shared__ float vm[RPP][D];
   const int64_t nch = (N + kVChunk - 1) / kVChunk;
   const int64_t g = cta - q_ctas - k_ctas;  // bh * nch + chunk
   const int64_t bh = g / nch;
   const int r0 = (int)(g % nch) * kVChunk, r1 = min(N, r0 + kVChunk);
+  const __nv_bfloat16* X = V + bh * (int64_t)N * D;
+  float m8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int r = r0 + lr; r < r1; r += RPP) {
+    const uint4 u = *reinterpret_cast<const uint4*>(X + (int64_t)r * D + c0);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      m8[2 * j] = fmaxf(m8[2 * j], fabsf(f.x));
+      m8[2 * j + 1] = fmaxf(m8[2 * j + 1], fabsf(f.y));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) vm[lr][c0 + j] = m8[j];
+  __syncthreads();
   if (tid < D) {
-    const __nv_bfloat16* X = V + bh * (int64_t)N * D + tid;
     float amax = 0.0f;
-    for (int r = r0; r < r1; ++r) amax = fmaxf(amax, fabsf(__bfloat162float(X[(int64_t)r * D])));
+#pragma unroll
+    for (int k = 0; k < RPP; ++k) amax = fmaxf(amax, vm[k][tid]);
     vpart[g * D + tid] = amax;
   }
 }

@@ -422,8 +422,10 @@ int oracle_attention_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* 
 //   * P: e4m3 relative to a running integer log2 maximum, in the order the
 //     kept key tiles (64 keys, ascending blocks) are visited:
 //       x_j   = float(S_j) * c, c = float(log2(e)/sqrt(d)) / (s_q * s_k) in float;
-//       m     = max(m, ceil(max_j x_j)) per tile, the accumulators scaled by
-//               2^(m_old - m_new) (exact) when m grows;
+//       m     = ceil(max_j x_j) of the first tile; afterwards it moves up to
+//               a tile's ceil(max_j x_j) only when that exceeds m + 8, the
+//               accumulators then scaled by 2^(m_old - m_new) (exact), so
+//               every e_j <= 2^8 stays inside e4m3's range;
 //       e_j   = 2^(x_j - m), x_j - m in float; p_j = e4m3(e_j);
 //       l += e_j (the normaliser is not quantised: only the operands of the
 //       two products are); acc += p_j v8_j;
@@ -554,13 +556,15 @@ int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_
           x[j - key0] = static_cast<float>(S) * c;
           mt = std::max(mt, x[j - key0]);
         }
-        const float m_new = std::max(m, std::ceil(mt));
-        if (m_new > m && l > 0.0) {
-          const double f = std::exp2(static_cast<double>(m - m_new));
+        const float cm = std::ceil(mt);
+        if (m == -std::numeric_limits<float>::infinity()) {
+          m = cm;
+        } else if (cm > m + 8.0f) {
+          const double f = std::exp2(static_cast<double>(m - cm));
           l *= f;
           for (int cc = 0; cc < d; ++cc) acc[cc] *= f;
+          m = cm;
         }
-        m = m_new;
         for (int64_t j = key0; j < key1; ++j) {
           const float y = x[j - key0] - m;
           const double ej = std::exp2(static_cast<double>(y));
