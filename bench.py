@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="480p", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="bf16", choices=["bf16", "q8"],
+                    help="q8: the low-bit sparse branch (int8 Q/K codes, e4m3 P and V), no linear branch")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -169,7 +171,7 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
-def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1):
+def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16"):
     """Times the oracle on a bounded sample: the mask of `heads` head(s) and the
     attention of `n_qblocks` query blocks of the first head, and returns
     (effective FLOP/s, description, threads)."""
@@ -182,9 +184,12 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1):
     t_mask = time.perf_counter() - t0
     qbs = np.linspace(0, w.nqb - 1, n_qblocks).astype(np.int64)
     rows = np.concatenate([np.arange(qb * w.bq, min(w.N, qb * w.bq + w.bq)) for qb in qbs]).astype(np.int64)
-    mode = "sla2" if w.sla2 else "sparse"
+    mode = "q8" if variant == "q8" else ("sla2" if w.sla2 else "sparse")
     t0 = time.perf_counter()
-    oracle.attention_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, alpha[:heads].numpy(), mode=mode, rows=rows)
+    if mode == "q8":
+        oracle.attention_q8_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, rows)
+    else:
+        oracle.attention_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, alpha[:heads].numpy(), mode=mode, rows=rows)
     t_attn = time.perf_counter() - t0
     flops = 0.0
     for qb in qbs:
@@ -205,7 +210,7 @@ def run_reference(args, w, rank, world):
     Q, K, V, alpha = synth.make_workload(w, heads=[(0, 0)])
     vals = []
     for i in range(args.warmup + args.steps):
-        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4)
+        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4, variant=args.variant)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals) / 1e12
@@ -214,7 +219,9 @@ def run_reference(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
-                   "topk": w.topk, "topp": w.topp},
+                   "topk": w.topk, "topp": w.topp,
+                   "path": "oracle: low-bit sparse branch" if args.variant == "q8" else
+                           ("oracle: sparse + linear mix" if w.sla2 else "oracle: sparse branch")},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -234,8 +241,12 @@ def run_ours(args, w, rank, world, local_rank):
     B, H, N, d = Q.shape
     shape = sparge.make_shape(Q, w.bq, w.bk)
     ws_mask = torch.empty(max(1, sparge.workspace_bytes(sparge.OP_MASK, shape)), dtype=torch.uint8, device=dev)
-    n_sla2 = sparge.workspace_bytes(sparge.OP_SLA2, shape) if w.sla2 else 0
+    q8 = args.variant == "q8"
+    sla2 = w.sla2 and not q8  # the low-bit variant is the sparse branch alone
+    n_sla2 = sparge.workspace_bytes(sparge.OP_SLA2, shape) if sla2 else 0
     ws_sla2 = torch.empty(max(1, n_sla2), dtype=torch.uint8, device=dev)
+    n_q8 = sparge.workspace_bytes(sparge.OP_ATTN_Q8, shape) if q8 else 0
+    ws_q8 = torch.empty(max(1, n_q8), dtype=torch.uint8, device=dev)
     kv_idx = torch.empty((B, H, w.nqb, w.nkb), dtype=torch.int32, device=dev)
     kv_cnt = torch.empty((B, H, w.nqb), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
@@ -245,14 +256,17 @@ def run_ours(args, w, rank, world, local_rank):
         sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
         if ev_a is not None:
             ev_a.record(stream)
-        if w.sla2:
+        if q8:
+            sparge.sparge_attn_fwd_q8(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, workspace=ws_q8)
+        elif sla2:
             sparge.sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, w.bq, w.bk, O=O, workspace=ws_sla2)
         else:
             sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O)
         if ev_b is not None:
             ev_b.record(stream)
 
-    launches_per_step = sparge.MASK_LAUNCHES + (sparge.SLA2_LAUNCHES if w.sla2 else sparge.ATTN_LAUNCHES)
+    launches_per_step = sparge.MASK_LAUNCHES + (sparge.Q8_LAUNCHES if q8 else
+                                                sparge.SLA2_LAUNCHES if sla2 else sparge.ATTN_LAUNCHES)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -313,23 +327,30 @@ def run_ours(args, w, rank, world, local_rank):
     burst = clocks["sm_mhz"] is not None and clocks["sm_max_mhz"] and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
     peak = float(peaks["bf16_tflops"] if burst else peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     peak_desc = f"{peak_kind} bf16 {'burst (SM clock at max during the timed region)' if burst else 'sustained'}"
+    if q8:
+        # int8 and e4m3 MMAs: the measured bf16 peak times the nominal 8-bit / bf16 ratio (4.5 / 2.25).
+        peak *= 2.0
+        peak_desc += " x 2 (nominal int8 / e4m3 to bf16 ratio)"
     achieved = flops / (attn_avg * 1e-3) / 1e12
     # The timed span is one library call: attn_fwd_kernel alone for the pure
     # sparse path; linear_summary + linear_reduce + attn_fwd_kernel<128, 1>
     # for the sparse + linear mix (the attention kernel is about 96% of it).
-    kernel_name = f"attn_fwd_kernel<{d}, 1>" if w.sla2 else f"attn_fwd_kernel<{d}, 0>"
-    span = "sla2_attn_fwd (3 launches)" if w.sla2 else "sparge_attn_fwd (1 launch)"
-    traffic = dram_traffic(w.name, kernel_name)
+    kernel_name = "attn_q8_kernel" if q8 else (f"attn_fwd_kernel<{d}, 1>" if sla2 else f"attn_fwd_kernel<{d}, 0>")
+    span = ("sparge_attn_fwd_q8 (3 launches: codes, V codes, attention)" if q8 else
+            "sla2_attn_fwd (4 launches)" if sla2 else "sparge_attn_fwd (1 launch)")
+    traffic = dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h)
+        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant)
         cpu = {"value": v / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-shaped Q/K/V, see synth.py)",
+        "vs_baseline": None, "dtype": "int8+e4m3" if q8 else "bf16",
+        "data": "synthetic (seeded video-shaped Q/K/V, see synth.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
-                   "topk": w.topk, "topp": w.topp, "alpha": "U[0.6,1] per head" if w.sla2 else 1.0,
+                   "topk": w.topk, "topp": w.topp, "alpha": "U[0.6,1] per head" if sla2 else 1.0,
+                   "path": "sparge_attn_fwd_q8" if q8 else ("sla2_attn_fwd" if sla2 else "sparge_attn_fwd"),
                    "l2": f"inputs larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V per rank)",
                    "parallelism": f"independent replicas x{world}"},
         "kept_fraction": flops / dense_flops,

@@ -50,13 +50,14 @@ def _load():
         lib.oracle_mask.argtypes = [p, p, i64, i64, i32, i32, i32, dbl, dbl, i32, p, p, p]
         lib.oracle_attention_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, i32,
                                               p, i64, p, p]
+        lib.oracle_mask_router.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, i64, i32, dbl, dbl, i32, p, p, p]
         lib.oracle_quant_q8.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         lib.oracle_e4m3.argtypes = [p, i64, p]
         lib.oracle_attention_q8_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, p]
         for f in (lib.oracle_pool_f64, lib.oracle_pool_f32, lib.oracle_block_probs_f64,
                   lib.oracle_block_probs_f32, lib.oracle_select_row, lib.oracle_mask,
                   lib.oracle_attention_rows, lib.oracle_quant_q8, lib.oracle_e4m3,
-                  lib.oracle_attention_q8_rows):
+                  lib.oracle_attention_q8_rows, lib.oracle_mask_router):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -144,6 +145,27 @@ def mask(Q, K, bq: int, bk: int, topk: float, topp: float, precision: int = 32):
     P = np.zeros((B, H, nqb, nkb), np.float64)
     _check(_load().oracle_mask(_ptr(q), _ptr(k), B * H, N, d, bq, bk, float(topk), float(topp),
                                precision, _ptr(kv_idx), _ptr(kv_cnt), _ptr(P)), "mask")
+    return kv_idx, kv_cnt, P
+
+
+def mask_router(Q, K, bq: int, bk: int, Wq, Wk, topk: float, topp: float, precision: int = 32):
+    """Block mask with a learnt router: pooled blocks projected by Wq / Wk
+    (float32 [H, d, dr], one pair per head) before scoring.
+
+    Returns (kv_idx, kv_cnt, P) like mask()."""
+    q, k = _bits(Q), _bits(K)
+    B, H, N, d = q.shape
+    wq = np.ascontiguousarray(np.asarray(Wq), np.float32)
+    wk = np.ascontiguousarray(np.asarray(Wk), np.float32)
+    assert wq.shape == wk.shape and wq.shape[:2] == (H, d), (wq.shape, wk.shape)
+    dr = wq.shape[2]
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx = np.zeros((B, H, nqb, nkb), np.int32)
+    kv_cnt = np.zeros((B, H, nqb), np.int32)
+    P = np.zeros((B, H, nqb, nkb), np.float64)
+    _check(_load().oracle_mask_router(_ptr(q), _ptr(k), B * H, N, d, bq, bk, _ptr(wq), _ptr(wk), H, dr,
+                                      float(topk), float(topp), precision, _ptr(kv_idx), _ptr(kv_cnt), _ptr(P)),
+           "mask_router")
     return kv_idx, kv_cnt, P
 
 

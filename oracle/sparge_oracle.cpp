@@ -250,24 +250,76 @@ int oracle_select_row(const double* P, int64_t Nkb, double topk, double topp, in
 // valid, ascending), kv_cnt [B*H, Nqb]. precision: 32 (the kernel's decision
 // precision) or 64 (the double definition). P_out: optional [B*H, Nqb, Nkb].
 // ---------------------------------------------------------------------------
-int oracle_mask(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int d, int bq,
-                int bk, double topk, double topp, int precision, int32_t* kv_idx,
-                int32_t* kv_cnt, double* P_out) {
+// ---------------------------------------------------------------------------
+// Block mask with a learnt router [SLA2 s2]: the article replaces the
+// heuristic routing by a router with two learnable projection matrices that
+// map the query and key features into a space suited to the routing
+// decision. Reading: the pooled block vectors are projected,
+//   qhat_I = qbar_I Wq_h,  khat_J = kbar_J Wk_h   (W: [d, dr] per head h),
+// and the block importance is softmax_J(qhat_I . khat_J / sqrt(dr)), followed
+// by the same hybrid selection. Single precision: each projected entry is a
+// sequential fused multiply-add over the d input channels in order.
+// Wq / Wk: fp32 [H, d, dr] (row c, column c'); H = BH / (heads per batch).
+// ---------------------------------------------------------------------------
+int oracle_mask_router(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int d, int bq, int bk,
+                       const float* Wq, const float* Wk, int64_t H, int dr, double topk, double topp, int precision,
+                       int32_t* kv_idx, int32_t* kv_cnt, double* P_out) {
   if (!Q || !K || !kv_idx || !kv_cnt || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
   if (precision != 32 && precision != 64) return ERR_ARG;
+  const bool routed = Wq != nullptr || Wk != nullptr;
+  if (routed && (!Wq || !Wk || H <= 0 || BH % H != 0 || dr <= 0)) return ERR_ARG;
+  const int dd = routed ? dr : d;
   const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
   std::vector<double> P(static_cast<size_t>(BH * Nqb * Nkb));
   if (precision == 64) {
     std::vector<double> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
     oracle_pool_f64(Q, BH, N, d, bq, qb.data());
     oracle_pool_f64(K, BH, N, d, bk, kb.data());
-    oracle_block_probs_f64(qb.data(), kb.data(), BH, Nqb, Nkb, d, P.data());
+    if (routed) {
+      std::vector<double> qh(static_cast<size_t>(BH * Nqb * dr)), kh(static_cast<size_t>(BH * Nkb * dr));
+      for (int pass = 0; pass < 2; ++pass) {
+        const std::vector<double>& in = pass == 0 ? qb : kb;
+        std::vector<double>& out = pass == 0 ? qh : kh;
+        const float* W = pass == 0 ? Wq : Wk;
+        const int64_t nb = pass == 0 ? Nqb : Nkb;
+        for (int64_t bh = 0; bh < BH; ++bh)
+          for (int64_t I = 0; I < nb; ++I)
+            for (int c2 = 0; c2 < dr; ++c2) {
+              double acc = 0.0;
+              for (int c = 0; c < d; ++c)
+                acc += in[(bh * nb + I) * d + c] * static_cast<double>(W[((bh % H) * d + c) * dr + c2]);
+              out[(bh * nb + I) * dr + c2] = acc;
+            }
+      }
+      oracle_block_probs_f64(qh.data(), kh.data(), BH, Nqb, Nkb, dd, P.data());
+    } else {
+      oracle_block_probs_f64(qb.data(), kb.data(), BH, Nqb, Nkb, dd, P.data());
+    }
   } else {
     std::vector<float> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
     std::vector<float> Pf(P.size());
     oracle_pool_f32(Q, BH, N, d, bq, qb.data());
     oracle_pool_f32(K, BH, N, d, bk, kb.data());
-    oracle_block_probs_f32(qb.data(), kb.data(), BH, Nqb, Nkb, d, Pf.data());
+    if (routed) {
+      std::vector<float> qh(static_cast<size_t>(BH * Nqb * dr)), kh(static_cast<size_t>(BH * Nkb * dr));
+      for (int pass = 0; pass < 2; ++pass) {
+        const std::vector<float>& in = pass == 0 ? qb : kb;
+        std::vector<float>& out = pass == 0 ? qh : kh;
+        const float* W = pass == 0 ? Wq : Wk;
+        const int64_t nb = pass == 0 ? Nqb : Nkb;
+        for (int64_t bh = 0; bh < BH; ++bh)
+          for (int64_t I = 0; I < nb; ++I)
+            for (int c2 = 0; c2 < dr; ++c2) {
+              float acc = 0.0f;
+              for (int c = 0; c < d; ++c)
+                acc = std::fma(in[(bh * nb + I) * d + c], W[((bh % H) * d + c) * dr + c2], acc);
+              out[(bh * nb + I) * dr + c2] = acc;
+            }
+      }
+      oracle_block_probs_f32(qh.data(), kh.data(), BH, Nqb, Nkb, dd, Pf.data());
+    } else {
+      oracle_block_probs_f32(qb.data(), kb.data(), BH, Nqb, Nkb, dd, Pf.data());
+    }
     for (size_t i = 0; i < P.size(); ++i) P[i] = static_cast<double>(Pf[i]);
   }
   for (int64_t row = 0; row < BH * Nqb; ++row) {
@@ -280,6 +332,14 @@ int oracle_mask(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int
   }
   if (P_out) std::memcpy(P_out, P.data(), P.size() * sizeof(double));
   return OK;
+}
+
+// Block mask without a router: pooled vectors scored directly.
+int oracle_mask(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int d, int bq,
+                int bk, double topk, double topp, int precision, int32_t* kv_idx,
+                int32_t* kv_cnt, double* P_out) {
+  return oracle_mask_router(Q, K, BH, N, d, bq, bk, nullptr, nullptr, 0, 0, topk, topp, precision, kv_idx, kv_cnt,
+                            P_out);
 }
 
 // ---------------------------------------------------------------------------

@@ -459,3 +459,53 @@ def test_q8_close_to_exact_sparse_attention(oracle_mod):
     rel = np.abs(a - e).sum() / np.abs(e).sum()
     assert rel < 0.06, rel
     assert rel > 1e-4  # the quantisation is really applied
+
+
+# ----------------------------------------------------------------------------- learnt router
+def _router_inputs(seed, H=2, N=2048, d=64, s=1.5):
+    Q, K, V = synth.make_qkv(1, H, N, d, grid=(2, 32, 32), s=s, seed=seed)
+    return Q, K
+
+
+def test_router_identity_projection_is_the_plain_mask(oracle_mod):
+    Q, K = _router_inputs(50)
+    I = np.tile(np.eye(64, dtype=np.float32), (2, 1, 1))
+    for precision in (32, 64):
+        a = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=precision)
+        b = oracle_mod.mask_router(Q, K, 64, 64, I, I, 0.1, 0.9, precision=precision)
+        for x, y in zip(a, b):
+            np.testing.assert_array_equal(x, y)
+
+
+def test_router_probabilities_match_projected_softmax(oracle_mod):
+    Q, K = _router_inputs(51)
+    g = np.random.default_rng(5)
+    Wq = g.standard_normal((2, 64, 32)).astype(np.float32) / 8
+    Wk = g.standard_normal((2, 64, 32)).astype(np.float32) / 8
+    _, _, P = oracle_mod.mask_router(Q, K, 64, 64, Wq, Wk, 0.1, 0.9, precision=64)
+    qb = oracle_mod.pool(Q, 64, precision=64)[0]  # [H, Nqb, d]
+    kb = oracle_mod.pool(K, 64, precision=64)[0]
+    for h in range(2):
+        z = (qb[h] @ Wq[h].astype(np.float64)) @ (kb[h] @ Wk[h].astype(np.float64)).T / math.sqrt(32)
+        ref = torch.softmax(torch.from_numpy(z), dim=-1).numpy()
+        np.testing.assert_allclose(P[0, h], ref, rtol=1e-10, atol=1e-15)
+
+
+def test_router_orthogonal_projection_keeps_the_probabilities(oracle_mod):
+    Q, K = _router_inputs(52)
+    R = np.linalg.qr(np.random.default_rng(6).standard_normal((64, 64)))[0].astype(np.float32)
+    W = np.stack([R, R])
+    _, _, P0 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=64)
+    _, _, P1 = oracle_mod.mask_router(Q, K, 64, 64, W, W, 0.1, 0.9, precision=64)
+    np.testing.assert_allclose(P1, P0, rtol=1e-5, atol=1e-9)  # R R^T = I up to the fp32 rounding of R
+
+
+def test_router_power_of_two_rescaling_is_exact(oracle_mod):
+    Q, K = _router_inputs(53)
+    g = np.random.default_rng(7)
+    Wq = g.standard_normal((2, 64, 64)).astype(np.float32) / 8
+    Wk = g.standard_normal((2, 64, 64)).astype(np.float32) / 8
+    a = oracle_mod.mask_router(Q, K, 64, 64, Wq, Wk, 0.1, 0.9, precision=32)
+    b = oracle_mod.mask_router(Q, K, 64, 64, Wq * 2, Wk / 2, 0.1, 0.9, precision=32)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
