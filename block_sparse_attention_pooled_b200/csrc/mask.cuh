@@ -79,6 +79,52 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ----------------------------------------------------------------------------
+// Learnt router (SLA2 article, arXiv:2602.12675, section 2: a router with two
+// learnable projection matrices maps the query and key features into a space
+// suited to the routing decision): pooled block vectors are projected,
+//   out[g, c'] = sum_c in[g, c] * W_h[c, c'],  W_h = W + h * D * DR,
+// each entry a sequential fused multiply-add over c in order. One CTA = up to
+// 32 pooled blocks of one (b, h) (CTA = bh * chunks + chunk), so every row uses
+// the same W_h; thread t computes column t % DR for rows t / DR, t / DR + G,
+// ... (G = 128 / DR row groups), reading each W_h entry once per CTA.
+// ----------------------------------------------------------------------------
+constexpr int kProjRows = 32;
+
+template <int D, int DR>
+__global__ void __launch_bounds__(128) project_kernel(const float* __restrict__ in, int64_t nb, int H,
+                                                      const float* __restrict__ W, float* __restrict__ out) {
+  constexpr int G = 128 / DR, RPT = kProjRows / G;  // row groups, rows per thread
+  __shared__ __align__(16) float sx[kProjRows][D];
+  const int64_t chunks = (nb + kProjRows - 1) / kProjRows;
+  const int64_t bh = blockIdx.x / chunks;
+  const int64_t r0 = (blockIdx.x % chunks) * kProjRows;
+  const int nr = (int)(nb - r0 < kProjRows ? nb - r0 : kProjRows);
+  const float* src = in + (bh * nb + r0) * D;
+  for (int e = threadIdx.x; e < kProjRows * (D / 4); e += 128) {
+    const int r = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < nr) v = *reinterpret_cast<const float4*>(src + (int64_t)r * D + c4);
+    *reinterpret_cast<float4*>(&sx[r][c4]) = v;
+  }
+  __syncthreads();
+  const int col = threadIdx.x % DR, grp = threadIdx.x / DR;
+  const float* w = W + (bh % H) * D * DR + col;
+  float acc[RPT];
+#pragma unroll
+  for (int k = 0; k < RPT; ++k) acc[k] = 0.0f;
+#pragma unroll 4
+  for (int c = 0; c < D; ++c) {
+    const float wc = __ldg(w + c * DR);
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) acc[k] = __fmaf_rn(sx[grp + k * G][c], wc, acc[k]);
+  }
+  float* dst = out + (bh * nb + r0) * DR + col;
+#pragma unroll
+  for (int k = 0; k < RPT; ++k)
+    if (grp + k * G < nr) dst[(int64_t)(grp + k * G) * DR] = acc[k];
+}
+
+// ----------------------------------------------------------------------------
 // Scaled scores z[I, J] = (q̄_I . k̄_J) * (float)(1/sqrt(d)). One CTA = 32
 // query-block rows x 64 key blocks of one (b,h); each thread owns 4 rows x 4
 // key blocks (8 shared-memory vector loads per 64 fused multiply-adds) and

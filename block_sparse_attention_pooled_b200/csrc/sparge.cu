@@ -66,6 +66,24 @@ MaskWs mask_ws(const sparge_shape* s, const Dims& d) {
   return w;
 }
 
+// The router's scratch: the mask's, then the projected blocks q^ and k^
+// (sized for the widest supported router width).
+constexpr int kMaxRouterDim = 128;
+
+struct RouterWs {
+  MaskWs mask;
+  size_t qhat, khat, total;
+};
+
+RouterWs router_ws(const sparge_shape* s, const Dims& d) {
+  RouterWs w;
+  w.mask = mask_ws(s, d);
+  w.qhat = w.mask.total;
+  w.khat = w.qhat + align256((size_t)d.BH * d.nqb * kMaxRouterDim * 4);
+  w.total = w.khat + align256((size_t)d.BH * d.nkb * kMaxRouterDim * 4);
+  return w;
+}
+
 // ---------------------------------------------------------------------------
 // TMA descriptors through the driver entry point (no link-time libcuda).
 // ---------------------------------------------------------------------------
@@ -114,10 +132,34 @@ cudaError_t ensure_smem(K kernel, int bytes, int slot) {
   return e;
 }
 
+// Scores of DD-wide pooled (or projected) vectors into P.
+template <int DD>
+cudaError_t launch_scores(const float* a, const float* b, const Dims& dm, float* P, cudaStream_t st) {
+  const float scale = (float)(1.0 / std::sqrt((double)DD));
+  const int ssm = score_smem_bytes<DD>();
+  cudaError_t e = ensure_smem(score_kernel<DD>, ssm, DD == 64 ? 0 : 1);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows) * ceil_div(dm.nkb, kScoreTileJ);
+  score_kernel<DD><<<(unsigned)tiles, 128, ssm, st>>>(a, b, (int)dm.nqb, (int)dm.nkb, scale, P);
+  return cudaGetLastError();
+}
+
+// Router projections of the pooled vectors (DR output columns).
+template <int D, int DR>
+void launch_projection(const float* qbar, const float* kbar, const Dims& dm, int H, const float* Wq, const float* Wk,
+                       float* qhat, float* khat, cudaStream_t st) {
+  const unsigned gq = (unsigned)(ceil_div(dm.nqb, kProjRows) * dm.BH);
+  const unsigned gk = (unsigned)(ceil_div(dm.nkb, kProjRows) * dm.BH);
+  project_kernel<D, DR><<<gq, 128, 0, st>>>(qbar, dm.nqb, H, Wq, qhat);
+  project_kernel<D, DR><<<gk, 128, 0, st>>>(kbar, dm.nkb, H, Wk, khat);
+}
+
+// Pool, (project,) score, select. Wq / Wk null: no router.
 template <int D>
 sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, const Dims& dm, int kc, double topp,
                           int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs, uint8_t* ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, const float* Wq = nullptr, const float* Wk = nullptr, int dr = 0,
+                          float* qhat = nullptr, float* khat = nullptr) {
   const MaskWs w = mask_ws(s, dm);
   float* qbar = reinterpret_cast<float*>(ws + w.qbar);
   float* kbar = reinterpret_cast<float*>(ws + w.kbar);
@@ -127,13 +169,21 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
   pool_kernel<D><<<(unsigned)(gq + gk), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(Q),
                                                      static_cast<const __nv_bfloat16*>(K), dm.BH, s->N, s->bq,
                                                      s->bk, gq, qbar, kbar);
-  const float scale = (float)(1.0 / std::sqrt((double)D));
-  const int ssm = score_smem_bytes<D>();
-  cudaError_t e = ensure_smem(score_kernel<D>, ssm, D == 64 ? 0 : 1);
-  if (e != cudaSuccess) return cuda_status(e);
   const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows) * ceil_div(dm.nkb, kScoreTileJ);
   if (tiles > INT32_MAX) return SPARGE_ERR_UNSUPPORTED;
-  score_kernel<D><<<(unsigned)tiles, 128, ssm, st>>>(qbar, kbar, (int)dm.nqb, (int)dm.nkb, scale, P);
+  cudaError_t e;
+  if (Wq != nullptr) {
+    if (dr == 64) {
+      launch_projection<D, 64>(qbar, kbar, dm, s->H, Wq, Wk, qhat, khat, st);
+      e = launch_scores<64>(qhat, khat, dm, P, st);
+    } else {
+      launch_projection<D, 128>(qbar, kbar, dm, s->H, Wq, Wk, qhat, khat, st);
+      e = launch_scores<128>(qhat, khat, dm, P, st);
+    }
+  } else {
+    e = launch_scores<D>(qbar, kbar, dm, P, st);
+  }
+  if (e != cudaSuccess) return cuda_status(e);
   const int sel_sm = select_smem_bytes((int)dm.nkb);
   e = ensure_smem(select_kernel, sel_sm, 2);
   if (e != cudaSuccess) return cuda_status(e);
@@ -354,6 +404,8 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
       return shape->d == 128 ? sla2_ws(shape, dm).total : 0;
     case SPARGE_OP_ATTN_Q8:
       return shape->d == 128 ? q8_ws(shape, dm).total : 0;
+    case SPARGE_OP_MASK_ROUTER:
+      return router_ws(shape, dm).total;
     default:
       return 0;
   }
@@ -380,6 +432,37 @@ sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shap
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (shape->d == 64) return launch_mask<64>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
   return launch_mask<128>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s);
+}
+
+sparge_status sparge_mask_router(const void* Q, const void* K, const sparge_shape* shape, const float* Wq,
+                                 const float* Wk, int dr, double topk_frac, double topp, int32_t* kv_idx,
+                                 int32_t* kv_cnt, float* row_thresh, float* probs, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !Wq || !Wk || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || (probs && !aligned16(probs))) return SPARGE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(Wq) & 3u) || (reinterpret_cast<uintptr_t>(Wk) & 3u)) return SPARGE_ERR_INVALID_ARG;
+  if (!(topk_frac >= 0.0 && topk_frac <= 1.0) || !(topp >= 0.0 && topp <= 1.0)) return SPARGE_ERR_INVALID_ARG;
+  if (dr != 64 && dr != 128) return SPARGE_ERR_UNSUPPORTED;
+  const RouterWs w = router_ws(shape, dm);
+  if (workspace == nullptr || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
+  int kc = 0;
+  if (topk_frac > 0.0) {
+    const double c = std::ceil(topk_frac * (double)dm.nkb - 1e-9);
+    kc = (int)std::min<double>(std::max<double>(c, 0.0), (double)dm.nkb);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* qhat = reinterpret_cast<float*>(ws + w.qhat);
+  float* khat = reinterpret_cast<float*>(ws + w.khat);
+  if (shape->d == 64)
+    return launch_mask<64>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s, Wq, Wk, dr, qhat,
+                           khat);
+  return launch_mask<128>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s, Wq, Wk, dr, qhat,
+                          khat);
 }
 
 sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_shape* shape, double topk_frac,

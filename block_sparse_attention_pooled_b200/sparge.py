@@ -20,14 +20,15 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
-OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8 = 0, 1, 2, 3
+OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8, OP_MASK_ROUTER = 0, 1, 2, 3, 4
 
 # Kernel launches per call of each entry point (for launch accounting).
-MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES = 3, 1, 4, 3
+MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES, ROUTER_LAUNCHES = 3, 1, 4, 3, 5
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
-           "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8")
+           "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8",
+           "sparge_mask_router")
 
 
 class Shape(ctypes.Structure):
@@ -38,6 +39,8 @@ _vp, _sz, _dbl = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_double
 _lib.sparge_workspace_bytes.argtypes = [ctypes.c_int, ctypes.POINTER(Shape)]
 _lib.sparge_workspace_bytes.restype = _sz
 _lib.sparge_mask.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _dbl, _dbl, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sparge_mask_router.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _vp, _vp, ctypes.c_int, _dbl, _dbl, _vp, _vp,
+                                     _vp, _vp, _vp, _sz, _vp]
 _lib.sparge_mask_noalloc.argtypes = [_vp, _vp, ctypes.POINTER(Shape), _dbl, _dbl, _vp, _vp, _vp, _vp, _vp]
 _lib.sparge_mask_noalloc.restype = ctypes.c_int
 _lib.sparge_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -46,7 +49,7 @@ _lib.sparge_attn_fwd_q8.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _
 _lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 _lib.sparge_status_string.argtypes = [ctypes.c_int]
 _lib.sparge_status_string.restype = ctypes.c_char_p
-for _f in ("sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
+for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -119,6 +122,33 @@ def sparge_mask(Q, K, bq: int, bk: int, topk: float, topp: float, kv_idx=None, k
     _check(_lib.sparge_mask(_ptr(Q), _ptr(K), ctypes.byref(shape), float(topk), float(topp), _ptr(kv_idx),
                             _ptr(kv_cnt), _ptr(row_thresh), _ptr(probs), _ptr(workspace), nws, _stream(stream)),
            "sparge_mask")
+    return kv_idx, kv_cnt
+
+
+def sparge_mask_router(Q, K, Wq, Wk, bq: int, bk: int, topk: float, topp: float, kv_idx=None, kv_cnt=None,
+                       row_thresh=None, probs=None, workspace=None, stream=None):
+    """Block mask scored through the learnt router projections Wq, Wk (fp32 [H, d, dr]).
+    Returns (kv_idx, kv_cnt)."""
+    _check_qkv(Q, K)
+    H, d = Q.shape[1], Q.shape[3]
+    for W in (Wq, Wk):
+        if W.dtype != torch.float32 or not W.is_cuda or not W.is_contiguous() or W.dim() != 3 \
+                or W.shape[0] != H or W.shape[1] != d or W.shape != Wq.shape:
+            raise ValueError("Wq/Wk must be contiguous fp32 CUDA tensors of shape [H, d, dr]")
+    shape = make_shape(Q, bq, bk)
+    B, _, N, _ = Q.shape
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, H, nqb, nkb), dtype=torch.int32, device=Q.device)
+    if kv_cnt is None:
+        kv_cnt = torch.empty((B, H, nqb), dtype=torch.int32, device=Q.device)
+    if workspace is None:
+        workspace, nws = _workspace(OP_MASK_ROUTER, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sparge_mask_router(_ptr(Q), _ptr(K), ctypes.byref(shape), _ptr(Wq), _ptr(Wk), int(Wq.shape[2]),
+                                   float(topk), float(topp), _ptr(kv_idx), _ptr(kv_cnt), _ptr(row_thresh),
+                                   _ptr(probs), _ptr(workspace), nws, _stream(stream)), "sparge_mask_router")
     return kv_idx, kv_cnt
 
 

@@ -39,6 +39,7 @@ _N_SINUSOIDS = 16
 # Stream ids keep every tensor of every head reproducible on its own, so a
 # subset of heads can be regenerated without drawing the others.
 _STREAM_FIELD, _STREAM_EPS_Q, _STREAM_EPS_K, _STREAM_V, _STREAM_ALPHA = 1, 2, 3, 4, 5
+_STREAM_ROUTER_BASE, _STREAM_ROUTER_Q, _STREAM_ROUTER_K = 6, 7, 8
 
 
 @dataclasses.dataclass(frozen=True)
@@ -161,6 +162,31 @@ def make_alpha(H: int, seed: int = 0, sla2: bool = True) -> torch.Tensor:
         return torch.ones(H, dtype=torch.float32)
     rng = _rng(seed, 0, 0, _STREAM_ALPHA)
     return torch.from_numpy(rng.uniform(0.6, 1.0, size=H).astype(np.float32))
+
+
+def make_router(H: int, d: int, dr: int, seed: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Router projections Wq, Wk, float32 [H, d, dr], standing in for trained ones.
+
+    Per head: a random partial isometry (QR of a seeded Gaussian matrix:
+    orthonormal columns when dr <= d, orthonormal rows when dr > d), times
+    (max(d, dr) / min(d, dr))^(1/4) so that the projected dot products over
+    sqrt(dr) keep, on average, the scale of the pooled ones over sqrt(d),
+    plus independent N(0, 0.1^2/d) perturbations for Wq and Wk, so the two
+    differ."""
+    Wq = np.zeros((H, d, dr), np.float32)
+    Wk = np.zeros((H, d, dr), np.float32)
+    gain = (max(d, dr) / min(d, dr)) ** 0.25
+    for h in range(H):
+        g = _rng(seed, 0, h, _STREAM_ROUTER_BASE)
+        if dr <= d:
+            base = np.linalg.qr(g.standard_normal((d, dr)))[0]
+        else:
+            base = np.linalg.qr(g.standard_normal((dr, d)))[0].T
+        eq = _rng(seed, 0, h, _STREAM_ROUTER_Q).standard_normal((d, dr)) * (0.1 / math.sqrt(d))
+        ek = _rng(seed, 0, h, _STREAM_ROUTER_K).standard_normal((d, dr)) * (0.1 / math.sqrt(d))
+        Wq[h] = base * gain + eq
+        Wk[h] = base * gain + ek
+    return torch.from_numpy(Wq), torch.from_numpy(Wk)
 
 
 def make_workload(w: Workload, heads=None):

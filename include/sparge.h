@@ -1,8 +1,8 @@
 /*
  * sparge.h - C ABI of the pooled block-sparse attention library (sm_100a).
  *
- * Three operations, each one stream-ordered launch sequence on the caller's
- * CUDA stream:
+ * Each operation is one stream-ordered launch sequence on the caller's CUDA
+ * stream. The three of the hot path:
  *
  *   sparge_mask      block mask: mean-pool Q and K per block, score the
  *                    pooled blocks with softmax(qbar . kbar / sqrt(d)) along
@@ -22,6 +22,11 @@
  *                    SLA2 article, section 1 (sparse attention for important
  *                    regions, linear attention for the rest) and section 2
  *                    (learnable mixing ratio alpha).
+ *
+ * and three variants of them: sparge_mask_router (the mask scored through
+ * learnt projections of the pooled blocks, SLA2 article section 2),
+ * sparge_attn_fwd_q8 (the sparse branch on int8 / fp8 operand codes, SLA2
+ * article section 3) and sparge_mask_noalloc (the mask with a static scratch).
  *
  * Conventions shared by every entry point
  *   - Q, K, V, O: bf16, [B, H, N, d] contiguous (d fastest), device memory,
@@ -73,7 +78,13 @@ typedef struct {
   int32_t bq, bk;     /* query rows per block, keys per block */
 } sparge_shape;
 
-enum { SPARGE_OP_MASK = 0, SPARGE_OP_ATTN = 1, SPARGE_OP_SLA2 = 2, SPARGE_OP_ATTN_Q8 = 3 };
+enum {
+  SPARGE_OP_MASK = 0,
+  SPARGE_OP_ATTN = 1,
+  SPARGE_OP_SLA2 = 2,
+  SPARGE_OP_ATTN_Q8 = 3,
+  SPARGE_OP_MASK_ROUTER = 4
+};
 
 /* Workspace bytes the operation needs for this shape (0 if none, or if the
  * shape is invalid). */
@@ -98,6 +109,24 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape);
 sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shape, double topk_frac,
                           double topp, int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block mask through a learnt router (SLA2 article, arXiv:2602.12675,
+ * section 2: two learnable projections map the pooled query and key block
+ * features before they are scored). Same steps and outputs as sparge_mask,
+ * with one step added between pooling and scoring:
+ *   q^_I = q-bar_I . Wq_h,   k^_J = k-bar_J . Wk_h       (h = head of the row)
+ *   P[I, :] = softmax_J(q^_I . k^_J / sqrt(dr))
+ *   Wq, Wk      fp32 [H, d, dr] row-major, device, 4-byte aligned, read only;
+ *               the caller owns them (no copy is kept).
+ *   dr          router width: 64 or 128 (else SPARGE_ERR_UNSUPPORTED).
+ * Precision: each projected entry is one fp32 fused-multiply-add chain over
+ * the d channels in order; the rest as in sparge_mask.
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_MASK_ROUTER, shape) (pooled
+ * and projected blocks, probability rows), 256-byte aligned. */
+sparge_status sparge_mask_router(const void* Q, const void* K, const sparge_shape* shape, const float* Wq,
+                                 const float* Wk, int dr, double topk_frac, double topp, int32_t* kv_idx,
+                                 int32_t* kv_cnt, float* row_thresh, float* probs, void* workspace,
+                                 size_t workspace_bytes, void* stream);
 
 /* The same block mask as sparge_mask, for callers that cannot allocate
  * device memory: code hosted inside a framework or runtime that owns every

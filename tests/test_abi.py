@@ -59,6 +59,10 @@ def test_workspace_bytes_host_arithmetic(lib):
     need_q8 = lib.workspace_bytes(lib.OP_ATTN_Q8, s)
     assert need_q8 >= 3 * 40 * 75600 * 128 + 4 * 40 * (nqb + nkb + 128)
     assert lib.workspace_bytes(lib.OP_ATTN_Q8, lib.Shape(1, 1, 4096, 64, 64, 64)) == 0  # d = 128 only
+    # Learnt router: the mask's scratch plus the projected blocks at the widest router width.
+    need_r = lib.workspace_bytes(lib.OP_MASK_ROUTER, s)
+    assert need_r >= need + 40 * (nqb + nkb) * 128 * 4
+    assert lib.workspace_bytes(lib.OP_MASK_ROUTER, bad) == 0
 
 
 def test_invalid_arguments_rejected_before_any_launch(lib):
@@ -92,6 +96,24 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s128), P, P, P, None, 0, None) == lib.ERR_WORKSPACE
     assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s128), P, P, P, P, 64, None) == lib.ERR_WORKSPACE
     assert raw.sparge_attn_fwd_q8(P, None, P, ctypes.byref(s128), P, P, P, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    # Learnt router: both projections required, 4-byte aligned; dr 64 or 128; workspace sized for it.
+    W, big = ctypes.c_void_p(32 * 1024), 1 << 30
+    assert raw.sparge_mask_router(P, P, ctypes.byref(s), None, W, 64, 0.1, 0.9, P, P, None, None, P, big,
+                                  None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_mask_router(P, P, ctypes.byref(s), W, None, 64, 0.1, 0.9, P, P, None, None, P, big,
+                                  None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_mask_router(P, P, ctypes.byref(s), ctypes.c_void_p(32 * 1024 + 2), W, 64, 0.1, 0.9, P, P,
+                                  None, None, P, big, None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_mask_router(P, P, ctypes.byref(s), W, W, 64, 1.5, 0.9, P, P, None, None, P, big,
+                                  None) == lib.ERR_INVALID_ARG
+    for dr in (0, 32, 96, 256):
+        assert raw.sparge_mask_router(P, P, ctypes.byref(s), W, W, dr, 0.1, 0.9, P, P, None, None, P, big,
+                                      None) == lib.ERR_UNSUPPORTED
+    mask_only = lib.workspace_bytes(lib.OP_MASK, s)
+    assert raw.sparge_mask_router(P, P, ctypes.byref(s), W, W, 64, 0.1, 0.9, P, P, None, None, P, mask_only,
+                                  None) == lib.ERR_WORKSPACE
+    assert raw.sparge_mask_router(P, P, ctypes.byref(s), W, W, 64, 0.1, 0.9, P, P, None, None,
+                                  ctypes.c_void_p(16 * 1024 + 16), big, None) == lib.ERR_WORKSPACE
 
 
 def test_binding_refuses_cpu_tensors(lib):
@@ -100,3 +122,6 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         lib.sparge_mask(q, q, 64, 64, 0.1, 0.9)
+    w = torch.zeros(1, 64, 64, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        lib.sparge_mask_router(q, q, w, w, 64, 64, 0.1, 0.9)

@@ -509,3 +509,18 @@ def test_router_power_of_two_rescaling_is_exact(oracle_mod):
     b = oracle_mod.mask_router(Q, K, 64, 64, Wq * 2, Wk / 2, 0.1, 0.9, precision=32)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+def test_router_generator_is_a_scaled_partial_isometry():
+    # The stand-in router weights: seeded, fp32 [H, d, dr], and without their
+    # perturbation a partial isometry times the stated gain.
+    for d, dr in ((128, 64), (64, 128), (128, 128)):
+        Wq, Wk = synth.make_router(3, d, dr, seed=2)
+        assert Wq.shape == (3, d, dr) and Wq.dtype == torch.float32
+        a, b = synth.make_router(3, d, dr, seed=2)
+        assert torch.equal(a, Wq) and torch.equal(b, Wk)
+        gain = (max(d, dr) / min(d, dr)) ** 0.25
+        base = (Wq.double() + Wk.double()).numpy() / (2 * gain)  # perturbations average out partly
+        for h in range(3):
+            gram = base[h].T @ base[h] if dr <= d else base[h] @ base[h].T
+            assert np.abs(gram - np.eye(min(d, dr))).max() < 0.1
