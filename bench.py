@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="bf16", choices=["bf16", "q8"],
                     help="q8: the low-bit sparse branch (int8 Q/K codes, e4m3 P and V), no linear branch")
+    ap.add_argument("--router", type=int, default=0, choices=[0, 64, 128],
+                    help="score the mask through a learnt router of this width (seeded stand-in projections)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -138,11 +140,15 @@ def _smi_id(dev) -> str:
         return ids[dev.index].strip() if dev.index < len(ids) else str(dev.index)
 
 
-def kernel_source_sha() -> str:
-    """Digest of the CUDA sources, to tell whether stored counters still apply."""
+# Source files each timed kernel is built from (its own header and the PTX helpers).
+KERNEL_SOURCES = {"attn_fwd_kernel": ("attn.cuh", "ptx.cuh"), "attn_q8_kernel": ("attn_q8.cuh", "ptx.cuh")}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """Digest of the CUDA sources of one kernel, to tell whether stored counters still apply."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_attention_pooled_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel.split("<")[0]]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -156,7 +162,7 @@ def dram_traffic(workload: str, kernel: str):
         return None
     with open(path) as f:
         entry = json.load(f).get(workload)
-    if not entry or entry.get("kernel") != kernel or entry.get("csrc_sha") != kernel_source_sha():
+    if not entry or entry.get("kernel") != kernel or entry.get("csrc_sha") != kernel_source_sha(kernel):
         return None
     return entry["dram_bytes_per_launch"]
 
@@ -171,7 +177,7 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
-def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16"):
+def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=None):
     """Times the oracle on a bounded sample: the mask of `heads` head(s) and the
     attention of `n_qblocks` query blocks of the first head, and returns
     (effective FLOP/s, description, threads)."""
@@ -180,7 +186,11 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16"):
     oracle.build()
     Qh, Kh, Vh = Q[:1, :heads].contiguous(), K[:1, :heads].contiguous(), V[:1, :heads].contiguous()
     t0 = time.perf_counter()
-    idx, cnt, _ = oracle.mask(Qh, Kh, w.bq, w.bk, w.topk, w.topp, precision=32)
+    if router is None:
+        idx, cnt, _ = oracle.mask(Qh, Kh, w.bq, w.bk, w.topk, w.topp, precision=32)
+    else:
+        Wq, Wk = (W[:heads].numpy() for W in router)
+        idx, cnt, _ = oracle.mask_router(Qh, Kh, w.bq, w.bk, Wq, Wk, w.topk, w.topp, precision=32)
     t_mask = time.perf_counter() - t0
     qbs = np.linspace(0, w.nqb - 1, n_qblocks).astype(np.int64)
     rows = np.concatenate([np.arange(qb * w.bq, min(w.N, qb * w.bq + w.bq)) for qb in qbs]).astype(np.int64)
@@ -198,7 +208,7 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16"):
         flops += 4.0 * w.d * nrows * keys
     # the mask's time is charged pro rata to the sampled query blocks
     t = t_attn + t_mask * (len(qbs) / (w.nqb * heads))
-    desc = (f"oracle mask of {heads} head(s) ({t_mask:.2f} s, charged pro rata) + {mode} attention of "
+    desc = (f"oracle {'router ' if router is not None else ''}mask of {heads} head(s) ({t_mask:.2f} s, charged pro rata) + {mode} attention of "
             f"{len(qbs)} query blocks x {w.bq} rows ({t_attn:.2f} s); {w.name} workload")
     return flops / t, desc, 1
 
@@ -208,9 +218,10 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     Q, K, V, alpha = synth.make_workload(w, heads=[(0, 0)])
+    router = synth.make_router(w.H, w.d, args.router, seed=w.seed) if args.router else None
     vals = []
     for i in range(args.warmup + args.steps):
-        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4, variant=args.variant)
+        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4, variant=args.variant, router=router)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals) / 1e12
@@ -221,7 +232,8 @@ def run_reference(args, w, rank, world):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
                    "topk": w.topk, "topp": w.topp,
                    "path": "oracle: low-bit sparse branch" if args.variant == "q8" else
-                           ("oracle: sparse + linear mix" if w.sla2 else "oracle: sparse branch")},
+                           ("oracle: sparse + linear mix" if w.sla2 else "oracle: sparse branch"),
+                   "router": args.router or None},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -240,7 +252,10 @@ def run_ours(args, w, rank, world, local_rank):
     Q, K, V, alpha = Qh.to(dev), Kh.to(dev), Vh.to(dev), alpha_h.to(dev)
     B, H, N, d = Q.shape
     shape = sparge.make_shape(Q, w.bq, w.bk)
-    ws_mask = torch.empty(max(1, sparge.workspace_bytes(sparge.OP_MASK, shape)), dtype=torch.uint8, device=dev)
+    router_h = synth.make_router(H, d, args.router, seed=w.seed) if args.router else None
+    mask_op = sparge.OP_MASK_ROUTER if router_h is not None else sparge.OP_MASK
+    ws_mask = torch.empty(max(1, sparge.workspace_bytes(mask_op, shape)), dtype=torch.uint8, device=dev)
+    Wq, Wk = (router_h[0].to(dev), router_h[1].to(dev)) if router_h is not None else (None, None)
     q8 = args.variant == "q8"
     sla2 = w.sla2 and not q8  # the low-bit variant is the sparse branch alone
     n_sla2 = sparge.workspace_bytes(sparge.OP_SLA2, shape) if sla2 else 0
@@ -253,7 +268,11 @@ def run_ours(args, w, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     def step(ev_a=None, ev_b=None):
-        sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
+        if Wq is not None:
+            sparge.sparge_mask_router(Q, K, Wq, Wk, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt,
+                                      workspace=ws_mask)
+        else:
+            sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
         if ev_a is not None:
             ev_a.record(stream)
         if q8:
@@ -265,7 +284,7 @@ def run_ours(args, w, rank, world, local_rank):
         if ev_b is not None:
             ev_b.record(stream)
 
-    launches_per_step = sparge.MASK_LAUNCHES + (sparge.Q8_LAUNCHES if q8 else
+    launches_per_step = (sparge.ROUTER_LAUNCHES if Wq is not None else sparge.MASK_LAUNCHES) + (sparge.Q8_LAUNCHES if q8 else
                                                 sparge.SLA2_LAUNCHES if sla2 else sparge.ATTN_LAUNCHES)
     for _ in range(args.warmup):
         step()
@@ -338,10 +357,11 @@ def run_ours(args, w, rank, world, local_rank):
     kernel_name = "attn_q8_kernel" if q8 else (f"attn_fwd_kernel<{d}, 1>" if sla2 else f"attn_fwd_kernel<{d}, 0>")
     span = ("sparge_attn_fwd_q8 (3 launches: codes, V codes, attention)" if q8 else
             "sla2_attn_fwd (4 launches)" if sla2 else "sparge_attn_fwd (1 launch)")
-    traffic = dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
+    # Counters were captured with the plain mask; a router mask keeps other tiles.
+    traffic = None if args.router else dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant)
+        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant, router=router_h)
         cpu = {"value": v / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -351,6 +371,7 @@ def run_ours(args, w, rank, world, local_rank):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
                    "topk": w.topk, "topp": w.topp, "alpha": "U[0.6,1] per head" if sla2 else 1.0,
                    "path": "sparge_attn_fwd_q8" if q8 else ("sla2_attn_fwd" if sla2 else "sparge_attn_fwd"),
+                   "mask": f"sparge_mask_router (dr {args.router})" if args.router else "sparge_mask",
                    "l2": f"inputs larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V per rank)",
                    "parallelism": f"independent replicas x{world}"},
         "kept_fraction": flops / dense_flops,
