@@ -53,6 +53,8 @@ def _load():
         lib.oracle_mask_router.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, i64, i32, dbl, dbl, i32, p, p, p]
         lib.oracle_quant_q8.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         lib.oracle_e4m3.argtypes = [p, i64, p]
+        lib.oracle_attention_bwd.argtypes = [p, p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, i32, p, i64, p, i64,
+                                             p, p, p, p]
         lib.oracle_attention_q8_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, p]
         for f in (lib.oracle_pool_f64, lib.oracle_pool_f32, lib.oracle_block_probs_f64,
                   lib.oracle_block_probs_f32, lib.oracle_select_row, lib.oracle_mask,
@@ -192,6 +194,32 @@ def attention_rows(Q, K, V, bq: int, bk: int, kv_idx=None, kv_cnt=None, alpha=No
                                          _ptr(cnt), _ptr(al), H, MODES[mode], _ptr(rows),
                                          rows.shape[0], _ptr(O), _ptr(lse)), "attention_rows")
     return O, lse
+
+
+def attention_bwd(Q, K, V, dO, bq: int, bk: int, kv_idx=None, kv_cnt=None, alpha=None, mode: str = "sparse",
+                  rows=None, kblocks=None, want_dalpha: bool = False):
+    """Double-precision gradients of the forward of attention_rows for dL/dO = dO (bf16).
+
+    rows: flat query rows b*H*N + h*N + i whose dQ is wanted (default: all).
+    kblocks: flat key blocks (b*H + h)*Nkb + J whose dK, dV are wanted
+    (default: all). Returns (dQ [nrows,d], dK [nblocks,bk,d], dV [nblocks,bk,d],
+    dalpha [H] or None), float64; dK / dV rows past N are zero."""
+    q, k, v, g = _bits(Q), _bits(K), _bits(V), _bits(dO)
+    B, H, N, d = q.shape
+    nkb = -(-N // bk)
+    rows = np.arange(B * H * N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, np.int64)
+    kb = np.arange(B * H * nkb, dtype=np.int64) if kblocks is None else np.ascontiguousarray(kblocks, np.int64)
+    idx = None if kv_idx is None else np.ascontiguousarray(np.asarray(kv_idx), np.int32)
+    cnt = None if kv_cnt is None else np.ascontiguousarray(np.asarray(kv_cnt), np.int32)
+    al = None if alpha is None else np.ascontiguousarray(np.asarray(alpha), np.float32)
+    dQ = np.zeros((rows.shape[0], d), np.float64)
+    dK = np.zeros((kb.shape[0], bk, d), np.float64)
+    dV = np.zeros((kb.shape[0], bk, d), np.float64)
+    da = np.zeros(H, np.float64) if want_dalpha else None
+    _check(_load().oracle_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B * H, N, d, bq, bk, _ptr(idx),
+                                        _ptr(cnt), _ptr(al), H, MODES[mode], _ptr(rows), rows.shape[0], _ptr(kb),
+                                        kb.shape[0], _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(da)), "attention_bwd")
+    return dQ, dK, dV, da
 
 
 def e4m3(x) -> np.ndarray:

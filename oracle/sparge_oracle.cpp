@@ -642,3 +642,207 @@ int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_
 
 }  // extern "C"
 
+
+// ===========================================================================
+// Gradients [SA2 s1 (trainable sparse attention), SLA2 s2]: for a loss L with
+// dL/dO = dO, the gradients of Q, K, V (and of alpha) through the forward of
+// oracle_attention_rows, written out from the chain rule in double:
+//
+//   sparse branch (g_i = alpha * dO_i; alpha = 1 outside the mix):
+//     P_ij = softmax over the kept keys of s_ij = q_i.k_j / sqrt(d),
+//     O_s,i = sum_j P_ij v_j,
+//     dV_j += P_ij g_i,      dP_ij = g_i . v_j,
+//     dS_ij = P_ij (dP_ij - g_i . O_s,i),
+//     dQ_i += sum_j dS_ij k_j / sqrt(d),   dK_j += dS_ij q_i / sqrt(d);
+//   linear branch (h_i = (1 - alpha) dO_i; dO_i outside the mix), over the
+//   keys j outside the kept blocks, w_ij = phi(q_i).phi(k_j),
+//   den_i = sum_j w_ij, O_l,i = sum_j w_ij v_j / den_i:
+//     dV_j += (w_ij / den_i) h_i,
+//     dw_ij = h_i . (v_j - O_l,i) / den_i,
+//     dQ_i += (sum_j dw_ij phi(k_j)) * phi'(q_i),
+//     dK_j += dw_ij phi(q_i) * phi'(k_j),   phi'(x) = 1 (x > 0), e^x (x <= 0);
+//     an empty complement (O_l = 0 by the forward's reading) gives nothing;
+//   the mix: dalpha_h = sum over the rows of head h of dO_i . (O_s,i - O_l,i).
+//
+// mode as in oracle_attention_rows (0 sparse, 1 linear, 2 mix, 3 dense).
+// dO: bf16 bits [BH, N, d] (widened exactly). Outputs:
+//   dQ [n_rows, d] for the flat rows q_rows[] (bh*N + i), if dQ is not null;
+//   dK, dV [n_blocks, bk, d] for the flat key blocks k_blocks[] (bh*Nkb + J),
+//     rows past N zero, if dK / dV are not null;
+//   dalpha [H] (mode 2 only, summed over every row of every head) if not null.
+// Every query row that feeds a requested output is visited (for dK / dV:
+// the rows whose block keeps J, plus every row of the head in modes 1 and 2).
+// ===========================================================================
+extern "C" {
+
+int oracle_attention_bwd(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* dO, int64_t BH,
+                         int64_t N, int d, int bq, int bk, const int32_t* kv_idx, const int32_t* kv_cnt,
+                         const float* alpha, int64_t H, int mode, const int64_t* q_rows, int64_t n_rows,
+                         const int64_t* k_blocks, int64_t n_blocks, double* dQ, double* dK, double* dV,
+                         double* dalpha) {
+  if (!Q || !K || !V || !dO || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
+  if (mode < 0 || mode > 3) return ERR_ARG;
+  if (mode != 3 && (!kv_idx || !kv_cnt)) return ERR_ARG;
+  if (mode == 2 && (!alpha || H <= 0 || BH % H != 0)) return ERR_ARG;
+  if (dalpha && mode != 2) return ERR_ARG;
+  if ((n_rows > 0 && (!q_rows || !dQ)) || (n_blocks > 0 && (!k_blocks || (!dK && !dV)))) return ERR_ARG;
+  const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
+  const double scale = 1.0 / std::sqrt(static_cast<double>(d));
+  const bool use_s = mode != 1, use_l = mode == 1 || mode == 2;
+  for (int64_t t = 0; t < n_rows; ++t)
+    if (q_rows[t] < 0 || q_rows[t] >= BH * N) return ERR_ARG;
+  for (int64_t t = 0; t < n_blocks; ++t)
+    if (k_blocks[t] < 0 || k_blocks[t] >= BH * Nkb) return ERR_ARG;
+  if (dQ) std::fill(dQ, dQ + n_rows * d, 0.0);
+  if (dK) std::fill(dK, dK + n_blocks * bk * d, 0.0);
+  if (dV) std::fill(dV, dV + n_blocks * bk * d, 0.0);
+  if (dalpha) std::fill(dalpha, dalpha + H, 0.0);
+
+  // kept[J] of query block I of head bh.
+  auto kept_row = [&](int64_t bh, int64_t I, std::vector<char>& kept) -> bool {
+    if (mode == 3) {
+      std::fill(kept.begin(), kept.end(), 1);
+      return true;
+    }
+    std::fill(kept.begin(), kept.end(), 0);
+    const int64_t cnt = kv_cnt[bh * Nqb + I];
+    if (cnt < 0 || cnt > Nkb) return false;
+    for (int64_t e = 0; e < cnt; ++e) {
+      const int32_t J = kv_idx[(bh * Nqb + I) * Nkb + e];
+      if (J < 0 || J >= Nkb) return false;
+      kept[J] = 1;
+    }
+    return true;
+  };
+
+  std::vector<double> Kd, Vd, phiK, q(d), phiq(d), g(d), hl(d), s, w, Os(d), Ol(d), dq(d), dphiq(d);
+  std::vector<char> kept(Nkb), qkeep(Nkb);
+  std::vector<int64_t> qslot, kslot;
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    // Requested outputs of this head.
+    qslot.assign(static_cast<size_t>(N), -1);
+    kslot.assign(static_cast<size_t>(Nkb), -1);
+    bool any = dalpha != nullptr;
+    for (int64_t t = 0; t < n_rows; ++t)
+      if (q_rows[t] / N == bh) qslot[q_rows[t] % N] = t, any = true;
+    for (int64_t t = 0; t < n_blocks; ++t)
+      if (k_blocks[t] / Nkb == bh) kslot[k_blocks[t] % Nkb] = t, any = true;
+    if (!any) continue;
+    Kd.assign(static_cast<size_t>(N * d), 0.0);
+    Vd.assign(static_cast<size_t>(N * d), 0.0);
+    phiK.assign(static_cast<size_t>(N * d), 0.0);
+    for (int64_t e = 0; e < N * d; ++e) {
+      Kd[e] = widen(K[bh * N * d + e]);
+      Vd[e] = widen(V[bh * N * d + e]);
+      phiK[e] = phi(Kd[e]);
+    }
+    const double a = mode == 2 ? static_cast<double>(alpha[bh % H]) : 1.0;
+    for (int64_t i = 0; i < N; ++i) {
+      const int64_t I = i / bq;
+      if (!kept_row(bh, I, kept)) return ERR_ARG;
+      // Does this row feed anything requested?
+      bool feeds = dalpha != nullptr || qslot[i] >= 0;
+      for (int64_t J = 0; J < Nkb && !feeds; ++J)
+        if (kslot[J] >= 0 && ((use_s && kept[J]) || (use_l && !kept[J]))) feeds = true;
+      if (!feeds) continue;
+      for (int c = 0; c < d; ++c) {
+        q[c] = widen(Q[(bh * N + i) * d + c]);
+        phiq[c] = phi(q[c]);
+        const double go = widen(dO[(bh * N + i) * d + c]);
+        g[c] = mode == 2 ? a * go : go;
+        hl[c] = mode == 2 ? (1.0 - a) * go : go;
+      }
+      std::fill(dq.begin(), dq.end(), 0.0);
+      std::fill(Os.begin(), Os.end(), 0.0);
+      std::fill(Ol.begin(), Ol.end(), 0.0);
+      // Sparse branch: forward (two passes), then its gradients.
+      if (use_s) {
+        double mx = -std::numeric_limits<double>::infinity();
+        s.assign(static_cast<size_t>(N), 0.0);
+        for (int64_t j = 0; j < N; ++j) {
+          if (!kept[j / bk]) continue;
+          double dot = 0.0;
+          for (int c = 0; c < d; ++c) dot += q[c] * Kd[j * d + c];
+          s[j] = dot * scale;
+          mx = std::max(mx, s[j]);
+        }
+        if (mx > -std::numeric_limits<double>::infinity()) {
+          double l = 0.0;
+          for (int64_t j = 0; j < N; ++j)
+            if (kept[j / bk]) l += std::exp(s[j] - mx);
+          for (int64_t j = 0; j < N; ++j) {
+            if (!kept[j / bk]) continue;
+            s[j] = std::exp(s[j] - mx) / l;  // s now holds P_ij
+            for (int c = 0; c < d; ++c) Os[c] += s[j] * Vd[j * d + c];
+          }
+          double gO = 0.0;
+          for (int c = 0; c < d; ++c) gO += g[c] * Os[c];
+          for (int64_t j = 0; j < N; ++j) {
+            if (!kept[j / bk]) continue;
+            double dP = 0.0;
+            for (int c = 0; c < d; ++c) dP += g[c] * Vd[j * d + c];
+            const double dS = s[j] * (dP - gO);
+            for (int c = 0; c < d; ++c) dq[c] += dS * Kd[j * d + c] * scale;
+            const int64_t ks = kslot[j / bk];
+            if (ks >= 0) {
+              const int64_t r = (ks * bk + j % bk) * d;
+              for (int c = 0; c < d; ++c) {
+                if (dK) dK[r + c] += dS * q[c] * scale;
+                if (dV) dV[r + c] += s[j] * g[c];
+              }
+            }
+          }
+        }
+      }
+      // Linear branch over the complement: forward, then its gradients.
+      if (use_l) {
+        w.assign(static_cast<size_t>(N), 0.0);
+        double den = 0.0;
+        for (int64_t j = 0; j < N; ++j) {
+          if (kept[j / bk]) continue;
+          double x = 0.0;
+          for (int c = 0; c < d; ++c) x += phiq[c] * phiK[j * d + c];
+          w[j] = x;
+          den += x;
+        }
+        if (den > 0.0) {
+          for (int64_t j = 0; j < N; ++j) {
+            if (kept[j / bk]) continue;
+            for (int c = 0; c < d; ++c) Ol[c] += w[j] * Vd[j * d + c];
+          }
+          for (int c = 0; c < d; ++c) Ol[c] /= den;
+          double hO = 0.0;
+          for (int c = 0; c < d; ++c) hO += hl[c] * Ol[c];
+          std::fill(dphiq.begin(), dphiq.end(), 0.0);
+          for (int64_t j = 0; j < N; ++j) {
+            if (kept[j / bk]) continue;
+            double hv = 0.0;
+            for (int c = 0; c < d; ++c) hv += hl[c] * Vd[j * d + c];
+            const double dw = (hv - hO) / den;
+            for (int c = 0; c < d; ++c) dphiq[c] += dw * phiK[j * d + c];
+            const int64_t ks = kslot[j / bk];
+            if (ks >= 0) {
+              const int64_t r = (ks * bk + j % bk) * d;
+              for (int c = 0; c < d; ++c) {
+                const double kc = Kd[j * d + c];
+                if (dK) dK[r + c] += dw * phiq[c] * (kc > 0.0 ? 1.0 : std::exp(kc));
+                if (dV) dV[r + c] += (w[j] / den) * hl[c];
+              }
+            }
+          }
+          for (int c = 0; c < d; ++c) dq[c] += dphiq[c] * (q[c] > 0.0 ? 1.0 : std::exp(q[c]));
+        }
+      }
+      if (qslot[i] >= 0)
+        for (int c = 0; c < d; ++c) dQ[qslot[i] * d + c] = dq[c];
+      if (dalpha) {
+        double x = 0.0;
+        for (int c = 0; c < d; ++c) x += widen(dO[(bh * N + i) * d + c]) * (Os[c] - Ol[c]);
+        dalpha[bh % H] += x;
+      }
+    }
+  }
+  return OK;
+}
+
+}  // extern "C"

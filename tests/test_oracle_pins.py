@@ -524,3 +524,137 @@ def test_router_generator_is_a_scaled_partial_isometry():
         for h in range(3):
             gram = base[h].T @ base[h] if dr <= d else base[h] @ base[h].T
             assert np.abs(gram - np.eye(min(d, dr))).max() < 0.1
+
+
+# ----------------------------------------------------------------------------- gradients
+def _bwd_case(N, bq, bk, d, seed, max_keep=None, keep_nonempty=True):
+    q, k, v = _rand_qkv(1, 2, N, d, seed, scale=1.5)
+    g = torch.Generator().manual_seed(seed + 1)
+    dO = _bf16(torch.randn(1, 2, N, d, generator=g))
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx, kv_cnt = synth.random_mask(1, 2, nqb, nkb, nkb if max_keep is None else max_keep, seed=seed)
+    if keep_nonempty:
+        empty = kv_cnt == 0
+        kv_cnt[empty] = 1
+        kv_idx[..., 0][empty] = 0
+    return q, k, v, dO, kv_idx, kv_cnt
+
+
+def _autograd(fn, q, k, v, dO, extra=()):
+    leaves = [t.double().requires_grad_(True) for t in (q, k, v)] + [t.requires_grad_(True) for t in extra]
+    O = fn(*leaves)
+    (O * dO.double()).sum().backward()
+    return O.detach(), [t.grad for t in leaves]
+
+
+def _kgrad(x, nkb, bk):
+    """[1,H,N,d] key-side gradient as the oracle's [H*nkb, bk, d] block layout."""
+    _, H, N, d = x.shape
+    out = torch.zeros(H, nkb * bk, d, dtype=torch.float64)
+    out[:, :N] = x[0]
+    return out.reshape(H * nkb, bk, d).numpy()
+
+
+@pytest.mark.parametrize("N,bq,bk", [(200, 64, 32), (130, 128, 64)])
+def test_sparse_gradients_match_sdpa_autograd(oracle_mod, N, bq, bk):
+    d = 16
+    q, k, v, dO, kv_idx, kv_cnt = _bwd_case(N, bq, bk, d, 40 + N)
+    m = torch.from_numpy(_block_bool_mask(kv_idx.numpy(), kv_cnt.numpy(), N, bq, bk))
+    O, (gq, gk, gv) = _autograd(lambda a, b, c: F.scaled_dot_product_attention(a, b, c, attn_mask=m), q, k, v, dO)
+    O_or, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    np.testing.assert_allclose(O_or.reshape(O.shape), O.numpy(), rtol=0, atol=1e-12)
+    dQ, dK, dV, _ = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    nkb = -(-N // bk)
+    np.testing.assert_allclose(dQ.reshape(gq.shape), gq.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dK, _kgrad(gk, nkb, bk), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dV, _kgrad(gv, nkb, bk), rtol=0, atol=1e-11)
+
+
+def test_linear_gradients_match_autograd(oracle_mod):
+    N, bq, bk, d = 200, 64, 32, 8
+    q, k, v, dO, kv_idx, kv_cnt = _bwd_case(N, bq, bk, d, 44, max_keep=6, keep_nonempty=False)
+    # one row keeps everything: its complement is empty, O_l = 0 and no gradient
+    nkb = -(-N // bk)
+    kv_idx[0, 1, 1, :nkb] = torch.arange(nkb, dtype=torch.int32)
+    kv_cnt[0, 1, 1] = nkb
+    keep = torch.from_numpy(_block_bool_mask(kv_idx.numpy(), kv_cnt.numpy(), N, bq, bk))
+
+    def lin(a, b, c):
+        W = (_phi_torch(a) @ _phi_torch(b).transpose(-1, -2)) * (~keep)
+        den = W.sum(-1, keepdim=True)
+        return torch.where(den > 0, (W @ c) / torch.where(den > 0, den, torch.ones_like(den)), torch.zeros_like(a))
+
+    O, (gq, gk, gv) = _autograd(lin, q, k, v, dO)
+    O_or, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="linear")
+    np.testing.assert_allclose(O_or.reshape(O.shape), O.numpy(), rtol=0, atol=1e-12)
+    dQ, dK, dV, _ = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, mode="linear")
+    np.testing.assert_allclose(dQ.reshape(gq.shape), gq.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dK, _kgrad(gk, nkb, bk), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dV, _kgrad(gv, nkb, bk), rtol=0, atol=1e-11)
+
+
+def test_mix_gradients_match_autograd_including_alpha(oracle_mod):
+    N, bq, bk, d = 200, 64, 32, 8
+    q, k, v, dO, kv_idx, kv_cnt = _bwd_case(N, bq, bk, d, 45, max_keep=5)
+    alpha = torch.tensor([0.7, 0.25], dtype=torch.float32)
+    keep = torch.from_numpy(_block_bool_mask(kv_idx.numpy(), kv_cnt.numpy(), N, bq, bk))
+    nkb = -(-N // bk)
+
+    def mix(a, b, c, al):
+        Os = F.scaled_dot_product_attention(a, b, c, attn_mask=keep)
+        W = (_phi_torch(a) @ _phi_torch(b).transpose(-1, -2)) * (~keep)
+        Ol = (W @ c) / W.sum(-1, keepdim=True)
+        w = al.view(1, 2, 1, 1)
+        return w * Os + (1 - w) * Ol
+
+    O, (gq, gk, gv, ga) = _autograd(mix, q, k, v, dO, extra=(alpha.double(),))
+    O_or, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, alpha=alpha, mode="sla2")
+    np.testing.assert_allclose(O_or.reshape(O.shape), O.numpy(), rtol=0, atol=1e-12)
+    dQ, dK, dV, da = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, alpha=alpha, mode="sla2",
+                                              want_dalpha=True)
+    np.testing.assert_allclose(dQ.reshape(gq.shape), gq.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dK, _kgrad(gk, nkb, bk), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dV, _kgrad(gv, nkb, bk), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(da, ga.numpy(), rtol=1e-12, atol=1e-11)
+
+
+def test_sparse_gradient_invariants(oracle_mod):
+    # Softmax rows sum to one, so each row's dS sums to zero: the key gradients of a
+    # head sum to zero, and the value gradients sum to the sum of dO over the rows.
+    N, bq, bk, d = 1000, 128, 64, 64
+    q, k, v, dO, kv_idx, kv_cnt = _bwd_case(N, bq, bk, d, 46, max_keep=5)
+    _, dK, dV, _ = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, mode="sparse", rows=[])
+    nkb = -(-N // bk)
+    dK = dK.reshape(2, nkb * bk, d)
+    dV = dV.reshape(2, nkb * bk, d)
+    scale = np.abs(dK).sum(1)
+    assert np.all(np.abs(dK.sum(1)) <= 1e-12 * scale + 1e-300)
+    np.testing.assert_allclose(dV.sum(1), dO.double().numpy()[0].sum(1), rtol=1e-12, atol=1e-10)
+
+
+def test_dalpha_is_do_dot_branch_difference(oracle_mod):
+    N, bq, bk, d = 300, 64, 64, 16
+    q, k, v, dO, kv_idx, kv_cnt = _bwd_case(N, bq, bk, d, 47, max_keep=3)
+    alpha = torch.tensor([0.9, 0.6], dtype=torch.float32)
+    Os, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse")
+    Ol, _ = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="linear")
+    ref = (dO.double().numpy().reshape(2, N, d) * (Os - Ol).reshape(2, N, d)).sum((1, 2))
+    _, _, _, da = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, alpha=alpha, mode="sla2",
+                                           rows=[], kblocks=[], want_dalpha=True)
+    np.testing.assert_allclose(da, ref, rtol=1e-12)
+
+
+def test_sampled_gradients_equal_full_gradients(oracle_mod):
+    N, bq, bk, d = 500, 128, 64, 32
+    q, k, v, dO, kv_idx, kv_cnt = _bwd_case(N, bq, bk, d, 48, max_keep=4)
+    alpha = torch.tensor([0.8, 0.7], dtype=torch.float32)
+    for mode in ("sparse", "sla2"):
+        al = alpha if mode == "sla2" else None
+        full = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, alpha=al, mode=mode)
+        rows = np.array([0, 17, 499, 500 + 250, 999])
+        kb = np.array([1, 7, 8 + 3])
+        part = oracle_mod.attention_bwd(q, k, v, dO, bq, bk, kv_idx, kv_cnt, alpha=al, mode=mode, rows=rows,
+                                        kblocks=kb)
+        np.testing.assert_array_equal(part[0], full[0][rows])
+        np.testing.assert_array_equal(part[1], full[1][kb])
+        np.testing.assert_array_equal(part[2], full[2][kb])
