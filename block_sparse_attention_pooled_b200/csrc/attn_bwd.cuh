@@ -1,0 +1,674 @@
+// Block-sparse attention backward on the 5th-generation tensor cores.
+//
+// What it computes (SpargeAttention2 article, arXiv:2602.13515, section 1:
+// the sparse attention is trainable, so its gradients flow through the kept
+// blocks; section 4: each block is either fully computed or fully skipped).
+// For the sparse forward O_i = sum_{j kept} P_ij v_j, P_ij = softmax_j(s_ij),
+// s_ij = q_i . k_j / sqrt(d), and dL/dO = dO:
+//   D_i   = dO_i . O_i
+//   P_ij  = exp(s_ij - lse_i)                 (lse from the forward)
+//   dP_ij = dO_i . v_j,   dS_ij = P_ij (dP_ij - D_i)
+//   dQ_i  = sum_j dS_ij k_j / sqrt(d)          (kept keys of i's block)
+//   dK_j  = sum_i dS_ij q_i / sqrt(d),  dV_j = sum_i P_ij dO_i
+//                                              (rows whose block keeps j's)
+//
+// Four launches, no atomics (bit-reproducible):
+//   bwd_dot_kernel         D_i for every row;
+//   mask_transpose_kernel  for every key block, the ascending list of query
+//                          blocks that keep it;
+//   attn_bwd_dq_kernel     one CTA per query tile, walking its kept key tiles
+//                          (the forward's structure): S = Q K^T and
+//                          dP = dO V^T into TMEM, dS written back over S as
+//                          bf16, dQ += dS K with dS read from TMEM;
+//   attn_bwd_dkdv_kernel   one CTA per 64-key tile, walking the query tiles
+//                          that keep it: S and dP as above; P and dS staged
+//                          as bf16 in shared memory; dV^T += dO^T P and
+//                          dK^T += Q^T dS accumulate in TMEM with the head
+//                          dimension on the lanes (M = d = 128), so the MMAs
+//                          keep M = 128 for 64-key blocks.
+// Warp roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer and
+// TMEM owner, warps 2..5 one row (TMEM lane) per thread. d = 128.
+#pragma once
+#include <cuda.h>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "attn.cuh"
+#include "ptx.cuh"
+
+namespace sparge {
+
+enum : unsigned int {
+  kErrBwdIn = 0x700, kErrBwdKFull, kErrBwdVFull, kErrBwdKEmpty, kErrBwdVEmpty, kErrBwdSFull, kErrBwdPFull,
+  kErrBwdFinal, kErrBwdDrain, kErrBwdStage, kErrBwdInEmpty, kErrBwdKV
+};
+
+struct BwdParams {
+  const int32_t* lst;  // dQ: kv_idx [BH, nqb, nkb]; dK/dV: query-block lists [BH, nkb, nqb]
+  const int32_t* cnt;  // dQ: kv_cnt [BH, nqb];       dK/dV: list lengths [BH, nkb]
+  const float* lse;    // [BH, N], natural log, from the forward
+  const float* dsum;   // [BH, N], D_i = dO_i . O_i
+  int N;
+  int nqb;
+  int nkb;
+  int bq;
+  int bk;
+  float scale_log2;  // log2(e) / sqrt(d)
+  float scale;       // 1 / sqrt(d)
+};
+
+// ---------------------------------------------------------------------------
+// D_i = sum_c dO_ic O_ic in fp32 (bf16 inputs); each thread takes 8 channels,
+// the row's threads combine by shuffles in a fixed order.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dot_kernel(const __nv_bfloat16* __restrict__ O,
+                                                      const __nv_bfloat16* __restrict__ dO, int64_t rows,
+                                                      float* __restrict__ dsum) {
+  constexpr int TPR = D / 8;
+  const int64_t g = (int64_t)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
+  const int c8 = (threadIdx.x % TPR) * 8;
+  float acc = 0.0f;
+  if (g < rows) {
+    const uint4 a = *reinterpret_cast<const uint4*>(O + g * D + c8);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + g * D + c8);
+    const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = __bfloat1622float2(ha[j]), y = __bfloat1622float2(hb[j]);
+      acc = __fmaf_rn(x.x, y.x, acc);
+      acc = __fmaf_rn(x.y, y.y, acc);
+    }
+  }
+#pragma unroll
+  for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (g < rows && threadIdx.x % TPR == 0) dsum[g] = acc;
+}
+
+// ---------------------------------------------------------------------------
+// Transposed mask: for key block J of head bh, the query blocks I whose kept
+// list holds J, ascending. One CTA = one head x 256 key blocks: a bit matrix
+// [Nqb][256] in shared memory is filled from the kept lists, then thread t
+// walks column t in query-block order. Entries outside [0, Nkb) are ignored.
+// ---------------------------------------------------------------------------
+constexpr int kTrCols = 256;
+
+__host__ __device__ constexpr int transpose_smem_bytes(int nqb) { return nqb * (kTrCols / 8); }
+
+__global__ void __launch_bounds__(kTrCols) mask_transpose_kernel(const int32_t* __restrict__ kv_idx,
+                                                                 const int32_t* __restrict__ kv_cnt, int nqb,
+                                                                 int nkb, int32_t* __restrict__ q_idx,
+                                                                 int32_t* __restrict__ q_cnt) {
+  extern __shared__ uint32_t bits[];  // [nqb][kTrCols / 32]
+  constexpr int W = kTrCols / 32;
+  const int chunks = (nkb + kTrCols - 1) / kTrCols;
+  const int64_t bh = blockIdx.x / chunks;
+  const int j0 = (int)(blockIdx.x % chunks) * kTrCols;
+  for (int e = threadIdx.x; e < nqb * W; e += kTrCols) bits[e] = 0u;
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int I = warp; I < nqb; I += kTrCols / 32) {
+    const int64_t row = bh * nqb + I;
+    const int c = min(max(__ldg(kv_cnt + row), 0), nkb);
+    const int32_t* lst = kv_idx + row * nkb;
+    for (int e = lane; e < c; e += 32) {
+      const int J = __ldg(lst + e) - j0;
+      if (J >= 0 && J < kTrCols) atomicOr(&bits[I * W + (J >> 5)], 1u << (J & 31));
+    }
+  }
+  __syncthreads();
+  const int J = j0 + threadIdx.x;
+  if (J < nkb) {
+    const int w = threadIdx.x >> 5;
+    const uint32_t m = 1u << (threadIdx.x & 31);
+    int32_t* out = q_idx + (bh * nkb + J) * (int64_t)nqb;
+    int n = 0;
+    for (int I = 0; I < nqb; ++I)
+      if (bits[I * W + w] & m) out[n++] = I;
+    q_cnt[bh * nkb + J] = n;
+  }
+}
+
+// ---------------------------------------------------------------- shared pieces
+// The row's 64 values of a TMEM block (S or dP) into registers.
+__device__ __forceinline__ void load_row64(uint32_t taddr, float (&s)[kTileK]) { load_scores(taddr, s); }
+
+// P_j = 2^(s_j * scale_log2 - lse2), dS_j = P_j (dP_j - D); keys at or past N
+// (and rows the caller marks invalid) give P = dS = 0.
+__device__ __forceinline__ void p_and_ds(const float (&s)[kTileK], const float (&dp)[kTileK], float scale_log2,
+                                         float lse2, float Di, int key0, int N, bool row_ok,
+                                         uint32_t (&pp)[kTileK / 2], uint32_t (&pds)[kTileK / 2]) {
+  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di);
+  const bool tail = key0 + kTileK > N;
+#pragma unroll
+  for (int k = 0; k < kTileK / 2; ++k) {
+    const float2 x = f2_split(fma2(f2(s[2 * k], s[2 * k + 1]), sc2, nl2));
+    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+    if (!row_ok || (tail && key0 + 2 * k >= N)) p0 = 0.0f;
+    if (!row_ok || (tail && key0 + 2 * k + 1 >= N)) p1 = 0.0f;
+    const float2 g = f2_split(add2(f2(dp[2 * k], dp[2 * k + 1]), nd2));
+    pp[k] = pack_bf16x2(p0, p1);
+    pds[k] = pack_bf16x2(p0 * g.x, p1 * g.y);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ: one CTA per (bh, query block), the forward's walk over kept key tiles.
+// TMEM columns: S(b) [64b, 64b+64), dP(b) [128+64b, 192+64b) for the two
+// tile buffers b, dQ [256, 384); dS(t) (bf16 pairs) over the first 32
+// columns of S(t)'s buffer. One CTA per SM (512 columns).
+// ---------------------------------------------------------------------------
+template <int D>
+struct BwdQSmem {
+  static constexpr int NS = 2;
+  static constexpr int kQBytes = kTileQ * D * 2;
+  static constexpr int kKBytes = kTileK * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kOffQ + kQBytes;
+  static constexpr int kOffK = kOffDO + kQBytes;
+  static constexpr int kOffV = kOffK + NS * kKBytes;
+  static constexpr int kOffBar = kOffV + NS * kKBytes;
+  static constexpr int kBarIn = 0, kBarKFull = 1, kBarVFull = 1 + NS, kBarKEmpty = 1 + 2 * NS,
+                       kBarVEmpty = 1 + 3 * NS, kBarSFull = 1 + 4 * NS, kBarPFull = 3 + 4 * NS,
+                       kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS;
+  static constexpr int kNumBars = 7 + 4 * NS;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffTmem + 16 + 1024;  // + room to align the base to 1024
+  static constexpr int kTmemCols = 512;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+  using L = BwdQSmem<D>;
+  constexpr int NS = L::NS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const uint32_t sQ = sbase + L::kOffQ, sDO = sbase + L::kOffDO, sK = sbase + L::kOffK, sV = sbase + L::kOffV;
+  const uint32_t bar0 = sbase + L::kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tile = blockIdx.x;  // (bh, query block), head-major
+  const int bh = tile / p.nqb;
+  const int q0 = (tile % p.nqb) * p.bq;
+  const int tiles_per_block = p.bk / kTileK;
+  const int cnt = min(max(__ldg(p.cnt + tile), 0), p.nkb);
+  const int T = cnt * tiles_per_block;
+  const int32_t* lst = p.lst + (int64_t)tile * p.nkb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::kBarIn), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(L::kBarKFull + s), 1);
+      mbar_init(bar(L::kBarVFull + s), 1);
+      mbar_init(bar(L::kBarKEmpty + s), 1);
+      mbar_init(bar(L::kBarVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::kBarSFull + s), 1);
+      mbar_init(bar(L::kBarPFull + s), 128);
+    }
+    mbar_init(bar(L::kBarFinal), 1);
+    mbar_init(bar(L::kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::kOffTmem, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && T > 0) {
+      int nk = 0, nv = 0;
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(bar(L::kBarIn), 2 * L::kQBytes);
+      for (int b = 0; b < D / 64; ++b) {
+        tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(L::kBarIn), b * 64, q0, bh);
+        tma_load_3d(sDO + b * (kTileQ * 128), &tmDO, bar(L::kBarIn), b * 64, q0, bh);
+      }
+      int key_next = tile_key0(lst, 0, tiles_per_block, p.bk);
+      for (int t = 0; t < T; ++t) {
+        const int slot = t % NS, round = t / NS;
+        const int key0 = key_next;
+        if (t + 1 < T) key_next = tile_key0(lst, t + 1, tiles_per_block, p.bk);
+        // V(t) feeds dP(t) only, so its slot frees early; K(t) also feeds dQ(t).
+        if (t >= NS && !role_wait(bar(L::kBarVEmpty + slot), (round - 1) & 1, kErrBwdVEmpty, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::kBarVFull + slot), L::kKBytes);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(sV + slot * L::kKBytes + b * (kTileK * 128), &tmV, bar(L::kBarVFull + slot), b * 64, key0, bh);
+        ++nv;
+        if (t >= NS && !role_wait(bar(L::kBarKEmpty + slot), (round - 1) & 1, kErrBwdKEmpty, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(L::kBarKFull + slot), L::kKBytes);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(sK + slot * L::kKBytes + b * (kTileK * 128), &tmK, bar(L::kBarKFull + slot), b * 64, key0, bh);
+        ++nk;
+      }
+      // Never leave with copies in flight.
+      mbar_wait(bar(L::kBarIn), 0, kErrBwdIn);
+      for (int t = (nk > NS ? nk - NS : 0); t < nk; ++t)
+        mbar_wait(bar(L::kBarKFull + t % NS), (t / NS) & 1, kErrBwdKFull);
+      for (int t = (nv > NS ? nv - NS : 0); t < nv; ++t)
+        mbar_wait(bar(L::kBarVFull + t % NS), (t / NS) & 1, kErrBwdVFull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (T > 0) {
+      const bool leader = elect_one();
+      constexpr uint32_t idS = idesc_bf16_f32(kTileQ, kTileK, false, false);
+      constexpr uint32_t idQ = idesc_bf16_f32(kTileQ, D, false, true);
+      const uint64_t dQd = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dDO = sdesc_sw128(sDO, 16, 1024);
+      const uint64_t dK = sdesc_sw128(sK, 16, 1024);                // K-major (S = Q K^T)
+      const uint64_t dKmn = sdesc_sw128(sK, kTileK * 128, 1024);    // MN-major (dQ += dS K)
+      const uint64_t dV = sdesc_sw128(sV, 16, 1024);                // K-major (dP = dO V^T)
+      auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
+        return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
+      };
+      bool ok = warp_wait(L::kBarIn, 0, kErrBwdIn);
+      tc_fence_after();
+      for (int t = 0; ok && t <= T; ++t) {
+        if (t < T) {
+          const int slot = t % NS, b = t & 1;
+          if (!warp_wait(L::kBarKFull + slot, (t / NS) & 1, kErrBwdKFull)) break;
+          if (!warp_wait(L::kBarVFull + slot, (t / NS) & 1, kErrBwdVFull)) break;
+          tc_fence_after();
+          if (leader) {
+            const uint64_t dKs = dK + (uint64_t)((slot * L::kKBytes) >> 4);
+            const uint64_t dVs = dV + (uint64_t)((slot * L::kKBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+              const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+              mma_ss(tS + b * 64, dQd + qo, dKs + ko, idS, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+              const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+              mma_ss(tP + b * 64, dDO + qo, dVs + ko, idS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(L::kBarSFull + b));
+            mma_commit(bar(L::kBarVEmpty + slot));
+          }
+          __syncwarp();
+        }
+        if (t >= 1) {
+          const int u = t - 1, ks = u % NS, b = u & 1;
+          if (!warp_wait(L::kBarPFull + b, (u >> 1) & 1, kErrBwdPFull)) break;
+          tc_fence_after();
+          if (leader) {
+            const uint64_t dKm = dKmn + (uint64_t)((ks * L::kKBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 keys = 2048 bytes of K = 8 packed dS columns
+              mma_ts(tQ, tS + b * 64 + kk * 8, dKm + kk * 128, idQ, (u > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(L::kBarKEmpty + ks));
+            if (u == T - 1) mma_commit(bar(L::kBarFinal));
+          }
+          __syncwarp();
+        }
+      }
+      if (leader) mma_commit(bar(L::kBarDrain));
+      __syncwarp();
+      mbar_wait(bar(L::kBarDrain), 0, kErrBwdDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ dS + epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool row_ok = r < p.bq && q0 + r < p.N;
+    const int64_t grow = (int64_t)bh * p.N + q0 + r;
+    const float lse2 = row_ok ? __ldg(p.lse + grow) * 1.4426950408889634f : 0.0f;
+    const float Di = row_ok ? __ldg(p.dsum + grow) : 0.0f;
+    bool ok = true;
+    int idx_cur = lane < cnt ? __ldg(lst + lane) : 0;
+    int idx_nxt = 32 + lane < cnt ? __ldg(lst + 32 + lane) : 0;
+    for (int t = 0; t < T; ++t) {
+      const int b = t & 1;
+      const int e = t / tiles_per_block, sub = t % tiles_per_block;
+      if (e > 0 && (e & 31) == 0 && sub == 0) {
+        idx_cur = idx_nxt;
+        idx_nxt = e + 32 + lane < cnt ? __ldg(lst + e + 32 + lane) : 0;
+      }
+      const int key0 = __shfl_sync(0xffffffffu, idx_cur, e & 31) * p.bk + sub * kTileK;
+      ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t >> 1) & 1, kErrBwdSFull, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kTileK], dp[kTileK];
+      load_row64(tS + lane_off + b * 64, s);
+      load_row64(tP + lane_off + b * 64, dp);
+      uint32_t pp[kTileK / 2], pds[kTileK / 2];
+      p_and_ds(s, dp, p.scale_log2, lse2, Di, key0, p.N, row_ok, pp, pds);
+      store_p(tS + lane_off + b * 64, pds);
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarPFull + b));
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarFinal), 0, kErrBwdFinal, abort_flag));
+      tc_fence_after();
+    }
+    // Epilogue: scale * dQ -> bf16 -> Q buffer (free: every MMA is done) -> TMA store.
+#pragma unroll 1
+    for (int c = 0; c < D; c += 16) {
+      uint32_t v[16];
+      if (T > 0 && ok) {
+        tmem_ld16(tQ + lane_off + c, v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0u;
+      }
+      float o[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v[j]) * p.scale;
+      stage_row16(sQ, r, c, o);
+    }
+    fence_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0) {
+      for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmDQ, sQ + b * (kTileQ * 128), b * 64, q0, bh);
+      tma_store_commit();
+      tma_store_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV: one CTA per (bh, 64-key tile), walking the query blocks that keep
+// the tile's block (lists from mask_transpose_kernel). Per query tile u:
+//   S(u) = Q_u K^T, dP(u) = dO_u V^T             (M = 128 query rows, N = 64)
+//   P(u), dS(u) -> bf16 staging tiles [128 rows][64 keys] (shared memory)
+//   dV^T += dO_u^T P(u), dK^T += Q_u^T dS(u)     (M = 128 channels, N = 64, K = 128 rows)
+// TMEM columns: S(b) [64b, 64b+64), dP(b) [128+64b, 192+64b), dV^T [256, 320),
+// dK^T [320, 384). One CTA per SM (512 columns).
+// ---------------------------------------------------------------------------
+template <int D>
+struct BwdKVSmem {
+  static constexpr int NS = 2;
+  static constexpr int kQBytes = kTileQ * D * 2;   // Q_u or dO_u
+  static constexpr int kKBytes = kTileK * D * 2;   // K or V of the key tile
+  static constexpr int kSlot = 2 * kQBytes;        // Q_u then dO_u
+  static constexpr int kStBytes = kTileQ * kTileK * 2;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKBytes;
+  static constexpr int kOffRing = kOffV + kKBytes;
+  static constexpr int kOffP = kOffRing + NS * kSlot;
+  static constexpr int kOffDS = kOffP + kStBytes;
+  static constexpr int kOffBar = kOffDS + kStBytes;
+  static constexpr int kBarKV = 0, kBarInFull = 1, kBarInEmpty = 1 + NS, kBarSFull = 1 + 2 * NS,
+                       kBarPReady = 3 + 2 * NS, kBarStage = 4 + 2 * NS, kBarFinal = 5 + 2 * NS,
+                       kBarDrain = 6 + 2 * NS;
+  static constexpr int kNumBars = 7 + 2 * NS;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffTmem + 16 + 1024;
+  static constexpr int kTmemCols = 512;
+};
+
+// 64 bf16 (pairs in pk) as row r of a [128 rows][64 columns] tile with the
+// 128-byte swizzle: the MN-major operand layout of a 64-wide N.
+__device__ __forceinline__ void stage_row64(uint32_t tile, int r, const uint32_t (&pk)[kTileK / 2]) {
+  const uint32_t row_addr = tile + r * 128;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_addr + ((ch ^ (r & 7)) * 16)),
+                 "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]), "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3])
+                 : "memory");
+}
+
+// Column c of a [64 keys][D] bf16 tile in TMA layout (64-column boxes of 64
+// rows, 128-byte swizzle) from the thread's 64 values, scaled by f.
+template <int D>
+__device__ __forceinline__ void stage_col64(uint32_t tile, int c, const float (&v)[kTileK], float f) {
+  const uint32_t base = tile + (c / 64) * (kTileK * 128) + (c % 8) * 2;
+  const int cc = (c % 64) / 8;
+#pragma unroll
+  for (int j = 0; j < kTileK; ++j) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v[j] * f);
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(&h);
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(base + j * 128 + ((cc ^ (j & 7)) * 16)), "h"(u) : "memory");
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                         const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
+                         const BwdParams p) {
+  using L = BwdKVSmem<D>;
+  constexpr int NS = L::NS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const uint32_t sK = sbase + L::kOffK, sV = sbase + L::kOffV, sRing = sbase + L::kOffRing;
+  const uint32_t sP = sbase + L::kOffP, sDS = sbase + L::kOffDS;
+  const uint32_t bar0 = sbase + L::kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nkt = (p.N + kTileK - 1) / kTileK;
+  const int bh = blockIdx.x / nkt;               // head-major: consecutive CTAs share a head's Q and dO
+  const int kt = blockIdx.x % nkt;
+  const int key0 = kt * kTileK;
+  const int64_t jrow = (int64_t)bh * p.nkb + key0 / p.bk;  // (bh, key block)
+  const int T = min(max(__ldg(p.cnt + jrow), 0), p.nqb);
+  const int32_t* lst = p.lst + jrow * p.nqb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::kBarKV), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(L::kBarInFull + s), 1);
+      mbar_init(bar(L::kBarInEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) mbar_init(bar(L::kBarSFull + s), 1);
+    mbar_init(bar(L::kBarPReady), 128);
+    mbar_init(bar(L::kBarStage), 1);
+    mbar_init(bar(L::kBarFinal), 1);
+    mbar_init(bar(L::kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + L::kOffTmem, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + 128, tDV = tmem + 256, tDK = tmem + 320;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && T > 0) {
+      int n_in = 0;
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDO);
+      mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes);
+      for (int b = 0; b < D / 64; ++b) {
+        tma_load_3d(sK + b * (kTileK * 128), &tmK, bar(L::kBarKV), b * 64, key0, bh);
+        tma_load_3d(sV + b * (kTileK * 128), &tmV, bar(L::kBarKV), b * 64, key0, bh);
+      }
+      for (int t = 0; t < T; ++t) {
+        const int slot = t % NS, round = t / NS;
+        const int q0 = __ldg(lst + t) * p.bq;
+        if (t >= NS && !role_wait(bar(L::kBarInEmpty + slot), (round - 1) & 1, kErrBwdInEmpty, abort_flag)) break;
+        const uint32_t dst = sRing + slot * L::kSlot;
+        mbar_arrive_expect_tx(bar(L::kBarInFull + slot), 2 * L::kQBytes);
+        for (int b = 0; b < D / 64; ++b) {
+          tma_load_3d(dst + b * (kTileQ * 128), &tmQ, bar(L::kBarInFull + slot), b * 64, q0, bh);
+          tma_load_3d(dst + L::kQBytes + b * (kTileQ * 128), &tmDO, bar(L::kBarInFull + slot), b * 64, q0, bh);
+        }
+        ++n_in;
+      }
+      mbar_wait(bar(L::kBarKV), 0, kErrBwdKV);
+      for (int t = (n_in > NS ? n_in - NS : 0); t < n_in; ++t)
+        mbar_wait(bar(L::kBarInFull + t % NS), (t / NS) & 1, kErrBwdIn);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (T > 0) {
+      const bool leader = elect_one();
+      constexpr uint32_t idS = idesc_bf16_f32(kTileQ, kTileK, false, false);
+      constexpr uint32_t idT = idesc_bf16_f32(D, kTileK, true, true);
+      const uint64_t dRingK = sdesc_sw128(sRing, 16, 1024);               // Q_u, dO_u as K-major A
+      const uint64_t dRingM = sdesc_sw128(sRing, kTileQ * 128, 1024);     // Q_u, dO_u as MN-major A
+      const uint64_t dK = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dPst = sdesc_sw128(sP, kTileQ * 128, 1024);          // MN-major B, one 64-wide atom
+      const uint64_t dDSst = sdesc_sw128(sDS, kTileQ * 128, 1024);
+      auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
+        return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
+      };
+      bool ok = warp_wait(L::kBarKV, 0, kErrBwdKV);
+      tc_fence_after();
+      for (int t = 0; ok && t <= T; ++t) {
+        if (t < T) {
+          const int slot = t % NS, b = t & 1;
+          if (!warp_wait(L::kBarInFull + slot, (t / NS) & 1, kErrBwdIn)) break;
+          tc_fence_after();
+          if (leader) {
+            const uint32_t so = (uint32_t)((slot * L::kSlot) >> 4);
+            const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+              const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+              mma_ss(tS + b * 64, dRingK + so + qo, dK + ko, idS, kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+              const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+              mma_ss(tP + b * 64, dRingK + doo + qo, dV + ko, idS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(L::kBarSFull + b));
+          }
+          __syncwarp();
+        }
+        if (t >= 1) {
+          const int u = t - 1, slot = u % NS;
+          if (!warp_wait(L::kBarPReady, u & 1, kErrBwdPFull)) break;
+          tc_fence_after();
+          if (leader) {
+            const uint32_t so = (uint32_t)((slot * L::kSlot) >> 4);
+            const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kTileQ / 16; ++kk)  // 16 query rows = 2048 bytes of each operand
+              mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < kTileQ / 16; ++kk)
+              mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar(L::kBarInEmpty + slot));
+            mma_commit(bar(L::kBarStage));
+            if (u == T - 1) mma_commit(bar(L::kBarFinal));
+          }
+          __syncwarp();
+        }
+      }
+      if (leader) mma_commit(bar(L::kBarDrain));
+      __syncwarp();
+      mbar_wait(bar(L::kBarDrain), 0, kErrBwdDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ P, dS + epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // query row of the tile; in the epilogue, the channel
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    int idx_cur = lane < T ? __ldg(lst + lane) : 0;
+    int idx_nxt = 32 + lane < T ? __ldg(lst + 32 + lane) : 0;
+    for (int t = 0; t < T; ++t) {
+      const int b = t & 1;
+      if (t > 0 && (t & 31) == 0) {
+        idx_cur = idx_nxt;
+        idx_nxt = t + 32 + lane < T ? __ldg(lst + t + 32 + lane) : 0;
+      }
+      const int q0 = __shfl_sync(0xffffffffu, idx_cur, t & 31) * p.bq;
+      const bool row_ok = r < p.bq && q0 + r < p.N;
+      const int64_t grow = (int64_t)bh * p.N + q0 + r;
+      const float lse2 = row_ok ? __ldg(p.lse + grow) * 1.4426950408889634f : 0.0f;
+      const float Di = row_ok ? __ldg(p.dsum + grow) : 0.0f;
+      ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t >> 1) & 1, kErrBwdSFull, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kTileK], dp[kTileK];
+      load_row64(tS + lane_off + b * 64, s);
+      load_row64(tP + lane_off + b * 64, dp);
+      uint32_t pp[kTileK / 2], pds[kTileK / 2];
+      p_and_ds(s, dp, p.scale_log2, lse2, Di, key0, p.N, row_ok, pp, pds);
+      // The staging tiles are free once the MMAs of the previous tile have read them.
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarStage), (t - 1) & 1, kErrBwdStage, abort_flag));
+        if (!ok) break;
+      }
+      stage_row64(sP, r, pp);
+      stage_row64(sDS, r, pds);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarPReady));
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarFinal), 0, kErrBwdFinal, abort_flag));
+      tc_fence_after();
+    }
+    // Epilogue: lane r holds channel r of dV^T and dK^T; stage both tiles
+    // transposed into the first ring slot (free: every MMA and load is done).
+    const uint32_t sOutV = sRing, sOutK = sRing + L::kKBytes;
+    float v[kTileK];
+    if (T > 0 && ok) {
+      load_row64(tDV + lane_off, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kTileK; ++j) v[j] = 0.0f;
+    }
+    stage_col64<D>(sOutV, r, v, 1.0f);
+    if (T > 0 && ok) load_row64(tDK + lane_off, v);
+    stage_col64<D>(sOutK, r, v, p.scale);
+    fence_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0) {
+      for (int b = 0; b < D / 64; ++b) {
+        tma_store_3d(&tmDV, sOutV + b * (kTileK * 128), b * 64, key0, bh);
+        tma_store_3d(&tmDK, sOutK + b * (kTileK * 128), b * 64, key0, bh);
+      }
+      tma_store_commit();
+      tma_store_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace sparge

@@ -17,6 +17,7 @@
 #include "lin_out.cuh"
 #include "quant.cuh"
 #include "attn_q8.cuh"
+#include "attn_bwd.cuh"
 
 namespace {
 
@@ -205,6 +206,70 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t BH, int N, int box_ro
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Workspace of the backward: D_i per row, the transposed mask (query-block
+// lists per key block and their lengths).
+struct BwdWs {
+  size_t dsum, qidx, qcnt, total;
+};
+
+BwdWs bwd_ws(const sparge_shape* s, const Dims& d) {
+  BwdWs w;
+  w.dsum = 0;
+  w.qidx = w.dsum + align256((size_t)d.BH * s->N * 4);
+  w.qcnt = w.qidx + align256((size_t)d.BH * d.nkb * d.nqb * 4);
+  w.total = w.qcnt + align256((size_t)d.BH * d.nkb * 4);
+  return w;
+}
+
+constexpr int kMaxTransposeSmem = 200 * 1024;
+
+sparge_status launch_bwd(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
+                         const int32_t* kv_idx, const int32_t* kv_cnt, const void* O, const float* lse,
+                         const void* dO, void* dQ, void* dK, void* dV, uint8_t* ws, cudaStream_t st) {
+  constexpr int D = 128;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
+  if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mdo, dO, dm.BH, s->N, D, kTileQ) ||
+      !make_map_bhnd(&mdq, dQ, dm.BH, s->N, D, s->bq) || !make_map_bhnd(&mdk, dK, dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mdv, dV, dm.BH, s->N, D, kTileK))
+    return SPARGE_ERR_CUDA;
+  const BwdWs w = bwd_ws(s, dm);
+  float* dsum = reinterpret_cast<float*>(ws + w.dsum);
+  int32_t* q_idx = reinterpret_cast<int32_t*>(ws + w.qidx);
+  int32_t* q_cnt = reinterpret_cast<int32_t*>(ws + w.qcnt);
+  const int64_t rows = dm.BH * s->N;
+  bwd_dot_kernel<D><<<(unsigned)ceil_div(rows, 256 / (D / 8)), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), rows, dsum);
+  const int tsm = transpose_smem_bytes((int)dm.nqb);
+  cudaError_t e = ensure_smem(mask_transpose_kernel, tsm, 10);
+  if (e != cudaSuccess) return cuda_status(e);
+  mask_transpose_kernel<<<(unsigned)(dm.BH * ceil_div(dm.nkb, kTrCols)), kTrCols, tsm, st>>>(
+      kv_idx, kv_cnt, (int)dm.nqb, (int)dm.nkb, q_idx, q_cnt);
+  BwdParams p;
+  p.lse = lse;
+  p.dsum = dsum;
+  p.N = s->N;
+  p.nqb = (int)dm.nqb;
+  p.nkb = (int)dm.nkb;
+  p.bq = s->bq;
+  p.bk = s->bk;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.scale = (float)(1.0 / std::sqrt((double)D));
+  p.lst = kv_idx;
+  p.cnt = kv_cnt;
+  e = ensure_smem(attn_bwd_dq_kernel<D>, BwdQSmem<D>::kBytes, 11);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_bwd_dq_kernel<D><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, BwdQSmem<D>::kBytes, st>>>(mq, mk, mv, mdo,
+                                                                                               mdq, p);
+  p.lst = q_idx;
+  p.cnt = q_cnt;
+  e = ensure_smem(attn_bwd_dkdv_kernel<D>, BwdKVSmem<D>::kBytes, 12);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_bwd_dkdv_kernel<D><<<(unsigned)(dm.BH * ceil_div(s->N, kTileK)), kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(
+      mq, mk, mv, mdo, mdk, mdv, p);
+  return cuda_status(cudaGetLastError());
 }
 
 // Workspace of the low-bit sparse branch: codes and scales of Q, K, V.
@@ -406,6 +471,8 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
       return shape->d == 128 ? q8_ws(shape, dm).total : 0;
     case SPARGE_OP_MASK_ROUTER:
       return router_ws(shape, dm).total;
+    case SPARGE_OP_ATTN_BWD:
+      return shape->d == 128 ? bwd_ws(shape, dm).total : 0;
     default:
       return 0;
   }
@@ -548,6 +615,26 @@ sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const s
   st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, z_tile, alpha, O, s);
   if (st != SPARGE_OK) return st;
   return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, alpha, s);
+}
+
+sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, const void* O, const float* lse,
+                              const void* dO, void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !V || !O || !lse || !dO || !dQ || !dK || !dV || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
+      !aligned16(dK) || !aligned16(dV))
+    return SPARGE_ERR_INVALID_ARG;
+  if (shape->d != 128 || transpose_smem_bytes((int)dm.nqb) > kMaxTransposeSmem) return SPARGE_ERR_UNSUPPORTED;
+  if ((int64_t)dm.BH * ceil_div(shape->N, kTileK) > INT32_MAX) return SPARGE_ERR_UNSUPPORTED;
+  const BwdWs w = bwd_ws(shape, dm);
+  if (workspace == nullptr || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
+  return launch_bwd(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, dO, dQ, dK, dV, static_cast<uint8_t*>(workspace),
+                    static_cast<cudaStream_t>(stream));
 }
 
 sparge_status sparge_device_status(void* stream, int32_t* code) {

@@ -20,15 +20,15 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
-OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8, OP_MASK_ROUTER = 0, 1, 2, 3, 4
+OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8, OP_MASK_ROUTER, OP_ATTN_BWD = 0, 1, 2, 3, 4, 5
 
 # Kernel launches per call of each entry point (for launch accounting).
-MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES, ROUTER_LAUNCHES = 3, 1, 4, 3, 5
+MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES, ROUTER_LAUNCHES, BWD_LAUNCHES = 3, 1, 4, 3, 5, 4
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
            "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8",
-           "sparge_mask_router")
+           "sparge_mask_router", "sparge_attn_bwd")
 
 
 class Shape(ctypes.Structure):
@@ -46,10 +46,12 @@ _lib.sparge_mask_noalloc.restype = ctypes.c_int
 _lib.sparge_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sla2_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sparge_attn_fwd_q8.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.sparge_attn_bwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _sz, _vp]
 _lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 _lib.sparge_status_string.argtypes = [ctypes.c_int]
 _lib.sparge_status_string.restype = ctypes.c_char_p
-for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
+for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_bwd", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -165,6 +167,26 @@ def sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, bq: int, bk: int, O=None, lse=None,
     _check(_lib.sparge_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt), _ptr(O),
                                 _ptr(lse), _ptr(workspace), nws, _stream(stream)), "sparge_attn_fwd")
     return O
+
+
+def sparge_attn_bwd(Q, K, V, kv_idx, kv_cnt, O, lse, dO, bq: int, bk: int, dQ=None, dK=None, dV=None,
+                    workspace=None, stream=None):
+    """Gradients of sparge_attn_fwd (O and lse from that call) for dL/dO = dO. Returns (dQ, dK, dV)."""
+    _check_qkv(Q, K, V, O, dO)
+    if lse is None or lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous float32 CUDA log-sum-exp [B,H,N]")
+    shape = make_shape(Q, bq, bk)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    if workspace is None:
+        workspace, nws = _workspace(OP_ATTN_BWD, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sparge_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt), _ptr(O),
+                                _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace), nws,
+                                _stream(stream)), "sparge_attn_bwd")
+    return dQ, dK, dV
 
 
 def sparge_attn_fwd_q8(Q, K, V, kv_idx, kv_cnt, bq: int, bk: int, O=None, workspace=None, stream=None):

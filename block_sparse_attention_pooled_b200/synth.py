@@ -40,6 +40,7 @@ _N_SINUSOIDS = 16
 # subset of heads can be regenerated without drawing the others.
 _STREAM_FIELD, _STREAM_EPS_Q, _STREAM_EPS_K, _STREAM_V, _STREAM_ALPHA = 1, 2, 3, 4, 5
 _STREAM_ROUTER_BASE, _STREAM_ROUTER_Q, _STREAM_ROUTER_K = 6, 7, 8
+_STREAM_DOUT = 9
 
 
 @dataclasses.dataclass(frozen=True)
@@ -187,6 +188,17 @@ def make_router(H: int, d: int, dr: int, seed: int = 0) -> Tuple[torch.Tensor, t
         Wq[h] = base * gain + eq
         Wk[h] = base * gain + ek
     return torch.from_numpy(Wq), torch.from_numpy(Wk)
+
+
+def make_dout(B: int, H: int, N: int, d: int, seed: int = 0, heads=None) -> torch.Tensor:
+    """Output gradient dL/dO for the backward, bf16 [B,H,N,d]: N(0, 1) per
+    element, one seeded stream per (b, h); `heads` as in make_qkv."""
+    pairs = list(heads) if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    out = torch.empty((B, H, N, d) if heads is None else (1, len(pairs), N, d), dtype=torch.bfloat16)
+    o2 = out.view(len(pairs), N, d)
+    for i, (b, h) in enumerate(pairs):
+        o2[i] = _to_bf16(_rng(seed, b, h, _STREAM_DOUT).standard_normal((N, d), dtype=np.float32))
+    return out
 
 
 def make_workload(w: Workload, heads=None):

@@ -83,7 +83,8 @@ enum {
   SPARGE_OP_ATTN = 1,
   SPARGE_OP_SLA2 = 2,
   SPARGE_OP_ATTN_Q8 = 3,
-  SPARGE_OP_MASK_ROUTER = 4
+  SPARGE_OP_MASK_ROUTER = 4,
+  SPARGE_OP_ATTN_BWD = 5
 };
 
 /* Workspace bytes the operation needs for this shape (0 if none, or if the
@@ -165,6 +166,30 @@ sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_sha
 sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                               const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention backward: gradients of sparge_attn_fwd for a loss L
+ * with dL/dO = dO (SpargeAttention2 article, section 1: the sparse attention
+ * is trainable; section 4: blocks computed whole or skipped whole, so the
+ * gradients flow through the kept blocks only).
+ *   D_i = dO_i . O_i,  P_ij = exp(q_i . k_j / sqrt(d) - lse_i),
+ *   dS_ij = P_ij (dO_i . v_j - D_i) over the kept keys of i's block,
+ *   dQ_i = sum_j dS_ij k_j / sqrt(d),  dK_j = sum_i dS_ij q_i / sqrt(d),
+ *   dV_j = sum_i P_ij dO_i.
+ *   O, lse      the forward's output and log-sum-exp (sparge_attn_fwd with
+ *               lse requested) for the same Q, K, V and mask.
+ *   dO          bf16 [B,H,N,d], device. dQ, dK, dV: bf16 [B,H,N,d] outputs;
+ *               keys no query block keeps get dK = dV = 0, rows whose block
+ *               keeps nothing get dQ = 0.
+ * Precision: fp32 scores, P and dS rounded to bf16 as MMA operands, fp32
+ * accumulation; D_i from the bf16 O and dO in fp32.
+ * d must be 128 (else SPARGE_ERR_UNSUPPORTED), and Nqb * 32 bytes must not
+ * exceed 200 KiB (the transposed-mask bit matrix of one CTA).
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN_BWD, shape) (D_i, and for
+ * every key block the ascending list of query blocks that keep it). */
+sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, const void* O, const float* lse,
+                              const void* dO, void* dQ, void* dK, void* dV, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /* Low-bit block-sparse attention forward (SLA2 article, section 3: the
  * sparse branch computes with Q, K, the attention probabilities P and V in
