@@ -42,8 +42,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="480p", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="bf16", choices=["bf16", "q8"],
-                    help="q8: the low-bit sparse branch (int8 Q/K codes, e4m3 P and V), no linear branch")
+    ap.add_argument("--variant", default="bf16", choices=["bf16", "q8", "bwd"],
+                    help="q8: the low-bit sparse branch (int8 Q/K codes, e4m3 P and V), no linear branch; "
+                         "bwd: a training step of the sparse branch (mask, forward with lse, backward)")
     ap.add_argument("--router", type=int, default=0, choices=[0, 64, 128],
                     help="score the mask through a learnt router of this width (seeded stand-in projections)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -177,7 +178,7 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
-def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=None):
+def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=None, dO=None):
     """Times the oracle on a bounded sample: the mask of `heads` head(s) and the
     attention of `n_qblocks` query blocks of the first head, and returns
     (effective FLOP/s, description, threads)."""
@@ -194,9 +195,13 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=N
     t_mask = time.perf_counter() - t0
     qbs = np.linspace(0, w.nqb - 1, n_qblocks).astype(np.int64)
     rows = np.concatenate([np.arange(qb * w.bq, min(w.N, qb * w.bq + w.bq)) for qb in qbs]).astype(np.int64)
-    mode = "q8" if variant == "q8" else ("sla2" if w.sla2 else "sparse")
+    mode = variant if variant in ("q8", "bwd") else ("sla2" if w.sla2 else "sparse")
     t0 = time.perf_counter()
-    if mode == "q8":
+    if mode == "bwd":
+        # forward and backward of the sampled rows' dQ (their kept keys)
+        oracle.attention_bwd(Qh, Kh, Vh, dO[:1, :heads].contiguous(), w.bq, w.bk, idx, cnt, mode="sparse", rows=rows,
+                             kblocks=np.zeros(0, np.int64))
+    elif mode == "q8":
         oracle.attention_q8_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, rows)
     else:
         oracle.attention_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, alpha[:heads].numpy(), mode=mode, rows=rows)
@@ -205,7 +210,7 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=N
     for qb in qbs:
         nrows = min(w.bq, w.N - qb * w.bq)
         keys = sum(min(w.bk, w.N - int(J) * w.bk) for J in idx[0, 0, qb, : cnt[0, 0, qb]])
-        flops += 4.0 * w.d * nrows * keys
+        flops += 4.0 * w.d * nrows * keys * (3.5 if mode == "bwd" else 1.0)
     # the mask's time is charged pro rata to the sampled query blocks
     t = t_attn + t_mask * (len(qbs) / (w.nqb * heads))
     desc = (f"oracle {'router ' if router is not None else ''}mask of {heads} head(s) ({t_mask:.2f} s, charged pro rata) + {mode} attention of "
@@ -219,9 +224,10 @@ def run_reference(args, w, rank, world):
         return
     Q, K, V, alpha = synth.make_workload(w, heads=[(0, 0)])
     router = synth.make_router(w.H, w.d, args.router, seed=w.seed) if args.router else None
+    dO = synth.make_dout(w.B, w.H, w.N, w.d, seed=w.seed, heads=[(0, 0)]) if args.variant == "bwd" else None
     vals = []
     for i in range(args.warmup + args.steps):
-        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4, variant=args.variant, router=router)
+        v, desc, cores = cpu_sample(w, Q, K, V, alpha, n_qblocks=4, variant=args.variant, router=router, dO=dO)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals) / 1e12
@@ -232,6 +238,7 @@ def run_reference(args, w, rank, world):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
                    "topk": w.topk, "topp": w.topp,
                    "path": "oracle: low-bit sparse branch" if args.variant == "q8" else
+                           "oracle: sparse branch forward + backward (dQ of the sampled rows)" if args.variant == "bwd" else
                            ("oracle: sparse + linear mix" if w.sla2 else "oracle: sparse branch"),
                    "router": args.router or None},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
@@ -257,7 +264,8 @@ def run_ours(args, w, rank, world, local_rank):
     ws_mask = torch.empty(max(1, sparge.workspace_bytes(mask_op, shape)), dtype=torch.uint8, device=dev)
     Wq, Wk = (router_h[0].to(dev), router_h[1].to(dev)) if router_h is not None else (None, None)
     q8 = args.variant == "q8"
-    sla2 = w.sla2 and not q8  # the low-bit variant is the sparse branch alone
+    bwd = args.variant == "bwd"
+    sla2 = w.sla2 and not q8 and not bwd  # the low-bit and backward variants run the sparse branch alone
     n_sla2 = sparge.workspace_bytes(sparge.OP_SLA2, shape) if sla2 else 0
     ws_sla2 = torch.empty(max(1, n_sla2), dtype=torch.uint8, device=dev)
     n_q8 = sparge.workspace_bytes(sparge.OP_ATTN_Q8, shape) if q8 else 0
@@ -265,6 +273,12 @@ def run_ours(args, w, rank, world, local_rank):
     kv_idx = torch.empty((B, H, w.nqb, w.nkb), dtype=torch.int32, device=dev)
     kv_cnt = torch.empty((B, H, w.nqb), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
+    if bwd:
+        dOh = pin(synth.make_dout(w.B, w.H, w.N, w.d, seed=w.seed + rank))
+        dO = dOh.to(dev)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+        ws_bwd = torch.empty(sparge.workspace_bytes(sparge.OP_ATTN_BWD, shape), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev_a=None, ev_b=None):
@@ -273,6 +287,14 @@ def run_ours(args, w, rank, world, local_rank):
                                       workspace=ws_mask)
         else:
             sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
+        if bwd:
+            sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, lse=lse)
+            if ev_a is not None:
+                ev_a.record(stream)
+            sparge.sparge_attn_bwd(Q, K, V, kv_idx, kv_cnt, O, lse, dO, w.bq, w.bk, dQ, dK, dV, workspace=ws_bwd)
+            if ev_b is not None:
+                ev_b.record(stream)
+            return
         if ev_a is not None:
             ev_a.record(stream)
         if q8:
@@ -284,14 +306,19 @@ def run_ours(args, w, rank, world, local_rank):
         if ev_b is not None:
             ev_b.record(stream)
 
-    launches_per_step = (sparge.ROUTER_LAUNCHES if Wq is not None else sparge.MASK_LAUNCHES) + (sparge.Q8_LAUNCHES if q8 else
-                                                sparge.SLA2_LAUNCHES if sla2 else sparge.ATTN_LAUNCHES)
+    launches_per_step = ((sparge.ROUTER_LAUNCHES if Wq is not None else sparge.MASK_LAUNCHES) +
+                         (sparge.Q8_LAUNCHES if q8 else sparge.SLA2_LAUNCHES if sla2 else sparge.ATTN_LAUNCHES) +
+                         (sparge.BWD_LAUNCHES if bwd else 0))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
     flops = kept_flops(kv_idx, kv_cnt, N, d, w.bq, w.bk)
     dense_flops = 4.0 * B * H * N * N * d
+    # A training step counts the forward's kept-block FLOPs once and the
+    # backward's five products (S, dP, dV, dK, dQ) as 2.5 times them.
+    step_flops = flops * (3.5 if bwd else 1.0)
+    span_flops = flops * (2.5 if bwd else 1.0)
 
     # ---- device-timed region (inputs resident in HBM, larger than L2)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -310,31 +337,37 @@ def run_ours(args, w, rank, world, local_rank):
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     attn_ms = [a.elapsed_time(b) for a, b in evs]
     ms_step = ms_total / args.steps
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = step_flops * world / (ms_step * 1e-3) / 1e12
     attn_avg = sum(attn_ms) / len(attn_ms)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-        for _ in range(2):
-            Q.copy_(Qh, non_blocking=True); K.copy_(Kh, non_blocking=True); V.copy_(Vh, non_blocking=True)
+        outs = (dQ, dK, dV) if bwd else (O,)
+        hosts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+        ins = [(Q, Qh), (K, Kh), (V, Vh)] + ([(dO, dOh)] if bwd else [])
+
+        def e2e_step():
+            for dst, src in ins:
+                dst.copy_(src, non_blocking=True)
             step()
-            Oh.copy_(O, non_blocking=True)
+            for h, t in zip(hosts, outs):
+                h.copy_(t, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ksteps = max(3, args.steps // 4)
         e0.record(stream)
         for _ in range(ksteps):
-            Q.copy_(Qh, non_blocking=True); K.copy_(Kh, non_blocking=True); V.copy_(Vh, non_blocking=True)
-            step()
-            Oh.copy_(O, non_blocking=True)
+            e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / ksteps, world, dev)
-        h2d = 3 * Q.numel() * Q.element_size()
-        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": O.numel() * O.element_size(), "ms_per_step": e2e_ms}
+        h2d = sum(t.numel() * t.element_size() for t, _ in ins)
+        e2e = {"value": step_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs), "ms_per_step": e2e_ms}
     assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
 
     if rank != 0:
@@ -350,18 +383,22 @@ def run_ours(args, w, rank, world, local_rank):
         # int8 and e4m3 MMAs: the measured bf16 peak times the nominal 8-bit / bf16 ratio (4.5 / 2.25).
         peak *= 2.0
         peak_desc += " x 2 (nominal int8 / e4m3 to bf16 ratio)"
-    achieved = flops / (attn_avg * 1e-3) / 1e12
+    achieved = span_flops / (attn_avg * 1e-3) / 1e12
     # The timed span is one library call: attn_fwd_kernel alone for the pure
     # sparse path; linear_summary + linear_reduce + attn_fwd_kernel<128, 1>
     # for the sparse + linear mix (the attention kernel is about 96% of it).
     kernel_name = "attn_q8_kernel" if q8 else (f"attn_fwd_kernel<{d}, 1>" if sla2 else f"attn_fwd_kernel<{d}, 0>")
-    span = ("sparge_attn_fwd_q8 (3 launches: codes, V codes, attention)" if q8 else
+    if bwd:
+        kernel_name = "attn_bwd_dq_kernel + attn_bwd_dkdv_kernel"
+    span = ("sparge_attn_bwd (4 launches: D_i, transposed mask, dQ, dK/dV)" if bwd else
+            "sparge_attn_fwd_q8 (3 launches: codes, V codes, attention)" if q8 else
             "sla2_attn_fwd (4 launches)" if sla2 else "sparge_attn_fwd (1 launch)")
     # Counters were captured with the plain mask; a router mask keeps other tiles.
-    traffic = None if args.router else dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
+    traffic = None if (args.router or bwd) else dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant, router=router_h)
+        v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant, router=router_h,
+                                    dO=dOh if bwd else None)
         cpu = {"value": v / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -370,7 +407,9 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded video-shaped Q/K/V, see synth.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
                    "topk": w.topk, "topp": w.topp, "alpha": "U[0.6,1] per head" if sla2 else 1.0,
-                   "path": "sparge_attn_fwd_q8" if q8 else ("sla2_attn_fwd" if sla2 else "sparge_attn_fwd"),
+                   "path": "sparge_attn_fwd_q8" if q8 else "sparge_attn_fwd + sparge_attn_bwd" if bwd else
+                           ("sla2_attn_fwd" if sla2 else "sparge_attn_fwd"),
+                   "flops": "kept-block FLOPs x 3.5 (forward + backward)" if bwd else "kept-block FLOPs",
                    "mask": f"sparge_mask_router (dr {args.router})" if args.router else "sparge_mask",
                    "l2": f"inputs larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V per rank)",
                    "parallelism": f"independent replicas x{world}"},

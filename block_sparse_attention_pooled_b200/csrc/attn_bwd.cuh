@@ -153,38 +153,67 @@ __device__ __forceinline__ void p_and_ds(const float (&s)[kTileK], const float (
   }
 }
 
+// Entries of a block list, 32 at a time, one per lane, a chunk ahead of use,
+// so no tile waits on a global load. The whole warp calls get() with the
+// same non-decreasing entry index.
+struct ListChunks {
+  int cur, nxt, chunk;
+  __device__ __forceinline__ ListChunks(const int32_t* lst, int n, int lane) : chunk(0) {
+    cur = lane < n ? __ldg(lst + lane) : 0;
+    nxt = 32 + lane < n ? __ldg(lst + 32 + lane) : 0;
+  }
+  __device__ __forceinline__ int get(const int32_t* lst, int n, int e, int lane) {
+    while ((e >> 5) != chunk) {
+      ++chunk;
+      cur = nxt;
+      nxt = 32 * (chunk + 1) + lane < n ? __ldg(lst + 32 * (chunk + 1) + lane) : 0;
+    }
+    return __shfl_sync(0xffffffffu, cur, e & 31);
+  }
+};
+
 // ---------------------------------------------------------------------------
 // dQ: one CTA per (bh, query block), the forward's walk over kept key tiles.
-// TMEM columns: S(b) [64b, 64b+64), dP(b) [128+64b, 192+64b) for the two
-// tile buffers b, dQ [256, 384); dS(t) (bf16 pairs) over the first 32
-// columns of S(t)'s buffer. One CTA per SM (512 columns).
+// TMEM columns: S(b) [64b, 64b+64), dP(b) [192+64b, 256+64b) for the three
+// tile buffers b = t % 3, dQ [384, 512); dS(t) (bf16 pairs) over the first 32
+// columns of S(t)'s buffer. One CTA per SM (512 columns), so two dS warpgroups
+// share the SM: warps 2..5 take the even tiles, warps 6..9 the odd ones, and
+// each writes half of the dQ columns in the epilogue. With three buffers the
+// MMA warp computes S and dP two tiles ahead, so a warpgroup that finishes a
+// tile finds its next one ready.
 // ---------------------------------------------------------------------------
+constexpr int kBwdQThreads = 320;
+constexpr int kBwdQBufs = 3;
+
 template <int D>
 struct BwdQSmem {
-  static constexpr int NS = 2;
+  // K(t) is held until dQ(t) has read it, one softmax period after S(t): a
+  // four-slot K ring keeps its loads two tiles ahead. V(t) frees after dP(t).
+  static constexpr int NSK = 4, NSV = 2;
   static constexpr int kQBytes = kTileQ * D * 2;
   static constexpr int kKBytes = kTileK * D * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffDO = kOffQ + kQBytes;
   static constexpr int kOffK = kOffDO + kQBytes;
-  static constexpr int kOffV = kOffK + NS * kKBytes;
-  static constexpr int kOffBar = kOffV + NS * kKBytes;
-  static constexpr int kBarIn = 0, kBarKFull = 1, kBarVFull = 1 + NS, kBarKEmpty = 1 + 2 * NS,
-                       kBarVEmpty = 1 + 3 * NS, kBarSFull = 1 + 4 * NS, kBarPFull = 3 + 4 * NS,
-                       kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS;
-  static constexpr int kNumBars = 7 + 4 * NS;
+  static constexpr int kOffV = kOffK + NSK * kKBytes;
+  static constexpr int kOffBar = kOffV + NSV * kKBytes;
+  static constexpr int kBarIn = 0, kBarKFull = 1, kBarKEmpty = 1 + NSK, kBarVFull = 1 + 2 * NSK,
+                       kBarVEmpty = 1 + 2 * NSK + NSV, kBarSFull = 1 + 2 * NSK + 2 * NSV,
+                       kBarPFull = 4 + 2 * NSK + 2 * NSV, kBarFinal = 7 + 2 * NSK + 2 * NSV,
+                       kBarDrain = 8 + 2 * NSK + 2 * NSV;
+  static constexpr int kNumBars = 9 + 2 * NSK + 2 * NSV;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;  // + room to align the base to 1024
   static constexpr int kTmemCols = 512;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kBwdQThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                        const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using L = BwdQSmem<D>;
-  constexpr int NS = L::NS;
+  constexpr int NSK = L::NSK, NSV = L::NSV;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -206,13 +235,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarIn), 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(bar(L::kBarKFull + s), 1);
-      mbar_init(bar(L::kBarVFull + s), 1);
       mbar_init(bar(L::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(bar(L::kBarVFull + s), 1);
       mbar_init(bar(L::kBarVEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kBwdQBufs; ++s) {
       mbar_init(bar(L::kBarSFull + s), 1);
       mbar_init(bar(L::kBarPFull + s), 128);
     }
@@ -229,42 +260,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+  const uint32_t tS = tmem, tP = tmem + 64 * kBwdQBufs, tQ = tmem + 128 * kBwdQBufs;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && T > 0) {
+    // The whole warp walks the list (indices by shuffle); lane 0 waits and issues.
+    if (T > 0) {
       int nk = 0, nv = 0;
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(bar(L::kBarIn), 2 * L::kQBytes);
-      for (int b = 0; b < D / 64; ++b) {
-        tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(L::kBarIn), b * 64, q0, bh);
-        tma_load_3d(sDO + b * (kTileQ * 128), &tmDO, bar(L::kBarIn), b * 64, q0, bh);
+      bool ok = true;
+      if (lane == 0) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        mbar_arrive_expect_tx(bar(L::kBarIn), 2 * L::kQBytes);
+        for (int b = 0; b < D / 64; ++b) {
+          tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(L::kBarIn), b * 64, q0, bh);
+          tma_load_3d(sDO + b * (kTileQ * 128), &tmDO, bar(L::kBarIn), b * 64, q0, bh);
+        }
       }
-      int key_next = tile_key0(lst, 0, tiles_per_block, p.bk);
+      ListChunks lc(lst, cnt, lane);
       for (int t = 0; t < T; ++t) {
-        const int slot = t % NS, round = t / NS;
-        const int key0 = key_next;
-        if (t + 1 < T) key_next = tile_key0(lst, t + 1, tiles_per_block, p.bk);
-        // V(t) feeds dP(t) only, so its slot frees early; K(t) also feeds dQ(t).
-        if (t >= NS && !role_wait(bar(L::kBarVEmpty + slot), (round - 1) & 1, kErrBwdVEmpty, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::kBarVFull + slot), L::kKBytes);
-        for (int b = 0; b < D / 64; ++b)
-          tma_load_3d(sV + slot * L::kKBytes + b * (kTileK * 128), &tmV, bar(L::kBarVFull + slot), b * 64, key0, bh);
-        ++nv;
-        if (t >= NS && !role_wait(bar(L::kBarKEmpty + slot), (round - 1) & 1, kErrBwdKEmpty, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::kBarKFull + slot), L::kKBytes);
-        for (int b = 0; b < D / 64; ++b)
-          tma_load_3d(sK + slot * L::kKBytes + b * (kTileK * 128), &tmK, bar(L::kBarKFull + slot), b * 64, key0, bh);
-        ++nk;
+        const int key0 = lc.get(lst, cnt, t / tiles_per_block, lane) * p.bk + (t % tiles_per_block) * kTileK;
+        if (lane == 0) {
+          const int ks = t % NSK, vs = t % NSV;
+          // V(t) feeds dP(t) only, so its slot frees early; K(t) also feeds dQ(t).
+          ok = t < NSV || role_wait(bar(L::kBarVEmpty + vs), (t / NSV - 1) & 1, kErrBwdVEmpty, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(bar(L::kBarVFull + vs), L::kKBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(sV + vs * L::kKBytes + b * (kTileK * 128), &tmV, bar(L::kBarVFull + vs), b * 64, key0,
+                          bh);
+            ++nv;
+            ok = t < NSK || role_wait(bar(L::kBarKEmpty + ks), (t / NSK - 1) & 1, kErrBwdKEmpty, abort_flag);
+          }
+          if (ok) {
+            mbar_arrive_expect_tx(bar(L::kBarKFull + ks), L::kKBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(sK + ks * L::kKBytes + b * (kTileK * 128), &tmK, bar(L::kBarKFull + ks), b * 64, key0,
+                          bh);
+            ++nk;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
       // Never leave with copies in flight.
-      mbar_wait(bar(L::kBarIn), 0, kErrBwdIn);
-      for (int t = (nk > NS ? nk - NS : 0); t < nk; ++t)
-        mbar_wait(bar(L::kBarKFull + t % NS), (t / NS) & 1, kErrBwdKFull);
-      for (int t = (nv > NS ? nv - NS : 0); t < nv; ++t)
-        mbar_wait(bar(L::kBarVFull + t % NS), (t / NS) & 1, kErrBwdVFull);
+      if (lane == 0) {
+        mbar_wait(bar(L::kBarIn), 0, kErrBwdIn);
+        for (int t = (nk > NSK ? nk - NSK : 0); t < nk; ++t)
+          mbar_wait(bar(L::kBarKFull + t % NSK), (t / NSK) & 1, kErrBwdKFull);
+        for (int t = (nv > NSV ? nv - NSV : 0); t < nv; ++t)
+          mbar_wait(bar(L::kBarVFull + t % NSV), (t / NSV) & 1, kErrBwdVFull);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -282,15 +327,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       bool ok = warp_wait(L::kBarIn, 0, kErrBwdIn);
       tc_fence_after();
-      for (int t = 0; ok && t <= T; ++t) {
+      // S(t) and dP(t) run kBwdQBufs - 1 tiles ahead of dQ(t): buffer t % kBwdQBufs
+      // was last read by dQ(t - kBwdQBufs), issued (and its dS written) before.
+      for (int t = 0; ok && t < T + kBwdQBufs - 1; ++t) {
         if (t < T) {
-          const int slot = t % NS, b = t & 1;
-          if (!warp_wait(L::kBarKFull + slot, (t / NS) & 1, kErrBwdKFull)) break;
-          if (!warp_wait(L::kBarVFull + slot, (t / NS) & 1, kErrBwdVFull)) break;
+          const int ks = t % NSK, vs = t % NSV, b = t % kBwdQBufs;
+          if (!warp_wait(L::kBarKFull + ks, (t / NSK) & 1, kErrBwdKFull)) break;
+          if (!warp_wait(L::kBarVFull + vs, (t / NSV) & 1, kErrBwdVFull)) break;
           tc_fence_after();
           if (leader) {
-            const uint64_t dKs = dK + (uint64_t)((slot * L::kKBytes) >> 4);
-            const uint64_t dVs = dV + (uint64_t)((slot * L::kKBytes) >> 4);
+            const uint64_t dKs = dK + (uint64_t)((ks * L::kKBytes) >> 4);
+            const uint64_t dVs = dV + (uint64_t)((vs * L::kKBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
@@ -304,13 +351,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               mma_ss(tP + b * 64, dDO + qo, dVs + ko, idS, kk > 0 ? 1u : 0u);
             }
             mma_commit(bar(L::kBarSFull + b));
-            mma_commit(bar(L::kBarVEmpty + slot));
+            mma_commit(bar(L::kBarVEmpty + vs));
           }
           __syncwarp();
         }
-        if (t >= 1) {
-          const int u = t - 1, ks = u % NS, b = u & 1;
-          if (!warp_wait(L::kBarPFull + b, (u >> 1) & 1, kErrBwdPFull)) break;
+        if (t >= kBwdQBufs - 1) {
+          const int u = t - (kBwdQBufs - 1), ks = u % NSK, b = u % kBwdQBufs;
+          if (!warp_wait(L::kBarPFull + b, (u / kBwdQBufs) & 1, kErrBwdPFull)) break;
           tc_fence_after();
           if (leader) {
             const uint64_t dKm = dKmn + (uint64_t)((ks * L::kKBytes) >> 4);
@@ -329,6 +376,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dS + epilogue
+    const int wg = (warp - 2) >> 2;  // 0: even tiles, 1: odd tiles
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -337,17 +385,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float lse2 = row_ok ? __ldg(p.lse + grow) * 1.4426950408889634f : 0.0f;
     const float Di = row_ok ? __ldg(p.dsum + grow) : 0.0f;
     bool ok = true;
-    int idx_cur = lane < cnt ? __ldg(lst + lane) : 0;
-    int idx_nxt = 32 + lane < cnt ? __ldg(lst + 32 + lane) : 0;
-    for (int t = 0; t < T; ++t) {
-      const int b = t & 1;
-      const int e = t / tiles_per_block, sub = t % tiles_per_block;
-      if (e > 0 && (e & 31) == 0 && sub == 0) {
-        idx_cur = idx_nxt;
-        idx_nxt = e + 32 + lane < cnt ? __ldg(lst + e + 32 + lane) : 0;
-      }
-      const int key0 = __shfl_sync(0xffffffffu, idx_cur, e & 31) * p.bk + sub * kTileK;
-      ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t >> 1) & 1, kErrBwdSFull, abort_flag));
+    ListChunks lc(lst, cnt, lane);
+    for (int t = wg; t < T; t += 2) {
+      const int b = t % kBwdQBufs;
+      const int key0 = lc.get(lst, cnt, t / tiles_per_block, lane) * p.bk + (t % tiles_per_block) * kTileK;
+      ok = __all_sync(0xffffffffu,
+                      role_wait(bar(L::kBarSFull + b), (t / kBwdQBufs) & 1, kErrBwdSFull, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float s[kTileK], dp[kTileK];
@@ -363,9 +406,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarFinal), 0, kErrBwdFinal, abort_flag));
       tc_fence_after();
     }
-    // Epilogue: scale * dQ -> bf16 -> Q buffer (free: every MMA is done) -> TMA store.
+    // Epilogue: scale * dQ -> bf16 -> Q buffer (free: every MMA is done) ->
+    // TMA store; warpgroup wg takes columns [wg * D/2, (wg + 1) * D/2).
 #pragma unroll 1
-    for (int c = 0; c < D; c += 16) {
+    for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 16) {
       uint32_t v[16];
       if (T > 0 && ok) {
         tmem_ld16(tQ + lane_off + c, v);
@@ -380,7 +424,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       stage_row16(sQ, r, c, o);
     }
     fence_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (warp == 2 && lane == 0) {
       for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmDQ, sQ + b * (kTileQ * 128), b * 64, q0, bh);
       tma_store_commit();
@@ -418,10 +462,12 @@ struct BwdKVSmem {
   static constexpr int kOffP = kOffRing + NS * kSlot;
   static constexpr int kOffDS = kOffP + kStBytes;
   static constexpr int kOffBar = kOffDS + kStBytes;
-  static constexpr int kBarKV = 0, kBarInFull = 1, kBarInEmpty = 1 + NS, kBarSFull = 1 + 2 * NS,
-                       kBarPReady = 3 + 2 * NS, kBarStage = 4 + 2 * NS, kBarFinal = 5 + 2 * NS,
-                       kBarDrain = 6 + 2 * NS;
-  static constexpr int kNumBars = 7 + 2 * NS;
+  // Q_u and dO_u have their own barriers: dO_u frees after dV(u), Q_u after
+  // dK(u), so the next loads into the slot start as early as possible.
+  static constexpr int kBarKV = 0, kBarQFull = 1, kBarDOFull = 1 + NS, kBarQEmpty = 1 + 2 * NS,
+                       kBarDOEmpty = 1 + 3 * NS, kBarSFull = 1 + 4 * NS, kBarPReady = 3 + 4 * NS,
+                       kBarStage = 4 + 4 * NS, kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS;
+  static constexpr int kNumBars = 7 + 4 * NS;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;
   static constexpr int kTmemCols = 512;
@@ -483,8 +529,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarKV), 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(bar(L::kBarInFull + s), 1);
-      mbar_init(bar(L::kBarInEmpty + s), 1);
+      mbar_init(bar(L::kBarQFull + s), 1);
+      mbar_init(bar(L::kBarDOFull + s), 1);
+      mbar_init(bar(L::kBarQEmpty + s), 1);
+      mbar_init(bar(L::kBarDOEmpty + s), 1);
     }
     for (int s = 0; s < 2; ++s) mbar_init(bar(L::kBarSFull + s), 1);
     mbar_init(bar(L::kBarPReady), 128);
@@ -506,30 +554,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && T > 0) {
+    // The whole warp walks the list (indices by shuffle); lane 0 waits and issues.
+    if (T > 0) {
       int n_in = 0;
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmDO);
-      mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes);
-      for (int b = 0; b < D / 64; ++b) {
-        tma_load_3d(sK + b * (kTileK * 128), &tmK, bar(L::kBarKV), b * 64, key0, bh);
-        tma_load_3d(sV + b * (kTileK * 128), &tmV, bar(L::kBarKV), b * 64, key0, bh);
-      }
-      for (int t = 0; t < T; ++t) {
-        const int slot = t % NS, round = t / NS;
-        const int q0 = __ldg(lst + t) * p.bq;
-        if (t >= NS && !role_wait(bar(L::kBarInEmpty + slot), (round - 1) & 1, kErrBwdInEmpty, abort_flag)) break;
-        const uint32_t dst = sRing + slot * L::kSlot;
-        mbar_arrive_expect_tx(bar(L::kBarInFull + slot), 2 * L::kQBytes);
+      bool ok = true;
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmDO);
+        mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes);
         for (int b = 0; b < D / 64; ++b) {
-          tma_load_3d(dst + b * (kTileQ * 128), &tmQ, bar(L::kBarInFull + slot), b * 64, q0, bh);
-          tma_load_3d(dst + L::kQBytes + b * (kTileQ * 128), &tmDO, bar(L::kBarInFull + slot), b * 64, q0, bh);
+          tma_load_3d(sK + b * (kTileK * 128), &tmK, bar(L::kBarKV), b * 64, key0, bh);
+          tma_load_3d(sV + b * (kTileK * 128), &tmV, bar(L::kBarKV), b * 64, key0, bh);
         }
-        ++n_in;
       }
-      mbar_wait(bar(L::kBarKV), 0, kErrBwdKV);
-      for (int t = (n_in > NS ? n_in - NS : 0); t < n_in; ++t)
-        mbar_wait(bar(L::kBarInFull + t % NS), (t / NS) & 1, kErrBwdIn);
+      ListChunks lc(lst, T, lane);
+      int n_do = 0;
+      for (int t = 0; t < T; ++t) {
+        const int q0 = lc.get(lst, T, t, lane) * p.bq;
+        if (lane == 0) {
+          const int slot = t % NS, round = t / NS;
+          const uint32_t dst = sRing + slot * L::kSlot;
+          ok = t < NS || role_wait(bar(L::kBarDOEmpty + slot), (round - 1) & 1, kErrBwdInEmpty, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(bar(L::kBarDOFull + slot), L::kQBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(dst + L::kQBytes + b * (kTileQ * 128), &tmDO, bar(L::kBarDOFull + slot), b * 64, q0, bh);
+            ++n_do;
+            ok = t < NS || role_wait(bar(L::kBarQEmpty + slot), (round - 1) & 1, kErrBwdInEmpty, abort_flag);
+          }
+          if (ok) {
+            mbar_arrive_expect_tx(bar(L::kBarQFull + slot), L::kQBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_3d(dst + b * (kTileQ * 128), &tmQ, bar(L::kBarQFull + slot), b * 64, q0, bh);
+            ++n_in;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
+      if (lane == 0) {
+        mbar_wait(bar(L::kBarKV), 0, kErrBwdKV);
+        for (int t = (n_in > NS ? n_in - NS : 0); t < n_in; ++t)
+          mbar_wait(bar(L::kBarQFull + t % NS), (t / NS) & 1, kErrBwdIn);
+        for (int t = (n_do > NS ? n_do - NS : 0); t < n_do; ++t)
+          mbar_wait(bar(L::kBarDOFull + t % NS), (t / NS) & 1, kErrBwdIn);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -546,51 +614,61 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
         return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
       };
+      // dP(t) and S(t) for tile t into TMEM buffer t & 1.
+      auto issue_sdp = [&](int t) -> bool {
+        const int slot = t % NS, b = t & 1;
+        const uint32_t so = (uint32_t)((slot * L::kSlot) >> 4);
+        const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
+        if (!warp_wait(L::kBarDOFull + slot, (t / NS) & 1, kErrBwdIn)) return false;
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+            mma_ss(tP + b * 64, dRingK + doo + qo, dV + ko, idS, kk > 0 ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+        if (!warp_wait(L::kBarQFull + slot, (t / NS) & 1, kErrBwdIn)) return false;
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+            mma_ss(tS + b * 64, dRingK + so + qo, dK + ko, idS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::kBarSFull + b));
+        }
+        __syncwarp();
+        return true;
+      };
       bool ok = warp_wait(L::kBarKV, 0, kErrBwdKV);
       tc_fence_after();
-      for (int t = 0; ok && t <= T; ++t) {
-        if (t < T) {
-          const int slot = t % NS, b = t & 1;
-          if (!warp_wait(L::kBarInFull + slot, (t / NS) & 1, kErrBwdIn)) break;
-          tc_fence_after();
-          if (leader) {
-            const uint32_t so = (uint32_t)((slot * L::kSlot) >> 4);
-            const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
+      // S and dP run two tiles ahead; dV(u) and dK(u) are issued as soon as
+      // P(u) and dS(u) are staged, before the loads of tile u + 2 are awaited.
+      for (int t = 0; ok && t < T && t < 2; ++t) ok = issue_sdp(t);
+      for (int u = 0; ok && u < T; ++u) {
+        const int slot = u % NS;
+        if (!warp_wait(L::kBarPReady, u & 1, kErrBwdPFull)) break;
+        tc_fence_after();
+        if (leader) {
+          const uint32_t so = (uint32_t)((slot * L::kSlot) >> 4);
+          const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
-              const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
-              mma_ss(tS + b * 64, dRingK + so + qo, dK + ko, idS, kk > 0 ? 1u : 0u);
-            }
+          for (int kk = 0; kk < kTileQ / 16; ++kk)  // 16 query rows = 2048 bytes of each operand
+            mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::kBarDOEmpty + slot));
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
-              const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
-              mma_ss(tP + b * 64, dRingK + doo + qo, dV + ko, idS, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(bar(L::kBarSFull + b));
-          }
-          __syncwarp();
+          for (int kk = 0; kk < kTileQ / 16; ++kk)
+            mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::kBarQEmpty + slot));
+          mma_commit(bar(L::kBarStage));
+          if (u == T - 1) mma_commit(bar(L::kBarFinal));
         }
-        if (t >= 1) {
-          const int u = t - 1, slot = u % NS;
-          if (!warp_wait(L::kBarPReady, u & 1, kErrBwdPFull)) break;
-          tc_fence_after();
-          if (leader) {
-            const uint32_t so = (uint32_t)((slot * L::kSlot) >> 4);
-            const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < kTileQ / 16; ++kk)  // 16 query rows = 2048 bytes of each operand
-              mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-            for (int kk = 0; kk < kTileQ / 16; ++kk)
-              mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(bar(L::kBarInEmpty + slot));
-            mma_commit(bar(L::kBarStage));
-            if (u == T - 1) mma_commit(bar(L::kBarFinal));
-          }
-          __syncwarp();
-        }
+        __syncwarp();
+        if (u + 2 < T) ok = issue_sdp(u + 2);
       }
       if (leader) mma_commit(bar(L::kBarDrain));
       __syncwarp();
@@ -602,15 +680,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int r = q * 32 + lane;  // query row of the tile; in the epilogue, the channel
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     bool ok = true;
-    int idx_cur = lane < T ? __ldg(lst + lane) : 0;
-    int idx_nxt = 32 + lane < T ? __ldg(lst + 32 + lane) : 0;
+    ListChunks lc(lst, T, lane);
     for (int t = 0; t < T; ++t) {
       const int b = t & 1;
-      if (t > 0 && (t & 31) == 0) {
-        idx_cur = idx_nxt;
-        idx_nxt = t + 32 + lane < T ? __ldg(lst + t + 32 + lane) : 0;
-      }
-      const int q0 = __shfl_sync(0xffffffffu, idx_cur, t & 31) * p.bq;
+      const int q0 = lc.get(lst, T, t, lane) * p.bq;
       const bool row_ok = r < p.bq && q0 + r < p.N;
       const int64_t grow = (int64_t)bh * p.N + q0 + r;
       const float lse2 = row_ok ? __ldg(p.lse + grow) * 1.4426950408889634f : 0.0f;

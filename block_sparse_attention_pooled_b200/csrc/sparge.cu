@@ -261,7 +261,7 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   p.cnt = kv_cnt;
   e = ensure_smem(attn_bwd_dq_kernel<D>, BwdQSmem<D>::kBytes, 11);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dq_kernel<D><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, BwdQSmem<D>::kBytes, st>>>(mq, mk, mv, mdo,
+  attn_bwd_dq_kernel<D><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D>::kBytes, st>>>(mq, mk, mv, mdo,
                                                                                                mdq, p);
   p.lst = q_idx;
   p.cnt = q_cnt;
