@@ -130,16 +130,102 @@ __global__ void __launch_bounds__(kTrCols) mask_transpose_kernel(const int32_t* 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Row pass of the SLA2 backward (SLA2 article, arXiv:2602.12675, section 2:
+// O = alpha_h O_s + (1 - alpha_h) O_l). Row i of head bh, h = bh % H:
+//   D_i = alpha_h dO_i . O_s,i     (the sparse backward's D for dO -> alpha_h dO)
+//   f_i = dO_i . O_l,i,  c_i = (1 - alpha_h) / den_i (0 where the linear
+//   branch is off, den_i = 0), e_i = c_i f_i,
+//   and dO_i . (O_s,i - O_l,i), the row's share of dalpha_h.
+// One CTA = kRowsPerCta rows of one (bh), 16 threads per row; each CTA's
+// dalpha share goes to part[] and sla2_dalpha_kernel adds them in order.
+// ---------------------------------------------------------------------------
+constexpr int kRowsPerCta = 256;
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    sla2_bwd_rows_kernel(const __nv_bfloat16* __restrict__ Os, const __nv_bfloat16* __restrict__ Ol,
+                         const __nv_bfloat16* __restrict__ dO, const float* __restrict__ den,
+                         const float* __restrict__ alpha, int H, int N, int chunks, float* __restrict__ dsum,
+                         float* __restrict__ cw, float* __restrict__ fw, float* __restrict__ ew,
+                         float* __restrict__ part) {
+  constexpr int TPR = D / 8, RPP = 256 / TPR;
+  __shared__ float red[8];
+  const int64_t bh = blockIdx.x / chunks;
+  const int r0 = (int)(blockIdx.x % chunks) * kRowsPerCta;
+  const float a = __ldg(alpha + bh % H);
+  const int c8 = (threadIdx.x % TPR) * 8;
+  float acc = 0.0f;
+  for (int k = 0; k < kRowsPerCta / RPP; ++k) {
+    const int r = r0 + k * RPP + threadIdx.x / TPR;
+    float ds = 0.0f, dl = 0.0f;
+    if (r < N) {
+      const int64_t g = (bh * N + r) * D + c8;
+      const uint4 uo = *reinterpret_cast<const uint4*>(Os + g);
+      const uint4 ul = *reinterpret_cast<const uint4*>(Ol + g);
+      const uint4 ud = *reinterpret_cast<const uint4*>(dO + g);
+      const __nv_bfloat162* ho = reinterpret_cast<const __nv_bfloat162*>(&uo);
+      const __nv_bfloat162* hl = reinterpret_cast<const __nv_bfloat162*>(&ul);
+      const __nv_bfloat162* hd = reinterpret_cast<const __nv_bfloat162*>(&ud);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 xo = __bfloat1622float2(ho[j]), xl = __bfloat1622float2(hl[j]), xd = __bfloat1622float2(hd[j]);
+        ds = __fmaf_rn(xd.x, xo.x, ds);
+        ds = __fmaf_rn(xd.y, xo.y, ds);
+        dl = __fmaf_rn(xd.x, xl.x, dl);
+        dl = __fmaf_rn(xd.y, xl.y, dl);
+      }
+    }
+#pragma unroll
+    for (int o = TPR / 2; o > 0; o >>= 1) {
+      ds += __shfl_xor_sync(0xffffffffu, ds, o);
+      dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    }
+    if (r < N && threadIdx.x % TPR == 0) {
+      const int64_t row = bh * N + r;
+      const float dn = __ldg(den + row);
+      const float c = dn > 0.0f ? (1.0f - a) / dn : 0.0f;
+      dsum[row] = a * ds;
+      fw[row] = dl;
+      cw[row] = c;
+      ew[row] = c * dl;
+      acc += ds - dl;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w];
+    part[blockIdx.x] = t;
+  }
+}
+
+// dalpha_h = the row shares of every batch of head h, in (batch, chunk) order.
+__global__ void __launch_bounds__(128) sla2_dalpha_kernel(const float* __restrict__ part, int B, int H, int chunks,
+                                                          float* __restrict__ dalpha) {
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    float acc = 0.0f;
+    for (int b = 0; b < B; ++b)
+      for (int k = 0; k < chunks; ++k) acc += part[(int64_t)(b * H + h) * chunks + k];
+    dalpha[h] = acc;
+  }
+}
+
 // ---------------------------------------------------------------- shared pieces
 // The row's 64 values of a TMEM block (S or dP) into registers.
 __device__ __forceinline__ void load_row64(uint32_t taddr, float (&s)[kTileK]) { load_scores(taddr, s); }
 
-// P_j = 2^(s_j * scale_log2 - lse2), dS_j = P_j (dP_j - D); keys at or past N
-// (and rows the caller marks invalid) give P = dS = 0.
+// P_j = 2^(s_j * scale_log2 - lse2); pp = a P, pds = dS = P (a dP - D) (a:
+// the branch weight alpha_h of the SLA2 mix, 1 for the sparse branch alone);
+// keys at or past N (and rows the caller marks invalid) give zeros.
 __device__ __forceinline__ void p_and_ds(const float (&s)[kTileK], const float (&dp)[kTileK], float scale_log2,
-                                         float lse2, float Di, int key0, int N, bool row_ok,
+                                         float lse2, float Di, float a, int key0, int N, bool row_ok,
                                          uint32_t (&pp)[kTileK / 2], uint32_t (&pds)[kTileK / 2]) {
-  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di);
+  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di), a2 = f2(a, a);
   const bool tail = key0 + kTileK > N;
 #pragma unroll
   for (int k = 0; k < kTileK / 2; ++k) {
@@ -147,8 +233,8 @@ __device__ __forceinline__ void p_and_ds(const float (&s)[kTileK], const float (
     float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
     if (!row_ok || (tail && key0 + 2 * k >= N)) p0 = 0.0f;
     if (!row_ok || (tail && key0 + 2 * k + 1 >= N)) p1 = 0.0f;
-    const float2 g = f2_split(add2(f2(dp[2 * k], dp[2 * k + 1]), nd2));
-    pp[k] = pack_bf16x2(p0, p1);
+    const float2 g = f2_split(fma2(f2(dp[2 * k], dp[2 * k + 1]), a2, nd2));
+    pp[k] = pack_bf16x2(a * p0, a * p1);
     pds[k] = pack_bf16x2(p0 * g.x, p1 * g.y);
   }
 }
@@ -174,51 +260,96 @@ struct ListChunks {
 
 // ---------------------------------------------------------------------------
 // dQ: one CTA per (bh, query block), the forward's walk over kept key tiles.
-// TMEM columns: S(b) [64b, 64b+64), dP(b) [192+64b, 256+64b) for the three
-// tile buffers b = t % 3, dQ [384, 512); dS(t) (bf16 pairs) over the first 32
-// columns of S(t)'s buffer. One CTA per SM (512 columns), so two dS warpgroups
-// share the SM: warps 2..5 take the even tiles, warps 6..9 the odd ones, and
-// each writes half of the dQ columns in the epilogue. With three buffers the
-// MMA warp computes S and dP two tiles ahead, so a warpgroup that finishes a
-// tile finds its next one ready.
+// TMEM columns: S(b) [64b, 64b+64) and dP(b) [64 NB + 64b, ...) for NB tile
+// buffers b = t % NB, dQ [128 NB, 128 NB + 128); dS(t) (bf16 pairs) over the
+// first 32 columns of S(t)'s buffer. One CTA per SM (512 columns), so two dS
+// warpgroups share the SM: warps 2..5 take the even tiles, warps 6..9 the odd
+// ones, and each writes half of the dQ columns in the epilogue. With three
+// buffers (sparse branch alone) the MMA warp computes S and dP two tiles
+// ahead, so a warpgroup that finishes a tile finds its next one ready.
+//
+// SLA2 = true adds the linear branch's query gradient (SLA2 article,
+// arXiv:2602.12675, sections 1 and 2). With c_i = (1 - alpha_h) / den_i,
+// f_i = dO_i . O_l,i (den_i, O_l from the forward's linear branch) and the
+// complement of i's kept keys:
+//   dphi(q_i) = c_i sum_{j not kept} (dP_ij - f_i) phi(k_j)
+//             = c_i (S_all dO_i - f_i z_all + sum_{j kept} (f_i - dP_ij) phi(k_j))
+// so a second accumulator L [128 NB + 128, +128) starts as dO S_all^T (one MMA
+// from a bf16 copy of S_all) and gains X(t) phi(K_t) per kept tile, X = f - dP
+// written as bf16 over dP(t)'s first 32 columns; the epilogue forms
+//   dq_i = scale * dQ_i + c_i (L_i - f_i z_all) * phi'(q_i).
+// The sparse part uses alpha_h dO: dS = P (alpha_h dP - D_i), D_i = alpha_h dO_i . O_s,i.
+// NB = 2 then (TMEM: 4 x 64 + 128 + 128 columns).
 // ---------------------------------------------------------------------------
 constexpr int kBwdQThreads = 320;
-constexpr int kBwdQBufs = 3;
 
-template <int D>
+template <int D, bool SLA2>
 struct BwdQSmem {
   // K(t) is held until dQ(t) has read it, one softmax period after S(t): a
   // four-slot K ring keeps its loads two tiles ahead. V(t) frees after dP(t).
-  static constexpr int NSK = 4, NSV = 2;
+  // SLA2: phi(K_t) rides with K(t); the bf16 S_all tile sits after dO.
+  static constexpr int NB = SLA2 ? 2 : 3;
+  static constexpr int NSK = SLA2 ? 2 : 4, NSV = 2;
   static constexpr int kQBytes = kTileQ * D * 2;
   static constexpr int kKBytes = kTileK * D * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffDO = kOffQ + kQBytes;
-  static constexpr int kOffK = kOffDO + kQBytes;
-  static constexpr int kOffV = kOffK + NSK * kKBytes;
+  static constexpr int kOffSall = kOffDO + kQBytes;
+  static constexpr int kOffK = kOffSall + (SLA2 ? kQBytes : 0);
+  static constexpr int kOffPK = kOffK + NSK * kKBytes;
+  static constexpr int kOffV = kOffPK + (SLA2 ? NSK * kKBytes : 0);
   static constexpr int kOffBar = kOffV + NSV * kKBytes;
   static constexpr int kBarIn = 0, kBarKFull = 1, kBarKEmpty = 1 + NSK, kBarVFull = 1 + 2 * NSK,
                        kBarVEmpty = 1 + 2 * NSK + NSV, kBarSFull = 1 + 2 * NSK + 2 * NSV,
-                       kBarPFull = 4 + 2 * NSK + 2 * NSV, kBarFinal = 7 + 2 * NSK + 2 * NSV,
-                       kBarDrain = 8 + 2 * NSK + 2 * NSV;
-  static constexpr int kNumBars = 9 + 2 * NSK + 2 * NSV;
+                       kBarPFull = kBarSFull + NB, kBarFinal = kBarPFull + NB, kBarDrain = kBarFinal + 1;
+  static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;  // + room to align the base to 1024
   static constexpr int kTmemCols = 512;
 };
 
-template <int D>
+// Per-row inputs of the SLA2 backward (null for the sparse branch alone).
+struct BwdLinParams {
+  const float* alpha;  // [H]
+  const float* cw;     // [BH, N] c_i
+  const float* fw;     // [BH, N] f_i
+  const float* z_all;  // [BH, d]
+  int H;
+};
+
+// dS = P (alpha dP - D) (bf16 pairs) and, with SLA2, X = f - dP (bf16 pairs).
+template <bool SLA2>
+__device__ __forceinline__ void ds_and_x(const float (&s)[kTileK], const float (&dp)[kTileK], float scale_log2,
+                                         float lse2, float Di, float a, float f, int key0, int N, bool row_ok,
+                                         uint32_t (&pds)[kTileK / 2], uint32_t (&px)[kTileK / 2]) {
+  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di), a2 = f2(a, a);
+  const bool tail = key0 + kTileK > N;
+#pragma unroll
+  for (int k = 0; k < kTileK / 2; ++k) {
+    const float2 x = f2_split(fma2(f2(s[2 * k], s[2 * k + 1]), sc2, nl2));
+    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+    if (!row_ok || (tail && key0 + 2 * k >= N)) p0 = 0.0f;
+    if (!row_ok || (tail && key0 + 2 * k + 1 >= N)) p1 = 0.0f;
+    const float2 g = f2_split(fma2(f2(dp[2 * k], dp[2 * k + 1]), a2, nd2));
+    pds[k] = pack_bf16x2(p0 * g.x, p1 * g.y);
+    if (SLA2) px[k] = row_ok ? pack_bf16x2(f - dp[2 * k], f - dp[2 * k + 1]) : 0u;
+  }
+}
+
+template <int D, bool SLA2>
 __global__ void __launch_bounds__(kBwdQThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
-  using L = BwdQSmem<D>;
-  constexpr int NSK = L::NSK, NSV = L::NSV;
+                       const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmPK,
+                       const __grid_constant__ CUtensorMap tmSall, const BwdParams p, const BwdLinParams lp) {
+  using L = BwdQSmem<D, SLA2>;
+  constexpr int NSK = L::NSK, NSV = L::NSV, NB = L::NB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw);
   const uint32_t sQ = sbase + L::kOffQ, sDO = sbase + L::kOffDO, sK = sbase + L::kOffK, sV = sbase + L::kOffV;
+  const uint32_t sSall = sbase + L::kOffSall, sPK = sbase + L::kOffPK;
   const uint32_t bar0 = sbase + L::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
@@ -232,6 +363,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
   const int cnt = min(max(__ldg(p.cnt + tile), 0), p.nkb);
   const int T = cnt * tiles_per_block;
   const int32_t* lst = p.lst + (int64_t)tile * p.nkb;
+  const bool work = T > 0 || SLA2;  // the linear branch has a term even when nothing is kept
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarIn), 1);
@@ -243,7 +375,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
       mbar_init(bar(L::kBarVFull + s), 1);
       mbar_init(bar(L::kBarVEmpty + s), 1);
     }
-    for (int s = 0; s < kBwdQBufs; ++s) {
+    for (int s = 0; s < NB; ++s) {
       mbar_init(bar(L::kBarSFull + s), 1);
       mbar_init(bar(L::kBarPFull + s), 128);
     }
@@ -260,21 +392,23 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 64 * kBwdQBufs, tQ = tmem + 128 * kBwdQBufs;
+  const uint32_t tS = tmem, tP = tmem + 64 * NB, tQ = tmem + 128 * NB, tL = tQ + 128;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // The whole warp walks the list (indices by shuffle); lane 0 waits and issues.
-    if (T > 0) {
+    if (work) {
+      constexpr uint32_t kKTx = (SLA2 ? 2 : 1) * L::kKBytes;
       int nk = 0, nv = 0;
       bool ok = true;
       if (lane == 0) {
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
-        mbar_arrive_expect_tx(bar(L::kBarIn), 2 * L::kQBytes);
+        mbar_arrive_expect_tx(bar(L::kBarIn), (SLA2 ? 3 : 2) * L::kQBytes);
         for (int b = 0; b < D / 64; ++b) {
           tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(L::kBarIn), b * 64, q0, bh);
           tma_load_3d(sDO + b * (kTileQ * 128), &tmDO, bar(L::kBarIn), b * 64, q0, bh);
+          if (SLA2) tma_load_3d(sSall + b * (kTileQ * 128), &tmSall, bar(L::kBarIn), b * 64, 0, bh);
         }
       }
       ListChunks lc(lst, cnt, lane);
@@ -293,10 +427,14 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
             ok = t < NSK || role_wait(bar(L::kBarKEmpty + ks), (t / NSK - 1) & 1, kErrBwdKEmpty, abort_flag);
           }
           if (ok) {
-            mbar_arrive_expect_tx(bar(L::kBarKFull + ks), L::kKBytes);
-            for (int b = 0; b < D / 64; ++b)
+            mbar_arrive_expect_tx(bar(L::kBarKFull + ks), kKTx);
+            for (int b = 0; b < D / 64; ++b) {
               tma_load_3d(sK + ks * L::kKBytes + b * (kTileK * 128), &tmK, bar(L::kBarKFull + ks), b * 64, key0,
                           bh);
+              if (SLA2)
+                tma_load_3d(sPK + ks * L::kKBytes + b * (kTileK * 128), &tmPK, bar(L::kBarKFull + ks), b * 64,
+                            key0, bh);
+            }
             ++nk;
           }
         }
@@ -313,25 +451,39 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (T > 0) {
+    if (work) {
       const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16_f32(kTileQ, kTileK, false, false);
       constexpr uint32_t idQ = idesc_bf16_f32(kTileQ, D, false, true);
+      constexpr uint32_t idL = idesc_bf16_f32(kTileQ, D, false, false);
       const uint64_t dQd = sdesc_sw128(sQ, 16, 1024);
       const uint64_t dDO = sdesc_sw128(sDO, 16, 1024);
+      const uint64_t dSall = sdesc_sw128(sSall, 16, 1024);           // K-major B (row = feature)
       const uint64_t dK = sdesc_sw128(sK, 16, 1024);                // K-major (S = Q K^T)
       const uint64_t dKmn = sdesc_sw128(sK, kTileK * 128, 1024);    // MN-major (dQ += dS K)
+      const uint64_t dPKmn = sdesc_sw128(sPK, kTileK * 128, 1024);  // MN-major (L += X phi(K))
       const uint64_t dV = sdesc_sw128(sV, 16, 1024);                // K-major (dP = dO V^T)
       auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
         return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
       };
       bool ok = warp_wait(L::kBarIn, 0, kErrBwdIn);
       tc_fence_after();
-      // S(t) and dP(t) run kBwdQBufs - 1 tiles ahead of dQ(t): buffer t % kBwdQBufs
-      // was last read by dQ(t - kBwdQBufs), issued (and its dS written) before.
-      for (int t = 0; ok && t < T + kBwdQBufs - 1; ++t) {
+      if (SLA2 && ok) {
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+            mma_ss(tL, dDO + qo, dSall + qo, idL, kk > 0 ? 1u : 0u);
+          }
+          if (T == 0) mma_commit(bar(L::kBarFinal));
+        }
+        __syncwarp();
+      }
+      // S(t) and dP(t) run NB - 1 tiles ahead of dQ(t): buffer t % NB was last
+      // read by dQ(t - NB), issued (and its dS written) before.
+      for (int t = 0; ok && t < T + NB - 1; ++t) {
         if (t < T) {
-          const int ks = t % NSK, vs = t % NSV, b = t % kBwdQBufs;
+          const int ks = t % NSK, vs = t % NSV, b = t % NB;
           if (!warp_wait(L::kBarKFull + ks, (t / NSK) & 1, kErrBwdKFull)) break;
           if (!warp_wait(L::kBarVFull + vs, (t / NSV) & 1, kErrBwdVFull)) break;
           tc_fence_after();
@@ -355,15 +507,21 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
           }
           __syncwarp();
         }
-        if (t >= kBwdQBufs - 1) {
-          const int u = t - (kBwdQBufs - 1), ks = u % NSK, b = u % kBwdQBufs;
-          if (!warp_wait(L::kBarPFull + b, (u / kBwdQBufs) & 1, kErrBwdPFull)) break;
+        if (t >= NB - 1) {
+          const int u = t - (NB - 1), ks = u % NSK, b = u % NB;
+          if (!warp_wait(L::kBarPFull + b, (u / NB) & 1, kErrBwdPFull)) break;
           tc_fence_after();
           if (leader) {
             const uint64_t dKm = dKmn + (uint64_t)((ks * L::kKBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 keys = 2048 bytes of K = 8 packed dS columns
               mma_ts(tQ, tS + b * 64 + kk * 8, dKm + kk * 128, idQ, (u > 0 || kk > 0) ? 1u : 0u);
+            if (SLA2) {
+              const uint64_t dPKm = dPKmn + (uint64_t)((ks * L::kKBytes) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kTileK / 16; ++kk)
+                mma_ts(tL, tP + b * 64 + kk * 8, dPKm + kk * 128, idQ, 1u);
+            }
             mma_commit(bar(L::kBarKEmpty + ks));
             if (u == T - 1) mma_commit(bar(L::kBarFinal));
           }
@@ -384,30 +542,33 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
     const int64_t grow = (int64_t)bh * p.N + q0 + r;
     const float lse2 = row_ok ? __ldg(p.lse + grow) * 1.4426950408889634f : 0.0f;
     const float Di = row_ok ? __ldg(p.dsum + grow) : 0.0f;
+    const float a_h = SLA2 ? __ldg(lp.alpha + (bh % lp.H)) : 1.0f;
+    const float fi = SLA2 && row_ok ? __ldg(lp.fw + grow) : 0.0f;
+    const float ci = SLA2 && row_ok ? __ldg(lp.cw + grow) : 0.0f;
     bool ok = true;
     ListChunks lc(lst, cnt, lane);
     for (int t = wg; t < T; t += 2) {
-      const int b = t % kBwdQBufs;
+      const int b = t % NB;
       const int key0 = lc.get(lst, cnt, t / tiles_per_block, lane) * p.bk + (t % tiles_per_block) * kTileK;
-      ok = __all_sync(0xffffffffu,
-                      role_wait(bar(L::kBarSFull + b), (t / kBwdQBufs) & 1, kErrBwdSFull, abort_flag));
+      ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t / NB) & 1, kErrBwdSFull, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float s[kTileK], dp[kTileK];
       load_row64(tS + lane_off + b * 64, s);
       load_row64(tP + lane_off + b * 64, dp);
-      uint32_t pp[kTileK / 2], pds[kTileK / 2];
-      p_and_ds(s, dp, p.scale_log2, lse2, Di, key0, p.N, row_ok, pp, pds);
+      uint32_t pds[kTileK / 2], px[kTileK / 2];
+      ds_and_x<SLA2>(s, dp, p.scale_log2, lse2, Di, a_h, fi, key0, p.N, row_ok, pds, px);
       store_p(tS + lane_off + b * 64, pds);
+      if (SLA2) store_p(tP + lane_off + b * 64, px);
       tc_fence_before();
       mbar_arrive(bar(L::kBarPFull + b));
     }
-    if (ok && T > 0) {
+    if (ok && work) {
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarFinal), 0, kErrBwdFinal, abort_flag));
       tc_fence_after();
     }
-    // Epilogue: scale * dQ -> bf16 -> Q buffer (free: every MMA is done) ->
-    // TMA store; warpgroup wg takes columns [wg * D/2, (wg + 1) * D/2).
+    // Epilogue: scale * dQ (+ the linear term) -> bf16 -> Q buffer (free: every
+    // MMA is done) -> TMA store; warpgroup wg takes columns [wg D/2, (wg + 1) D/2).
 #pragma unroll 1
     for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 16) {
       uint32_t v[16];
@@ -421,6 +582,24 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
       float o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j] = __uint_as_float(v[j]) * p.scale;
+      if (SLA2) {
+        uint32_t l[16];
+        if (ok) {
+          tmem_ld16(tL + lane_off + c, l);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) l[j] = 0u;
+        }
+        float qv[16];
+        read_row16(sQ, r, c, qv);
+        const float* z = lp.z_all + (int64_t)bh * D + c;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float dphi = ci * (__uint_as_float(l[j]) - fi * __ldg(z + j));
+          o[j] += dphi * (qv[j] > 0.0f ? 1.0f : __expf(qv[j]));
+        }
+      }
       stage_row16(sQ, r, c, o);
     }
     fence_async_smem();
@@ -448,6 +627,24 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
 //   dV^T += dO_u^T P(u), dK^T += Q_u^T dS(u)     (M = 128 channels, N = 64, K = 128 rows)
 // TMEM columns: S(b) [64b, 64b+64), dP(b) [128+64b, 192+64b), dV^T [256, 320),
 // dK^T [320, 384). One CTA per SM (512 columns).
+//
+// MODE 0: the sparse branch alone; bf16 dK, dV.
+// MODE 1: the sparse part of the SLA2 backward: dV stages alpha_h P, dS uses
+//         alpha_h dP (D_i already carries alpha_h); fp32 partials out.
+// MODE 2: the linear part of the SLA2 backward (SLA2 article, sections 1 and
+//         2), over the same kept pairs, with phi(Q), phi(K) in place of Q, K
+//         and W = phi(Q_u) phi(K)^T in place of S. For key j and the query
+//         rows i whose block does NOT keep j's (c_i, f_i as in the dQ kernel):
+//           dphi(k_j) = sum_i c_i (dP_ij - f_i) phi(q_i)
+//                     = G_all v_j - g_all + sum_{i kept} c_i (f_i - dP_ij) phi(q_i)
+//           dv_j      = G_all^T phi(k_j) - sum_{i kept} c_i W_ij dO_i
+//         (G_all = sum_i phi(q_i) (c_i dO_i)^T, g_all = sum_i c_i f_i phi(q_i)
+//         over every row of the head). The accumulators start as
+//         dphiK^T = G_all V^T and dV^T = G_all^T phi(K)^T (two MMAs with the
+//         bf16 G_all tile in the staging area), gain the kept-pair terms with
+//         the staged -c W and c (f - dP), and the epilogue adds the MODE 1
+//         partials: dK = dK_sparse + (dphiK - g_all) * phi'(k), phi'(k) =
+//         min(phi(k), 1); dV = dV_sparse + dV_linear.
 // ---------------------------------------------------------------------------
 template <int D>
 struct BwdKVSmem {
@@ -460,7 +657,7 @@ struct BwdKVSmem {
   static constexpr int kOffV = kOffK + kKBytes;
   static constexpr int kOffRing = kOffV + kKBytes;
   static constexpr int kOffP = kOffRing + NS * kSlot;
-  static constexpr int kOffDS = kOffP + kStBytes;
+  static constexpr int kOffDS = kOffP + kStBytes;  // P and dS staging: together one [128][128] tile
   static constexpr int kOffBar = kOffDS + kStBytes;
   // Q_u and dO_u have their own barriers: dO_u frees after dV(u), Q_u after
   // dK(u), so the next loads into the slot start as early as possible.
@@ -498,12 +695,28 @@ __device__ __forceinline__ void stage_col64(uint32_t tile, int c, const float (&
   }
 }
 
-template <int D>
+// Element (row j, column c) of such a tile, as float.
+__device__ __forceinline__ float tile_at(const uint8_t* tile, int j, int c) {
+  const int cc = (c % 64) / 8;
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+      tile + (c / 64) * (kTileK * 128) + j * 128 + ((cc ^ (j & 7)) * 16) + (c % 8) * 2));
+}
+
+// Inputs and outputs of the SLA2 modes of the dK/dV kernel.
+struct BwdKVLin {
+  const float* alpha;   // [H] (MODE 1)
+  float* dk_part;       // [BH, N, d] fp32: MODE 1 writes scale * dK_sparse, MODE 2 reads it
+  float* dv_part;       // [BH, N, d] fp32: MODE 1 writes dV_sparse, MODE 2 reads it
+  const float* g_all;   // [BH, d] (MODE 2)
+  int H;
+};
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-                         const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tmG, const BwdParams p, const BwdKVLin lk) {
   using L = BwdKVSmem<D>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -525,6 +738,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int64_t jrow = (int64_t)bh * p.nkb + key0 / p.bk;  // (bh, key block)
   const int T = min(max(__ldg(p.cnt + jrow), 0), p.nqb);
   const int32_t* lst = p.lst + jrow * p.nqb;
+  const bool work = T > 0 || MODE == 2;  // the linear part has the G_all terms even when nothing is kept
+  // The staging tiles are free for tile t once phase t - 1 (MODE 2: t, the
+  // first phase being the G_all MMAs) of the stage barrier has completed.
+  constexpr int kStageShift = MODE == 2 ? 0 : 1;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarKV), 1);
@@ -555,16 +772,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // The whole warp walks the list (indices by shuffle); lane 0 waits and issues.
-    if (T > 0) {
+    if (work) {
       int n_in = 0;
       bool ok = true;
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmDO);
-        mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes);
+        mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes + (MODE == 2 ? 2 * L::kStBytes : 0));
         for (int b = 0; b < D / 64; ++b) {
           tma_load_3d(sK + b * (kTileK * 128), &tmK, bar(L::kBarKV), b * 64, key0, bh);
           tma_load_3d(sV + b * (kTileK * 128), &tmV, bar(L::kBarKV), b * 64, key0, bh);
+          if (MODE == 2) tma_load_3d(sP + b * (kTileQ * 128), &tmG, bar(L::kBarKV), b * 64, 0, bh);
         }
       }
       ListChunks lc(lst, T, lane);
@@ -601,16 +819,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (T > 0) {
+    if (work) {
       const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16_f32(kTileQ, kTileK, false, false);
       constexpr uint32_t idT = idesc_bf16_f32(D, kTileK, true, true);
+      constexpr uint32_t idGK = idesc_bf16_f32(D, kTileK, false, false);  // G_all V^T
       const uint64_t dRingK = sdesc_sw128(sRing, 16, 1024);               // Q_u, dO_u as K-major A
       const uint64_t dRingM = sdesc_sw128(sRing, kTileQ * 128, 1024);     // Q_u, dO_u as MN-major A
       const uint64_t dK = sdesc_sw128(sK, 16, 1024);
       const uint64_t dV = sdesc_sw128(sV, 16, 1024);
       const uint64_t dPst = sdesc_sw128(sP, kTileQ * 128, 1024);          // MN-major B, one 64-wide atom
       const uint64_t dDSst = sdesc_sw128(sDS, kTileQ * 128, 1024);
+      const uint64_t dGk = sdesc_sw128(sP, 16, 1024);                     // G_all as K-major A
+      const uint64_t dGm = sdesc_sw128(sP, kTileQ * 128, 1024);           // G_all^T as MN-major A
       auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
         return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
       };
@@ -646,6 +867,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       bool ok = warp_wait(L::kBarKV, 0, kErrBwdKV);
       tc_fence_after();
+      if (MODE == 2 && ok) {
+        // dphiK^T = G_all V^T and dV^T = G_all^T phi(K)^T (K = the d features).
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t go = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+            const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+            mma_ss(tDK, dGk + go, dV + ko, idGK, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
+            mma_ss(tDV, dGm + kk * 128, dK + ko, idGK | (1u << 15), kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::kBarStage));  // the staging area (G_all) is free again
+          if (T == 0) mma_commit(bar(L::kBarFinal));
+        }
+        __syncwarp();
+      }
       // S and dP run two tiles ahead; dV(u) and dK(u) are issued as soon as
       // P(u) and dS(u) are staged, before the loads of tile u + 2 are awaited.
       for (int t = 0; ok && t < T && t < 2; ++t) ok = issue_sdp(t);
@@ -658,11 +898,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTileQ / 16; ++kk)  // 16 query rows = 2048 bytes of each operand
-            mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (MODE == 2 || u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::kBarDOEmpty + slot));
 #pragma unroll
           for (int kk = 0; kk < kTileQ / 16; ++kk)
-            mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (MODE == 2 || u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::kBarQEmpty + slot));
           mma_commit(bar(L::kBarStage));
           if (u == T - 1) mma_commit(bar(L::kBarFinal));
@@ -675,10 +915,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(bar(L::kBarDrain), 0, kErrBwdDrain);
     }
   } else {
-    // ------------------------------------------------------------ P, dS + epilogue
+    // ------------------------------------------------------------ staging + epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;  // query row of the tile; in the epilogue, the channel
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float a_h = MODE == 1 ? __ldg(lk.alpha + (bh % lk.H)) : 1.0f;
     bool ok = true;
     ListChunks lc(lst, T, lane);
     for (int t = 0; t < T; ++t) {
@@ -686,8 +927,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int q0 = lc.get(lst, T, t, lane) * p.bq;
       const bool row_ok = r < p.bq && q0 + r < p.N;
       const int64_t grow = (int64_t)bh * p.N + q0 + r;
-      const float lse2 = row_ok ? __ldg(p.lse + grow) * 1.4426950408889634f : 0.0f;
-      const float Di = row_ok ? __ldg(p.dsum + grow) : 0.0f;
+      // MODE 0/1: lse and D of the row; MODE 2: c_i and f_i.
+      const float x0 = row_ok ? __ldg(p.lse + grow) : 0.0f;
+      const float x1 = row_ok ? __ldg(p.dsum + grow) : 0.0f;
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t >> 1) & 1, kErrBwdSFull, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -695,10 +937,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       load_row64(tS + lane_off + b * 64, s);
       load_row64(tP + lane_off + b * 64, dp);
       uint32_t pp[kTileK / 2], pds[kTileK / 2];
-      p_and_ds(s, dp, p.scale_log2, lse2, Di, key0, p.N, row_ok, pp, pds);
-      // The staging tiles are free once the MMAs of the previous tile have read them.
-      if (t > 0) {
-        ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarStage), (t - 1) & 1, kErrBwdStage, abort_flag));
+      if (MODE == 2) {
+        // -c W for dV, c (f - dP) for dphi(K); zero on rows outside the block.
+        const float ci = row_ok ? x0 : 0.0f;
+#pragma unroll
+        for (int k = 0; k < kTileK / 2; ++k) {
+          pp[k] = pack_bf16x2(-ci * s[2 * k], -ci * s[2 * k + 1]);
+          pds[k] = pack_bf16x2(ci * (x1 - dp[2 * k]), ci * (x1 - dp[2 * k + 1]));
+        }
+      } else {
+        p_and_ds(s, dp, p.scale_log2, x0 * 1.4426950408889634f, x1, a_h, key0, p.N, row_ok, pp, pds);
+      }
+      // The staging tiles are free once the MMAs of the previous tile (MODE 2
+      // at t = 0: the G_all MMAs) have read them.
+      if (t + 1 - kStageShift > 0) {
+        ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarStage), (t - kStageShift) & 1, kErrBwdStage, abort_flag));
         if (!ok) break;
       }
       stage_row64(sP, r, pp);
@@ -707,32 +960,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(L::kBarPReady));
     }
-    if (ok && T > 0) {
+    if (ok && work) {
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarFinal), 0, kErrBwdFinal, abort_flag));
       tc_fence_after();
     }
-    // Epilogue: lane r holds channel r of dV^T and dK^T; stage both tiles
-    // transposed into the first ring slot (free: every MMA and load is done).
+    // Epilogue: lane r holds channel r of dV^T and dK^T (keys along the columns).
     const uint32_t sOutV = sRing, sOutK = sRing + L::kKBytes;
     float v[kTileK];
-    if (T > 0 && ok) {
+    if (work && ok) {
       load_row64(tDV + lane_off, v);
     } else {
 #pragma unroll
       for (int j = 0; j < kTileK; ++j) v[j] = 0.0f;
     }
-    stage_col64<D>(sOutV, r, v, 1.0f);
-    if (T > 0 && ok) load_row64(tDK + lane_off, v);
-    stage_col64<D>(sOutK, r, v, p.scale);
-    fence_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (warp == 2 && lane == 0) {
-      for (int b = 0; b < D / 64; ++b) {
-        tma_store_3d(&tmDV, sOutV + b * (kTileK * 128), b * 64, key0, bh);
-        tma_store_3d(&tmDK, sOutK + b * (kTileK * 128), b * 64, key0, bh);
+    const int64_t obase = ((int64_t)bh * p.N + key0) * D + r;
+    const int nvalid = min(kTileK, p.N - key0);
+    if (MODE == 1) {
+#pragma unroll
+      for (int j = 0; j < kTileK; ++j)
+        if (j < nvalid) lk.dv_part[obase + (int64_t)j * D] = v[j];
+    } else {
+      if (MODE == 2) {
+#pragma unroll
+        for (int j = 0; j < kTileK; ++j)
+          if (j < nvalid) v[j] += lk.dv_part[obase + (int64_t)j * D];
       }
-      tma_store_commit();
-      tma_store_wait0();
+      stage_col64<D>(sOutV, r, v, 1.0f);
+    }
+    if (work && ok) {
+      load_row64(tDK + lane_off, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kTileK; ++j) v[j] = 0.0f;
+    }
+    if (MODE == 1) {
+#pragma unroll
+      for (int j = 0; j < kTileK; ++j)
+        if (j < nvalid) lk.dk_part[obase + (int64_t)j * D] = v[j] * p.scale;
+    } else {
+      if (MODE == 2) {
+        const float g = __ldg(lk.g_all + (int64_t)bh * D + r);
+#pragma unroll
+        for (int j = 0; j < kTileK; ++j)
+          if (j < nvalid)
+            v[j] = lk.dk_part[obase + (int64_t)j * D] + (v[j] - g) * fminf(tile_at(sgen + L::kOffK, j, r), 1.0f);
+      }
+      stage_col64<D>(sOutK, r, v, MODE == 0 ? p.scale : 1.0f);
+    }
+    if (MODE != 1) {
+      fence_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (warp == 2 && lane == 0) {
+        for (int b = 0; b < D / 64; ++b) {
+          tma_store_3d(&tmDV, sOutV + b * (kTileK * 128), b * 64, key0, bh);
+          tma_store_3d(&tmDK, sOutK + b * (kTileK * 128), b * 64, key0, bh);
+        }
+        tma_store_commit();
+        tma_store_wait0();
+      }
     }
   }
   tc_fence_before();

@@ -78,6 +78,7 @@ struct LoParams {
   const float* z_all;     // [BH, 128] fp32
   const float* z_tile;    // [BH, ntiles, 128] fp32
   const float* alpha;     // [H]
+  float* den_out;         // [BH, N] or null: phi(q) . z_c per row (0 where the branch is off)
   int H;
   int N;
   int ntiles;             // ceil(N / 64)
@@ -265,23 +266,24 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       tc_fence_before();
       mbar_arrive(bar(L::kBarInit));
     }
-    // z_kept[r] over the kept tiles, four loads in flight at a time.
+    // z_kept[r] over the kept tiles, four loads in flight at a time. A last
+    // 128-key block may hold a single 64-key tile: its second tile lies past
+    // N, has no z_tile entry and adds nothing.
     float zk = 0.0f;
     {
       const float* zt = p.z_tile + (int64_t)bh * p.ntiles * 128 + r;
+      auto ztile = [&](int tt) {
+        const int tile64 = (__ldg(lst + tt / tiles_per_block) * p.bk + (tt % tiles_per_block) * 64) / 64;
+        return tile64 < p.ntiles ? __ldg(zt + (int64_t)tile64 * 128) : 0.0f;
+      };
       int t = 0;
       for (; t + 4 <= T; t += 4) {
         float v[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int tt = t + u;
-          const int tile64 = (__ldg(lst + tt / tiles_per_block) * p.bk + (tt % tiles_per_block) * 64) / 64;
-          v[u] = __ldg(zt + (int64_t)tile64 * 128);
-        }
+        for (int u = 0; u < 4; ++u) v[u] = ztile(t + u);
         zk += (v[0] + v[1]) + (v[2] + v[3]);
       }
-      for (; t < T; ++t)
-        zk += __ldg(zt + (int64_t)((__ldg(lst + t / tiles_per_block) * p.bk + (t % tiles_per_block) * 64) / 64) * 128);
+      for (; t < T; ++t) zk += ztile(t);
     }
     bool ok = warp_wait(L::kBarKept, 0, kErrLoKept);
     tc_fence_after();
@@ -337,6 +339,8 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     }
     const float a_h = __ldg(p.alpha + (bh % p.H));
     const float wl = (cnt < p.nkb && den > 0.0f) ? (1.0f - a_h) / den : 0.0f;
+    if (p.den_out != nullptr && r < p.bq && q0 + r < p.N)
+      p.den_out[(int64_t)bh * p.N + q0 + r] = (cnt < p.nkb && den > 0.0f) ? den : 0.0f;
     if (ok) ok = warp_wait(L::kBarOut, 0, kErrLoOut);
     tc_fence_after();
     // 4. O tile = (1 - alpha_h) numerator / denominator, bf16, TMA store.

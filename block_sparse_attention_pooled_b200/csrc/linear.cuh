@@ -11,6 +11,14 @@
 // The attention kernel subtracts the kept blocks' share of S_all and z_all to
 // get the complement's summaries.
 //
+// With GRAD = true the same kernel gives the summaries the backward of the
+// linear branch needs (rows are query rows then, with per-row weights c_i and
+// e_i from the backward's row pass):
+//   phiQ  = phi(Q)                         bf16 [N, d]
+//   G_all = sum_i phi(q_i) (c_i dO_i)^T     fp32 [d, d]
+//   g_all = sum_i e_i phi(q_i)              fp32 [d]
+// (K -> Q, V -> dO with row i scaled by c_i, the ones column -> e_i; no z_tile).
+//
 // One CTA handles a run of 64-key tiles of one head: TMA loads K and V tiles,
 // the 128 threads apply phi to the K tile in place in shared memory (rows past
 // N are zeroed), a TMA store writes the phi(K) tile out, and one thread issues
@@ -47,7 +55,9 @@ constexpr int kLinPartial = 128 * 129;  // per CTA: [feature][128 value columns 
 
 struct LinParams {
   float* partial;  // [BH, ctas_per_head, 128, 129]
-  float* z_tile;   // [BH, ntiles, 128]
+  float* z_tile;   // [BH, ntiles, 128] (null with GRAD)
+  const float* row_scale;  // GRAD: c_i [BH, N]
+  const float* row_w;      // GRAD: e_i [BH, N]
   int N;
   int ntiles;         // ceil(N / 64)
   int ctas_per_head;
@@ -66,6 +76,7 @@ __device__ __forceinline__ uint4 phi8(uint4 v) {
   return v;
 }
 
+template <bool GRAD>
 __global__ void __launch_bounds__(kLinThreads)
     linear_summary_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const __grid_constant__ CUtensorMap tmPhiK, const LinParams p) {
@@ -143,6 +154,29 @@ __global__ void __launch_bounds__(kLinThreads)
       const int row = (u * 16 % 8192) / 128;          // key row inside the box
       tile[u] = (key0 + row < p.N) ? phi8(tile[u]) : make_uint4(0u, 0u, 0u, 0u);
     }
+    if (GRAD) {
+      // dO rows scaled by c_i (zero past N); the ones column carries e_i.
+      uint4* vt = reinterpret_cast<uint4*>(sgen + slot * L::kSlot + L::kK);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int u = tid + kLinThreads * j;
+        const int row = (u * 16 % 8192) / 128;
+        const float c = key0 + row < p.N ? __ldg(p.row_scale + (int64_t)bh * p.N + key0 + row) : 0.0f;
+        uint4 v = vt[u];
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h[k]);
+          h[k] = __floats2bfloat162_rn(f.x * c, f.y * c);
+        }
+        vt[u] = v;
+      }
+      if (tid < 64) {
+        const float e = key0 + tid < p.N ? __ldg(p.row_w + (int64_t)bh * p.N + key0 + tid) : 0.0f;
+        uint8_t* ones = sgen + slot * L::kSlot + L::kK + 64 * 128 * 2;
+        *reinterpret_cast<__nv_bfloat16*>(ones + tid * 128 + ((tid & 7) << 4)) = __float2bfloat16_rn(e);
+      }
+    }
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -157,7 +191,7 @@ __global__ void __launch_bounds__(kLinThreads)
       }
       mma_commit(bar_mma(slot));
     }
-    {
+    if (!GRAD) {
       // z_tile: thread = feature; column sum over the tile's 64 rows of the
       // swizzled phi(K) tile (a warp reads 64 contiguous bytes per row).
       const int a = tid, col = a & 63;
@@ -219,8 +253,10 @@ __global__ void __launch_bounds__(kLinThreads)
 
 // S_all / z_all of each head = the sum of its CTAs' partials, in CTA order.
 // One thread per element of the [128][129] summary.
+// s_bf16 (optional): a bf16 copy of S_all, [BH, 128, 128] row-major.
 __global__ void __launch_bounds__(256) linear_reduce_kernel(const float* __restrict__ partial, int ctas_per_head,
-                                                            float* __restrict__ s_all, float* __restrict__ z_all) {
+                                                            float* __restrict__ s_all, float* __restrict__ z_all,
+                                                            __nv_bfloat16* __restrict__ s_bf16) {
   const int bh = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;
   if (e >= kLinPartial) return;
@@ -228,9 +264,10 @@ __global__ void __launch_bounds__(256) linear_reduce_kernel(const float* __restr
   float acc = 0.0f;
   for (int k = 0; k < ctas_per_head; ++k) acc += src[(int64_t)k * kLinPartial];
   const int a = e / 129, c = e % 129;
-  if (c < 128)
+  if (c < 128) {
     s_all[((int64_t)bh * 128 + a) * 128 + c] = acc;
-  else
+    if (s_bf16 != nullptr) s_bf16[((int64_t)bh * 128 + a) * 128 + c] = __float2bfloat16_rn(acc);
+  } else
     z_all[(int64_t)bh * 128 + a] = acc;
 }
 

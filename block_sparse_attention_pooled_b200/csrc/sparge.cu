@@ -123,7 +123,7 @@ bool make_map_bhnd(CUtensorMap* m, const void* base, int64_t BH, int N, int d, i
 // Raises a kernel's dynamic shared memory limit once per device.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int bytes, int slot) {
-  static int done[64][16];  // [device][slot]: one slot per kernel
+  static int done[64][32];  // [device][slot]: one slot per kernel
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -259,16 +259,18 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   p.scale = (float)(1.0 / std::sqrt((double)D));
   p.lst = kv_idx;
   p.cnt = kv_cnt;
-  e = ensure_smem(attn_bwd_dq_kernel<D>, BwdQSmem<D>::kBytes, 11);
+  const BwdLinParams lp{};
+  e = ensure_smem(attn_bwd_dq_kernel<D, false>, BwdQSmem<D, false>::kBytes, 11);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dq_kernel<D><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D>::kBytes, st>>>(mq, mk, mv, mdo,
-                                                                                               mdq, p);
+  attn_bwd_dq_kernel<D, false><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D, false>::kBytes, st>>>(
+      mq, mk, mv, mdo, mdq, mk, mq, p, lp);
   p.lst = q_idx;
   p.cnt = q_cnt;
-  e = ensure_smem(attn_bwd_dkdv_kernel<D>, BwdKVSmem<D>::kBytes, 12);
+  const BwdKVLin lk{};
+  e = ensure_smem(attn_bwd_dkdv_kernel<D, 0>, BwdKVSmem<D>::kBytes, 12);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dkdv_kernel<D><<<(unsigned)(dm.BH * ceil_div(s->N, kTileK)), kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, p);
+  attn_bwd_dkdv_kernel<D, 0><<<(unsigned)(dm.BH * ceil_div(s->N, kTileK)), kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(
+      mq, mk, mv, mdo, mdk, mdv, mq, p, lk);
   return cuda_status(cudaGetLastError());
 }
 
@@ -381,7 +383,7 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
 sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape* s, const Dims& dm,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, const void* phik, const float* s_all,
                                 const float* z_all, const float* z_tile, const float* alpha, void* O,
-                                cudaStream_t st) {
+                                cudaStream_t st, float* den_out = nullptr) {
   CUtensorMap mq, mv, mp, mo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, 128, 128) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
@@ -393,6 +395,7 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   p.z_all = z_all;
   p.z_tile = z_tile;
   p.alpha = alpha;
+  p.den_out = den_out;
   p.H = s->H;
   p.N = s->N;
   p.ntiles = (int)ceil_div(s->N, 64);
@@ -407,7 +410,9 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
 }
 
 sparge_status launch_summaries(const void* K, const void* V, const sparge_shape* s, const Dims& dm, void* phik,
-                               float* partial, float* s_all, float* z_all, float* z_tile, cudaStream_t st) {
+                               float* partial, float* s_all, float* z_all, float* z_tile, cudaStream_t st,
+                               __nv_bfloat16* s_bf16 = nullptr, const float* row_scale = nullptr,
+                               const float* row_w = nullptr) {
   CUtensorMap mk, mv, mp;
   if (!make_map_bhnd(&mk, K, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64))
@@ -415,14 +420,159 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
   LinParams p;
   p.partial = partial;
   p.z_tile = z_tile;
+  p.row_scale = row_scale;
+  p.row_w = row_w;
   p.N = s->N;
   p.ntiles = (int)ceil_div(s->N, 64);
   p.ctas_per_head = lin_ctas_per_head(s->N);
-  cudaError_t e = ensure_smem(linear_summary_kernel, LinSmem::kBytes, 6);
+  const unsigned grid = (unsigned)(dm.BH * p.ctas_per_head);
+  cudaError_t e;
+  if (row_scale != nullptr) {  // the backward's G_all / g_all (K -> Q, V -> dO)
+    e = ensure_smem(linear_summary_kernel<true>, LinSmem::kBytes, 13);
+    if (e != cudaSuccess) return cuda_status(e);
+    linear_summary_kernel<true><<<grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+  } else {
+    e = ensure_smem(linear_summary_kernel<false>, LinSmem::kBytes, 6);
+    if (e != cudaSuccess) return cuda_status(e);
+    linear_summary_kernel<false><<<grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+  }
+  dim3 rgrid((unsigned)ceil_div(kLinPartial, 256), (unsigned)dm.BH);
+  linear_reduce_kernel<<<rgrid, 256, 0, st>>>(partial, p.ctas_per_head, s_all, z_all, s_bf16);
+  return cuda_status(cudaGetLastError());
+}
+
+// Workspace of the SLA2 backward: the forward's linear summaries and the
+// recomputed branch outputs, the row pass, the gradient summaries, the
+// transposed mask and the fp32 sparse partials of dK and dV.
+struct Sla2BwdWs {
+  Sla2Ws f;  // phi(K), S_all, z_all, z_tile, summary partials
+  size_t s_bf16, os, lse, ol, den, alpha0, dsum, cw, fw, ew, dpart, phiq, g, gall, g_bf16, qidx, qcnt, dkp, dvp,
+      total;
+};
+
+inline int sla2_row_chunks(int N) { return (int)ceil_div(N, kRowsPerCta); }
+
+Sla2BwdWs sla2_bwd_ws(const sparge_shape* s, const Dims& d) {
+  Sla2BwdWs w;
+  w.f = sla2_ws(s, d);
+  const size_t tens = align256((size_t)d.BH * s->N * s->d * 2), rows = align256((size_t)d.BH * s->N * 4);
+  const size_t mat32 = align256((size_t)d.BH * s->d * s->d * 4), mat16 = align256((size_t)d.BH * s->d * s->d * 2);
+  w.s_bf16 = w.f.total;
+  w.os = w.s_bf16 + mat16;
+  w.lse = w.os + tens;
+  w.ol = w.lse + rows;
+  w.den = w.ol + tens;
+  w.alpha0 = w.den + rows;
+  w.dsum = w.alpha0 + align256((size_t)s->H * 4);
+  w.cw = w.dsum + rows;
+  w.fw = w.cw + rows;
+  w.ew = w.fw + rows;
+  w.dpart = w.ew + rows;
+  w.phiq = w.dpart + align256((size_t)d.BH * sla2_row_chunks(s->N) * 4);
+  w.g = w.phiq + tens;
+  w.gall = w.g + mat32;
+  w.g_bf16 = w.gall + align256((size_t)d.BH * s->d * 4);
+  w.qidx = w.g_bf16 + mat16;
+  w.qcnt = w.qidx + align256((size_t)d.BH * d.nkb * d.nqb * 4);
+  w.dkp = w.qcnt + align256((size_t)d.BH * d.nkb * 4);
+  w.dvp = w.dkp + align256((size_t)d.BH * s->N * s->d * 4);
+  w.total = w.dvp + align256((size_t)d.BH * s->N * s->d * 4);
+  return w;
+}
+
+sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
+                              const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, const void* dO,
+                              void* dQ, void* dK, void* dV, float* dalpha, uint8_t* ws, cudaStream_t st) {
+  constexpr int D = 128;
+  const Sla2BwdWs w = sla2_bwd_ws(s, dm);
+  auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
+  auto fat = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  __nv_bfloat16* s_bf16 = static_cast<__nv_bfloat16*>(at(w.s_bf16));
+  __nv_bfloat16* g_bf16 = static_cast<__nv_bfloat16*>(at(w.g_bf16));
+  // 1. The forward's pieces: summaries (and a bf16 S_all), O_l unscaled with
+  //    its denominators (alpha = 0 gives weight 1), the sparse branch with lse.
+  sparge_status r = launch_summaries(K, V, s, dm, at(w.f.phik), fat(w.f.partial), fat(w.f.s_all), fat(w.f.z_all),
+                                     fat(w.f.z_tile), st, s_bf16);
+  if (r != SPARGE_OK) return r;
+  cudaError_t e = cudaMemsetAsync(at(w.alpha0), 0, (size_t)s->H * 4, st);
   if (e != cudaSuccess) return cuda_status(e);
-  linear_summary_kernel<<<(unsigned)(dm.BH * p.ctas_per_head), kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
-  dim3 grid((unsigned)ceil_div(kLinPartial, 256), (unsigned)dm.BH);
-  linear_reduce_kernel<<<grid, 256, 0, st>>>(partial, p.ctas_per_head, s_all, z_all);
+  r = launch_linear_out(Q, V, s, dm, kv_idx, kv_cnt, at(w.f.phik), fat(w.f.s_all), fat(w.f.z_all), fat(w.f.z_tile),
+                        fat(w.alpha0), at(w.ol), st, fat(w.den));
+  if (r != SPARGE_OK) return r;
+  r = launch_attn<D, false>(Q, K, V, s, dm, kv_idx, kv_cnt, at(w.os), fat(w.lse), nullptr, st);
+  if (r != SPARGE_OK) return r;
+  // 2. Row pass and dalpha.
+  const int chunks = sla2_row_chunks(s->N);
+  sla2_bwd_rows_kernel<D><<<(unsigned)(dm.BH * chunks), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(at(w.os)), static_cast<const __nv_bfloat16*>(at(w.ol)),
+      static_cast<const __nv_bfloat16*>(dO), fat(w.den), alpha, s->H, s->N, chunks, fat(w.dsum), fat(w.cw),
+      fat(w.fw), fat(w.ew), fat(w.dpart));
+  sla2_dalpha_kernel<<<1, 128, 0, st>>>(fat(w.dpart), s->B, s->H, chunks, dalpha);
+  // 3. G_all, g_all and phi(Q) (the summary kernel on Q and dO with c_i, e_i).
+  r = launch_summaries(Q, dO, s, dm, at(w.phiq), fat(w.f.partial), fat(w.g), fat(w.gall), nullptr, st, g_bf16,
+                       fat(w.cw), fat(w.ew));
+  if (r != SPARGE_OK) return r;
+  // 4. Transposed mask.
+  int32_t* q_idx = reinterpret_cast<int32_t*>(ws + w.qidx);
+  int32_t* q_cnt = reinterpret_cast<int32_t*>(ws + w.qcnt);
+  const int tsm = transpose_smem_bytes((int)dm.nqb);
+  e = ensure_smem(mask_transpose_kernel, tsm, 10);
+  if (e != cudaSuccess) return cuda_status(e);
+  mask_transpose_kernel<<<(unsigned)(dm.BH * ceil_div(dm.nkb, kTrCols)), kTrCols, tsm, st>>>(
+      kv_idx, kv_cnt, (int)dm.nqb, (int)dm.nkb, q_idx, q_cnt);
+  // 5. dQ (sparse + linear), then dK and dV: sparse part into fp32 partials,
+  //    linear part and the combination into bf16.
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, mpq, msall, mg;
+  if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mdo, dO, dm.BH, s->N, D, kTileQ) ||
+      !make_map_bhnd(&mdq, dQ, dm.BH, s->N, D, s->bq) || !make_map_bhnd(&mdk, dK, dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mdv, dV, dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mpk, at(w.f.phik), dm.BH, s->N, D, kTileK) ||
+      !make_map_bhnd(&mpq, at(w.phiq), dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&msall, s_bf16, dm.BH, D, D, kTileQ) ||
+      !make_map_bhnd(&mg, g_bf16, dm.BH, D, D, kTileQ))
+    return SPARGE_ERR_CUDA;
+  BwdParams p;
+  p.lse = fat(w.lse);
+  p.dsum = fat(w.dsum);
+  p.N = s->N;
+  p.nqb = (int)dm.nqb;
+  p.nkb = (int)dm.nkb;
+  p.bq = s->bq;
+  p.bk = s->bk;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.scale = (float)(1.0 / std::sqrt((double)D));
+  p.lst = kv_idx;
+  p.cnt = kv_cnt;
+  BwdLinParams lp;
+  lp.alpha = alpha;
+  lp.cw = fat(w.cw);
+  lp.fw = fat(w.fw);
+  lp.z_all = fat(w.f.z_all);
+  lp.H = s->H;
+  e = ensure_smem(attn_bwd_dq_kernel<D, true>, BwdQSmem<D, true>::kBytes, 14);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_bwd_dq_kernel<D, true><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D, true>::kBytes, st>>>(
+      mq, mk, mv, mdo, mdq, mpk, msall, p, lp);
+  p.lst = q_idx;
+  p.cnt = q_cnt;
+  BwdKVLin lk;
+  lk.alpha = alpha;
+  lk.dk_part = fat(w.dkp);
+  lk.dv_part = fat(w.dvp);
+  lk.g_all = fat(w.gall);
+  lk.H = s->H;
+  const unsigned kgrid = (unsigned)(dm.BH * ceil_div(s->N, kTileK));
+  e = ensure_smem(attn_bwd_dkdv_kernel<D, 1>, BwdKVSmem<D>::kBytes, 15);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_bwd_dkdv_kernel<D, 1><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, p,
+                                                                              lk);
+  BwdParams pl = p;
+  pl.lse = fat(w.cw);
+  pl.dsum = fat(w.fw);
+  e = ensure_smem(attn_bwd_dkdv_kernel<D, 2>, BwdKVSmem<D>::kBytes, 16);
+  if (e != cudaSuccess) return cuda_status(e);
+  attn_bwd_dkdv_kernel<D, 2><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mpq, mpk, mv, mdo, mdk, mdv, mg, pl,
+                                                                              lk);
   return cuda_status(cudaGetLastError());
 }
 
@@ -473,6 +623,8 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
       return router_ws(shape, dm).total;
     case SPARGE_OP_ATTN_BWD:
       return shape->d == 128 ? bwd_ws(shape, dm).total : 0;
+    case SPARGE_OP_SLA2_BWD:
+      return shape->d == 128 ? sla2_bwd_ws(shape, dm).total : 0;
     default:
       return 0;
   }
@@ -635,6 +787,27 @@ sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const
     return SPARGE_ERR_WORKSPACE;
   return launch_bwd(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, dO, dQ, dK, dV, static_cast<uint8_t*>(workspace),
                     static_cast<cudaStream_t>(stream));
+}
+
+sparge_status sla2_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                            const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, const void* dO, void* dQ,
+                            void* dK, void* dV, float* dalpha, void* workspace, size_t workspace_bytes, void* stream) {
+  Dims dm;
+  sparge_status st = check_shape(shape, &dm);
+  if (st != SPARGE_OK) return st;
+  if (!Q || !K || !V || !dO || !dQ || !dK || !dV || !dalpha || !kv_idx || !kv_cnt || !alpha)
+    return SPARGE_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dK) ||
+      !aligned16(dV))
+    return SPARGE_ERR_INVALID_ARG;
+  if (shape->d != 128 || dm.BH > 65535 || transpose_smem_bytes((int)dm.nqb) > kMaxTransposeSmem)
+    return SPARGE_ERR_UNSUPPORTED;
+  if ((int64_t)dm.BH * ceil_div(shape->N, kTileK) > INT32_MAX) return SPARGE_ERR_UNSUPPORTED;
+  const Sla2BwdWs w = sla2_bwd_ws(shape, dm);
+  if (workspace == nullptr || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
+  return launch_sla2_bwd(Q, K, V, shape, dm, kv_idx, kv_cnt, alpha, dO, dQ, dK, dV, dalpha,
+                         static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 sparge_status sparge_device_status(void* stream, int32_t* code) {

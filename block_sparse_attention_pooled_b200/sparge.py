@@ -20,15 +20,18 @@ if not os.path.exists(_LIB_PATH):
 _lib = ctypes.CDLL(_LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
-OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8, OP_MASK_ROUTER, OP_ATTN_BWD = 0, 1, 2, 3, 4, 5
+OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8, OP_MASK_ROUTER, OP_ATTN_BWD, OP_SLA2_BWD = 0, 1, 2, 3, 4, 5, 6
 
 # Kernel launches per call of each entry point (for launch accounting).
 MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES, ROUTER_LAUNCHES, BWD_LAUNCHES = 3, 1, 4, 3, 5, 4
+# sla2_attn_bwd: summaries + reduce, linear_out, sparse forward, row pass, dalpha, gradient summaries
+# + reduce, transposed mask, dQ, dK/dV sparse part, dK/dV linear part (the memset is not a kernel).
+SLA2_BWD_LAUNCHES = 12
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
            "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8",
-           "sparge_mask_router", "sparge_attn_bwd")
+           "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd")
 
 
 class Shape(ctypes.Structure):
@@ -48,10 +51,12 @@ _lib.sla2_attn_fwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _
 _lib.sparge_attn_fwd_q8.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sparge_attn_bwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _sz, _vp]
+_lib.sla2_attn_bwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                               _vp]
 _lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 _lib.sparge_status_string.argtypes = [ctypes.c_int]
 _lib.sparge_status_string.restype = ctypes.c_char_p
-for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_bwd", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
+for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -187,6 +192,27 @@ def sparge_attn_bwd(Q, K, V, kv_idx, kv_cnt, O, lse, dO, bq: int, bk: int, dQ=No
                                 _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace), nws,
                                 _stream(stream)), "sparge_attn_bwd")
     return dQ, dK, dV
+
+
+def sla2_attn_bwd(Q, K, V, kv_idx, kv_cnt, alpha, dO, bq: int, bk: int, dQ=None, dK=None, dV=None, dalpha=None,
+                  workspace=None, stream=None):
+    """Gradients of sla2_attn_fwd for dL/dO = dO. Returns (dQ, dK, dV, dalpha)."""
+    _check_qkv(Q, K, V, dO)
+    if alpha.dtype != torch.float32 or not alpha.is_cuda or alpha.numel() != Q.shape[1]:
+        raise ValueError("alpha must be a float32 CUDA tensor with one value per head")
+    shape = make_shape(Q, bq, bk)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    dalpha = torch.empty(Q.shape[1], dtype=torch.float32, device=Q.device) if dalpha is None else dalpha
+    if workspace is None:
+        workspace, nws = _workspace(OP_SLA2_BWD, shape, Q.device)
+    else:
+        nws = workspace.numel() * workspace.element_size()
+    _check(_lib.sla2_attn_bwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt),
+                              _ptr(alpha), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dalpha), _ptr(workspace), nws,
+                              _stream(stream)), "sla2_attn_bwd")
+    return dQ, dK, dV, dalpha
 
 
 def sparge_attn_fwd_q8(Q, K, V, kv_idx, kv_cnt, bq: int, bk: int, O=None, workspace=None, stream=None):

@@ -84,7 +84,8 @@ enum {
   SPARGE_OP_SLA2 = 2,
   SPARGE_OP_ATTN_Q8 = 3,
   SPARGE_OP_MASK_ROUTER = 4,
-  SPARGE_OP_ATTN_BWD = 5
+  SPARGE_OP_ATTN_BWD = 5,
+  SPARGE_OP_SLA2_BWD = 6
 };
 
 /* Workspace bytes the operation needs for this shape (0 if none, or if the
@@ -190,6 +191,28 @@ sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const
                               const int32_t* kv_idx, const int32_t* kv_cnt, const void* O, const float* lse,
                               const void* dO, void* dQ, void* dK, void* dV, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* SLA2 backward: gradients of sla2_attn_fwd for a loss L with dL/dO = dO
+ * (SLA2 article, sections 1 and 2: O = alpha_h O_sparse + (1 - alpha_h) O_linear,
+ * both branches and alpha trainable).
+ *   sparse branch with alpha_h dO (as sparge_attn_bwd);
+ *   linear branch, over the keys outside i's kept blocks, w_ij = phi(q_i).phi(k_j),
+ *   den_i = sum_j w_ij, O_l,i = sum_j w_ij v_j / den_i, h_i = (1 - alpha_h) dO_i:
+ *     dV_j += (w_ij / den_i) h_i,  dw_ij = h_i . (v_j - O_l,i) / den_i,
+ *     dQ_i += (sum_j dw_ij phi(k_j)) * phi'(q_i),  dK_j += (sum_i dw_ij phi(q_i)) * phi'(k_j);
+ *   dalpha_h = sum over the rows of head h (every batch) of dO_i . (O_s,i - O_l,i).
+ *   alpha       float [H], device.  dO: bf16 [B,H,N,d].
+ *   dQ, dK, dV  bf16 [B,H,N,d] outputs; dalpha float [H] output, device.
+ * The call recomputes what it needs of the forward (the linear summaries,
+ * O_linear and its denominators, the sparse branch and its log-sum-exp), so
+ * it takes no forward outputs. Precision: as sparge_attn_bwd for the sparse
+ * part; the linear part's products take bf16 operands (S_all, G_all, phi(Q),
+ * phi(K)) with fp32 accumulation; row scalars in fp32.
+ * d must be 128 and Nqb * 32 bytes must not exceed 200 KiB.
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_SLA2_BWD, shape). */
+sparge_status sla2_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
+                            const int32_t* kv_idx, const int32_t* kv_cnt, const float* alpha, const void* dO, void* dQ,
+                            void* dK, void* dV, float* dalpha, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Low-bit block-sparse attention forward (SLA2 article, section 3: the
  * sparse branch computes with Q, K, the attention probabilities P and V in

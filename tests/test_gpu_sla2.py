@@ -32,6 +32,7 @@ def _check(Q, K, V, idx, cnt, alpha, bq, bk, rows=None):
 
 
 @pytest.mark.parametrize("N,bq,bk,max_keep", [(1000, 128, 64, 6), (777, 64, 64, 5), (2000, 128, 128, 4),
+                                              (777, 64, 128, 4), (1000, 128, 128, 5),
                                                (130, 128, 64, 3), (64, 64, 64, 1), (4100, 128, 64, 20)])
 def test_sla2_random_masks(N, bq, bk, max_keep):
     Q, K, V = synth.make_qkv(1, 3, N, 128, grid=None, s=1.5, seed=N + bq)
