@@ -44,7 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="bf16", choices=["bf16", "q8", "bwd"],
                     help="q8: the low-bit sparse branch (int8 Q/K codes, e4m3 P and V), no linear branch; "
-                         "bwd: a training step of the sparse branch (mask, forward with lse, backward)")
+                         "bwd: a training step (mask, forward, backward; the sparse + linear mix on SLA2 "
+                         "workloads, whose backward recomputes its forward pieces)")
     ap.add_argument("--router", type=int, default=0, choices=[0, 64, 128],
                     help="score the mask through a learnt router of this width (seeded stand-in projections)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -198,9 +199,10 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=N
     mode = variant if variant in ("q8", "bwd") else ("sla2" if w.sla2 else "sparse")
     t0 = time.perf_counter()
     if mode == "bwd":
-        # forward and backward of the sampled rows' dQ (their kept keys)
-        oracle.attention_bwd(Qh, Kh, Vh, dO[:1, :heads].contiguous(), w.bq, w.bk, idx, cnt, mode="sparse", rows=rows,
-                             kblocks=np.zeros(0, np.int64))
+        # forward and backward of the sampled rows' dQ (the sparse + linear mix on SLA2 workloads)
+        oracle.attention_bwd(Qh, Kh, Vh, dO[:1, :heads].contiguous(), w.bq, w.bk, idx, cnt,
+                             alpha=alpha[:heads].numpy() if w.sla2 else None, mode="sla2" if w.sla2 else "sparse",
+                             rows=rows, kblocks=np.zeros(0, np.int64))
     elif mode == "q8":
         oracle.attention_q8_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, rows)
     else:
@@ -265,7 +267,7 @@ def run_ours(args, w, rank, world, local_rank):
     Wq, Wk = (router_h[0].to(dev), router_h[1].to(dev)) if router_h is not None else (None, None)
     q8 = args.variant == "q8"
     bwd = args.variant == "bwd"
-    sla2 = w.sla2 and not q8 and not bwd  # the low-bit and backward variants run the sparse branch alone
+    sla2 = w.sla2 and not q8  # the low-bit variant runs the sparse branch alone
     n_sla2 = sparge.workspace_bytes(sparge.OP_SLA2, shape) if sla2 else 0
     ws_sla2 = torch.empty(max(1, n_sla2), dtype=torch.uint8, device=dev)
     n_q8 = sparge.workspace_bytes(sparge.OP_ATTN_Q8, shape) if q8 else 0
@@ -278,7 +280,9 @@ def run_ours(args, w, rank, world, local_rank):
         dO = dOh.to(dev)
         lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
         dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
-        ws_bwd = torch.empty(sparge.workspace_bytes(sparge.OP_ATTN_BWD, shape), dtype=torch.uint8, device=dev)
+        ws_bwd = torch.empty(sparge.workspace_bytes(sparge.OP_SLA2_BWD if sla2 else sparge.OP_ATTN_BWD, shape),
+                             dtype=torch.uint8, device=dev)
+        dalpha = torch.empty(H, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev_a=None, ev_b=None):
@@ -288,10 +292,17 @@ def run_ours(args, w, rank, world, local_rank):
         else:
             sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
         if bwd:
-            sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, lse=lse)
+            if sla2:
+                sparge.sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, w.bq, w.bk, O=O, workspace=ws_sla2)
+            else:
+                sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, lse=lse)
             if ev_a is not None:
                 ev_a.record(stream)
-            sparge.sparge_attn_bwd(Q, K, V, kv_idx, kv_cnt, O, lse, dO, w.bq, w.bk, dQ, dK, dV, workspace=ws_bwd)
+            if sla2:
+                sparge.sla2_attn_bwd(Q, K, V, kv_idx, kv_cnt, alpha, dO, w.bq, w.bk, dQ, dK, dV, dalpha,
+                                     workspace=ws_bwd)
+            else:
+                sparge.sparge_attn_bwd(Q, K, V, kv_idx, kv_cnt, O, lse, dO, w.bq, w.bk, dQ, dK, dV, workspace=ws_bwd)
             if ev_b is not None:
                 ev_b.record(stream)
             return
@@ -308,7 +319,7 @@ def run_ours(args, w, rank, world, local_rank):
 
     launches_per_step = ((sparge.ROUTER_LAUNCHES if Wq is not None else sparge.MASK_LAUNCHES) +
                          (sparge.Q8_LAUNCHES if q8 else sparge.SLA2_LAUNCHES if sla2 else sparge.ATTN_LAUNCHES) +
-                         (sparge.BWD_LAUNCHES if bwd else 0))
+                         ((sparge.SLA2_BWD_LAUNCHES if sla2 else sparge.BWD_LAUNCHES) if bwd else 0))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -343,7 +354,7 @@ def run_ours(args, w, rank, world, local_rank):
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        outs = (dQ, dK, dV) if bwd else (O,)
+        outs = ((dQ, dK, dV) + ((dalpha,) if sla2 else ())) if bwd else (O,)
         hosts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
         ins = [(Q, Qh), (K, Kh), (V, Vh)] + ([(dO, dOh)] if bwd else [])
 
@@ -390,7 +401,9 @@ def run_ours(args, w, rank, world, local_rank):
     kernel_name = "attn_q8_kernel" if q8 else (f"attn_fwd_kernel<{d}, 1>" if sla2 else f"attn_fwd_kernel<{d}, 0>")
     if bwd:
         kernel_name = "attn_bwd_dq_kernel + attn_bwd_dkdv_kernel"
-    span = ("sparge_attn_bwd (4 launches: D_i, transposed mask, dQ, dK/dV)" if bwd else
+    span = (("sla2_attn_bwd (12 launches: forward pieces, row pass, gradient summaries, transposed mask, dQ, "
+             "dK/dV sparse and linear parts)" if sla2 else
+             "sparge_attn_bwd (4 launches: D_i, transposed mask, dQ, dK/dV)") if bwd else
             "sparge_attn_fwd_q8 (3 launches: codes, V codes, attention)" if q8 else
             "sla2_attn_fwd (4 launches)" if sla2 else "sparge_attn_fwd (1 launch)")
     # Counters were captured with the plain mask; a router mask keeps other tiles.
@@ -407,9 +420,11 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded video-shaped Q/K/V, see synth.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
                    "topk": w.topk, "topp": w.topp, "alpha": "U[0.6,1] per head" if sla2 else 1.0,
-                   "path": "sparge_attn_fwd_q8" if q8 else "sparge_attn_fwd + sparge_attn_bwd" if bwd else
+                   "path": "sparge_attn_fwd_q8" if q8 else
+                           ("sla2_attn_fwd + sla2_attn_bwd" if sla2 else "sparge_attn_fwd + sparge_attn_bwd") if bwd else
                            ("sla2_attn_fwd" if sla2 else "sparge_attn_fwd"),
-                   "flops": "kept-block FLOPs x 3.5 (forward + backward)" if bwd else "kept-block FLOPs",
+                   "flops": ("kept-block FLOPs x 3.5 (forward + backward; the linear branch's work is not counted)"
+                             if bwd else "kept-block FLOPs"),
                    "mask": f"sparge_mask_router (dr {args.router})" if args.router else "sparge_mask",
                    "l2": f"inputs larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V per rank)",
                    "parallelism": f"independent replicas x{world}"},

@@ -663,11 +663,13 @@ struct BwdKVSmem {
   // dK(u), so the next loads into the slot start as early as possible.
   static constexpr int kBarKV = 0, kBarQFull = 1, kBarDOFull = 1 + NS, kBarQEmpty = 1 + 2 * NS,
                        kBarDOEmpty = 1 + 3 * NS, kBarSFull = 1 + 4 * NS, kBarPReady = 3 + 4 * NS,
-                       kBarStage = 4 + 4 * NS, kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS;
-  static constexpr int kNumBars = 7 + 4 * NS;
+                       kBarStage = 4 + 4 * NS, kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS,
+                       kBarPart = 7 + 4 * NS;
+  static constexpr int kNumBars = 8 + 4 * NS;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;
   static constexpr int kTmemCols = 512;
+  static constexpr int kPartBytes = kTileK * D * 4;  // one fp32 partial tile, four 32-column boxes
 };
 
 // 64 bf16 (pairs in pk) as row r of a [128 rows][64 columns] tile with the
@@ -716,7 +718,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-                         const __grid_constant__ CUtensorMap tmG, const BwdParams p, const BwdKVLin lk) {
+                         const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmKp,
+                         const __grid_constant__ CUtensorMap tmVp, const BwdParams p, const BwdKVLin lk) {
   using L = BwdKVSmem<D>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -756,6 +759,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar(L::kBarStage), 1);
     mbar_init(bar(L::kBarFinal), 1);
     mbar_init(bar(L::kBarDrain), 1);
+    mbar_init(bar(L::kBarPart), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -965,7 +969,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
     }
     // Epilogue: lane r holds channel r of dV^T and dK^T (keys along the columns).
-    const uint32_t sOutV = sRing, sOutK = sRing + L::kKBytes;
+    // MODE 2 brings the fp32 sparse partials of the tile into the (now idle)
+    // ring by TMA and stages its outputs in the staging area instead.
+    const uint32_t sOutV = MODE == 2 ? sP : sRing, sOutK = MODE == 2 ? sDS : sRing + L::kKBytes;
+    const uint8_t* partK = sgen + L::kOffRing;
+    const uint8_t* partV = sgen + L::kOffRing + L::kPartBytes;
+    if (MODE == 2) {
+      if (warp == 2 && lane == 0 && ok) {
+        mbar_arrive_expect_tx(bar(L::kBarPart), 2 * L::kPartBytes);
+        for (int b = 0; b < D / 32; ++b) {
+          tma_load_3d(sRing + b * (kTileK * 128), &tmKp, bar(L::kBarPart), b * 32, key0, bh);
+          tma_load_3d(sRing + L::kPartBytes + b * (kTileK * 128), &tmVp, bar(L::kBarPart), b * 32, key0, bh);
+        }
+      }
+      if (ok) ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarPart), 0, kErrBwdIn, abort_flag));
+    }
+    // Element (key j, channel r) of a loaded partial tile: 32-column boxes of 64 rows.
+    auto part_at = [&](const uint8_t* t, int j) {
+      return *reinterpret_cast<const float*>(t + (r / 32) * (kTileK * 128) + j * 128 + (r % 32) * 4);
+    };
     float v[kTileK];
     if (work && ok) {
       load_row64(tDV + lane_off, v);
@@ -982,8 +1004,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else {
       if (MODE == 2) {
 #pragma unroll
-        for (int j = 0; j < kTileK; ++j)
-          if (j < nvalid) v[j] += lk.dv_part[obase + (int64_t)j * D];
+        for (int j = 0; j < kTileK; ++j) v[j] += part_at(partV, j);
       }
       stage_col64<D>(sOutV, r, v, 1.0f);
     }
@@ -1002,8 +1023,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float g = __ldg(lk.g_all + (int64_t)bh * D + r);
 #pragma unroll
         for (int j = 0; j < kTileK; ++j)
-          if (j < nvalid)
-            v[j] = lk.dk_part[obase + (int64_t)j * D] + (v[j] - g) * fminf(tile_at(sgen + L::kOffK, j, r), 1.0f);
+          v[j] = part_at(partK, j) + (v[j] - g) * fminf(tile_at(sgen + L::kOffK, j, r), 1.0f);
       }
       stage_col64<D>(sOutK, r, v, MODE == 0 ? p.scale : 1.0f);
     }

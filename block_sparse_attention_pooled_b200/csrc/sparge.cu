@@ -208,6 +208,20 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t BH, int N, int box_ro
   return r == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map over [BH][N][128] with (32 columns x rows x 1) boxes, no swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, int64_t BH, int N, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {128 * 4, (cuuint64_t)N * 128 * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Workspace of the backward: D_i per row, the transposed mask (query-block
 // lists per key block and their lengths).
 struct BwdWs {
@@ -270,7 +284,7 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   e = ensure_smem(attn_bwd_dkdv_kernel<D, 0>, BwdKVSmem<D>::kBytes, 12);
   if (e != cudaSuccess) return cuda_status(e);
   attn_bwd_dkdv_kernel<D, 0><<<(unsigned)(dm.BH * ceil_div(s->N, kTileK)), kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, mq, p, lk);
+      mq, mk, mv, mdo, mdk, mdv, mq, mq, mq, p, lk);
   return cuda_status(cudaGetLastError());
 }
 
@@ -522,14 +536,15 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
       kv_idx, kv_cnt, (int)dm.nqb, (int)dm.nkb, q_idx, q_cnt);
   // 5. dQ (sparse + linear), then dK and dV: sparse part into fp32 partials,
   //    linear part and the combination into bf16.
-  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, mpq, msall, mg;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, mpq, msall, mg, mkp, mvp;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mdo, dO, dm.BH, s->N, D, kTileQ) ||
       !make_map_bhnd(&mdq, dQ, dm.BH, s->N, D, s->bq) || !make_map_bhnd(&mdk, dK, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mdv, dV, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mpk, at(w.f.phik), dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mpq, at(w.phiq), dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&msall, s_bf16, dm.BH, D, D, kTileQ) ||
-      !make_map_bhnd(&mg, g_bf16, dm.BH, D, D, kTileQ))
+      !make_map_bhnd(&mg, g_bf16, dm.BH, D, D, kTileQ) || !make_map_f32(&mkp, ws + w.dkp, dm.BH, s->N, kTileK) ||
+      !make_map_f32(&mvp, ws + w.dvp, dm.BH, s->N, kTileK))
     return SPARGE_ERR_CUDA;
   BwdParams p;
   p.lse = fat(w.lse);
@@ -564,15 +579,15 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   const unsigned kgrid = (unsigned)(dm.BH * ceil_div(s->N, kTileK));
   e = ensure_smem(attn_bwd_dkdv_kernel<D, 1>, BwdKVSmem<D>::kBytes, 15);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dkdv_kernel<D, 1><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, p,
-                                                                              lk);
+  attn_bwd_dkdv_kernel<D, 1><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mkp,
+                                                                              mvp, p, lk);
   BwdParams pl = p;
   pl.lse = fat(w.cw);
   pl.dsum = fat(w.fw);
   e = ensure_smem(attn_bwd_dkdv_kernel<D, 2>, BwdKVSmem<D>::kBytes, 16);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dkdv_kernel<D, 2><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mpq, mpk, mv, mdo, mdk, mdv, mg, pl,
-                                                                              lk);
+  attn_bwd_dkdv_kernel<D, 2><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mpq, mpk, mv, mdo, mdk, mdv, mg,
+                                                                              mkp, mvp, pl, lk);
   return cuda_status(cudaGetLastError());
 }
 

@@ -96,6 +96,24 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s128), P, P, P, None, 0, None) == lib.ERR_WORKSPACE
     assert raw.sparge_attn_fwd_q8(P, P, P, ctypes.byref(s128), P, P, P, P, 64, None) == lib.ERR_WORKSPACE
     assert raw.sparge_attn_fwd_q8(P, None, P, ctypes.byref(s128), P, P, P, P, 1 << 30, None) == lib.ERR_INVALID_ARG
+    # Backward entry points: d = 128 only, every buffer required, workspace sized for them.
+    s128b = lib.Shape(1, 2, 4096, 128, 128, 64)
+    nb = lib.workspace_bytes(lib.OP_ATTN_BWD, s128b)
+    assert nb > 0 and lib.workspace_bytes(lib.OP_ATTN_BWD, s) == 0
+    assert raw.sparge_attn_bwd(P, P, P, ctypes.byref(s), P, P, P, P, P, P, P, P, P, 1 << 30, None) == lib.ERR_UNSUPPORTED
+    assert raw.sparge_attn_bwd(P, P, P, ctypes.byref(s128b), P, P, P, None, P, P, P, P, P, 1 << 30,
+                               None) == lib.ERR_INVALID_ARG  # lse required
+    assert raw.sparge_attn_bwd(P, P, P, ctypes.byref(s128b), P, P, P, P, P, P, P, P, P, nb - 1,
+                               None) == lib.ERR_WORKSPACE
+    ns = lib.workspace_bytes(lib.OP_SLA2_BWD, s128b)
+    assert ns > nb
+    assert raw.sla2_attn_bwd(P, P, P, ctypes.byref(s128b), P, P, None, P, P, P, P, P, P, 1 << 34,
+                             None) == lib.ERR_INVALID_ARG  # alpha required
+    assert raw.sla2_attn_bwd(P, P, P, ctypes.byref(s128b), P, P, P, P, P, P, P, None, P, 1 << 34,
+                             None) == lib.ERR_INVALID_ARG  # dalpha required
+    assert raw.sla2_attn_bwd(P, P, P, ctypes.byref(s128b), P, P, P, P, P, P, P, P, P, ns - 1,
+                             None) == lib.ERR_WORKSPACE
+    assert raw.sla2_attn_bwd(P, P, P, ctypes.byref(s), P, P, P, P, P, P, P, P, P, 1 << 34, None) == lib.ERR_UNSUPPORTED
     # Learnt router: both projections required, 4-byte aligned; dr 64 or 128; workspace sized for it.
     W, big = ctypes.c_void_p(32 * 1024), 1 << 30
     assert raw.sparge_mask_router(P, P, ctypes.byref(s), None, W, 64, 0.1, 0.9, P, P, None, None, P, big,
