@@ -275,6 +275,7 @@ def run_ours(args, w, rank, world, local_rank):
     kv_idx = torch.empty((B, H, w.nqb, w.nkb), dtype=torch.int32, device=dev)
     kv_cnt = torch.empty((B, H, w.nqb), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
+    ws_attn = torch.empty(sparge.workspace_bytes(sparge.OP_ATTN, shape), dtype=torch.uint8, device=dev)
     if bwd:
         dOh = pin(synth.make_dout(w.B, w.H, w.N, w.d, seed=w.seed + rank))
         dO = dOh.to(dev)
@@ -295,7 +296,7 @@ def run_ours(args, w, rank, world, local_rank):
             if sla2:
                 sparge.sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, w.bq, w.bk, O=O, workspace=ws_sla2)
             else:
-                sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, lse=lse)
+                sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, lse=lse, workspace=ws_attn)
             if ev_a is not None:
                 ev_a.record(stream)
             if sla2:
@@ -313,13 +314,15 @@ def run_ours(args, w, rank, world, local_rank):
         elif sla2:
             sparge.sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, w.bq, w.bk, O=O, workspace=ws_sla2)
         else:
-            sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O)
+            sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, workspace=ws_attn)
         if ev_b is not None:
             ev_b.record(stream)
 
+    n_order = sparge.order_launches(shape)
     launches_per_step = ((sparge.ROUTER_LAUNCHES if Wq is not None else sparge.MASK_LAUNCHES) +
                          (sparge.Q8_LAUNCHES if q8 else sparge.SLA2_LAUNCHES if sla2 else sparge.ATTN_LAUNCHES) +
-                         ((sparge.SLA2_BWD_LAUNCHES if sla2 else sparge.BWD_LAUNCHES) if bwd else 0))
+                         n_order + ((sparge.SLA2_BWD_LAUNCHES if sla2 else sparge.BWD_LAUNCHES) + n_order
+                                    if bwd else 0))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -395,17 +398,17 @@ def run_ours(args, w, rank, world, local_rank):
         peak *= 2.0
         peak_desc += " x 2 (nominal int8 / e4m3 to bf16 ratio)"
     achieved = span_flops / (attn_avg * 1e-3) / 1e12
-    # The timed span is one library call: attn_fwd_kernel alone for the pure
-    # sparse path; linear_summary + linear_reduce + attn_fwd_kernel<128, 1>
-    # for the sparse + linear mix (the attention kernel is about 96% of it).
+    # The timed span is one library call: tile order + attn_fwd_kernel for the
+    # pure sparse path; tile order, linear summaries, linear_out and
+    # attn_fwd_kernel<128, 1> for the sparse + linear mix.
     kernel_name = "attn_q8_kernel" if q8 else (f"attn_fwd_kernel<{d}, 1>" if sla2 else f"attn_fwd_kernel<{d}, 0>")
     if bwd:
         kernel_name = "attn_bwd_dq_kernel + attn_bwd_dkdv_kernel"
-    span = (("sla2_attn_bwd (12 launches: forward pieces, row pass, gradient summaries, transposed mask, dQ, "
+    span = (("sla2_attn_bwd (12-13 launches: forward pieces, row pass, gradient summaries, transposed mask, dQ, "
              "dK/dV sparse and linear parts)" if sla2 else
-             "sparge_attn_bwd (4 launches: D_i, transposed mask, dQ, dK/dV)") if bwd else
-            "sparge_attn_fwd_q8 (3 launches: codes, V codes, attention)" if q8 else
-            "sla2_attn_fwd (4 launches)" if sla2 else "sparge_attn_fwd (1 launch)")
+             "sparge_attn_bwd (D_i, transposed mask, tile order when used, dQ, dK/dV)") if bwd else
+            "sparge_attn_fwd_q8 (codes, V codes, tile order when used, attention)" if q8 else
+            "sla2_attn_fwd (4-5 launches)" if sla2 else "sparge_attn_fwd (tile order when used, attention)")
     # Counters were captured with the plain mask; a router mask keeps other tiles.
     traffic = None if (args.router or bwd) else dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
     cpu = None

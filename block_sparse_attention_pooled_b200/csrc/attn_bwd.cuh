@@ -46,6 +46,7 @@ enum : unsigned int {
 struct BwdParams {
   const int32_t* lst;  // dQ: kv_idx [BH, nqb, nkb]; dK/dV: query-block lists [BH, nkb, nqb]
   const int32_t* cnt;  // dQ: kv_cnt [BH, nqb];       dK/dV: list lengths [BH, nkb]
+  const int32_t* order;  // dQ: launch order of the query tiles (as the forward's), or null
   const float* lse;    // [BH, N], natural log, from the forward
   const float* dsum;   // [BH, N], D_i = dO_i . O_i
   int N;
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int tile = blockIdx.x;  // (bh, query block), head-major
+  const int tile = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;  // (bh, query block)
   const int bh = tile / p.nqb;
   const int q0 = (tile % p.nqb) * p.bq;
   const int tiles_per_block = p.bk / kTileK;

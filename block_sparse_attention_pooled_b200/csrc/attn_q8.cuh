@@ -49,6 +49,7 @@ enum : unsigned int {
 struct Q8Params {
   const int32_t* kv_idx;  // [BH, nqb, nkb]
   const int32_t* kv_cnt;  // [BH, nqb]
+  const int32_t* order;   // [BH * nqb] launch order of the tiles, or null (head-major)
   const float* sq;        // [BH, nqb]
   const float* sk;        // [BH, nkb]
   const float* sv;        // [BH, 128]
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kQ8Threads, 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int tile = blockIdx.x;  // (bh, query block), head-major
+  const int tile = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;  // (bh, query block)
   const int bh = tile / p.nqb;
   const int qb = tile % p.nqb;
   const int q0 = qb * p.bq;

@@ -475,4 +475,73 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restric
   }
 }
 
+// ----------------------------------------------------------------------------
+// Launch order of the query tiles for the kernels that walk a tile's kept
+// blocks (their work is proportional to the kept count, which varies several
+// times over between tiles). Heads go in groups of G, so the K and V of a
+// group stay resident in L2 while its tiles run; inside a group the tiles
+// with more kept blocks come first, so the last wave of the grid holds the
+// lightest tiles. order[] is a permutation of [0, BH * Nqb); one CTA sorts
+// one group by counting (kept counts are at most Nkb). The order of equal
+// counts depends on scheduling; the kernels' results do not depend on the
+// order at all.
+// ----------------------------------------------------------------------------
+constexpr int kOrderThreads = 1024;
+
+__host__ __device__ constexpr int tile_order_smem_bytes(int nkb) { return (nkb + 1) * 4 + 32 * 4; }
+
+__global__ void __launch_bounds__(kOrderThreads) tile_order_kernel(const int32_t* __restrict__ kv_cnt, int64_t BH,
+                                                                   int nqb, int nkb, int G,
+                                                                   int32_t* __restrict__ order) {
+  extern __shared__ int hist[];  // [nkb + 1] bins (descending kept count), then 32 warp totals
+  int* wsum = hist + nkb + 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t h0 = (int64_t)blockIdx.x * G;
+  const int nh = (int)(BH - h0 < G ? BH - h0 : G);
+  const int n = nh * nqb;
+  const int64_t t0 = h0 * nqb;
+  for (int b = tid; b <= nkb; b += kOrderThreads) hist[b] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kOrderThreads) {
+    const int c = min(max(__ldg(kv_cnt + t0 + i), 0), nkb);
+    atomicAdd(&hist[nkb - c], 1);
+  }
+  __syncthreads();
+  // Exclusive scan of the bins: each thread owns a run of `per` bins.
+  const int per = (nkb + 1 + kOrderThreads - 1) / kOrderThreads;
+  const int b0 = tid * per, b1 = min(nkb + 1, b0 + per);
+  int run = 0;
+  for (int b = b0; b < b1; ++b) run += hist[b];
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
+    }
+    wsum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int off = incl - run + (warp > 0 ? wsum[warp - 1] : 0);
+  for (int b = b0; b < b1; ++b) {
+    const int c = hist[b];
+    hist[b] = off;
+    off += c;
+  }
+  __syncthreads();
+  for (int i = tid; i < n; i += kOrderThreads) {
+    const int c = min(max(__ldg(kv_cnt + t0 + i), 0), nkb);
+    const int pos = atomicAdd(&hist[nkb - c], 1);
+    order[t0 + pos] = (int32_t)(t0 + i);
+  }
+}
+
 }  // namespace sparge

@@ -133,6 +133,26 @@ cudaError_t ensure_smem(K kernel, int bytes, int slot) {
   return e;
 }
 
+// Launch order of the query tiles (tile_order_kernel): heads in groups whose
+// K and V (2 N d bf16 each) fit in 64 MB of L2, heaviest tiles first. When not
+// even two heads fit, the grid stays head-major (sorting inside one head
+// measured slower: it breaks the locality of neighbouring query blocks, which
+// keep mostly the same key blocks), and *order is set to null.
+cudaError_t launch_tile_order(const int32_t* kv_cnt, const sparge_shape* s, const Dims& dm, int32_t** order,
+                              cudaStream_t st) {
+  const int64_t per_head = 4 * (int64_t)s->N * s->d;
+  const int64_t G = std::min<int64_t>(dm.BH, (int64_t(64) << 20) / per_head);
+  if (G < 2) {
+    *order = nullptr;
+    return cudaSuccess;
+  }
+  tile_order_kernel<<<(unsigned)ceil_div(dm.BH, G), kOrderThreads, tile_order_smem_bytes((int)dm.nkb), st>>>(
+      kv_cnt, dm.BH, (int)dm.nqb, (int)dm.nkb, (int)G, *order);
+  return cudaGetLastError();
+}
+
+inline size_t order_bytes(const Dims& d) { return align256((size_t)d.BH * d.nqb * 4); }
+
 // Scores of DD-wide pooled (or projected) vectors into P.
 template <int DD>
 cudaError_t launch_scores(const float* a, const float* b, const Dims& dm, float* P, cudaStream_t st) {
@@ -225,7 +245,7 @@ bool make_map_f32(CUtensorMap* m, const void* base, int64_t BH, int N, int box_r
 // Workspace of the backward: D_i per row, the transposed mask (query-block
 // lists per key block and their lengths).
 struct BwdWs {
-  size_t dsum, qidx, qcnt, total;
+  size_t dsum, qidx, qcnt, order, total;
 };
 
 BwdWs bwd_ws(const sparge_shape* s, const Dims& d) {
@@ -233,7 +253,8 @@ BwdWs bwd_ws(const sparge_shape* s, const Dims& d) {
   w.dsum = 0;
   w.qidx = w.dsum + align256((size_t)d.BH * s->N * 4);
   w.qcnt = w.qidx + align256((size_t)d.BH * d.nkb * d.nqb * 4);
-  w.total = w.qcnt + align256((size_t)d.BH * d.nkb * 4);
+  w.order = w.qcnt + align256((size_t)d.BH * d.nkb * 4);
+  w.total = w.order + order_bytes(d);
   return w;
 }
 
@@ -271,6 +292,10 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   p.bk = s->bk;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.scale = (float)(1.0 / std::sqrt((double)D));
+  int32_t* order = reinterpret_cast<int32_t*>(ws + w.order);
+  e = launch_tile_order(kv_cnt, s, dm, &order, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  p.order = order;
   p.lst = kv_idx;
   p.cnt = kv_cnt;
   const BwdLinParams lp{};
@@ -278,6 +303,7 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   if (e != cudaSuccess) return cuda_status(e);
   attn_bwd_dq_kernel<D, false><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D, false>::kBytes, st>>>(
       mq, mk, mv, mdo, mdq, mk, mq, p, lp);
+  p.order = nullptr;
   p.lst = q_idx;
   p.cnt = q_cnt;
   const BwdKVLin lk{};
@@ -290,7 +316,7 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
 
 // Workspace of the low-bit sparse branch: codes and scales of Q, K, V.
 struct Q8Ws {
-  size_t q8, k8, v8, sq, sk, sv, vpart, total;
+  size_t q8, k8, v8, sq, sk, sv, vpart, order, total;
 };
 
 Q8Ws q8_ws(const sparge_shape* s, const Dims& d) {
@@ -304,7 +330,8 @@ Q8Ws q8_ws(const sparge_shape* s, const Dims& d) {
   w.sk = w.sq + align256((size_t)d.BH * d.nqb * 4);
   w.sv = w.sk + align256((size_t)d.BH * d.nkb * 4);
   w.vpart = w.sv + align256((size_t)d.BH * s->d * 4);
-  w.total = w.vpart + align256((size_t)d.BH * nch * s->d * 4);
+  w.order = w.vpart + align256((size_t)d.BH * nch * s->d * 4);
+  w.total = w.order + order_bytes(d);
   return w;
 }
 
@@ -331,9 +358,13 @@ sparge_status launch_q8(const void* Q, const void* K, const void* V, const sparg
   if (!make_map_u8(&mq, q8, dm.BH, s->N, kTileQ) || !make_map_u8(&mk, k8, dm.BH, s->N, kTileK) ||
       !make_map_u8(&mv, v8, dm.BH, s->N, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
     return SPARGE_ERR_CUDA;
+  int32_t* order = reinterpret_cast<int32_t*>(ws + w.order);
+  cudaError_t eo = launch_tile_order(kv_cnt, s, dm, &order, st);
+  if (eo != cudaSuccess) return cuda_status(eo);
   Q8Params p;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
+  p.order = order;
   p.sq = sq;
   p.sk = sk;
   p.sv = sv;
@@ -350,7 +381,7 @@ sparge_status launch_q8(const void* Q, const void* K, const void* V, const sparg
 }
 
 struct Sla2Ws {
-  size_t phik, s_all, z_all, z_tile, partial, total;
+  size_t phik, s_all, z_all, z_tile, partial, order, total;
 };
 
 inline int lin_ctas_per_head(int N) { return (int)ceil_div(ceil_div(N, 64), kLinTilesPerCta); }
@@ -362,14 +393,15 @@ Sla2Ws sla2_ws(const sparge_shape* s, const Dims& d) {
   w.z_all = w.s_all + align256((size_t)d.BH * s->d * s->d * 4);
   w.z_tile = w.z_all + align256((size_t)d.BH * s->d * 4);
   w.partial = w.z_tile + align256((size_t)d.BH * ceil_div(s->N, 64) * s->d * 4);
-  w.total = w.partial + align256((size_t)d.BH * lin_ctas_per_head(s->N) * kLinPartial * 4);
+  w.order = w.partial + align256((size_t)d.BH * lin_ctas_per_head(s->N) * kLinPartial * 4);
+  w.total = w.order + order_bytes(d);
   return w;
 }
 
 template <int D, bool MIX>
 sparge_status launch_attn(const void* Q, const void* K, const void* V, const sparge_shape* s, const Dims& dm,
                           const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, const float* alpha,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int32_t* order = nullptr) {
   CUtensorMap mq, mk, mv, mo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mo, O, dm.BH, s->N, D, s->bq))
@@ -379,6 +411,7 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
   p.H = s->H;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
+  p.order = order;
   p.lse = lse;
   p.N = s->N;
   p.nqb = (int)dm.nqb;
@@ -397,7 +430,7 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
 sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape* s, const Dims& dm,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, const void* phik, const float* s_all,
                                 const float* z_all, const float* z_tile, const float* alpha, void* O,
-                                cudaStream_t st, float* den_out = nullptr) {
+                                cudaStream_t st, float* den_out = nullptr, const int32_t* order = nullptr) {
   CUtensorMap mq, mv, mp, mo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, 128, 128) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
@@ -405,6 +438,7 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   LoParams p;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
+  p.order = order;
   p.s_all = s_all;
   p.z_all = z_all;
   p.z_tile = z_tile;
@@ -510,10 +544,13 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   if (r != SPARGE_OK) return r;
   cudaError_t e = cudaMemsetAsync(at(w.alpha0), 0, (size_t)s->H * 4, st);
   if (e != cudaSuccess) return cuda_status(e);
+  int32_t* order = reinterpret_cast<int32_t*>(ws + w.f.order);
+  e = launch_tile_order(kv_cnt, s, dm, &order, st);
+  if (e != cudaSuccess) return cuda_status(e);
   r = launch_linear_out(Q, V, s, dm, kv_idx, kv_cnt, at(w.f.phik), fat(w.f.s_all), fat(w.f.z_all), fat(w.f.z_tile),
-                        fat(w.alpha0), at(w.ol), st, fat(w.den));
+                        fat(w.alpha0), at(w.ol), st, fat(w.den), order);
   if (r != SPARGE_OK) return r;
-  r = launch_attn<D, false>(Q, K, V, s, dm, kv_idx, kv_cnt, at(w.os), fat(w.lse), nullptr, st);
+  r = launch_attn<D, false>(Q, K, V, s, dm, kv_idx, kv_cnt, at(w.os), fat(w.lse), nullptr, st, order);
   if (r != SPARGE_OK) return r;
   // 2. Row pass and dalpha.
   const int chunks = sla2_row_chunks(s->N);
@@ -556,6 +593,7 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   p.bk = s->bk;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.scale = (float)(1.0 / std::sqrt((double)D));
+  p.order = order;
   p.lst = kv_idx;
   p.cnt = kv_cnt;
   BwdLinParams lp;
@@ -568,6 +606,7 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   if (e != cudaSuccess) return cuda_status(e);
   attn_bwd_dq_kernel<D, true><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D, true>::kBytes, st>>>(
       mq, mk, mv, mdo, mdq, mpk, msall, p, lp);
+  p.order = nullptr;
   p.lst = q_idx;
   p.cnt = q_cnt;
   BwdKVLin lk;
@@ -629,7 +668,7 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape) {
     case SPARGE_OP_MASK:
       return mask_ws(shape, dm).total;
     case SPARGE_OP_ATTN:
-      return 0;
+      return order_bytes(dm);
     case SPARGE_OP_SLA2:
       return shape->d == 128 ? sla2_ws(shape, dm).total : 0;
     case SPARGE_OP_ATTN_Q8:
@@ -729,17 +768,20 @@ sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_sha
 sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                               const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse, void* workspace,
                               size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   Dims dm;
   sparge_status st = check_shape(shape, &dm);
   if (st != SPARGE_OK) return st;
   if (!Q || !K || !V || !O || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARGE_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < order_bytes(dm) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SPARGE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* order = static_cast<int32_t*>(workspace);
+  cudaError_t e = launch_tile_order(kv_cnt, shape, dm, &order, s);
+  if (e != cudaSuccess) return cuda_status(e);
   if (shape->d == 64)
-    return launch_attn<64, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s);
-  return launch_attn<128, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s);
+    return launch_attn<64, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s, order);
+  return launch_attn<128, false>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, lse, nullptr, s, order);
 }
 
 sparge_status sparge_attn_fwd_q8(const void* Q, const void* K, const void* V, const sparge_shape* shape,
@@ -777,11 +819,14 @@ sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const s
   float* z_all = reinterpret_cast<float*>(ws + w.z_all);
   float* z_tile = reinterpret_cast<float*>(ws + w.z_tile);
   float* partial = reinterpret_cast<float*>(ws + w.partial);
+  int32_t* order = reinterpret_cast<int32_t*>(ws + w.order);
+  cudaError_t e = launch_tile_order(kv_cnt, shape, dm, &order, s);
+  if (e != cudaSuccess) return cuda_status(e);
   st = launch_summaries(K, V, shape, dm, phik, partial, s_all, z_all, z_tile, s);
   if (st != SPARGE_OK) return st;
-  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, z_tile, alpha, O, s);
+  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, z_tile, alpha, O, s, nullptr, order);
   if (st != SPARGE_OK) return st;
-  return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, alpha, s);
+  return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, alpha, s, order);
 }
 
 sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,

@@ -26,12 +26,19 @@ OP_MASK, OP_ATTN, OP_SLA2, OP_ATTN_Q8, OP_MASK_ROUTER, OP_ATTN_BWD, OP_SLA2_BWD 
 MASK_LAUNCHES, ATTN_LAUNCHES, SLA2_LAUNCHES, Q8_LAUNCHES, ROUTER_LAUNCHES, BWD_LAUNCHES = 3, 1, 4, 3, 5, 4
 # sla2_attn_bwd: summaries + reduce, linear_out, sparse forward, row pass, dalpha, gradient summaries
 # + reduce, transposed mask, dQ, dK/dV sparse part, dK/dV linear part (the memset is not a kernel).
+# The attention, SLA2 and low-bit forward calls and both backward calls add order_launches(shape).
 SLA2_BWD_LAUNCHES = 12
 
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
            "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8",
            "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd")
+
+
+def order_launches(shape) -> int:
+    """Launches of the tile-order kernel per attention call for this shape (launch accounting):
+    1 when at least two heads' K and V (4 N d bytes each) fit in 64 MB, else 0."""
+    return 1 if min(shape.B * shape.H, (64 << 20) // (4 * shape.N * shape.d)) >= 2 else 0
 
 
 class Shape(ctypes.Structure):

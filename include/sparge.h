@@ -163,7 +163,11 @@ sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_sha
  *              softmax_j(q_i . k_j / sqrt(d)) v_j, in fp32, stored as bf16.
  *   lse         optional output, float [B,H,N]: natural-log log-sum-exp of the
  *               scaled scores over the kept keys; -inf where nothing is kept.
- * A row whose block keeps nothing gets O = 0. Workspace: none (0 bytes). */
+ * A row whose block keeps nothing gets O = 0.
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN, shape) (4 bytes per query
+ * tile: the launch order of the tiles, heavier kept lists first within groups
+ * of heads whose K and V fit in 64 MB of L2; the result does not depend on
+ * it). Two launches (one when not even two heads fit: head-major order). */
 sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                               const int32_t* kv_idx, const int32_t* kv_cnt, void* O, float* lse,
                               void* workspace, size_t workspace_bytes, void* stream);
@@ -185,8 +189,9 @@ sparge_status sparge_attn_fwd(const void* Q, const void* K, const void* V, const
  * accumulation; D_i from the bf16 O and dO in fp32.
  * d must be 128 (else SPARGE_ERR_UNSUPPORTED), and Nqb * 32 bytes must not
  * exceed 200 KiB (the transposed-mask bit matrix of one CTA).
- * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN_BWD, shape) (D_i, and for
- * every key block the ascending list of query blocks that keep it). */
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN_BWD, shape) (D_i, for
+ * every key block the ascending list of query blocks that keep it, and the
+ * query tiles' launch order as in sparge_attn_fwd). */
 sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                               const int32_t* kv_idx, const int32_t* kv_cnt, const void* O, const float* lse,
                               const void* dO, void* dQ, void* dK, void* dV, void* workspace,
@@ -228,7 +233,8 @@ sparge_status sla2_attn_bwd(const void* Q, const void* K, const void* V, const s
  *         the kept key tiles (64 keys, ascending); the normaliser sums e.
  *   O     = sum(P * v_codes) / (sum(e) * s_v), stored as bf16.
  * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN_Q8, shape) (codes and
- * scales). Three launches: Q/K codes with V channel maxima, V codes, attention. */
+ * scales, the tiles' launch order). Three or four launches: Q/K codes with V channel maxima,
+ * V codes, the launch order of the query tiles (as sparge_attn_fwd), attention. */
 sparge_status sparge_attn_fwd_q8(const void* Q, const void* K, const void* V, const sparge_shape* shape,
                                  const int32_t* kv_idx, const int32_t* kv_cnt, void* O, void* workspace,
                                  size_t workspace_bytes, void* stream);
@@ -240,8 +246,9 @@ sparge_status sparge_attn_fwd_q8(const void* Q, const void* K, const void* V, co
  *   phi(x) = elu(x) + 1; O_linear = 0 when every block is kept.
  *   alpha       float [H], device.
  * d must be 128. Workspace: sparge_workspace_bytes(SPARGE_OP_SLA2, shape).
- * Four launches: phi(K) and per-CTA partial sums of phi(K)^T [V | 1]; their
- * fixed-order reduction to the per-head totals; the linear branch of every
+ * Four or five launches: the launch order of the query tiles (as sparge_attn_fwd);
+ * phi(K) and per-CTA partial sums of phi(K)^T [V | 1]; their fixed-order
+ * reduction to the per-head totals; the linear branch of every
  * query block, written into O as (1 - alpha[h]) O_linear (bf16); the sparse
  * branch, which reads that tile back and adds alpha[h] O_sparse. O is
  * therefore also scratch between the last two launches. */

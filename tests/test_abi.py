@@ -52,7 +52,7 @@ def test_workspace_bytes_host_arithmetic(lib):
     nqb, nkb = 591, 1182
     need = lib.workspace_bytes(lib.OP_MASK, s)
     assert need >= 40 * (nqb + nkb) * 128 * 4 + 40 * nqb * nkb * 4
-    assert lib.workspace_bytes(lib.OP_ATTN, s) == 0
+    assert lib.workspace_bytes(lib.OP_ATTN, s) >= 40 * nqb * 4  # the tiles' launch order
     bad = lib.Shape(1, 1, 100, 96, 64, 64)  # unsupported head dim
     assert lib.workspace_bytes(lib.OP_MASK, bad) == 0
     # Low-bit branch: three code tensors of one byte per element plus the scales.
