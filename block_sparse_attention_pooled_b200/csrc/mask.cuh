@@ -62,12 +62,12 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
     }
   };
   int r = 0;
-  for (; r + 8 <= rows; r += 8) {
-    uint4 v[8];
+  for (; r + 16 <= rows; r += 16) {  // 16 rows in flight per thread, added in order
+    uint4 v[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + (int64_t)(r + u) * (D / 8));
+    for (int u = 0; u < 16; ++u) v[u] = __ldg(src + (int64_t)(r + u) * (D / 8));
 #pragma unroll
-    for (int u = 0; u < 8; ++u) add_row(v[u]);  // rows in order
+    for (int u = 0; u < 16; ++u) add_row(v[u]);
   }
   for (; r < rows; ++r) add_row(__ldg(src + (int64_t)r * (D / 8)));
   const float cnt = (float)rows;
@@ -157,17 +157,31 @@ __global__ void __launch_bounds__(128) score_kernel(const float* __restrict__ qb
   const int nrows = min(kScoreRows, nqb - I0);
   const int nj = min(kScoreTileJ, nkb - J0);
   const int tid = threadIdx.x;
-  for (int e = tid; e < kScoreRows * (D / 4); e += 128) {
-    const int i = e / (D / 4), c4 = (e % (D / 4)) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < nrows) v = *reinterpret_cast<const float4*>(qbar + (bh * nqb + I0 + i) * D + c4);
-    *reinterpret_cast<float4*>(sq + i * D + c4) = v;
+  // Every load of the tile is issued before the first store (unrolled), so
+  // the CTA waits for one round trip to L2 rather than one per 128 vectors.
+  constexpr int kQVec = kScoreRows * (D / 4) / 128, kKVec = kScoreTileJ * (D / 4) / 128;
+  float4 vq[kQVec], vk[kKVec];
+#pragma unroll
+  for (int u = 0; u < kQVec; ++u) {
+    const int e = tid + 128 * u, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    vq[u] = i < nrows ? *reinterpret_cast<const float4*>(qbar + (bh * nqb + I0 + i) * D + c4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int e = tid; e < kScoreTileJ * (D / 4); e += 128) {
-    const int j = e / (D / 4), c4 = (e % (D / 4)) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < nj) v = *reinterpret_cast<const float4*>(kbar + (bh * nkb + J0 + j) * D + c4);
-    *reinterpret_cast<float4*>(sk + j * (D + 4) + c4) = v;
+#pragma unroll
+  for (int u = 0; u < kKVec; ++u) {
+    const int e = tid + 128 * u, j = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    vk[u] = j < nj ? *reinterpret_cast<const float4*>(kbar + (bh * nkb + J0 + j) * D + c4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int u = 0; u < kQVec; ++u) {
+    const int e = tid + 128 * u, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    *reinterpret_cast<float4*>(sq + i * D + c4) = vq[u];
+  }
+#pragma unroll
+  for (int u = 0; u < kKVec; ++u) {
+    const int e = tid + 128 * u, j = e / (D / 4), c4 = (e % (D / 4)) * 4;
+    *reinterpret_cast<float4*>(sk + j * (D + 4) + c4) = vk[u];
   }
   __syncthreads();
   const int jl = tid % 16;   // key blocks jl, jl+16, jl+32, jl+48 of the tile
