@@ -490,6 +490,205 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restric
 }
 
 // ----------------------------------------------------------------------------
+// The same selection with one warp per row (eight rows per CTA), for rows of
+// at most kSelWarpMaxNkb blocks: every step is the arithmetic of
+// select_kernel (the softmax's 32 interleaved partial sums are exactly one
+// warp's lanes; the running weights are exact integers; the radix passes
+// walk the same 8-bit digits), but the row's steps synchronise with warp
+// barriers instead of block barriers. Each warp owns its row's P (then keys)
+// and a 256-bucket histogram in shared memory.
+// ----------------------------------------------------------------------------
+constexpr int kSelWarpRows = 8;
+constexpr int kSelWarpMaxNkb = 1024;
+
+__host__ __device__ constexpr int select_warp_bytes(int nkb) { return (nkb + 3) / 4 * 16 + 256 * 12 + 16; }
+__host__ __device__ constexpr int select_warp_smem_bytes(int nkb) { return kSelWarpRows * select_warp_bytes(nkb); }
+
+// One radix pass of the warp version (see radix_pass): returns the selected
+// digit and updates prefix / above_w / above_c; called by all 32 lanes.
+__device__ __forceinline__ void radix_pass_warp(const unsigned int* keys, int nkb, int shift, unsigned int hi_mask,
+                                                bool by_weight, unsigned long long target, unsigned int* prefix,
+                                                unsigned long long* above_w, int* above_c, unsigned int* hcnt,
+                                                unsigned long long* hsum) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    hcnt[lane * 8 + i] = 0u;
+    hsum[lane * 8 + i] = 0ull;
+  }
+  __syncwarp();
+  const unsigned int pre = *prefix;
+  for (int j = lane; j < nkb; j += 32) {
+    const unsigned int k = keys[j];
+    if ((k & hi_mask) == pre) {
+      const unsigned int d = (k >> shift) & 255u;
+      atomicAdd(&hcnt[d], 1u);
+      if (by_weight) atomicAdd(&hsum[d], p_fixed62(k));
+    }
+  }
+  __syncwarp();
+  // Lane l owns buckets 255-8l ... 248-8l (descending).
+  unsigned long long lw = 0ull;
+  unsigned int lc = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = 255 - 8 * lane - i;
+    lw += hsum[b];
+    lc += hcnt[b];
+  }
+  unsigned long long xw = lw;
+  unsigned int xc = lc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long yw = __shfl_up_sync(0xffffffffu, xw, o);
+    const unsigned int yc = __shfl_up_sync(0xffffffffu, xc, o);
+    if (lane >= o) {
+      xw += yw;
+      xc += yc;
+    }
+  }
+  const unsigned long long aw = *above_w + xw - lw;
+  const unsigned int ac = (unsigned int)*above_c + xc - lc;
+  const bool reach = by_weight ? (aw + lw >= target) : ((unsigned long long)(ac + lc) >= target);
+  const unsigned int ballot = __ballot_sync(0xffffffffu, reach);
+  const int first = __ffs(ballot) - 1;
+  unsigned long long w = aw;
+  unsigned int c = ac;
+  int bsel = 255 - 8 * lane - 7;
+  if (lane == first) {
+    for (int i = 0; i < 8; ++i) {
+      const int b = 255 - 8 * lane - i;
+      const bool hit = by_weight ? (w + hsum[b] >= target) : ((unsigned long long)(c + hcnt[b]) >= target);
+      if (hit) {
+        bsel = b;
+        break;
+      }
+      w += hsum[b];
+      c += hcnt[b];
+    }
+  }
+  bsel = __shfl_sync(0xffffffffu, bsel, first);
+  c = __shfl_sync(0xffffffffu, c, first);
+  w = __shfl_sync(0xffffffffu, w, first);
+  *prefix = pre | ((unsigned int)bsel << shift);
+  *above_c = (int)c;
+  *above_w = w;
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(float* __restrict__ P, int64_t rows, int nkb,
+                                                                        int kc, double topp,
+                                                                        int32_t* __restrict__ kv_idx,
+                                                                        int32_t* __restrict__ kv_cnt,
+                                                                        float* __restrict__ row_thresh) {
+  extern __shared__ __align__(16) unsigned char smraw[];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t row = (int64_t)blockIdx.x * kSelWarpRows + wid;
+  if (row >= rows) return;  // whole warps only: no block barrier follows
+  unsigned char* mine = smraw + wid * select_warp_bytes(nkb);
+  float* ev = reinterpret_cast<float*>(mine);                                      // [nkb], then the keys
+  unsigned int* keys = reinterpret_cast<unsigned int*>(mine);
+  unsigned long long* hsum = reinterpret_cast<unsigned long long*>(mine + (nkb + 3) / 4 * 16);  // [256]
+  unsigned int* hcnt = reinterpret_cast<unsigned int*>(hsum + 256);                // [256]
+  float* prow = P + row * (int64_t)nkb;
+
+  // 0. Row softmax: max, exponentials, lane l's partial sum over l, l+32, ...
+  float mx = -INFINITY;
+  for (int j = lane; j < nkb; j += 32) {
+    const float z = prow[j];
+    ev[j] = z;
+    mx = fmaxf(mx, z);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float part = 0.0f;
+  for (int j = lane; j < nkb; j += 32) {
+    const float e = expf(__fsub_rn(ev[j], mx));
+    ev[j] = e;
+    part = __fadd_rn(part, e);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+  const float rsum = part;
+  unsigned long long tot = 0ull;  // total weight (exact integer sum)
+  for (int j = lane; j < nkb; j += 32) {
+    const float pj = __fdiv_rn(ev[j], rsum);
+    prow[j] = pj;
+    keys[j] = __float_as_uint(pj);
+    tot += p_fixed62(__float_as_uint(pj));
+  }
+  __syncwarp();
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+
+  // 2. Top-p count.
+  int pc = 0;
+  unsigned int p_key = 0u;
+  int p_above = 0;
+  bool have_p = false;
+  if (topp > 0.0) {
+    const unsigned long long target = (unsigned long long)ceil(topp * 4611686018427387904.0);  // p * 2^62
+    if (tot < target) {
+      pc = nkb;
+    } else {
+      unsigned int prefix = 0u;
+      unsigned long long above_w = 0ull;
+      int above_c = 0;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        const unsigned int hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        radix_pass_warp(keys, nkb, shift, hi_mask, true, target, &prefix, &above_w, &above_c, hcnt, hsum);
+      }
+      const unsigned long long wt = p_fixed62(prefix);
+      const unsigned long long need = target - above_w;
+      const unsigned long long c = wt ? (need + wt - 1) / wt : 0ull;
+      pc = above_c + (int)c;
+      p_key = prefix;
+      p_above = above_c;
+      have_p = true;
+    }
+  }
+  const int m = min(nkb, max(max(kc, pc), 1));
+
+  // 3. Key of the m-th largest block, and how many of its ties are kept.
+  unsigned int tkey = p_key;
+  int above_m = p_above;
+  if (!(have_p && m == pc)) {
+    unsigned int prefix = 0u;
+    unsigned long long above_w = 0ull;
+    int above_c = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      const unsigned int hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+      radix_pass_warp(keys, nkb, shift, hi_mask, false, (unsigned long long)m, &prefix, &above_w, &above_c, hcnt,
+                      hsum);
+    }
+    tkey = prefix;
+    above_m = above_c;
+  }
+  const int ties_kept = m - above_m;
+
+  // 4. Compaction in block order, 32 blocks per round: ties at the threshold
+  //    key are kept lowest index first.
+  int32_t* out = kv_idx + row * (int64_t)nkb;
+  const unsigned int lt = (1u << lane) - 1u;
+  int ties_before = 0, kept_before = 0;
+  for (int j0 = 0; j0 < nkb; j0 += 32) {
+    const int j = j0 + lane;
+    const unsigned int k = j < nkb ? keys[j] : 0u;
+    const bool tie = j < nkb && k == tkey;
+    const unsigned int tb = __ballot_sync(0xffffffffu, tie);
+    const bool keep = j < nkb && (k > tkey || (tie && ties_before + __popc(tb & lt) < ties_kept));
+    const unsigned int kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[kept_before + __popc(kb & lt)] = j;
+    ties_before += __popc(tb);
+    kept_before += __popc(kb);
+  }
+  if (lane == 0) {
+    kv_cnt[row] = m;
+    if (row_thresh) row_thresh[row] = __uint_as_float(tkey);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Launch order of the query tiles for the kernels that walk a tile's kept
 // blocks (their work is proportional to the kept count, which varies several
 // times over between tiles). Heads go in groups of G, so the K and V of a

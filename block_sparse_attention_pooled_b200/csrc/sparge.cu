@@ -205,6 +205,14 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
     e = launch_scores<D>(qbar, kbar, dm, P, st);
   }
   if (e != cudaSuccess) return cuda_status(e);
+  if (dm.nkb <= kSelWarpMaxNkb) {  // one warp per row
+    const int sel_sm = select_warp_smem_bytes((int)dm.nkb);
+    e = ensure_smem(select_warp_kernel, sel_sm, 17);
+    if (e != cudaSuccess) return cuda_status(e);
+    select_warp_kernel<<<(unsigned)ceil_div(dm.BH * dm.nqb, kSelWarpRows), kSelWarpRows * 32, sel_sm, st>>>(
+        P, dm.BH * dm.nqb, (int)dm.nkb, kc, topp, kv_idx, kv_cnt, row_thresh);
+    return cuda_status(cudaGetLastError());
+  }
   const int sel_sm = select_smem_bytes((int)dm.nkb);
   e = ensure_smem(select_kernel, sel_sm, 2);
   if (e != cudaSuccess) return cuda_status(e);
