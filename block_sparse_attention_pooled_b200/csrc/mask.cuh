@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(float* __restric
 // and a 256-bucket histogram in shared memory.
 // ----------------------------------------------------------------------------
 constexpr int kSelWarpRows = 8;
-constexpr int kSelWarpMaxNkb = 1024;
+constexpr int kSelWarpMaxNkb = 2048;
 
 __host__ __device__ constexpr int select_warp_bytes(int nkb) { return (nkb + 3) / 4 * 16 + 256 * 12 + 16; }
 __host__ __device__ constexpr int select_warp_smem_bytes(int nkb) { return kSelWarpRows * select_warp_bytes(nkb); }
