@@ -282,7 +282,38 @@ struct ListChunks {
 // The sparse part uses alpha_h dO: dS = P (alpha_h dP - D_i), D_i = alpha_h dO_i . O_s,i.
 // NB = 2 then (TMEM: 4 x 64 + 128 + 128 columns).
 // ---------------------------------------------------------------------------
-constexpr int kBwdQThreads = 320;
+// dS warpgroups of the dQ kernel: three for the sparse branch alone (each
+// takes every third tile and owns one of the three S / dP buffers; dS is
+// formed half a tile at a time so 448 threads fit the register file), two
+// with SLA2 (the linear accumulator leaves room for two buffers).
+template <bool SLA2>
+__host__ __device__ constexpr int bwd_q_wgs() { return SLA2 ? 2 : 3; }
+template <bool SLA2>
+__host__ __device__ constexpr int bwd_q_threads() { return 64 + 128 * bwd_q_wgs<SLA2>(); }
+
+// dS = P (dP - D) for 32 keys (half a tile) of the sparse branch, read from
+// TMEM at the given S and dP columns; 16 bf16 pairs out.
+__device__ __forceinline__ void ds_half(uint32_t ts, uint32_t tp, float scale_log2, float lse2, float Di, int key0,
+                                        int N, bool row_ok, uint32_t (&pds)[16]) {
+  uint32_t sv[2][16], pv[2][16];
+  tmem_ld16(ts, sv[0]);
+  tmem_ld16(ts + 16, sv[1]);
+  tmem_ld16(tp, pv[0]);
+  tmem_ld16(tp + 16, pv[1]);
+  tmem_ld_wait();
+  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di);
+  const bool tail = key0 + 32 > N;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int h = k / 8, c = (2 * k) % 16;
+    const float2 x = f2_split(fma2(f2(__uint_as_float(sv[h][c]), __uint_as_float(sv[h][c + 1])), sc2, nl2));
+    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+    if (!row_ok || (tail && key0 + 2 * k >= N)) p0 = 0.0f;
+    if (!row_ok || (tail && key0 + 2 * k + 1 >= N)) p1 = 0.0f;
+    const float2 g = f2_split(add2(f2(__uint_as_float(pv[h][c]), __uint_as_float(pv[h][c + 1])), nd2));
+    pds[k] = pack_bf16x2(p0 * g.x, p1 * g.y);
+  }
+}
 
 template <int D, bool SLA2>
 struct BwdQSmem {
@@ -338,7 +369,7 @@ __device__ __forceinline__ void ds_and_x(const float (&s)[kTileK], const float (
 }
 
 template <int D, bool SLA2>
-__global__ void __launch_bounds__(kBwdQThreads, 1)
+__global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                        const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmPK,
@@ -535,7 +566,8 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dS + epilogue
-    const int wg = (warp - 2) >> 2;  // 0: even tiles, 1: odd tiles
+    constexpr int WG = bwd_q_wgs<SLA2>();
+    const int wg = (warp - 2) >> 2;  // takes tiles wg, wg + WG, ...
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -548,19 +580,32 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
     const float ci = SLA2 && row_ok ? __ldg(lp.cw + grow) : 0.0f;
     bool ok = true;
     ListChunks lc(lst, cnt, lane);
-    for (int t = wg; t < T; t += 2) {
+    for (int t = wg; t < T; t += WG) {
       const int b = t % NB;
       const int key0 = lc.get(lst, cnt, t / tiles_per_block, lane) * p.bk + (t % tiles_per_block) * kTileK;
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t / NB) & 1, kErrBwdSFull, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float s[kTileK], dp[kTileK];
-      load_row64(tS + lane_off + b * 64, s);
-      load_row64(tP + lane_off + b * 64, dp);
-      uint32_t pds[kTileK / 2], px[kTileK / 2];
-      ds_and_x<SLA2>(s, dp, p.scale_log2, lse2, Di, a_h, fi, key0, p.N, row_ok, pds, px);
-      store_p(tS + lane_off + b * 64, pds);
-      if (SLA2) store_p(tP + lane_off + b * 64, px);
+      if (SLA2) {
+        float s[kTileK], dp[kTileK];
+        load_row64(tS + lane_off + b * 64, s);
+        load_row64(tP + lane_off + b * 64, dp);
+        uint32_t pds[kTileK / 2], px[kTileK / 2];
+        ds_and_x<SLA2>(s, dp, p.scale_log2, lse2, Di, a_h, fi, key0, p.N, row_ok, pds, px);
+        store_p(tS + lane_off + b * 64, pds);
+        store_p(tP + lane_off + b * 64, px);
+      } else {
+        // Half a tile at a time; the half written back (columns 16h..16h+15 of
+        // S) holds S values already read.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pds[16];
+          ds_half(tS + lane_off + b * 64 + 32 * h, tP + lane_off + b * 64 + 32 * h, p.scale_log2, lse2, Di,
+                  key0 + 32 * h, p.N, row_ok, pds);
+          tmem_st16(tS + lane_off + b * 64 + 16 * h, pds);
+        }
+        tmem_st_wait();
+      }
       tc_fence_before();
       mbar_arrive(bar(L::kBarPFull + b));
     }
@@ -569,9 +614,10 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
       tc_fence_after();
     }
     // Epilogue: scale * dQ (+ the linear term) -> bf16 -> Q buffer (free: every
-    // MMA is done) -> TMA store; warpgroup wg takes columns [wg D/2, (wg + 1) D/2).
+    // MMA is done) -> TMA store; warpgroup wg takes a run of 16-column groups.
+    constexpr int kCols = (D / 16 + WG - 1) / WG * 16;
 #pragma unroll 1
-    for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 16) {
+    for (int c = wg * kCols; c < min(D, (wg + 1) * kCols); c += 16) {
       uint32_t v[16];
       if (T > 0 && ok) {
         tmem_ld16(tQ + lane_off + c, v);
@@ -604,7 +650,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
       stage_row16(sQ, r, c, o);
     }
     fence_async_smem();
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(128 * WG) : "memory");
     if (warp == 2 && lane == 0) {
       for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmDQ, sQ + b * (kTileQ * 128), b * 64, q0, bh);
       tma_store_commit();

@@ -309,7 +309,8 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   const BwdLinParams lp{};
   e = ensure_smem(attn_bwd_dq_kernel<D, false>, BwdQSmem<D, false>::kBytes, 11);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dq_kernel<D, false><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D, false>::kBytes, st>>>(
+  attn_bwd_dq_kernel<D, false><<<(unsigned)(dm.BH * dm.nqb), bwd_q_threads<false>(), BwdQSmem<D, false>::kBytes,
+                                 st>>>(
       mq, mk, mv, mdo, mdq, mk, mq, p, lp);
   p.order = nullptr;
   p.lst = q_idx;
@@ -612,7 +613,8 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   lp.H = s->H;
   e = ensure_smem(attn_bwd_dq_kernel<D, true>, BwdQSmem<D, true>::kBytes, 14);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dq_kernel<D, true><<<(unsigned)(dm.BH * dm.nqb), kBwdQThreads, BwdQSmem<D, true>::kBytes, st>>>(
+  attn_bwd_dq_kernel<D, true><<<(unsigned)(dm.BH * dm.nqb), bwd_q_threads<true>(), BwdQSmem<D, true>::kBytes,
+                                st>>>(
       mq, mk, mv, mdo, mdq, mpk, msall, p, lp);
   p.order = nullptr;
   p.lst = q_idx;
