@@ -12,10 +12,12 @@
 //   dK_j  = sum_i dS_ij q_i / sqrt(d),  dV_j = sum_i P_ij dO_i
 //                                              (rows whose block keeps j's)
 //
-// Four launches, no atomics (bit-reproducible):
+// Four or five launches, no atomics (bit-reproducible):
 //   bwd_dot_kernel         D_i for every row;
 //   mask_transpose_kernel  for every key block, the ascending list of query
 //                          blocks that keep it;
+//   tile_order_kernel      the query tiles' launch order (as the forward's),
+//                          when groups of heads fit in L2;
 //   attn_bwd_dq_kernel     one CTA per query tile, walking its kept key tiles
 //                          (the forward's structure): S = Q K^T and
 //                          dP = dO V^T into TMEM, dS written back over S as
@@ -27,7 +29,9 @@
 //                          dimension on the lanes (M = d = 128), so the MMAs
 //                          keep M = 128 for 64-key blocks.
 // Warp roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer and
-// TMEM owner, warps 2..5 one row (TMEM lane) per thread. d = 128.
+// TMEM owner, then one row (TMEM lane) per thread in warpgroups of four
+// warps (three in the sparse dQ kernel, two in the SLA2 dQ kernel, one in the
+// dK/dV kernel). d = 128.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
