@@ -100,3 +100,27 @@ def test_sla2_is_deterministic():
     a = _gpu_sla2(Q, K, V, idx, cnt, np.array([0.7, 0.9], np.float32), 128, 64)
     b = _gpu_sla2(Q, K, V, idx, cnt, np.array([0.7, 0.9], np.float32), 128, 64)
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("kind", ["random", "windows"])
+def test_sla2_many_query_tiles(kind):
+    # Many query tiles over many heads, with masks whose neighbouring rows
+    # change a lot (random) or by a few blocks at a time (sliding windows).
+    B, H, N, d, bq, bk = 1, 96, 8192, 128, 128, 64
+    g = torch.Generator().manual_seed(31)
+    Q, K, V = ((torch.randn(B, H, N, d, generator=g) * s).to(torch.bfloat16) for s in (1.5, 1.5, 1.0))
+    nqb, nkb = N // bq, N // bk
+    if kind == "random":
+        idx, cnt = (np.asarray(a) for a in synth.random_mask(B, H, nqb, nkb, 8, seed=5))
+    else:
+        idx = np.zeros((B, H, nqb, nkb), np.int32)
+        cnt = np.zeros((B, H, nqb), np.int32)
+        for h in range(H):
+            for I in range(nqb):
+                w = sorted({(2 * I + k + h) % nkb for k in range(6)})
+                idx[0, h, I, :len(w)] = w
+                cnt[0, h, I] = len(w)
+    alpha = np.linspace(0.6, 0.95, H).astype(np.float32)
+    rows = sample_rows(B, H, N, bq, 64, seed=3)
+    max_abs, mean_rel = _check(Q, K, V, idx, cnt, alpha, bq, bk, rows=rows)
+    print(f"{kind}: max-abs {max_abs:.2e} mean-rel-L1 {mean_rel:.2e}")
