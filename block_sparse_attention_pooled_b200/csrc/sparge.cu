@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -120,16 +121,25 @@ bool make_map_bhnd(CUtensorMap* m, const void* base, int64_t BH, int N, int d, i
   return r == CUDA_SUCCESS;
 }
 
-// Raises a kernel's dynamic shared memory limit once per device.
+// Raises a kernel's dynamic shared memory limit once per device. Any host
+// thread may launch: the fast path reads an atomic table, and the attribute
+// is only ever raised (to the largest size asked for so far) under a lock, so
+// a thread asking for less cannot lower a limit another thread relies on.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int bytes, int slot) {
-  static int done[64][32];  // [device][slot]: one slot per kernel
+  static std::atomic<int> done[64][32];  // [device][slot]: one slot per kernel
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 64 && done[dev][slot] >= bytes) return cudaSuccess;
+  if (dev < 0 || dev >= 64 || slot < 0 || slot >= 32)
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (done[dev][slot].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  const int have = done[dev][slot].load(std::memory_order_relaxed);
+  if (have >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev < 64) done[dev][slot] = bytes;
+  if (e == cudaSuccess) done[dev][slot].store(bytes, std::memory_order_release);
   return e;
 }
 
