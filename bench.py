@@ -208,11 +208,15 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=N
     else:
         oracle.attention_rows(Qh, Kh, Vh, w.bq, w.bk, idx, cnt, alpha[:heads].numpy(), mode=mode, rows=rows)
     t_attn = time.perf_counter() - t0
+    # Credit only the products the sample computes. The backward sample takes
+    # dQ of its rows: the forward's two products plus the backward's S, dP and
+    # dQ (its dK and dV products are not sampled), 2.5 times the forward's
+    # kept-block FLOPs; the GPU step's 3.5 adds dV and dK.
     flops = 0.0
     for qb in qbs:
         nrows = min(w.bq, w.N - qb * w.bq)
         keys = sum(min(w.bk, w.N - int(J) * w.bk) for J in idx[0, 0, qb, : cnt[0, 0, qb]])
-        flops += 4.0 * w.d * nrows * keys * (3.5 if mode == "bwd" else 1.0)
+        flops += 4.0 * w.d * nrows * keys * (2.5 if mode == "bwd" else 1.0)
     # the mask's time is charged pro rata to the sampled query blocks
     t = t_attn + t_mask * (len(qbs) / (w.nqb * heads))
     desc = (f"oracle {'router ' if router is not None else ''}mask of {heads} head(s) ({t_mask:.2f} s, charged pro rata) + {mode} attention of "
