@@ -169,6 +169,65 @@ def dram_traffic(workload: str, kernel: str):
     return entry["dram_bytes_per_launch"]
 
 
+# ----------------------------------------------------------------------------- end-to-end timing
+def e2e_serial_ms(k, step, io, host_ins, hosts, stream, cuda=torch.cuda):
+    """ms per step when each step copies its inputs in, runs, and copies its
+    results out, all on the compute stream (the copies' time adds to the
+    step's). io = (device inputs, device results) as step(io=...) takes them."""
+    e0, e1 = cuda.Event(enable_timing=True), cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(k):
+        for dst, src in zip(io[0], host_ins):
+            dst.copy_(src, non_blocking=True)
+        step(io=io)
+        for h, t in zip(hosts, io[1]):
+            h.copy_(t, non_blocking=True)
+    e1.record(stream)
+    cuda.synchronize()
+    return e0.elapsed_time(e1) / k
+
+
+def e2e_overlapped_ms(k, step, sets, host_ins, hosts, stream, s_in, s_out, cuda=torch.cuda):
+    """ms per step when step i copies its inputs in on s_in and its results
+    out on s_out, through buffer set i % 2 (sets[b] = (device inputs, device
+    results), hosts[b] = host result buffers), so that step i's work overlaps
+    the copy-in of step i + 1 and the copy-out of step i - 1. Events order the
+    reuse of a set: step i + 2's copy-in waits until step i has run, and step
+    i + 2 waits until step i's results have been copied out. The timed region
+    ends once every copy-out has finished."""
+    in_ready = [cuda.Event() for _ in range(2)]
+    ran = [cuda.Event() for _ in range(2)]
+    out_done = [cuda.Event() for _ in range(2)]
+    e0, e1 = cuda.Event(enable_timing=True), cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(k):
+        b = i & 1
+        ins, outs = sets[b]
+        if i >= 2:
+            s_in.wait_event(ran[b])
+        with cuda.stream(s_in):
+            for dst, src in zip(ins, host_ins):
+                dst.copy_(src, non_blocking=True)
+        in_ready[b].record(s_in)
+        stream.wait_event(in_ready[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])
+        step(io=sets[b])
+        ran[b].record(stream)
+        s_out.wait_event(ran[b])
+        with cuda.stream(s_out):
+            for h, t in zip(hosts[b], outs):
+                h.copy_(t, non_blocking=True)
+        out_done[b].record(s_out)
+    for b in range(min(2, k)):
+        stream.wait_event(out_done[b])
+    e1.record(stream)
+    cuda.synchronize()
+    return e0.elapsed_time(e1) / k
+
+
 # ----------------------------------------------------------------------------- peaks
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -279,6 +338,7 @@ def run_ours(args, w, rank, world, local_rank):
     kv_idx = torch.empty((B, H, w.nqb, w.nkb), dtype=torch.int32, device=dev)
     kv_cnt = torch.empty((B, H, w.nqb), dtype=torch.int32, device=dev)
     O = torch.empty_like(Q)
+    O_fwd = O
     ws_attn = torch.empty(sparge.workspace_bytes(sparge.OP_ATTN, shape), dtype=torch.uint8, device=dev)
     if bwd:
         dOh = pin(synth.make_dout(w.B, w.H, w.N, w.d, seed=w.seed + rank))
@@ -289,8 +349,18 @@ def run_ours(args, w, rank, world, local_rank):
                              dtype=torch.uint8, device=dev)
         dalpha = torch.empty(H, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    # One set of device buffers: the step's inputs (read) and results (written).
+    io0 = ([Q, K, V] + ([dO] if bwd else []), ([dQ, dK, dV] + ([dalpha] if sla2 else [])) if bwd else [O])
 
-    def step(ev_a=None, ev_b=None):
+    def step(ev_a=None, ev_b=None, io=None):
+        ins, outs = io0 if io is None else io
+        Q, K, V = ins[0], ins[1], ins[2]
+        if bwd:
+            dO, (dQ, dK, dV) = ins[3], outs[:3]
+            dalpha_ = outs[3] if sla2 else None
+            O = O_fwd  # the forward's output feeds the backward only
+        else:
+            O = outs[0]
         if Wq is not None:
             sparge.sparge_mask_router(Q, K, Wq, Wk, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt,
                                       workspace=ws_mask)
@@ -304,7 +374,7 @@ def run_ours(args, w, rank, world, local_rank):
             if ev_a is not None:
                 ev_a.record(stream)
             if sla2:
-                sparge.sla2_attn_bwd(Q, K, V, kv_idx, kv_cnt, alpha, dO, w.bq, w.bk, dQ, dK, dV, dalpha,
+                sparge.sla2_attn_bwd(Q, K, V, kv_idx, kv_cnt, alpha, dO, w.bq, w.bk, dQ, dK, dV, dalpha_,
                                      workspace=ws_bwd)
             else:
                 sparge.sparge_attn_bwd(Q, K, V, kv_idx, kv_cnt, O, lse, dO, w.bq, w.bk, dQ, dK, dV, workspace=ws_bwd)
@@ -361,31 +431,36 @@ def run_ours(args, w, rank, world, local_rank):
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        outs = ((dQ, dK, dV) + ((dalpha,) if sla2 else ())) if bwd else (O,)
-        hosts = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
-        ins = [(Q, Qh), (K, Kh), (V, Vh)] + ([(dO, dOh)] if bwd else [])
-
-        def e2e_step():
-            for dst, src in ins:
-                dst.copy_(src, non_blocking=True)
-            step()
-            for h, t in zip(hosts, outs):
-                h.copy_(t, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        host_ins = [Qh, Kh, Vh] + ([dOh] if bwd else [])
+        h2d = sum(t.numel() * t.element_size() for t in host_ins)
+        d2h = sum(t.numel() * t.element_size() for t in io0[1])
         ksteps = max(3, args.steps // 4)
-        e0.record(stream)
-        for _ in range(ksteps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / ksteps, world, dev)
-        h2d = sum(t.numel() * t.element_size() for t, _ in ins)
+        hosts0 = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in io0[1]]
+
+        e2e_serial_ms(2, step, io0, host_ins, hosts0, stream)
+        e2e_serial = max_over_ranks(e2e_serial_ms(ksteps, step, io0, host_ins, hosts0, stream), world, dev)
+        pipe, pipe_err = float("inf"), None
+        try:
+            sets = [io0, ([torch.empty_like(t) for t in io0[0]], [torch.empty_like(t) for t in io0[1]])]
+            hosts = [hosts0, [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in io0[1]]]
+            s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+            e2e_overlapped_ms(2, step, sets, host_ins, hosts, stream, s_in, s_out)
+            pipe = e2e_overlapped_ms(ksteps, step, sets, host_ins, hosts, stream, s_in, s_out)
+        except Exception as exc:  # the serial figure stands; the line says why
+            torch.cuda.synchronize()
+            pipe_err = f"{type(exc).__name__}: {exc}"[:300]
+        pipe = max_over_ranks(pipe, world, dev)  # every rank takes this collective
+        overlapped = math.isfinite(pipe)
+        e2e_ms = pipe if overlapped else e2e_serial
         e2e = {"value": step_flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs), "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "copies": ("overlapped: each step's inputs copied in on one stream and its results out on another, "
+                          "two buffer sets, while the neighbouring step runs" if overlapped else
+                          "serial: copy in, step, copy out on one stream"),
+               "serial_ms_per_step": e2e_serial,
+               "serial_value": step_flops * world / (e2e_serial * 1e-3) / 1e12}
+        if pipe_err is not None:
+            e2e["overlap_error"] = pipe_err
     assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
 
     if rank != 0:
