@@ -170,10 +170,11 @@ def dram_traffic(workload: str, kernel: str):
 
 
 # ----------------------------------------------------------------------------- end-to-end timing
-def e2e_serial_ms(k, step, io, host_ins, hosts, stream, cuda=torch.cuda):
+def e2e_serial_ms(k, step, io, host_ins, hosts, stream, cuda=None):
     """ms per step when each step copies its inputs in, runs, and copies its
     results out, all on the compute stream (the copies' time adds to the
     step's). io = (device inputs, device results) as step(io=...) takes them."""
+    cuda = torch.cuda if cuda is None else cuda
     e0, e1 = cuda.Event(enable_timing=True), cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(k):
@@ -187,7 +188,7 @@ def e2e_serial_ms(k, step, io, host_ins, hosts, stream, cuda=torch.cuda):
     return e0.elapsed_time(e1) / k
 
 
-def e2e_overlapped_ms(k, step, sets, host_ins, hosts, stream, s_in, s_out, cuda=torch.cuda):
+def e2e_overlapped_ms(k, step, sets, host_ins, hosts, stream, s_in, s_out, cuda=None):
     """ms per step when step i copies its inputs in on s_in and its results
     out on s_out, through buffer set i % 2 (sets[b] = (device inputs, device
     results), hosts[b] = host result buffers), so that step i's work overlaps
@@ -195,6 +196,7 @@ def e2e_overlapped_ms(k, step, sets, host_ins, hosts, stream, s_in, s_out, cuda=
     reuse of a set: step i + 2's copy-in waits until step i has run, and step
     i + 2 waits until step i's results have been copied out. The timed region
     ends once every copy-out has finished."""
+    cuda = torch.cuda if cuda is None else cuda
     in_ready = [cuda.Event() for _ in range(2)]
     ran = [cuda.Event() for _ in range(2)]
     out_done = [cuda.Event() for _ in range(2)]
