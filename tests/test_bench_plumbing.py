@@ -4,96 +4,21 @@ end-to-end schedules and the JSON line. Nothing here computes attention; it
 checks that the harness calls the library the way the timing claims and that
 every key of the line is present."""
 import argparse
-import contextlib
 import json
-import types
 
+import bench_fakes
 import pytest
-import torch
 
 import bench
 import block_sparse_attention_pooled_b200 as pkg
 from block_sparse_attention_pooled_b200 import synth
 
 
-class _Stream:
-    def wait_event(self, ev):
-        pass
-
-
-class _Event:
-    def __init__(self, enable_timing=False):
-        pass
-
-    def record(self, stream=None):
-        pass
-
-    def elapsed_time(self, other):
-        return 2.0
-
-
-def _fake_cuda():
-    ns = types.SimpleNamespace()
-    main = _Stream()
-    ns.set_device = lambda dev: None
-    ns.current_stream = lambda *a: main
-    ns.Stream = lambda device=None: _Stream()
-    ns.Event = _Event
-    ns.synchronize = lambda *a: None
-    ns.stream = lambda s: contextlib.nullcontext()
-
-    def no_props(dev):
-        raise RuntimeError("no device")
-
-    ns.get_device_properties = no_props
-    return ns
-
-
-class _Torch(types.ModuleType):
-    """The torch module with a CPU device and a fake CUDA namespace."""
-
-    def __getattr__(self, name):
-        return getattr(torch, name)
-
-
-def _fake_sparge(calls):
-    from block_sparse_attention_pooled_b200 import sparge as real
-
-    ns = types.SimpleNamespace(**{k: getattr(real, k) for k in dir(real) if k.isupper()})
-    ns.make_shape, ns.workspace_bytes, ns.order_launches = real.make_shape, real.workspace_bytes, real.order_launches
-
-    def mask(Q, K, bq, bk, topk, topp, kv_idx=None, kv_cnt=None, workspace=None, **kw):
-        calls.append(("mask", Q.data_ptr()))
-        nkb = kv_idx.shape[-1]
-        kv_idx.copy_(torch.arange(nkb, dtype=torch.int32).expand_as(kv_idx))
-        kv_cnt.fill_(min(2, nkb))
-
-    def record(name):
-        def f(*a, **kw):
-            calls.append((name, a[0].data_ptr()))
-        return f
-
-    ns.sparge_mask = mask
-    ns.sparge_mask_router = record("mask_router")
-    ns.sparge_attn_fwd = record("attn_fwd")
-    ns.sparge_attn_fwd_q8 = record("attn_fwd_q8")
-    ns.sla2_attn_fwd = record("sla2_attn_fwd")
-    ns.sparge_attn_bwd = record("attn_bwd")
-    ns.sla2_attn_bwd = record("sla2_attn_bwd")
-    ns.device_status = lambda *a: 0
-    return ns
-
-
 @pytest.mark.parametrize("variant,sla2,cpu", [("bf16", False, False), ("bf16", True, True), ("bwd", False, False),
                                               ("bwd", True, True), ("q8", False, False)])
 def test_bench_line_with_recorded_library_calls(monkeypatch, capsys, variant, sla2, cpu):
     calls = []
-    fake_torch = _Torch("torch")
-    fake_torch.device = lambda *a, **k: torch.device("cpu", 0)
-    fake_torch.cuda = _fake_cuda()
-    monkeypatch.setattr(bench, "torch", fake_torch)
-    monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self, *a, **k: self)
-    monkeypatch.setattr(pkg, "sparge", _fake_sparge(calls), raising=False)
+    bench_fakes.install(monkeypatch, bench, pkg, calls)
     w = synth.Workload("plumbing", 1, 2, 256, 64, (1, 16, 16), 64, 64, 0.1, 0.9, 1.5, sla2)
     steps, warmup = 8, 3
     args = argparse.Namespace(gpus=1, steps=steps, warmup=warmup, workload=w.name, impl="ours", variant=variant,
