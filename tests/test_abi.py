@@ -86,6 +86,10 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     for bad in (lib.Shape(1, 1, 100, 96, 64, 64), lib.Shape(1, 1, 100, 64, 32, 64), lib.Shape(1, 1, 100, 64, 64, 256),
                 lib.Shape(1, 1, 64 * 5000, 64, 64, 64)):
         assert raw.sparge_attn_fwd(P, P, P, ctypes.byref(bad), P, P, P, None, None, 0, None) == lib.ERR_UNSUPPORTED
+    # the block-count limit: 4096 key blocks per row, exactly
+    assert lib.workspace_bytes(lib.OP_MASK, lib.Shape(1, 1, 64 * 4096, 64, 64, 64)) > 0
+    assert lib.workspace_bytes(lib.OP_MASK, lib.Shape(1, 1, 64 * 4096 + 1, 64, 64, 64)) == 0
+    assert lib.workspace_bytes(lib.OP_MASK, lib.Shape(1, 1, 128 * 4096, 64, 128, 128)) > 0
     for bad in (lib.Shape(0, 1, 100, 64, 64, 64), lib.Shape(1, 1, -5, 64, 64, 64)):
         assert raw.sparge_attn_fwd(P, P, P, ctypes.byref(bad), P, P, P, None, None, 0, None) == lib.ERR_INVALID_ARG
     assert raw.sparge_attn_fwd(P, P, None, ctypes.byref(s), P, P, P, None, None, 0, None) == lib.ERR_INVALID_ARG

@@ -46,6 +46,17 @@ def test_mask_small(N, d, bq, bk, topk, topp):
     _check(Q, K, bq, bk, topk, topp)
 
 
+@pytest.mark.parametrize("nkb,topk,topp", [(2048, 0.03, 0.9), (2049, 0.03, 0.9), (2049, 0.0, 0.5),
+                                           (4096, 0.01, 0.0), (4096, 0.03, 0.9)])
+def test_mask_long_rows(nkb, topk, topp):
+    # Rows of up to 2048 blocks take the warp-per-row selection (2048 is its
+    # limit); longer rows take the CTA-per-row kernel, up to the 4096-block
+    # maximum the library accepts. The last key block is ragged.
+    N = nkb * 64 - 17
+    Q, K, _ = synth.make_qkv(1, 1, N, 64, grid=None, s=1.5, seed=nkb)
+    _check(Q, K, 128, 64, topk, topp)
+
+
 @pytest.mark.parametrize("name", ["tiny", "480p", "sla2_480p", "sweep_flat", "sweep_peaked"])
 def test_mask_workloads(name):
     w = synth.WORKLOADS[name]
