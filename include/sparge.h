@@ -53,6 +53,14 @@
  *     gives up records a code that sparge_device_status returns. Nothing
  *     crosses the ABI as an exception.
  *   - Determinism: identical inputs give bit-identical outputs.
+ *   - Host threads: any thread may call any entry point, on any stream and
+ *     device, concurrently with other threads; the host state the library
+ *     keeps (kernel attributes raised once per device, the tensor-map
+ *     encoder's address) is initialised under locks. The device error word
+ *     is one per device and shared by every caller: the first
+ *     sparge_device_status call after a kernel gave up returns the code and
+ *     clears it. sparge_mask_noalloc calls share one static scratch array
+ *     per device, so two of them must not overlap in time on the device.
  */
 #ifndef SPARGE_H_
 #define SPARGE_H_
