@@ -83,6 +83,23 @@ def test_attn_peaked_scores_rescale_path():
     _check_rows(Q, K, V, idx, cnt, bq, bk)
 
 
+def test_attn_long_rows_at_the_block_limit():
+    # 4096 key blocks per row (the library's maximum) with a ragged last
+    # block: one query block keeps every block (4096 kept-list entries, read
+    # 32 at a time), one keeps a scattered half, the rest keep a few.
+    N, d, bq, bk = 64 * 4096 - 17, 64, 128, 64
+    Q, K, V = synth.make_qkv(1, 1, N, d, grid=None, s=1.5, seed=4096)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    idx, cnt = (np.asarray(a) for a in synth.random_mask(1, 1, nqb, nkb, 6, seed=11))
+    idx[0, 0, 0] = np.arange(nkb, dtype=np.int32)
+    cnt[0, 0, 0] = nkb
+    half = np.sort(np.random.default_rng(5).choice(nkb, nkb // 2, replace=False)).astype(np.int32)
+    idx[0, 0, nqb - 1, : nkb // 2] = half
+    cnt[0, 0, nqb - 1] = nkb // 2
+    rows = np.concatenate([np.arange(0, 128, 5), np.arange((nqb - 1) * bq, N, 7), np.arange(700 * bq, 700 * bq + 64, 9)])
+    _check_rows(Q, K, V, idx, cnt, bq, bk, rows=rows.astype(np.int64))
+
+
 @pytest.mark.parametrize("name", ["tiny", "480p"])
 def test_attn_workload_oracle_mask(name):
     w = synth.WORKLOADS[name]
