@@ -111,6 +111,27 @@ def test_bwd_480p_sampled():
     _assert_grad("dV", _kblocks_layout(dV, w.bk)[kb], rV)
 
 
+def test_bwd_long_rows_at_the_block_limit():
+    # 4096 key blocks per row (the library's maximum), ragged last block: the
+    # first query block keeps every key block, the rest a few each. dQ is
+    # checked on rows of the full block and of the ragged last query block,
+    # dK and dV on the ragged last key block (which the full row keeps).
+    N, d, bq, bk = 64 * 4096 - 17, 128, 128, 64
+    Q, K, V = synth.make_qkv(1, 1, N, d, grid=None, s=1.5, seed=4097)
+    dO = synth.make_dout(1, 1, N, d, seed=4097)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx, kv_cnt = (np.asarray(a) for a in synth.random_mask(1, 1, nqb, nkb, 4, seed=12))
+    kv_idx[0, 0, 0] = np.arange(nkb, dtype=np.int32)
+    kv_cnt[0, 0, 0] = nkb
+    dQ, dK, dV = _fwd_bwd(Q, K, V, dO, kv_idx, kv_cnt, bq, bk)
+    rows = np.concatenate([np.arange(0, 128, 11), np.arange((nqb - 1) * bq, N, 13)]).astype(np.int64)
+    kb = np.array([nkb - 1], np.int64)
+    rQ, rK, rV, _ = oracle.attention_bwd(Q, K, V, dO, bq, bk, kv_idx, kv_cnt, mode="sparse", rows=rows, kblocks=kb)
+    _assert_grad("dQ", dQ.float().cpu().numpy().reshape(-1, d)[rows], rQ)
+    _assert_grad("dK", _kblocks_layout(dK, bk)[kb], rK)
+    _assert_grad("dV", _kblocks_layout(dV, bk)[kb], rV)
+
+
 def test_bwd_is_deterministic():
     Q, K, V = synth.make_qkv(1, 2, 4096, 128, grid=None, s=1.5, seed=11)
     dO = synth.make_dout(1, 2, 4096, 128, seed=11)
