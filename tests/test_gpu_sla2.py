@@ -76,6 +76,24 @@ def test_sla2_empty_and_full_rows():
     _check(Q, K, V, idx, cnt, np.array([0.7], np.float32), bq, bk)
 
 
+def test_sla2_long_rows_at_the_block_limit():
+    # 4096 key blocks per row (the library's maximum), ragged last block: the
+    # first query block keeps every block (empty complement, O_l = 0), the
+    # last keeps a scattered half, the rest a few (complements of ~262k keys).
+    N, bq, bk = 64 * 4096 - 17, 128, 64
+    Q, K, V = synth.make_qkv(1, 1, N, 128, grid=None, s=1.5, seed=4098)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    idx, cnt = (np.asarray(a) for a in synth.random_mask(1, 1, nqb, nkb, 5, seed=13))
+    idx[0, 0, 0] = np.arange(nkb, dtype=np.int32)
+    cnt[0, 0, 0] = nkb
+    half = np.sort(np.random.default_rng(6).choice(nkb, nkb // 2, replace=False)).astype(np.int32)
+    idx[0, 0, nqb - 1, : nkb // 2] = half
+    cnt[0, 0, nqb - 1] = nkb // 2
+    rows = np.concatenate([np.arange(0, 128, 17), np.arange((nqb - 1) * bq, N, 19),
+                           np.arange(900 * bq, 900 * bq + 128, 23)]).astype(np.int64)
+    _check(Q, K, V, idx, cnt, np.array([0.75], np.float32), bq, bk, rows=rows)
+
+
 @pytest.mark.parametrize("name", ["sla2_480p", "720p"])
 def test_sla2_workload_oracle_mask(name):
     w = synth.WORKLOADS[name]
