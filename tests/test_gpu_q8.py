@@ -64,6 +64,27 @@ def test_q8_attention_matches_oracle(N, bq, bk, mask):
     assert np.abs(got - ref).max() < 1e-2
 
 
+def test_q8_long_rows_at_the_block_limit():
+    # 4096 key blocks per row (the library's maximum), ragged last block: V's
+    # channel scales reduce 256 chunk maxima; one query block keeps every
+    # key block, the last a scattered half, the rest a few.
+    N, bq, bk = 64 * 4096 - 17, 128, 64
+    Q, K, V = synth.make_qkv(1, 1, N, 128, grid=None, s=2.0, seed=4099)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    kv_idx, kv_cnt = (np.asarray(a) for a in synth.random_mask(1, 1, nqb, nkb, 5, seed=14))
+    kv_idx[0, 0, 0] = np.arange(nkb, dtype=np.int32)
+    kv_cnt[0, 0, 0] = nkb
+    half = np.sort(np.random.default_rng(7).choice(nkb, nkb // 2, replace=False)).astype(np.int32)
+    kv_idx[0, 0, nqb - 1, : nkb // 2] = half
+    kv_cnt[0, 0, nqb - 1] = nkb // 2
+    O, _, _ = _run(Q, K, V, kv_idx, kv_cnt, bq, bk)
+    rows = np.concatenate([np.arange(0, 128, 17), np.arange((nqb - 1) * bq, N, 19),
+                           np.arange(900 * bq, 900 * bq + 128, 23)]).astype(np.int64)
+    ref = oracle.attention_q8_rows(Q, K, V, bq, bk, kv_idx, kv_cnt, rows)
+    got = O.float().cpu().numpy().reshape(-1, 128)[rows].astype(np.float64)
+    assert_outputs(got, ref)
+
+
 def test_q8_480p_sampled_rows():
     w = synth.WORKLOADS["480p"]
     Q, K, V, _ = synth.make_workload(w, heads=[(0, 0), (0, 5)])
