@@ -80,3 +80,12 @@ def test_router_is_deterministic():
     b = _run(Q, K, Wq, Wk, 128, 64, 0.05, 0.9)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("dr", [64, 128])
+def test_router_long_rows_at_the_block_limit(dr):
+    # 4096 key blocks per row, ragged last block: the CTA-per-row selection.
+    N = 64 * 4096 - 17
+    Q, K, _ = synth.make_qkv(1, 1, N, 64, grid=None, s=1.5, seed=4100)
+    Wq, Wk = synth.make_router(1, 64, dr, seed=dr + 1)
+    _check(Q, K, Wq, Wk, 128, 64, 0.03, 0.9)
