@@ -50,6 +50,8 @@ def parse():
                     help="score the mask through a learnt router of this width (seeded stand-in projections)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other headline shapes (720p sparse and SLA2, sla2_480p) timed after the 480p line")
     return ap.parse_args()
 
 
@@ -131,6 +133,91 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read in-process through NVML (read-only
+    queries) every few milliseconds during the timed region, so that even a
+    timed region of a few tens of milliseconds gets samples. Falls back to the
+    nvidia-smi sampler when NVML cannot be opened."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, gpu_id: str, period_s: float = 0.002):
+        self.gpu_id = gpu_id
+        self.period = period_s
+        self.samples = []  # (sm_mhz, max_mhz, reasons bitmask)
+        self._stop = threading.Event()
+        self._nvml = None
+        self._fallback = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id) if self.gpu_id.isdigit() else 0)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            self._max = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._nvml = (pynvml, h, get_reasons)
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._nvml = None
+            self._fallback = ClockSampler(self.gpu_id).__enter__()
+        return self
+
+    def _sample(self):
+        pynvml, h, get_reasons = self._nvml
+        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        reasons = get_reasons(h) if get_reasons is not None else 0
+        self.samples.append((float(sm), float(self._max), int(reasons)))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                break
+            self._stop.wait(self.period)
+
+    def __exit__(self, *exc):
+        if self._nvml is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            try:
+                self._sample()  # one sample at the end of the region
+                self._nvml[0].nvmlShutdown()
+            except Exception:
+                pass
+        if self._fallback is not None:
+            self._fallback.__exit__(*exc)
+
+    def summary(self):
+        if self._fallback is not None:
+            out = self._fallback.summary()
+            out["source"] = "nvidia-smi -lms 200"
+            return out
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({n for _, _, r in self.samples for n, bit in self.REASONS if r & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": self.samples[0][1] if self.samples else None,
+                "sm_mhz_min": min(sm) if sm else None, "reasons": reasons, "samples": len(sm),
+                "source": f"NVML in-process, every {self.period * 1e3:.0f} ms"}
+
+
+def clocks_at_max(clocks) -> bool:
+    """True when the sampled SM clock held >= 95% of its maximum, or when there
+    are no samples (unknown: the burst peak, the larger denominator, applies)."""
+    if not clocks.get("samples") or clocks.get("sm_mhz") is None or not clocks.get("sm_max_mhz"):
+        return True
+    return clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+
+
 def _smi_id(dev) -> str:
     """nvidia-smi --id for a torch device: its UUID when torch exposes it."""
     try:
@@ -156,9 +243,9 @@ def kernel_source_sha(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def dram_traffic(workload: str, kernel: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    capture, or None when there is none or the kernel changed since."""
+def _capture(workload: str, kernel: str):
+    """The committed ncu capture of the dominant kernel on this workload, or
+    None when there is none or the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -166,7 +253,21 @@ def dram_traffic(workload: str, kernel: str):
         entry = json.load(f).get(workload)
     if not entry or entry.get("kernel") != kernel or entry.get("csrc_sha") != kernel_source_sha(kernel):
         return None
-    return entry["dram_bytes_per_launch"]
+    return entry
+
+
+def dram_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    capture, or None when there is none or the kernel changed since."""
+    entry = _capture(workload, kernel)
+    return None if entry is None else entry["dram_bytes_per_launch"]
+
+
+def tensor_pipe_pct(workload: str, kernel: str):
+    """ncu's sm__pipe_tensor_cycles_active (% of peak sustained, active cycles)
+    from the same capture, or None."""
+    entry = _capture(workload, kernel)
+    return None if entry is None else entry.get("tensor_pipe_active_pct")
 
 
 # ----------------------------------------------------------------------------- end-to-end timing
@@ -250,10 +351,10 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=N
     Qh, Kh, Vh = Q[:1, :heads].contiguous(), K[:1, :heads].contiguous(), V[:1, :heads].contiguous()
     t0 = time.perf_counter()
     if router is None:
-        idx, cnt, _ = oracle.mask(Qh, Kh, w.bq, w.bk, w.topk, w.topp, precision=32)
+        idx, cnt, _ = oracle.mask(Qh, Kh, w.bq, w.bk, w.topk, w.topp)
     else:
         Wq, Wk = (W[:heads].numpy() for W in router)
-        idx, cnt, _ = oracle.mask_router(Qh, Kh, w.bq, w.bk, Wq, Wk, w.topk, w.topp, precision=32)
+        idx, cnt, _ = oracle.mask_router(Qh, Kh, w.bq, w.bk, Wq, Wk, w.topk, w.topp)
     t_mask = time.perf_counter() - t0
     qbs = np.linspace(0, w.nqb - 1, n_qblocks).astype(np.int64)
     rows = np.concatenate([np.arange(qb * w.bq, min(w.N, qb * w.bq + w.bq)) for qb in qbs]).astype(np.int64)
@@ -283,6 +384,116 @@ def cpu_sample(w, Q, K, V, alpha, n_qblocks=4, heads=1, variant="bf16", router=N
     desc = (f"oracle {'router ' if router is not None else ''}mask of {heads} head(s) ({t_mask:.2f} s, charged pro rata) + {mode} attention of "
             f"{len(qbs)} query blocks x {w.bq} rows ({t_attn:.2f} s); {w.name} workload")
     return flops / t, desc, 1
+
+
+# ----------------------------------------------------------------------------- timing
+L2_FLUSH_BYTES = 256 << 20  # written between timed steps: twice the 126 MB L2
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def timed_steps(step, steps, stream, flush, cuda=None):
+    """Runs `steps` steps, each bracketed by its own CUDA events on the
+    launching stream, with the L2 flushed (a buffer larger than L2 written)
+    before each step, outside its events. step(ev_a, ev_b) records ev_a / ev_b
+    around the library call it times (the attention span). Returns the
+    per-step and per-span milliseconds."""
+    cuda = torch.cuda if cuda is None else cuda
+    evs = [tuple(cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(steps)]
+    for e0, ea, eb, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step(ea, eb)
+        e1.record(stream)
+    cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, _, _, e1 in evs], [ea.elapsed_time(eb) for _, ea, eb, _ in evs]
+
+
+def roofline_peak(achieved, clocks, ratio=1.0):
+    """The measured bf16 peak a kernel timed alone is held to: the burst figure
+    when the SM clock held its maximum (or was not sampled), the sustained
+    (power-capped) one otherwise; both fractions and the nominal one are
+    returned. ratio scales the bf16 peaks for another operand type."""
+    peaks, peak_kind = measured_peaks()
+    burst = float(peaks["bf16_tflops"]) * ratio
+    sustained = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * ratio
+    at_max = clocks_at_max(clocks)
+    peak = burst if at_max else sustained
+    desc = (f"{peak_kind} bf16 {'burst' if at_max else 'sustained'}"
+            + (" (SM clock at max during the timed region)" if at_max and clocks.get("samples") else
+               " (no clock samples: burst)" if at_max else " (SM clock below max during the timed region)")
+            + (f" x {ratio:g} (nominal 8-bit / bf16 ratio)" if ratio != 1.0 else ""))
+    fracs = {"frac_vs_burst": achieved / burst, "frac_vs_sustained": achieved / sustained,
+             "frac_vs_nominal": achieved / (NOMINAL_BF16_TFLOPS * ratio)}
+    return peak, fracs, desc
+
+
+# The other shapes the metric is quoted at: (workload, library call).
+OTHER_WORKLOADS = (("720p", "sparge_attn_fwd"), ("720p", "sla2_attn_fwd"), ("sla2_480p", "sla2_attn_fwd"))
+
+
+def time_other_workloads(args, dev, stream, flush):
+    """Mask + attention steps of the other headline shapes on this GPU, timed
+    like the main line (per-step events, L2 flushed between steps)."""
+    from block_sparse_attention_pooled_b200 import sparge
+
+    out = {}
+    cache = {}
+    for name, call in OTHER_WORKLOADS:
+        w = synth.WORKLOADS[name]
+        if name not in cache:
+            cache.clear()
+            torch.cuda.empty_cache()
+            Qh, Kh, Vh, alpha_h = synth.make_workload(w)
+            cache[name] = (Qh.to(dev), Kh.to(dev), Vh.to(dev), alpha_h.to(dev))
+        Q, K, V, alpha = cache[name]
+        shape = sparge.make_shape(Q, w.bq, w.bk)
+        B, H, N, d = Q.shape
+        ws_mask = torch.empty(sparge.workspace_bytes(sparge.OP_MASK, shape), dtype=torch.uint8, device=dev)
+        op = sparge.OP_SLA2 if call == "sla2_attn_fwd" else sparge.OP_ATTN
+        ws = torch.empty(max(1, sparge.workspace_bytes(op, shape)), dtype=torch.uint8, device=dev)
+        kv_idx = torch.empty((B, H, w.nqb, w.nkb), dtype=torch.int32, device=dev)
+        kv_cnt = torch.empty((B, H, w.nqb), dtype=torch.int32, device=dev)
+        O = torch.empty_like(Q)
+
+        def step(ev_a=None, ev_b=None):
+            sparge.sparge_mask(Q, K, w.bq, w.bk, w.topk, w.topp, kv_idx=kv_idx, kv_cnt=kv_cnt, workspace=ws_mask)
+            if ev_a is not None:
+                ev_a.record(stream)
+            if call == "sla2_attn_fwd":
+                sparge.sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, w.bq, w.bk, O=O, workspace=ws)
+            else:
+                sparge.sparge_attn_fwd(Q, K, V, kv_idx, kv_cnt, w.bq, w.bk, O=O, workspace=ws)
+            if ev_b is not None:
+                ev_b.record(stream)
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
+        flops = kept_flops(kv_idx, kv_cnt, N, d, w.bq, w.bk)
+        with NvmlClockSampler(_smi_id(dev)) as clk:
+            step_ms, attn_ms = timed_steps(step, args.steps, stream, flush)
+        clocks = clk.summary()
+        ms = sum(step_ms) / len(step_ms)
+        span = sum(attn_ms) / len(attn_ms)
+        achieved = flops / (span * 1e-3) / 1e12
+        peak, fracs, desc = roofline_peak(achieved, clocks)
+        kernel = f"attn_fwd_kernel<{d}, {1 if call == 'sla2_attn_fwd' else 0}>"
+        out[f"{name}:{call}"] = {
+            "config": {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk, "topk": w.topk,
+                       "topp": w.topp, "alpha": "U[0.6,1] per head" if call == "sla2_attn_fwd" else 1.0},
+            "ms_per_step": ms, "ms_per_step_median": statistics.median(step_ms),
+            "kept_tflops": flops / (ms * 1e-3) / 1e12, "kept_fraction": flops / (4.0 * B * H * N * N * d),
+            "mask_ms": ms - span, "attn_ms": span,
+            "roofline": {"kernel": kernel, "timed_span": call, "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": desc, **fracs,
+                         "ncu_tensor_pipe_active_pct": tensor_pipe_pct(name, kernel)},
+            "clocks": clocks,
+        }
+        del ws_mask, ws, kv_idx, kv_cnt, O
+    cache.clear()
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- runs
@@ -410,23 +621,16 @@ def run_ours(args, w, rank, world, local_rank):
     step_flops = flops * (3.5 if bwd else 1.0)
     span_flops = flops * (2.5 if bwd else 1.0)
 
-    # ---- device-timed region (inputs resident in HBM, larger than L2)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- device-timed region (inputs resident in HBM; L2 flushed between steps)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(_smi_id(dev)) as clk:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(*evs[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
+    with NvmlClockSampler(_smi_id(dev)) as clk:
+        step_ms, attn_ms = timed_steps(step, args.steps, stream, flush)
     if world > 1:
         torch.distributed.barrier()
-    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
-    attn_ms = [a.elapsed_time(b) for a, b in evs]
-    ms_step = ms_total / args.steps
+    ms_step = max_over_ranks(sum(step_ms) / len(step_ms), world, dev)
     value = step_flops * world / (ms_step * 1e-3) / 1e12
     attn_avg = sum(attn_ms) / len(attn_ms)
 
@@ -467,18 +671,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     if rank != 0:
         return
-    peaks, peak_kind = measured_peaks()
     clocks = clk.summary()
-    # Burst peak when the clocks held their maximum through the timed region,
-    # the sustained (power-capped) one otherwise.
-    burst = clocks["sm_mhz"] is not None and clocks["sm_max_mhz"] and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
-    peak = float(peaks["bf16_tflops"] if burst else peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    peak_desc = f"{peak_kind} bf16 {'burst (SM clock at max during the timed region)' if burst else 'sustained'}"
-    if q8:
-        # int8 and e4m3 MMAs: the measured bf16 peak times the nominal 8-bit / bf16 ratio (4.5 / 2.25).
-        peak *= 2.0
-        peak_desc += " x 2 (nominal int8 / e4m3 to bf16 ratio)"
     achieved = span_flops / (attn_avg * 1e-3) / 1e12
+    peak, fracs, peak_desc = roofline_peak(achieved, clocks, 2.0 if q8 else 1.0)
     # The timed span is one library call: tile order + attn_fwd_kernel for the
     # pure sparse path; tile order, linear summaries, linear_out and
     # attn_fwd_kernel<128, 1> for the sparse + linear mix.
@@ -492,6 +687,7 @@ def run_ours(args, w, rank, world, local_rank):
             "sla2_attn_fwd (4-5 launches)" if sla2 else "sparge_attn_fwd (tile order when used, attention)")
     # Counters were captured with the plain mask; a router mask keeps other tiles.
     traffic = None if (args.router or bwd) else dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
+    tensor_pct = None if (args.router or bwd) else tensor_pipe_pct(w.name + ("_q8" if q8 else ""), kernel_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant, router=router_h,
@@ -510,19 +706,32 @@ def run_ours(args, w, rank, world, local_rank):
                    "flops": ("kept-block FLOPs x 3.5 (forward + backward; the linear branch's work is not counted)"
                              if bwd else "kept-block FLOPs"),
                    "mask": f"sparge_mask_router (dr {args.router})" if args.router else "sparge_mask",
-                   "l2": f"inputs larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V per rank)",
+                   "l2": (f"L2 flushed between steps (a {L2_FLUSH_BYTES >> 20} MB buffer written outside each "
+                          f"step's events); inputs also larger than L2 ({3 * Q.numel() * 2 / 1e6:.0f} MB of Q/K/V "
+                          f"per rank)"),
                    "parallelism": f"independent replicas x{world}"},
+        "timing": ("CUDA events around each step on the launching stream; ms_per_step = mean over the timed "
+                   "steps (max over ranks)"),
+        "ms_per_step_median": statistics.median(step_ms),
         "kept_fraction": flops / dense_flops,
         "dense_equiv_tflops": dense_flops * world / (ms_step * 1e-3) / 1e12,
         "attn_ms": attn_avg,
+        "attn_ms_median": statistics.median(attn_ms),
         "mask_ms": ms_step - attn_avg,
         "roofline": {"kernel": kernel_name, "timed_span": span, "bound": "tensor", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_desc, "traffic": traffic},
+                     "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": peak_desc, **fracs,
+                     "ncu_tensor_pipe_active_pct": tensor_pct, "traffic": traffic},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
+    if (w.name == "480p" and world == 1 and not getattr(args, "no_extra", False) and args.variant == "bf16"
+            and not args.router):
+        # The other headline shapes, timed in the same process (no e2e, no CPU leg).
+        del Q, K, V, O, ws_mask, ws_sla2, ws_q8, ws_attn, io0
+        torch.cuda.empty_cache()
+        line["per_workload"] = time_other_workloads(args, dev, stream, flush)
     print(json.dumps(line), flush=True)
 
 

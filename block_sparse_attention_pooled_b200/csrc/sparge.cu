@@ -55,21 +55,24 @@ sparge_status cuda_status(cudaError_t e) {
   return SPARGE_ERR_CUDA;
 }
 
+// The mask's scratch: pooled Q and K (double [BH, Nqb | Nkb, d]) and the
+// scaled scores (double [BH, Nqb, Nkb]) that the selection turns into
+// probabilities.
 struct MaskWs {
-  size_t qbar, kbar, probs, total;
+  size_t qbar, kbar, z, total;
 };
 
 MaskWs mask_ws(const sparge_shape* s, const Dims& d) {
   MaskWs w;
   w.qbar = 0;
-  w.kbar = w.qbar + align256((size_t)d.BH * d.nqb * s->d * 4);
-  w.probs = w.kbar + align256((size_t)d.BH * d.nkb * s->d * 4);
-  w.total = w.probs + align256((size_t)d.BH * d.nqb * d.nkb * 4);
+  w.kbar = w.qbar + align256((size_t)d.BH * d.nqb * s->d * 8);
+  w.z = w.kbar + align256((size_t)d.BH * d.nkb * s->d * 8);
+  w.total = w.z + align256((size_t)d.BH * d.nqb * d.nkb * 8);
   return w;
 }
 
 // The router's scratch: the mask's, then the projected blocks q^ and k^
-// (sized for the widest supported router width).
+// (double, sized for the widest supported router width).
 constexpr int kMaxRouterDim = 128;
 
 struct RouterWs {
@@ -81,8 +84,8 @@ RouterWs router_ws(const sparge_shape* s, const Dims& d) {
   RouterWs w;
   w.mask = mask_ws(s, d);
   w.qhat = w.mask.total;
-  w.khat = w.qhat + align256((size_t)d.BH * d.nqb * kMaxRouterDim * 4);
-  w.total = w.khat + align256((size_t)d.BH * d.nkb * kMaxRouterDim * 4);
+  w.khat = w.qhat + align256((size_t)d.BH * d.nqb * kMaxRouterDim * 8);
+  w.total = w.khat + align256((size_t)d.BH * d.nkb * kMaxRouterDim * 8);
   return w;
 }
 
@@ -163,26 +166,28 @@ cudaError_t launch_tile_order(const int32_t* kv_cnt, const sparge_shape* s, cons
 
 inline size_t order_bytes(const Dims& d) { return align256((size_t)d.BH * d.nqb * 4); }
 
-// Scores of DD-wide pooled (or projected) vectors into P.
+// Scaled scores of DD-wide pooled (or projected) vectors into Z.
 template <int DD>
-cudaError_t launch_scores(const float* a, const float* b, const Dims& dm, float* P, cudaStream_t st) {
-  const float scale = (float)(1.0 / std::sqrt((double)DD));
+cudaError_t launch_scores(const double* a, const double* b, const Dims& dm, double* Z, cudaStream_t st) {
+  const double scale = 1.0 / std::sqrt((double)DD);
   const int ssm = score_smem_bytes<DD>();
   cudaError_t e = ensure_smem(score_kernel<DD>, ssm, DD == 64 ? 0 : 1);
   if (e != cudaSuccess) return e;
   const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows) * ceil_div(dm.nkb, kScoreTileJ);
-  score_kernel<DD><<<(unsigned)tiles, 128, ssm, st>>>(a, b, (int)dm.nqb, (int)dm.nkb, scale, P);
+  score_kernel<DD><<<(unsigned)tiles, 128, ssm, st>>>(a, b, (int)dm.nqb, (int)dm.nkb, scale, Z);
   return cudaGetLastError();
 }
 
 // Router projections of the pooled vectors (DR output columns).
 template <int D, int DR>
-void launch_projection(const float* qbar, const float* kbar, const Dims& dm, int H, const float* Wq, const float* Wk,
-                       float* qhat, float* khat, cudaStream_t st) {
+cudaError_t launch_projection(const double* qbar, const double* kbar, const Dims& dm, int H, const float* Wq,
+                              const float* Wk, double* qhat, double* khat, cudaStream_t st) {
   const unsigned gq = (unsigned)(ceil_div(dm.nqb, kProjRows) * dm.BH);
   const unsigned gk = (unsigned)(ceil_div(dm.nkb, kProjRows) * dm.BH);
-  project_kernel<D, DR><<<gq, 128, 0, st>>>(qbar, dm.nqb, H, Wq, qhat);
-  project_kernel<D, DR><<<gk, 128, 0, st>>>(kbar, dm.nkb, H, Wk, khat);
+  constexpr int psm = project_smem_bytes<D>();
+  project_kernel<D, DR><<<gq, 128, psm, st>>>(qbar, dm.nqb, H, Wq, qhat);
+  project_kernel<D, DR><<<gk, 128, psm, st>>>(kbar, dm.nkb, H, Wk, khat);
+  return cudaGetLastError();
 }
 
 // Pool, (project,) score, select. Wq / Wk null: no router.
@@ -190,11 +195,11 @@ template <int D>
 sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, const Dims& dm, int kc, double topp,
                           int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs, uint8_t* ws,
                           cudaStream_t st, const float* Wq = nullptr, const float* Wk = nullptr, int dr = 0,
-                          float* qhat = nullptr, float* khat = nullptr) {
+                          double* qhat = nullptr, double* khat = nullptr) {
   const MaskWs w = mask_ws(s, dm);
-  float* qbar = reinterpret_cast<float*>(ws + w.qbar);
-  float* kbar = reinterpret_cast<float*>(ws + w.kbar);
-  float* P = probs ? probs : reinterpret_cast<float*>(ws + w.probs);
+  double* qbar = reinterpret_cast<double*>(ws + w.qbar);
+  double* kbar = reinterpret_cast<double*>(ws + w.kbar);
+  double* Z = reinterpret_cast<double*>(ws + w.z);
   constexpr int per_cta = 128 / (D / 8);
   const int64_t gq = ceil_div(dm.BH * dm.nqb, per_cta), gk = ceil_div(dm.BH * dm.nkb, per_cta);
   pool_kernel<D><<<(unsigned)(gq + gk), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(Q),
@@ -205,14 +210,14 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
   cudaError_t e;
   if (Wq != nullptr) {
     if (dr == 64) {
-      launch_projection<D, 64>(qbar, kbar, dm, s->H, Wq, Wk, qhat, khat, st);
-      e = launch_scores<64>(qhat, khat, dm, P, st);
+      e = launch_projection<D, 64>(qbar, kbar, dm, s->H, Wq, Wk, qhat, khat, st);
+      if (e == cudaSuccess) e = launch_scores<64>(qhat, khat, dm, Z, st);
     } else {
-      launch_projection<D, 128>(qbar, kbar, dm, s->H, Wq, Wk, qhat, khat, st);
-      e = launch_scores<128>(qhat, khat, dm, P, st);
+      e = launch_projection<D, 128>(qbar, kbar, dm, s->H, Wq, Wk, qhat, khat, st);
+      if (e == cudaSuccess) e = launch_scores<128>(qhat, khat, dm, Z, st);
     }
   } else {
-    e = launch_scores<D>(qbar, kbar, dm, P, st);
+    e = launch_scores<D>(qbar, kbar, dm, Z, st);
   }
   if (e != cudaSuccess) return cuda_status(e);
   if (dm.nkb <= kSelWarpMaxNkb) {  // one warp per row
@@ -220,14 +225,14 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
     e = ensure_smem(select_warp_kernel, sel_sm, 17);
     if (e != cudaSuccess) return cuda_status(e);
     select_warp_kernel<<<(unsigned)ceil_div(dm.BH * dm.nqb, kSelWarpRows), kSelWarpRows * 32, sel_sm, st>>>(
-        P, dm.BH * dm.nqb, (int)dm.nkb, kc, topp, kv_idx, kv_cnt, row_thresh);
+        Z, dm.BH * dm.nqb, (int)dm.nkb, kc, topp, kv_idx, kv_cnt, row_thresh, probs);
     return cuda_status(cudaGetLastError());
   }
   const int sel_sm = select_smem_bytes((int)dm.nkb);
   e = ensure_smem(select_kernel, sel_sm, 2);
   if (e != cudaSuccess) return cuda_status(e);
-  select_kernel<<<(unsigned)(dm.BH * dm.nqb), kSelectThreads, sel_sm, st>>>(P, dm.BH * dm.nqb, (int)dm.nkb, kc, topp,
-                                                                           kv_idx, kv_cnt, row_thresh);
+  select_kernel<<<(unsigned)(dm.BH * dm.nqb), kSelectThreads, sel_sm, st>>>(Z, dm.BH * dm.nqb, (int)dm.nkb, kc, topp,
+                                                                           kv_idx, kv_cnt, row_thresh, probs);
   return cuda_status(cudaGetLastError());
 }
 
@@ -749,8 +754,8 @@ sparge_status sparge_mask_router(const void* Q, const void* K, const sparge_shap
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* qhat = reinterpret_cast<float*>(ws + w.qhat);
-  float* khat = reinterpret_cast<float*>(ws + w.khat);
+  double* qhat = reinterpret_cast<double*>(ws + w.qhat);
+  double* khat = reinterpret_cast<double*>(ws + w.khat);
   if (shape->d == 64)
     return launch_mask<64>(Q, K, shape, dm, kc, topp, kv_idx, kv_cnt, row_thresh, probs, ws, s, Wq, Wk, dr, qhat,
                            khat);
@@ -767,11 +772,8 @@ sparge_status sparge_mask_noalloc(const void* Q, const void* K, const sparge_sha
   if (!Q || !K || !kv_idx || !kv_cnt) return SPARGE_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || (probs && !aligned16(probs))) return SPARGE_ERR_INVALID_ARG;
   if (!(topk_frac >= 0.0 && topk_frac <= 1.0) || !(topp >= 0.0 && topp <= 1.0)) return SPARGE_ERR_INVALID_ARG;
-  // Pooled Q and K always live in the scratch; the probability rows too
-  // unless the caller supplies `probs`.
-  const MaskWs w = mask_ws(shape, dm);
-  const size_t need = probs ? w.probs : w.total;
-  if (need > kNoAllocScratchBytes) return SPARGE_ERR_WORKSPACE;
+  // Pooled Q and K and the score rows live in the scratch.
+  if (mask_ws(shape, dm).total > kNoAllocScratchBytes) return SPARGE_ERR_WORKSPACE;
   uint8_t* ws = nullptr;
   st = noalloc_scratch(&ws);
   if (st != SPARGE_OK) return st;

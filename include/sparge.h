@@ -110,11 +110,15 @@ size_t sparge_workspace_bytes(int op, const sparge_shape* shape);
  *   kv_idx, kv_cnt  outputs (see conventions). Each row keeps
  *               max(kc, pc, 1) blocks: the union of two prefixes of one order.
  *   row_thresh  optional output, float [B,H,Nqb]: probability of the last
- *               kept block of each row (NULL to skip).
+ *               kept block of each row, rounded to float (NULL to skip).
  *   probs       optional output, float [B,H,Nqb,Nkb]: the pooled block
- *               probabilities (NULL to skip; the workspace holds them then).
- * Precision of the decision: fp32 pooling (row-order sums), fp32 scores
- * (channel-order fused multiply-adds), fp32 softmax, double running sums.
+ *               probabilities rounded to float (NULL to skip).
+ * Precision of the decision: double throughout (exact pooled sums, double
+ * scores and softmax, running sums in 2^-62 fixed point), so the kept set is
+ * the exact definition's except where two probabilities, or a running sum
+ * and topp, agree to within a few double rounding units.
+ * Workspace: sparge_workspace_bytes(SPARGE_OP_MASK, shape) (pooled Q and K
+ * and the score rows, in double), 256-byte aligned.
  * Limits: Nkb <= 4096. */
 sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shape, double topk_frac,
                           double topp, int32_t* kv_idx, int32_t* kv_cnt, float* row_thresh, float* probs,
@@ -129,8 +133,8 @@ sparge_status sparge_mask(const void* Q, const void* K, const sparge_shape* shap
  *   Wq, Wk      fp32 [H, d, dr] row-major, device, 4-byte aligned, read only;
  *               the caller owns them (no copy is kept).
  *   dr          router width: 64 or 128 (else SPARGE_ERR_UNSUPPORTED).
- * Precision: each projected entry is one fp32 fused-multiply-add chain over
- * the d channels in order; the rest as in sparge_mask.
+ * Precision: the projections in double (the fp32 weights widened exactly);
+ * the rest as in sparge_mask.
  * Workspace: sparge_workspace_bytes(SPARGE_OP_MASK_ROUTER, shape) (pooled
  * and projected blocks, probability rows), 256-byte aligned. */
 sparge_status sparge_mask_router(const void* Q, const void* K, const sparge_shape* shape, const float* Wq,
@@ -146,14 +150,15 @@ sparge_status sparge_mask_router(const void* Q, const void* K, const sparge_shap
  * counterpart; this is an interface convenience, not part of the method.
  *
  * Arguments and results are those of sparge_mask; the caller still passes
- * Q, K and every output. The scratch (pooled Q and K, and the probability
- * rows when `probs` is NULL) is a fixed 16 MiB array inside the library's
- * device code, so nothing is allocated: not by this call, not by the
- * library, not through any allocating library routine.
- *   - Limit: pooled Q + pooled K (+ probability rows when probs is NULL)
- *     must fit in 16 MiB: 4*B*H*d*(Nqb + Nkb) (+ 4*B*H*Nqb*Nkb) bytes, each
- *     part rounded up to 256. Larger shapes return SPARGE_ERR_WORKSPACE
- *     before anything is launched.
+ * Q, K and every output. The scratch (pooled Q and K and the score rows) is
+ * a fixed 16 MiB array inside the library's device code, so nothing is
+ * allocated: not by this call, not by the library, not through any
+ * allocating library routine.
+ *   - Limit: sparge_workspace_bytes(SPARGE_OP_MASK, shape) must not exceed
+ *     16 MiB: 8*B*H*d*(Nqb + Nkb) + 8*B*H*Nqb*Nkb bytes, each part rounded
+ *     up to 256 (for example B*H = 4 heads at N = 32760, d = 128, bq = 128,
+ *     bk = 64 take 7.3 MB). Larger shapes return SPARGE_ERR_WORKSPACE before
+ *     anything is launched.
  *   - The first call on a device looks up the array's device address on
  *     that device (cudaGetSymbolAddress, with the device current) and
  *     caches it; make that first call before any stream capture.

@@ -43,21 +43,18 @@ def _load():
         p = ctypes.c_void_p
         i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         lib.oracle_pool_f64.argtypes = [p, i64, i64, i32, i32, p]
-        lib.oracle_pool_f32.argtypes = [p, i64, i64, i32, i32, p]
         lib.oracle_block_probs_f64.argtypes = [p, p, i64, i64, i64, i32, p]
-        lib.oracle_block_probs_f32.argtypes = [p, p, i64, i64, i64, i32, p]
         lib.oracle_select_row.argtypes = [p, i64, dbl, dbl, p, p, p, p, p, p]
-        lib.oracle_mask.argtypes = [p, p, i64, i64, i32, i32, i32, dbl, dbl, i32, p, p, p]
+        lib.oracle_mask.argtypes = [p, p, i64, i64, i32, i32, i32, dbl, dbl, p, p, p]
         lib.oracle_attention_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, i32,
                                               p, i64, p, p]
-        lib.oracle_mask_router.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, i64, i32, dbl, dbl, i32, p, p, p]
+        lib.oracle_mask_router.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, i64, i32, dbl, dbl, p, p, p]
         lib.oracle_quant_q8.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         lib.oracle_e4m3.argtypes = [p, i64, p]
         lib.oracle_attention_bwd.argtypes = [p, p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, i32, p, i64, p, i64,
                                              p, p, p, p]
         lib.oracle_attention_q8_rows.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p, p, i64, p]
-        for f in (lib.oracle_pool_f64, lib.oracle_pool_f32, lib.oracle_block_probs_f64,
-                  lib.oracle_block_probs_f32, lib.oracle_select_row, lib.oracle_mask,
+        for f in (lib.oracle_pool_f64, lib.oracle_block_probs_f64, lib.oracle_select_row, lib.oracle_mask,
                   lib.oracle_attention_rows, lib.oracle_quant_q8, lib.oracle_e4m3,
                   lib.oracle_attention_q8_rows, lib.oracle_mask_router):
             f.restype = ctypes.c_int
@@ -89,33 +86,24 @@ def _check(rc: int, name: str):
         raise ValueError(f"{name}: invalid arguments (code {rc})")
 
 
-def pool(X, blk: int, precision: int = 64) -> np.ndarray:
-    """Mean-pool [B,H,N,d] bf16 over blocks of blk rows -> [B,H,ceil(N/blk),d]."""
+def pool(X, blk: int) -> np.ndarray:
+    """Mean-pool [B,H,N,d] bf16 over blocks of blk rows -> float64 [B,H,ceil(N/blk),d]."""
     x = _bits(X)
     B, H, N, d = x.shape
     nb = -(-N // blk)
-    if precision == 64:
-        out = np.empty((B, H, nb, d), np.float64)
-        _check(_load().oracle_pool_f64(_ptr(x), B * H, N, d, blk, _ptr(out)), "pool")
-    else:
-        out = np.empty((B, H, nb, d), np.float32)
-        _check(_load().oracle_pool_f32(_ptr(x), B * H, N, d, blk, _ptr(out)), "pool")
+    out = np.empty((B, H, nb, d), np.float64)
+    _check(_load().oracle_pool_f64(_ptr(x), B * H, N, d, blk, _ptr(out)), "pool")
     return out
 
 
 def block_probs(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
-    """Row softmax of pooled scores; float64 inputs -> float64, float32 -> float32."""
+    """Row softmax of pooled scores, in float64."""
     B, H, nqb, d = qbar.shape
     nkb = kbar.shape[2]
-    if qbar.dtype == np.float64:
-        qb, kb = np.ascontiguousarray(qbar), np.ascontiguousarray(kbar, np.float64)
-        out = np.empty((B, H, nqb, nkb), np.float64)
-        _check(_load().oracle_block_probs_f64(_ptr(qb), _ptr(kb), B * H, nqb, nkb, d, _ptr(out)), "probs")
-    else:
-        qb = np.ascontiguousarray(qbar, np.float32)
-        kb = np.ascontiguousarray(kbar, np.float32)
-        out = np.empty((B, H, nqb, nkb), np.float32)
-        _check(_load().oracle_block_probs_f32(_ptr(qb), _ptr(kb), B * H, nqb, nkb, d, _ptr(out)), "probs")
+    qb = np.ascontiguousarray(qbar, np.float64)
+    kb = np.ascontiguousarray(kbar, np.float64)
+    out = np.empty((B, H, nqb, nkb), np.float64)
+    _check(_load().oracle_block_probs_f64(_ptr(qb), _ptr(kb), B * H, nqb, nkb, d, _ptr(out)), "probs")
     return out
 
 
@@ -135,8 +123,8 @@ def select_row(P, topk: float, topp: float):
     return dict(kept=kept[: m.value].copy(), m=m.value, kc=kc.value, pc=pc.value, order=order, cum=cum)
 
 
-def mask(Q, K, bq: int, bk: int, topk: float, topp: float, precision: int = 32):
-    """Block mask for every query-block row.
+def mask(Q, K, bq: int, bk: int, topk: float, topp: float):
+    """Block mask for every query-block row (the double-precision definition).
 
     Returns (kv_idx int32 [B,H,Nqb,Nkb], kv_cnt int32 [B,H,Nqb], P float64 [B,H,Nqb,Nkb])."""
     q, k = _bits(Q), _bits(K)
@@ -146,11 +134,11 @@ def mask(Q, K, bq: int, bk: int, topk: float, topp: float, precision: int = 32):
     kv_cnt = np.zeros((B, H, nqb), np.int32)
     P = np.zeros((B, H, nqb, nkb), np.float64)
     _check(_load().oracle_mask(_ptr(q), _ptr(k), B * H, N, d, bq, bk, float(topk), float(topp),
-                               precision, _ptr(kv_idx), _ptr(kv_cnt), _ptr(P)), "mask")
+                               _ptr(kv_idx), _ptr(kv_cnt), _ptr(P)), "mask")
     return kv_idx, kv_cnt, P
 
 
-def mask_router(Q, K, bq: int, bk: int, Wq, Wk, topk: float, topp: float, precision: int = 32):
+def mask_router(Q, K, bq: int, bk: int, Wq, Wk, topk: float, topp: float):
     """Block mask with a learnt router: pooled blocks projected by Wq / Wk
     (float32 [H, d, dr], one pair per head) before scoring.
 
@@ -166,7 +154,7 @@ def mask_router(Q, K, bq: int, bk: int, Wq, Wk, topk: float, topp: float, precis
     kv_cnt = np.zeros((B, H, nqb), np.int32)
     P = np.zeros((B, H, nqb, nkb), np.float64)
     _check(_load().oracle_mask_router(_ptr(q), _ptr(k), B * H, N, d, bq, bk, _ptr(wq), _ptr(wk), H, dr,
-                                      float(topk), float(topp), precision, _ptr(kv_idx), _ptr(kv_cnt), _ptr(P)),
+                                      float(topk), float(topp), _ptr(kv_idx), _ptr(kv_cnt), _ptr(P)),
            "mask_router")
     return kv_idx, kv_cnt, P
 

@@ -40,14 +40,10 @@
 //     an empty complement gives O_l = 0;
 //   * no causal masking (bidirectional video attention).
 //
-// Precision: attention outputs are computed in double from the exactly widened
-// bf16 inputs. The block selection is an integer decision taken from floating
-// point, so it is offered in two precisions: the double-precision definition,
-// and the single-precision decision with a fixed operation order that the GPU
-// kernel also follows (pool: sequential float sum over rows, then divide by the
-// row count; score: sequential fused multiply-add over channels, then multiply
-// by (float)(1/sqrt(d)); softmax: expf(z - max) / sum, the row sum taken as
-// 32 interleaved partial sums combined pairwise).
+// Precision: everything is computed in double from the exactly widened bf16
+// inputs. The block selection is an integer decision taken from floating
+// point; it is the double-precision definition (pool, score, softmax, order,
+// running sums), with no single-precision variant.
 
 #include <algorithm>
 #include <cmath>
@@ -106,22 +102,6 @@ int oracle_pool_f64(const uint16_t* X, int64_t BH, int64_t N, int d, int blk, do
   return OK;
 }
 
-// Single-precision pooling with the GPU kernel's operation order.
-int oracle_pool_f32(const uint16_t* X, int64_t BH, int64_t N, int d, int blk, float* out) {
-  if (!X || !out || !shape_ok(BH, N, d, blk)) return ERR_ARG;
-  const int64_t nb = ceil_div(N, blk);
-  for (int64_t bh = 0; bh < BH; ++bh)
-    for (int64_t I = 0; I < nb; ++I) {
-      const int64_t r0 = I * blk, r1 = std::min<int64_t>(N, r0 + blk);
-      for (int c = 0; c < d; ++c) {
-        float acc = 0.0f;
-        for (int64_t r = r0; r < r1; ++r) acc = acc + widen_f(X[(bh * N + r) * d + c]);
-        out[(bh * nb + I) * d + c] = acc / static_cast<float>(r1 - r0);
-      }
-    }
-  return OK;
-}
-
 // ---------------------------------------------------------------------------
 // Pooled block importance [SA2 s4]: P[I, J] = softmax_J(qbar_I . kbar_J / sqrt d).
 // qbar [BH, Nqb, d], kbar [BH, Nkb, d], P [BH, Nqb, Nkb].
@@ -149,46 +129,6 @@ int oracle_block_probs_f64(const double* qbar, const double* kbar, int64_t BH, i
       }
       double* row = P + (bh * Nqb + I) * Nkb;
       for (int64_t J = 0; J < Nkb; ++J) row[J] = s[J] / sum;
-    }
-  return OK;
-}
-
-// Single precision with the GPU kernel's operation order: sequential fmaf over
-// channels, times (float)(1/sqrt(d)); expf(z - max); divide by the row sum
-// (32 interleaved partial sums combined pairwise).
-int oracle_block_probs_f32(const float* qbar, const float* kbar, int64_t BH, int64_t Nqb,
-                           int64_t Nkb, int d, float* P) {
-  if (!qbar || !kbar || !P || BH <= 0 || Nqb <= 0 || Nkb <= 0 || d <= 0) return ERR_ARG;
-  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
-  std::vector<float> z(Nkb);
-  for (int64_t bh = 0; bh < BH; ++bh)
-    for (int64_t I = 0; I < Nqb; ++I) {
-      const float* q = qbar + (bh * Nqb + I) * d;
-      float mx = -std::numeric_limits<float>::infinity();
-      for (int64_t J = 0; J < Nkb; ++J) {
-        const float* k = kbar + (bh * Nkb + J) * d;
-        float dot = 0.0f;
-        for (int c = 0; c < d; ++c) dot = std::fmaf(q[c], k[c], dot);
-        z[J] = dot * scale;
-        mx = std::max(mx, z[J]);
-      }
-      // Row sum in the kernel's order: 32 interleaved partial sums (partial
-      // l adds the terms l, l+32, l+64, ... in turn), then combined pairwise
-      // at distances 16, 8, 4, 2, 1.
-      float part[32];
-      for (int l = 0; l < 32; ++l) part[l] = 0.0f;
-      for (int64_t J = 0; J < Nkb; ++J) {
-        z[J] = std::exp(z[J] - mx);
-        part[J % 32] = part[J % 32] + z[J];
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        float nxt[32];
-        for (int l = 0; l < 32; ++l) nxt[l] = part[l] + part[l ^ o];
-        for (int l = 0; l < 32; ++l) part[l] = nxt[l];
-      }
-      const float sum = part[0];
-      float* row = P + (bh * Nqb + I) * Nkb;
-      for (int64_t J = 0; J < Nkb; ++J) row[J] = z[J] / sum;
     }
   return OK;
 }
@@ -245,82 +185,49 @@ int oracle_select_row(const double* P, int64_t Nkb, double topk, double topp, in
 }
 
 // ---------------------------------------------------------------------------
-// Full mask [SA2 s1, s4]: pool, score, select, for every query-block row.
-// Q, K: bf16 bits [B*H, N, d]. kv_idx [B*H, Nqb, Nkb] (first kv_cnt entries
-// valid, ascending), kv_cnt [B*H, Nqb]. precision: 32 (the kernel's decision
-// precision) or 64 (the double definition). P_out: optional [B*H, Nqb, Nkb].
-// ---------------------------------------------------------------------------
-// ---------------------------------------------------------------------------
 // Block mask with a learnt router [SLA2 s2]: the article replaces the
 // heuristic routing by a router with two learnable projection matrices that
 // map the query and key features into a space suited to the routing
 // decision. Reading: the pooled block vectors are projected,
 //   qhat_I = qbar_I Wq_h,  khat_J = kbar_J Wk_h   (W: [d, dr] per head h),
 // and the block importance is softmax_J(qhat_I . khat_J / sqrt(dr)), followed
-// by the same hybrid selection. Single precision: each projected entry is a
-// sequential fused multiply-add over the d input channels in order.
-// Wq / Wk: fp32 [H, d, dr] (row c, column c'); H = BH / (heads per batch).
+// by the same hybrid selection. Every step in double.
+// Q, K: bf16 bits [B*H, N, d]. Wq / Wk: fp32 [H, d, dr] (row c, column c'),
+// H = BH / (batches); both null for the plain mask. kv_idx [B*H, Nqb, Nkb]
+// (first kv_cnt entries valid, ascending), kv_cnt [B*H, Nqb]. P_out:
+// optional [B*H, Nqb, Nkb].
 // ---------------------------------------------------------------------------
 int oracle_mask_router(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int d, int bq, int bk,
-                       const float* Wq, const float* Wk, int64_t H, int dr, double topk, double topp, int precision,
+                       const float* Wq, const float* Wk, int64_t H, int dr, double topk, double topp,
                        int32_t* kv_idx, int32_t* kv_cnt, double* P_out) {
   if (!Q || !K || !kv_idx || !kv_cnt || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
-  if (precision != 32 && precision != 64) return ERR_ARG;
   const bool routed = Wq != nullptr || Wk != nullptr;
   if (routed && (!Wq || !Wk || H <= 0 || BH % H != 0 || dr <= 0)) return ERR_ARG;
   const int dd = routed ? dr : d;
   const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
   std::vector<double> P(static_cast<size_t>(BH * Nqb * Nkb));
-  if (precision == 64) {
-    std::vector<double> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
-    oracle_pool_f64(Q, BH, N, d, bq, qb.data());
-    oracle_pool_f64(K, BH, N, d, bk, kb.data());
-    if (routed) {
-      std::vector<double> qh(static_cast<size_t>(BH * Nqb * dr)), kh(static_cast<size_t>(BH * Nkb * dr));
-      for (int pass = 0; pass < 2; ++pass) {
-        const std::vector<double>& in = pass == 0 ? qb : kb;
-        std::vector<double>& out = pass == 0 ? qh : kh;
-        const float* W = pass == 0 ? Wq : Wk;
-        const int64_t nb = pass == 0 ? Nqb : Nkb;
-        for (int64_t bh = 0; bh < BH; ++bh)
-          for (int64_t I = 0; I < nb; ++I)
-            for (int c2 = 0; c2 < dr; ++c2) {
-              double acc = 0.0;
-              for (int c = 0; c < d; ++c)
-                acc += in[(bh * nb + I) * d + c] * static_cast<double>(W[((bh % H) * d + c) * dr + c2]);
-              out[(bh * nb + I) * dr + c2] = acc;
-            }
-      }
-      oracle_block_probs_f64(qh.data(), kh.data(), BH, Nqb, Nkb, dd, P.data());
-    } else {
-      oracle_block_probs_f64(qb.data(), kb.data(), BH, Nqb, Nkb, dd, P.data());
+  std::vector<double> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
+  oracle_pool_f64(Q, BH, N, d, bq, qb.data());
+  oracle_pool_f64(K, BH, N, d, bk, kb.data());
+  if (routed) {
+    std::vector<double> qh(static_cast<size_t>(BH * Nqb * dr)), kh(static_cast<size_t>(BH * Nkb * dr));
+    for (int pass = 0; pass < 2; ++pass) {
+      const std::vector<double>& in = pass == 0 ? qb : kb;
+      std::vector<double>& out = pass == 0 ? qh : kh;
+      const float* W = pass == 0 ? Wq : Wk;
+      const int64_t nb = pass == 0 ? Nqb : Nkb;
+      for (int64_t bh = 0; bh < BH; ++bh)
+        for (int64_t I = 0; I < nb; ++I)
+          for (int c2 = 0; c2 < dr; ++c2) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+              acc += in[(bh * nb + I) * d + c] * static_cast<double>(W[((bh % H) * d + c) * dr + c2]);
+            out[(bh * nb + I) * dr + c2] = acc;
+          }
     }
+    oracle_block_probs_f64(qh.data(), kh.data(), BH, Nqb, Nkb, dd, P.data());
   } else {
-    std::vector<float> qb(static_cast<size_t>(BH * Nqb * d)), kb(static_cast<size_t>(BH * Nkb * d));
-    std::vector<float> Pf(P.size());
-    oracle_pool_f32(Q, BH, N, d, bq, qb.data());
-    oracle_pool_f32(K, BH, N, d, bk, kb.data());
-    if (routed) {
-      std::vector<float> qh(static_cast<size_t>(BH * Nqb * dr)), kh(static_cast<size_t>(BH * Nkb * dr));
-      for (int pass = 0; pass < 2; ++pass) {
-        const std::vector<float>& in = pass == 0 ? qb : kb;
-        std::vector<float>& out = pass == 0 ? qh : kh;
-        const float* W = pass == 0 ? Wq : Wk;
-        const int64_t nb = pass == 0 ? Nqb : Nkb;
-        for (int64_t bh = 0; bh < BH; ++bh)
-          for (int64_t I = 0; I < nb; ++I)
-            for (int c2 = 0; c2 < dr; ++c2) {
-              float acc = 0.0f;
-              for (int c = 0; c < d; ++c)
-                acc = std::fma(in[(bh * nb + I) * d + c], W[((bh % H) * d + c) * dr + c2], acc);
-              out[(bh * nb + I) * dr + c2] = acc;
-            }
-      }
-      oracle_block_probs_f32(qh.data(), kh.data(), BH, Nqb, Nkb, dd, Pf.data());
-    } else {
-      oracle_block_probs_f32(qb.data(), kb.data(), BH, Nqb, Nkb, dd, Pf.data());
-    }
-    for (size_t i = 0; i < P.size(); ++i) P[i] = static_cast<double>(Pf[i]);
+    oracle_block_probs_f64(qb.data(), kb.data(), BH, Nqb, Nkb, dd, P.data());
   }
   for (int64_t row = 0; row < BH * Nqb; ++row) {
     int64_t m = 0;
@@ -334,12 +241,11 @@ int oracle_mask_router(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t
   return OK;
 }
 
-// Block mask without a router: pooled vectors scored directly.
+// Block mask without a router [SA2 s1, s4]: pool, score, select, for every
+// query-block row, the pooled vectors scored directly.
 int oracle_mask(const uint16_t* Q, const uint16_t* K, int64_t BH, int64_t N, int d, int bq,
-                int bk, double topk, double topp, int precision, int32_t* kv_idx,
-                int32_t* kv_cnt, double* P_out) {
-  return oracle_mask_router(Q, K, BH, N, d, bq, bk, nullptr, nullptr, 0, 0, topk, topp, precision, kv_idx, kv_cnt,
-                            P_out);
+                int bk, double topk, double topp, int32_t* kv_idx, int32_t* kv_cnt, double* P_out) {
+  return oracle_mask_router(Q, K, BH, N, d, bq, bk, nullptr, nullptr, 0, 0, topk, topp, kv_idx, kv_cnt, P_out);
 }
 
 // ---------------------------------------------------------------------------

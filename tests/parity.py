@@ -17,7 +17,7 @@ AMBIG_REL = 1e-6
 def compare_masks(g_idx, g_cnt, o_idx, o_cnt, P, topk, topp):
     """Returns (n_rows, n_mismatched_rows, n_ambiguous_rows); raises on a
     mismatch outside the ambiguity rule. Arrays are numpy; P is the oracle's
-    probability array in the decision precision."""
+    double-precision probability array."""
     g_idx = np.asarray(g_idx).reshape(-1, g_idx.shape[-1])
     o_idx = np.asarray(o_idx).reshape(-1, o_idx.shape[-1])
     g_cnt = np.asarray(g_cnt).reshape(-1)
@@ -55,6 +55,34 @@ def compare_masks(g_idx, g_cnt, o_idx, o_cnt, P, topk, topp):
                 f"({len(os_)}); unexplained blocks {sorted(diff - allowed)[:10]}, threshold {t}")
         n_amb += 1
     return len(g_cnt), len(bad_rows), n_amb
+
+
+def check_mask_outputs(gpu, ora, topk, topp):
+    """Checks a GPU mask (kv_idx, kv_cnt, probs as float, row thresholds as
+    float) against the oracle's (kv_idx, kv_cnt, P in double): kept sets under
+    the ambiguity rule, probabilities to float rounding, and, on the rows whose
+    kept sets agree, the threshold = the smallest kept probability (the last
+    kept block in the (P desc, index asc) order). Returns compare_masks'
+    counts."""
+    g_idx, g_cnt, g_P, g_thr = gpu
+    o_idx, o_cnt, o_P = ora
+    # float rounding (2^-24 relative) of a double that differs from the
+    # oracle's by a few double rounding units
+    np.testing.assert_allclose(g_P, o_P, rtol=1.2e-7, atol=1e-45)
+    n, bad, amb = compare_masks(g_idx, g_cnt, o_idx, o_cnt, o_P, topk, topp)
+    nkb = o_P.shape[-1]
+    oi = o_idx.reshape(-1, nkb)
+    oc = o_cnt.reshape(-1)
+    gi = g_idx.reshape(-1, nkb)
+    gc = g_cnt.reshape(-1)
+    P = o_P.reshape(-1, nkb)
+    cols = np.arange(nkb)[None, :]
+    valid = cols < oc[:, None]
+    same = (gc == oc) & np.all(np.where(valid, gi == oi, True), axis=1)
+    kept_P = np.where(valid, np.take_along_axis(P, np.clip(oi, 0, nkb - 1), axis=1), np.inf)
+    t = kept_P.min(axis=1)
+    np.testing.assert_allclose(g_thr.reshape(-1)[same], t[same], rtol=1.2e-7, atol=1e-45)
+    return n, bad, amb
 
 
 def output_errors(got, ref):

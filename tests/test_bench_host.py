@@ -100,3 +100,66 @@ def test_committed_traffic_entries_name_their_capture():
     for name, e in entries.items():
         assert e["dram_bytes_per_launch"] > 0 and e["kernel"].split("<")[0] in bench.KERNEL_SOURCES, name
         assert os.path.exists(os.path.join(bench.ROOT, e["source"])), name
+
+
+def test_burst_peak_applies_at_max_clock_or_without_samples(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
+                                                              "hbm_gbs": 6000.0}))
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 9}
+    capped = {"sm_mhz": 1600.0, "sm_max_mhz": 1965.0, "samples": 9}
+    none = {"sm_mhz": None, "sm_max_mhz": None, "samples": 0}
+    assert bench.clocks_at_max(at_max) and bench.clocks_at_max(none) and not bench.clocks_at_max(capped)
+    peak, fr, desc = bench.roofline_peak(800.0, at_max)
+    assert peak == 1600.0 and "burst" in desc and fr["frac_vs_burst"] == 0.5 and fr["frac_vs_sustained"] == 800 / 1400
+    assert fr["frac_vs_nominal"] == 800.0 / bench.NOMINAL_BF16_TFLOPS
+    peak, _, desc = bench.roofline_peak(800.0, none)
+    assert peak == 1600.0 and "no clock samples" in desc
+    peak, _, desc = bench.roofline_peak(800.0, capped)
+    assert peak == 1400.0 and "sustained" in desc
+    peak, fr, _ = bench.roofline_peak(800.0, at_max, ratio=2.0)
+    assert peak == 3200.0 and fr["frac_vs_burst"] == 0.25
+
+
+def test_timed_steps_flush_outside_each_steps_events():
+    """Every step is preceded by an L2 flush that lies outside its own events,
+    and each step records its span events between them."""
+    log = []
+
+    class Ev:
+        def __init__(self, enable_timing=False):
+            self.t = None
+
+        def record(self, stream=None):
+            self.t = len(log)
+            log.append("ev")
+
+        def elapsed_time(self, other):
+            return float(other.t - self.t)
+
+    class Flush:
+        def zero_(self):
+            log.append("flush")
+
+    class Cuda:
+        Event = Ev
+
+        @staticmethod
+        def synchronize():
+            log.append("sync")
+
+    def step(ea, eb):
+        ea.record()
+        log.append("work")
+        eb.record()
+
+    step_ms, attn_ms = bench.timed_steps(step, 3, None, Flush(), cuda=Cuda)
+    assert log == ["flush", "ev", "ev", "work", "ev", "ev"] * 3 + ["sync"]
+    assert step_ms == [4.0] * 3 and attn_ms == [2.0] * 3
+
+
+def test_nvml_sampler_falls_back_without_a_gpu():
+    with bench.NvmlClockSampler("GPU-00000000-0000-0000-0000-000000000000", period_s=0.001) as clk:
+        pass
+    s = clk.summary()
+    assert "samples" in s and "source" in s

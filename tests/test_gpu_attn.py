@@ -104,7 +104,7 @@ def test_attn_long_rows_at_the_block_limit():
 def test_attn_workload_oracle_mask(name):
     w = synth.WORKLOADS[name]
     Q, K, V, _ = synth.make_workload(w)
-    idx, cnt, _ = oracle.mask(Q, K, w.bq, w.bk, w.topk, w.topp, precision=32)
+    idx, cnt, _ = oracle.mask(Q, K, w.bq, w.bk, w.topk, w.topp)
     rows = None if name == "tiny" else sample_rows(w.B, w.H, w.N, w.bq, 96, seed=1)
     max_abs, mean_rel = _check_rows(Q, K, V, idx, cnt, w.bq, w.bk, rows=rows)
     print(f"{name}: max-abs {max_abs:.2e} mean-rel-L1 {mean_rel:.2e}")

@@ -1,12 +1,17 @@
-"""GPU block mask vs the CPU oracle (decision taken in single precision on
-both sides, same operation order; see the oracle's header)."""
+"""GPU block mask vs the CPU oracle's double-precision definition.
+
+The kept sets must be identical except where the ambiguity rule allows a
+difference (a block within 1e-6 relative of the row's threshold probability,
+or a Top-p boundary whose running sum lies within 1e-6 of p); such rows are
+counted and printed. The probabilities and the row thresholds the GPU
+returns (rounded to float) must equal the oracle's to float rounding."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from block_sparse_attention_pooled_b200 import synth
-from parity import compare_masks
+from parity import check_mask_outputs
 
 pytestmark = pytest.mark.gpu
 
@@ -26,15 +31,12 @@ def _run(Q, K, bq, bk, topk, topp):
     return idx.cpu().numpy(), cnt.cpu().numpy(), probs.cpu().numpy(), thr.cpu().numpy()
 
 
-def _check(Q, K, bq, bk, topk, topp):
-    g_idx, g_cnt, g_P, g_thr = _run(Q, K, bq, bk, topk, topp)
-    o_idx, o_cnt, o_P = oracle.mask(Q, K, bq, bk, topk, topp, precision=32)
-    # probabilities: same operation order except the row sum and expf rounding
-    np.testing.assert_allclose(g_P, o_P, rtol=1e-6, atol=1e-37)
-    n, bad, amb = compare_masks(g_idx, g_cnt, o_idx, o_cnt, o_P, topk, topp)
-    # threshold output: probability of the last kept block (rows that agree)
-    rows = g_cnt.reshape(-1) == o_cnt.reshape(-1)
-    assert np.all(g_thr.reshape(-1) > 0)
+def _check(Q, K, bq, bk, topk, topp, what=""):
+    g = _run(Q, K, bq, bk, topk, topp)
+    o_idx, o_cnt, o_P = oracle.mask(Q, K, bq, bk, topk, topp)
+    n, bad, amb = check_mask_outputs(g, (o_idx, o_cnt, o_P), topk, topp)
+    if what:
+        print(f"{what}: rows {n}, rows differing from the fp64 definition {bad} (all within the ambiguity rule)")
     return n, bad, amb
 
 
@@ -61,23 +63,22 @@ def test_mask_long_rows(nkb, topk, topp):
 def test_mask_workloads(name):
     w = synth.WORKLOADS[name]
     Q, K, _, _ = synth.make_workload(w)
-    n, bad, amb = _check(Q, K, w.bq, w.bk, w.topk, w.topp)
-    print(f"{name}: rows {n}, mismatched rows {bad} (all within the ambiguity rule)")
+    _check(Q, K, w.bq, w.bk, w.topk, w.topp, what=name)
 
 
 def test_mask_720p_all_heads():
     w = synth.WORKLOADS["720p"]
     Q, K, _, _ = synth.make_workload(w)
-    n, bad, amb = _check(Q, K, w.bq, w.bk, w.topk, w.topp)
-    print(f"720p: rows {n}, mismatched rows {bad} (all within the ambiguity rule)")
+    _check(Q, K, w.bq, w.bk, w.topk, w.topp, what="720p")
 
 
 @pytest.mark.parametrize("topk,topp", [(t, p) for t in synth.SWEEP_TOPK for p in synth.SWEEP_TOPP]
                          + [(0.05, 0.0), (0.0, 0.9)])
 def test_mask_sweep_regimes(topk, topp):
-    w = synth.WORKLOADS["sweep_peaked"]
-    Q, K, _ = synth.make_qkv(1, 4, w.N, w.d, w.grid, w.s, w.seed)
-    _check(Q, K, w.bq, w.bk, topk, topp)
+    for name in ("sweep_flat", "sweep_peaked"):
+        w = synth.WORKLOADS[name]
+        Q, K, _ = synth.make_qkv(1, 4, w.N, w.d, w.grid, w.s, w.seed)
+        _check(Q, K, w.bq, w.bk, topk, topp, what=f"{name} k={topk} p={topp} (4 heads)")
 
 
 def test_mask_is_deterministic():
@@ -104,8 +105,8 @@ def test_mask_exact_ties_take_lower_indices(topk, topp):
     Q, K, _ = synth.make_qkv(B, H, N, d, grid=None, s=1.5, seed=77)
     K = K[:, :, :bk].repeat(1, 1, N // bk, 1).contiguous()
     g_idx, g_cnt, g_P, _ = _run(Q, K, bq, bk, topk, topp)
-    o_idx, o_cnt, o_P = oracle.mask(Q, K, bq, bk, topk, topp, precision=32)
-    np.testing.assert_array_equal(g_P, o_P)
+    o_idx, o_cnt, o_P = oracle.mask(Q, K, bq, bk, topk, topp)
+    np.testing.assert_array_equal(g_P, o_P.astype(np.float32))
     np.testing.assert_array_equal(g_cnt, o_cnt)
     for r, c in enumerate(g_cnt.reshape(-1)):
         np.testing.assert_array_equal(g_idx.reshape(-1, g_idx.shape[-1])[r, :c], np.arange(c))

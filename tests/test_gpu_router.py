@@ -1,12 +1,13 @@
-"""Learnt-router block mask on the GPU against the CPU oracle (decision taken
-in single precision on both sides, same operation order)."""
+"""Learnt-router block mask on the GPU against the CPU oracle's
+double-precision definition, under the same ambiguity rule as the plain
+mask."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from block_sparse_attention_pooled_b200 import synth
-from parity import compare_masks
+from parity import check_mask_outputs
 
 pytestmark = pytest.mark.gpu
 
@@ -26,12 +27,12 @@ def _run(Q, K, Wq, Wk, bq, bk, topk, topp):
     return idx.cpu().numpy(), cnt.cpu().numpy(), probs.cpu().numpy(), thr.cpu().numpy()
 
 
-def _check(Q, K, Wq, Wk, bq, bk, topk, topp):
-    g_idx, g_cnt, g_P, g_thr = _run(Q, K, Wq, Wk, bq, bk, topk, topp)
-    o_idx, o_cnt, o_P = oracle.mask_router(Q, K, bq, bk, Wq, Wk, topk, topp, precision=32)
-    np.testing.assert_allclose(g_P, o_P, rtol=1e-6, atol=1e-37)
-    n, bad, amb = compare_masks(g_idx, g_cnt, o_idx, o_cnt, o_P, topk, topp)
-    assert np.all(g_thr > 0)
+def _check(Q, K, Wq, Wk, bq, bk, topk, topp, what=""):
+    g = _run(Q, K, Wq, Wk, bq, bk, topk, topp)
+    o = oracle.mask_router(Q, K, bq, bk, Wq, Wk, topk, topp)
+    n, bad, amb = check_mask_outputs(g, o, topk, topp)
+    if what:
+        print(f"{what}: rows {n}, rows differing from the fp64 definition {bad} (all within the ambiguity rule)")
     return n, bad, amb
 
 
@@ -62,8 +63,7 @@ def test_router_480p():
     w = synth.WORKLOADS["480p"]
     Q, K, _, _ = synth.make_workload(w)
     Wq, Wk = synth.make_router(w.H, w.d, 64, seed=1)
-    n, bad, amb = _check(Q, K, Wq, Wk, w.bq, w.bk, w.topk, w.topp)
-    print(f"480p router: rows {n}, mismatched rows {bad} (all within the ambiguity rule)")
+    _check(Q, K, Wq, Wk, w.bq, w.bk, w.topk, w.topp, what="480p router (dr 64)")
 
 
 def test_router_multi_batch_heads():

@@ -104,7 +104,7 @@ def test_sla2_workload_oracle_mask(name):
     else:
         Q, K, V, alpha = synth.make_workload(w)
         alpha = alpha.numpy()
-    idx, cnt, _ = oracle.mask(Q, K, w.bq, w.bk, w.topk, w.topp, precision=32)
+    idx, cnt, _ = oracle.mask(Q, K, w.bq, w.bk, w.topk, w.topp)
     B, H = Q.shape[:2]
     rows = sample_rows(B, H, w.N, w.bq, 48, seed=2)
     max_abs, mean_rel = _check(Q, K, V, idx, cnt, alpha, w.bq, w.bk, rows=rows)

@@ -53,7 +53,7 @@ def _phi_torch(x):
 # ----------------------------------------------------------------------------- pooling
 def test_pool_full_blocks_match_avg_pool(oracle_mod):
     q, _, _ = _rand_qkv(1, 2, 256, 16, 1)
-    got = oracle_mod.pool(q, 64, precision=64)
+    got = oracle_mod.pool(q, 64)
     x = q.double().reshape(2, 256, 16).transpose(1, 2)  # (BH, d, N)
     ref = F.avg_pool1d(x, kernel_size=64, stride=64).transpose(1, 2).reshape(1, 2, 4, 16)
     np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
@@ -64,19 +64,10 @@ def test_pool_ragged_block_averages_valid_rows_only(oracle_mod):
     x = torch.zeros(1, 1, 70, 4)
     x[0, 0, :64] = 3.0
     x[0, 0, 64:] = torch.arange(6, dtype=torch.float32)[:, None]  # rows 0..5 -> mean 2.5
-    got = oracle_mod.pool(_bf16(x), 64, precision=64)
+    got = oracle_mod.pool(_bf16(x), 64)
     assert got.shape == (1, 1, 2, 4)
     np.testing.assert_array_equal(got[0, 0, 0], 3.0)
     np.testing.assert_array_equal(got[0, 0, 1], 2.5)
-    got32 = oracle_mod.pool(_bf16(x), 64, precision=32)
-    np.testing.assert_array_equal(got32[0, 0, 1], np.float32(2.5))
-
-
-def test_pool_single_precision_close_to_double(oracle_mod):
-    q, _, _ = _rand_qkv(1, 2, 300, 32, 2, scale=3.0)
-    a = oracle_mod.pool(q, 128, 64)
-    b = oracle_mod.pool(q, 128, 32).astype(np.float64)
-    np.testing.assert_allclose(b, a, rtol=0, atol=1e-5)
 
 
 # ----------------------------------------------------------------------------- block scores
@@ -88,9 +79,6 @@ def test_block_probs_match_torch_softmax(oracle_mod):
     ref = torch.softmax(qb @ kb.transpose(-1, -2) / math.sqrt(16), dim=-1)
     np.testing.assert_allclose(got, ref.numpy(), rtol=1e-13, atol=1e-15)
     np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-12)
-    got32 = oracle_mod.block_probs(qb.numpy().astype(np.float32), kb.numpy().astype(np.float32))
-    np.testing.assert_allclose(got32, ref.numpy(), rtol=1e-4, atol=1e-6)
-    np.testing.assert_allclose(got32.sum(-1, dtype=np.float64), 1.0, atol=1e-5)
 
 
 # ----------------------------------------------------------------------------- selection
@@ -170,16 +158,6 @@ def test_select_invariants_random_rows(oracle_mod):
             assert r["cum"][r["pc"]] >= topp > r["cum"][r["pc"] - 1]
 
 
-def test_mask_single_precision_agrees_with_double(oracle_mod):
-    Q, K, _ = synth.make_qkv(1, 2, 2000, 64, grid=(2, 25, 40), s=1.5, seed=5)
-    i32, c32, P32 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=32)
-    i64, c64, P64 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=64)
-    np.testing.assert_allclose(P32, P64, rtol=1e-3, atol=1e-7)
-    same = (c32 == c64) & np.all(i32 == i64, axis=-1)
-    assert same.mean() > 0.95
-    np.testing.assert_allclose(P64.sum(-1), 1.0, atol=1e-12)
-
-
 # ----------------------------------------------------------------------------- attention
 def test_dense_matches_sdpa(oracle_mod):
     q, k, v = _rand_qkv(1, 2, 200, 16, 21, scale=1.5)
@@ -220,7 +198,7 @@ def test_all_blocks_kept_equals_dense(oracle_mod):
     # and the mask itself keeps all blocks when k = 1
     idx, cnt, _ = oracle_mod.mask(q, k, bq, bk, 1.0, 0.0)
     assert (cnt == nkb).all()
-    idx, cnt, _ = oracle_mod.mask(q, k, bq, bk, 0.0, 1.0, precision=64)
+    idx, cnt, _ = oracle_mod.mask(q, k, bq, bk, 0.0, 1.0)
     assert (cnt >= 1).all()
 
 
@@ -470,11 +448,10 @@ def _router_inputs(seed, H=2, N=2048, d=64, s=1.5):
 def test_router_identity_projection_is_the_plain_mask(oracle_mod):
     Q, K = _router_inputs(50)
     I = np.tile(np.eye(64, dtype=np.float32), (2, 1, 1))
-    for precision in (32, 64):
-        a = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=precision)
-        b = oracle_mod.mask_router(Q, K, 64, 64, I, I, 0.1, 0.9, precision=precision)
-        for x, y in zip(a, b):
-            np.testing.assert_array_equal(x, y)
+    a = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9)
+    b = oracle_mod.mask_router(Q, K, 64, 64, I, I, 0.1, 0.9)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
 
 
 def test_router_probabilities_match_projected_softmax(oracle_mod):
@@ -482,9 +459,9 @@ def test_router_probabilities_match_projected_softmax(oracle_mod):
     g = np.random.default_rng(5)
     Wq = g.standard_normal((2, 64, 32)).astype(np.float32) / 8
     Wk = g.standard_normal((2, 64, 32)).astype(np.float32) / 8
-    _, _, P = oracle_mod.mask_router(Q, K, 64, 64, Wq, Wk, 0.1, 0.9, precision=64)
-    qb = oracle_mod.pool(Q, 64, precision=64)[0]  # [H, Nqb, d]
-    kb = oracle_mod.pool(K, 64, precision=64)[0]
+    _, _, P = oracle_mod.mask_router(Q, K, 64, 64, Wq, Wk, 0.1, 0.9)
+    qb = oracle_mod.pool(Q, 64)[0]  # [H, Nqb, d]
+    kb = oracle_mod.pool(K, 64)[0]
     for h in range(2):
         z = (qb[h] @ Wq[h].astype(np.float64)) @ (kb[h] @ Wk[h].astype(np.float64)).T / math.sqrt(32)
         ref = torch.softmax(torch.from_numpy(z), dim=-1).numpy()
@@ -495,8 +472,8 @@ def test_router_orthogonal_projection_keeps_the_probabilities(oracle_mod):
     Q, K = _router_inputs(52)
     R = np.linalg.qr(np.random.default_rng(6).standard_normal((64, 64)))[0].astype(np.float32)
     W = np.stack([R, R])
-    _, _, P0 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9, precision=64)
-    _, _, P1 = oracle_mod.mask_router(Q, K, 64, 64, W, W, 0.1, 0.9, precision=64)
+    _, _, P0 = oracle_mod.mask(Q, K, 64, 64, 0.1, 0.9)
+    _, _, P1 = oracle_mod.mask_router(Q, K, 64, 64, W, W, 0.1, 0.9)
     np.testing.assert_allclose(P1, P0, rtol=1e-5, atol=1e-9)  # R R^T = I up to the fp32 rounding of R
 
 
@@ -505,8 +482,9 @@ def test_router_power_of_two_rescaling_is_exact(oracle_mod):
     g = np.random.default_rng(7)
     Wq = g.standard_normal((2, 64, 64)).astype(np.float32) / 8
     Wk = g.standard_normal((2, 64, 64)).astype(np.float32) / 8
-    a = oracle_mod.mask_router(Q, K, 64, 64, Wq, Wk, 0.1, 0.9, precision=32)
-    b = oracle_mod.mask_router(Q, K, 64, 64, Wq * 2, Wk / 2, 0.1, 0.9, precision=32)
+    # Doubling Wq and halving Wk scales every product by exactly 2 and 1/2.
+    a = oracle_mod.mask_router(Q, K, 64, 64, Wq, Wk, 0.1, 0.9)
+    b = oracle_mod.mask_router(Q, K, 64, 64, Wq * 2, Wk / 2, 0.1, 0.9)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
 

@@ -76,10 +76,10 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     from block_sparse_attention_pooled_b200 import sparge
 
     P = ctypes.c_void_p(16 * 1024)  # never dereferenced: the size check comes first
-    # 720p-sized mask: pooled Q/K 36 MB + probability rows 112 MB > 16 MiB.
+    # 720p-sized mask: pooled Q/K 73 MB + score rows 224 MB > 16 MiB.
     big = sparge.Shape(1, 40, 75600, 128, 128, 64)
     rc = sparge.raw().sparge_mask_noalloc(P, P, ctypes.byref(big), 0.03, 0.9, P, P, None, None, None)
     assert rc == sparge.ERR_WORKSPACE
-    # Still too large when the caller supplies the probability rows.
+    # Still too large when the caller also asks for the probability rows.
     rc = sparge.raw().sparge_mask_noalloc(P, P, ctypes.byref(big), 0.03, 0.9, P, P, None, P, None)
     assert rc == sparge.ERR_WORKSPACE
