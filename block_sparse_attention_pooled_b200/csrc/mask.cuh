@@ -134,27 +134,49 @@ __global__ void __launch_bounds__(128) project_kernel(const double* __restrict__
 }
 
 // ----------------------------------------------------------------------------
-// Scaled scores z[I, J] = (q̄_I . k̄_J) * (1/sqrt(d)), in double. One CTA = 32
-// query-block rows x 64 key blocks of one (b,h); each thread owns 4 rows x 4
-// key blocks (8 shared-memory loads per 16 fused multiply-adds). Pooled K
-// rows are padded by one double in shared memory so that the 16 rows a warp
-// reads at once fall in 16 different bank pairs. The row softmax happens in
-// the selection kernel, which reads the whole row anyway.
+// Scaled scores z[I, J] = (q̄_I . k̄_J) * (1/sqrt(d)), in double, on the fp64
+// tensor cores (mma.sync m8n8k4 .f64: each instruction is 256 fused
+// multiply-adds of one warp, its operands one double per lane). One CTA =
+// 64 query-block rows x 64 key blocks of one (b,h); warp w owns rows
+// 32 (w / 2) .. + 31 and key blocks 32 (w % 2) .. + 31 as 4 x 4 tiles of 8 x 8.
+// The pooled vectors pass through shared memory 32 channels at a time in a
+// two-stage cp.async ring; rows are padded to 36 doubles, so the 8 rows x 4
+// channels a fragment load touches fill the banks twice (256 bytes, the
+// minimum of two wavefronts). Rows past the tile's end are zero-filled.
+// The row softmax happens in the selection kernel, which reads the whole row
+// anyway.
 // ----------------------------------------------------------------------------
-constexpr int kScoreRows = 32;
-constexpr int kScoreTileJ = 64;
+constexpr int kScoreRows = 64;     // query-block rows per CTA
+constexpr int kScoreTileJ = 64;    // key blocks per CTA
+constexpr int kScoreChunk = 32;    // channels per stage
+constexpr int kScorePitch = 36;    // doubles per staged row
 
 template <int D>
 __host__ __device__ constexpr int score_smem_bytes() {
-  return (kScoreRows * D + kScoreTileJ * (D + 1)) * 8;
+  return 2 * (kScoreRows + kScoreTileJ) * kScorePitch * 8;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void dmma_884(double& c0, double& c1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(c0), "+d"(c1)
+               : "d"(a), "d"(b));
 }
 
 template <int D>
 __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                                                     int nqb, int nkb, double scale, double* __restrict__ Z) {
   extern __shared__ __align__(16) double smd[];
-  double* sq = smd;                                 // [32][D]
-  double* sk = sq + kScoreRows * D;                 // [64][D+1]
+  constexpr int kStage = (kScoreRows + kScoreTileJ) * kScorePitch;  // doubles per stage
+  constexpr int kChunks = D / kScoreChunk;
   const int tiles_q = (nqb + kScoreRows - 1) / kScoreRows;
   const int tiles_j = (nkb + kScoreTileJ - 1) / kScoreTileJ;
   const int64_t cta = blockIdx.x;
@@ -164,48 +186,77 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
   const int J0 = (rem % tiles_j) * kScoreTileJ;
   const int nrows = min(kScoreRows, nqb - I0);
   const int nj = min(kScoreTileJ, nkb - J0);
-  const int tid = threadIdx.x;
-  for (int e = tid; e < kScoreRows * (D / 2); e += 128) {
-    const int i = e / (D / 2), c2 = (e % (D / 2)) * 2;
-    double2 v = make_double2(0.0, 0.0);
-    if (i < nrows) v = *reinterpret_cast<const double2*>(qbar + (bh * nqb + I0 + i) * D + c2);
-    *reinterpret_cast<double2*>(sq + i * D + c2) = v;
-  }
-  for (int e = tid; e < kScoreTileJ * (D / 2); e += 128) {
-    const int j = e / (D / 2), c2 = (e % (D / 2)) * 2;
-    double2 v = make_double2(0.0, 0.0);
-    if (j < nj) v = *reinterpret_cast<const double2*>(kbar + (bh * nkb + J0 + j) * D + c2);
-    sk[j * (D + 1) + c2] = v.x;  // rows of D + 1 doubles: 8-byte stores only
-    sk[j * (D + 1) + c2 + 1] = v.y;
-  }
-  __syncthreads();
-  const int jl = tid % 16;   // key blocks jl, jl+16, jl+32, jl+48 of the tile
-  const int ig = tid / 16;   // query rows 4*ig .. 4*ig+3
-  double acc[4][4];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double* qsrc = qbar + (bh * nqb + I0) * D;
+  const double* ksrc = kbar + (bh * nkb + J0) * D;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smd);
+
+  // Stage `st` takes channels [ch * 32, ch * 32 + 32) of the tile's 64 + 64
+  // rows: 128 rows x 16 pieces of 16 bytes (2 doubles), 16 pieces per thread.
+  auto load_stage = [&](int st, int ch) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-#pragma unroll 4
-  for (int c = 0; c < D; ++c) {
-    double q[4], k[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) q[a] = sq[(4 * ig + a) * D + c];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) k[b] = sk[(jl + 16 * b) * (D + 1) + c];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(q[a], k[b], acc[a][b]);
-  }
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = jl + 16 * b;
-      if (j < nj && 4 * ig + a < nrows)
-        Z[(bh * nqb + I0 + 4 * ig + a) * (int64_t)nkb + J0 + j] = __dmul_rn(acc[a][b], scale);
+    for (int u = 0; u < 16; ++u) {
+      const int e = tid + 128 * u;          // 0 .. 2047
+      const int r = e >> 4, piece = e & 15;  // row 0 .. 127 (q rows, then k rows), piece 0 .. 15
+      const bool is_q = r < kScoreRows;
+      const int rr = is_q ? r : r - kScoreRows;
+      const bool valid = rr < (is_q ? nrows : nj);
+      const double* src = (is_q ? qsrc : ksrc) + (int64_t)(valid ? rr : 0) * D + ch * kScoreChunk + piece * 2;
+      const uint32_t dst = sbase + (uint32_t)((st * kStage + r * kScorePitch + piece * 2) * 8);
+      cp_async16(dst, src, valid ? 16 : 0);
     }
+  };
+
+  double acc[4][4][2];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
+  const int wr = 32 * (warp >> 1), wj = 32 * (warp & 1);
+  const int fr = lane >> 2, fc = lane & 3;  // fragment row (A row / B column) and channel
+
+  load_stage(0, 0);
+  cp_async_commit();
+#pragma unroll 1
+  for (int ch = 0; ch < kChunks; ++ch) {
+    if (ch + 1 < kChunks) {
+      load_stage((ch + 1) & 1, ch + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const double* sq = smd + (ch & 1) * kStage;
+    const double* sk = sq + kScoreRows * kScorePitch;
+#pragma unroll
+    for (int kk = 0; kk < kScoreChunk / 4; ++kk) {
+      double a[4], b[4];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) a[mt] = sq[(wr + 8 * mt + fr) * kScorePitch + 4 * kk + fc];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) b[nt] = sk[(wj + 8 * nt + fr) * kScorePitch + 4 * kk + fc];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) dmma_884(acc[mt][nt][0], acc[mt][nt][1], a[mt], b[nt]);
+    }
+    __syncthreads();  // the stage is refilled two chunks later
+  }
+  // Accumulator (c0, c1) of tile (mt, nt) sits at row 8 mt + lane / 4,
+  // columns 8 nt + 2 (lane % 4) + {0, 1}.
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int i = wr + 8 * mt + fr;
+    if (i >= nrows) continue;
+    double* zrow = Z + (bh * nqb + I0 + i) * (int64_t)nkb + J0;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int j = wj + 8 * nt + 2 * fc;
+      if (j < nj) zrow[j] = __dmul_rn(acc[mt][nt][0], scale);
+      if (j + 1 < nj) zrow[j + 1] = __dmul_rn(acc[mt][nt][1], scale);
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -216,19 +267,22 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
 // whatever the summation order (the truncation moves a row's total by less
 // than Nkb * 2^-62).
 //   0. P = exp(z - rowmax) / rowsum (double).
-//   1. Top-p: radix select (8-bit digits, most significant first) of the key
-//      at which the descending running weight first reaches p. It stops as
-//      soon as the digit bucket where p is reached holds a single block.
-//      At full resolution the blocks left tie exactly, all weigh the same, so
-//      the count needed follows by division.
+//   1. Top-p: a radix select of the key at which the descending running
+//      weight first reaches p. The first pass buckets the keys by binade
+//      below the row's largest (bucket 255 - (e_top - e)); the next passes
+//      take 8-bit digits of the mantissa inside the chosen binade. It stops
+//      as soon as the bucket where p is reached holds a single block (its
+//      index is recorded while the histogram is built). If the blocks left at
+//      full resolution tie exactly, they weigh the same and the count needed
+//      follows by division.
 //   2. m = max(kc, pc, 1). When m = pc the threshold is the one just found;
 //      otherwise a counting radix select finds the m-th largest key, stopping
-//      as soon as every block of the bucket where the count is reached is
-//      kept.
-//   3. The threshold is (key prefix T, resolution s, ties kept t): a block is
-//      kept if its key's bits from s up exceed T's, or equal them and fewer
-//      than t lower-indexed blocks share them. Kept flags are compacted in
-//      block order into the ascending kept list.
+//      as soon as the bucket where the count is reached holds one block, or
+//      is kept whole (its smallest key is then the threshold).
+//   3. The threshold is a full key T and a number t of the blocks equal to T
+//      that are kept (lowest indices first): a block is kept if its key
+//      exceeds T, or equals T and fewer than t lower-indexed blocks do.
+//      Kept flags are compacted in block order into the ascending kept list.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ unsigned long long p_fixed62(unsigned long long bits) {
   const int e = (int)((bits >> 52) & 0x7FFull);
@@ -239,67 +293,54 @@ __device__ __forceinline__ unsigned long long p_fixed62(unsigned long long bits)
   return (-sh >= 64) ? 0ull : (mant >> (-sh));
 }
 
-// The threshold of a row: see step 3 above.
-struct RowThreshold {
-  unsigned long long key;  // bits below `shift` are zero
-  int shift;
-  int ties_kept;
-};
-
-__device__ __forceinline__ bool above_threshold(unsigned long long k, const RowThreshold& t) {
-  return (k >> t.shift) > (t.key >> t.shift);
-}
-__device__ __forceinline__ bool at_threshold(unsigned long long k, const RowThreshold& t) {
-  return (k >> t.shift) == (t.key >> t.shift);
-}
-
 constexpr int kSelectThreads = 256;
 constexpr unsigned long long kWeightOne = 1ull << 62;
+constexpr int kAllTies = 1 << 30;  // "every block equal to the threshold key is kept"
 
-__host__ __device__ constexpr int select_smem_bytes(int nkb) {
-  // z / P / keys row (8 B per block) + histograms + scratch
-  return ((nkb + 1) / 2 * 2) * 8 + 256 * 12 + 1024;
-}
-
-// Block-wide exclusive scan of one int per thread (256 threads).
-__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) scratch[wid] = x;
-  __syncthreads();
-  int base = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kSelectThreads / 32; ++w) {
-    const int s = scratch[w];
-    if (w < wid) base += s;
-    tot += s;
-  }
-  __syncthreads();
-  *total = tot;
-  return base + x - v;
-}
-
-// Result of one radix pass: the selected digit's bucket and what lies above it.
-struct RadixState {
-  unsigned long long prefix;  // selected digits so far (bits below the pass's shift zero)
-  unsigned long long above_w; // weight of the keys above the selected bucket
-  int above_c;                // count of the keys above the selected bucket
-  int bucket_c;               // count of the keys in the selected bucket
+// The threshold of a row: see step 3 above.
+struct RowThreshold {
+  unsigned long long key;
+  int ties_kept;
+  int count;  // blocks kept when this threshold alone decides (pc or m)
 };
+
+__device__ __forceinline__ bool keep_key(unsigned long long k, const RowThreshold& t, int tie_rank) {
+  return k > t.key || (k == t.key && tie_rank < t.ties_kept);
+}
+
+// State of a radix select between passes.
+struct RadixState {
+  unsigned long long prefix;   // resolved bits of the selected class
+  unsigned long long mask;     // which bits are resolved
+  unsigned long long above_w;  // weight of the keys above the selected class
+  int above_c;                 // count of the keys above the selected class
+  int bucket_c;                // count of the keys in the selected class
+  int bsel;                    // selected bucket of the last pass
+  int bidx;                    // index of a key of that bucket (the key when bucket_c == 1)
+};
+
+// Bucket of key k in one pass: shift < 0 is the binade pass (every key is a
+// candidate; bucket 255 holds the binade of the row's largest key, bucket 0
+// everything 255 or more binades below, zeros included); otherwise the 8-bit
+// digit at `shift` of the keys in the selected class.
+__device__ __forceinline__ bool key_bucket(unsigned long long k, int shift, int e_top, const RadixState& st,
+                                           unsigned int* d) {
+  if (shift < 0) {
+    const int e = (int)((k >> 52) & 0x7FFull);
+    *d = 255u - (unsigned int)min(255, e_top - e);
+    return true;
+  }
+  *d = (unsigned int)(k >> shift) & 255u;
+  return (k & st.mask) == st.prefix;
+}
 
 // Finds, among 256 buckets held by lanes (lane l owns buckets 255-8l ...
 // 248-8l, descending), the first (from the largest key down) where the
 // running weight (by_weight) or count, starting from st's totals, reaches
-// `target`. Called by the 32 lanes of one warp; the result is returned to
-// all of them.
+// `target`. Called by the 32 lanes of one warp; every lane gets the result.
 __device__ __forceinline__ RadixState radix_scan_warp(const unsigned int* hcnt, const unsigned long long* hsum,
-                                                      bool by_weight, unsigned long long target, int shift,
-                                                      RadixState st) {
+                                                      const unsigned int* hidx, bool by_weight,
+                                                      unsigned long long target, int shift, RadixState st) {
   const int lane = threadIdx.x & 31;
   unsigned long long lw = 0ull;
   unsigned int lc = 0u;
@@ -328,14 +369,12 @@ __device__ __forceinline__ RadixState radix_scan_warp(const unsigned int* hcnt, 
   unsigned long long w = aw;
   unsigned int c = ac;
   int bsel = 255 - 8 * lane - 7;
-  unsigned int bcnt = 0u;
   if (lane == first) {
     for (int i = 0; i < 8; ++i) {
       const int b = 255 - 8 * lane - i;
       const bool hit = by_weight ? (w + hsum[b] >= target) : ((unsigned long long)(c + hcnt[b]) >= target);
       if (hit) {
         bsel = b;
-        bcnt = hcnt[b];
         break;
       }
       w += hsum[b];
@@ -343,112 +382,123 @@ __device__ __forceinline__ RadixState radix_scan_warp(const unsigned int* hcnt, 
     }
   }
   bsel = __shfl_sync(0xffffffffu, bsel, first);
-  bcnt = __shfl_sync(0xffffffffu, bcnt, first);
   c = __shfl_sync(0xffffffffu, c, first);
   w = __shfl_sync(0xffffffffu, w, first);
-  st.prefix |= (unsigned long long)bsel << shift;
+  st.bsel = bsel;
   st.above_c = (int)c;
   st.above_w = w;
-  st.bucket_c = (int)bcnt;
+  st.bucket_c = (int)hcnt[bsel];
+  st.bidx = (int)hidx[bsel];
+  if (shift >= 0) {
+    st.prefix |= (unsigned long long)bsel << shift;
+    st.mask |= 255ull << shift;
+  }
   return st;
 }
 
-// One radix pass of the CTA-per-row kernel: histogram of the digit at
-// `shift` over the keys matching the state's prefix, then the bucket scan by
-// warp 0. Called by all 256 threads.
-__device__ RadixState radix_pass_cta(const unsigned long long* keys, int nkb, int shift, bool by_weight,
-                                     unsigned long long target, RadixState st, unsigned int* hcnt,
-                                     unsigned long long* hsum, RadixState* shared_st) {
-  const int tid = threadIdx.x;
-  hcnt[tid] = 0u;
-  hsum[tid] = 0ull;
-  __syncthreads();
-  const unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-  const unsigned long long pre = st.prefix;
-  for (int j = tid; j < nkb; j += kSelectThreads) {
-    const unsigned long long k = keys[j];
-    if ((k & hi_mask) == pre) {
-      const unsigned int d = (unsigned int)(k >> shift) & 255u;
-      atomicAdd(&hcnt[d], 1u);
-      if (by_weight) atomicAdd(&hsum[d], p_fixed62(k));
+// Radix select over one row's keys. pass(shift, e_top, by_weight, target,
+// state) builds one histogram and scans it; class_min(state) returns the
+// smallest key of the selected class; key_at(j) reads key j. by_weight:
+// Top-p (target = p in fixed point; *count receives pc); otherwise the
+// target-th largest key (*count = target).
+template <typename Pass, typename ClassMin, typename KeyAt>
+__device__ __forceinline__ RowThreshold radix_select(Pass pass, ClassMin class_min, KeyAt key_at, int e_top,
+                                                     bool by_weight, unsigned long long target) {
+  RadixState st{0ull, 0ull, 0ull, 0, 0, 0, 0};
+  st = pass(-1, e_top, by_weight, target, st);  // binade pass
+  // Mantissa digits inside one binade (shifts 44, 36, ..., 4, then 0: the
+  // last digit overlaps the one before, whose bits are already resolved);
+  // the full key's digits (56, 48, ..., 0) when the chosen bucket mixes
+  // binades (255 or more below the largest key, zeros).
+  const bool mixed = st.bsel == 0;
+  int n = 0;
+  if (st.bucket_c != 1) {
+    if (mixed) {
+      st = RadixState{0ull, 0ull, 0ull, 0, 0, 0, 0};
+    } else {
+      st.prefix = (unsigned long long)(e_top - (255 - st.bsel)) << 52;  // sign 0 and the binade's exponent
+      st.mask = 0xFFFull << 52;
     }
   }
-  __syncthreads();
-  if (tid < 32) {
-    const RadixState s = radix_scan_warp(hcnt, hsum, by_weight, target, shift, st);
-    if (tid == 0) *shared_st = s;
-  }
-  __syncthreads();
-  st = *shared_st;
-  __syncthreads();
-  return st;
-}
-
-// One radix pass of the warp-per-row kernel (all 32 lanes of the row's warp).
-__device__ __forceinline__ RadixState radix_pass_warp(const unsigned long long* keys, int nkb, int shift,
-                                                      bool by_weight, unsigned long long target, RadixState st,
-                                                      unsigned int* hcnt, unsigned long long* hsum) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    hcnt[lane * 8 + i] = 0u;
-    hsum[lane * 8 + i] = 0ull;
-  }
-  __syncwarp();
-  const unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-  const unsigned long long pre = st.prefix;
-  for (int j = lane; j < nkb; j += 32) {
-    const unsigned long long k = keys[j];
-    if ((k & hi_mask) == pre) {
-      const unsigned int d = (unsigned int)(k >> shift) & 255u;
-      atomicAdd(&hcnt[d], 1u);
-      if (by_weight) atomicAdd(&hsum[d], p_fixed62(k));
+  for (;;) {
+    if (st.bucket_c == 1) {  // one block left in the class: it is the threshold
+      return RowThreshold{key_at(st.bidx), 1, st.above_c + 1};
     }
-  }
-  __syncwarp();
-  st = radix_scan_warp(hcnt, hsum, by_weight, target, shift, st);
-  __syncwarp();
-  return st;
-}
-
-// The Top-p threshold (and count pc) from the weight-driven passes, or the
-// m-th largest key from the counting passes. pass(shift, by_weight, target,
-// state) runs one radix pass and returns the new state.
-template <typename Pass>
-__device__ __forceinline__ RowThreshold select_by_weight(Pass pass, unsigned long long target, int* pc) {
-  RadixState st{0ull, 0ull, 0, 0};
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    st = pass(shift, true, target, st);
-    if (st.bucket_c == 1 || shift == 0) {
-      int need = 1;
-      if (shift == 0) {  // every key of the bucket equals the prefix: equal weights
-        const unsigned long long wt = p_fixed62(st.prefix);
-        const unsigned long long rem = target - st.above_w;  // > 0 by construction
-        need = wt ? (int)((rem + wt - 1) / wt) : st.bucket_c;
-        need = min(need, st.bucket_c);
-      }
-      *pc = st.above_c + need;
-      return RowThreshold{st.prefix, shift, need};
+    const int need_c = (int)target - st.above_c;
+    if (!by_weight && need_c == st.bucket_c) {  // the whole class is kept (never right after a reset: 0 < need_c)
+      return RowThreshold{class_min(st), kAllTies, (int)target};
     }
+    if (n == (mixed ? 8 : 7)) break;  // full key resolved
+    st = pass(mixed ? 56 - 8 * n : max(44 - 8 * n, 0), e_top, by_weight, target, st);
+    ++n;
   }
-  return RowThreshold{0ull, 0, 0};  // not reached
+  // Every key of the class equals st.prefix: ties.
+  int need = (int)target - st.above_c;
+  if (by_weight) {
+    const unsigned long long wt = p_fixed62(st.prefix);
+    const unsigned long long rem = target - st.above_w;  // > 0 by construction
+    need = wt ? (int)((rem + wt - 1) / wt) : st.bucket_c;
+  }
+  need = max(1, min(need, st.bucket_c));
+  return RowThreshold{st.prefix, need, st.above_c + need};
 }
 
-template <typename Pass>
-__device__ __forceinline__ RowThreshold select_by_count(Pass pass, int m) {
-  RadixState st{0ull, 0ull, 0, 0};
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    st = pass(shift, false, (unsigned long long)m, st);
-    const int need = m - st.above_c;
-    if (need == st.bucket_c || shift == 0) return RowThreshold{st.prefix, shift, need};
-  }
-  return RowThreshold{0ull, 0, 0};  // not reached
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
+  return a > b ? a : b;
 }
-
 __device__ __forceinline__ unsigned long long umin64(unsigned long long a, unsigned long long b) {
   return a < b ? a : b;
 }
 
+__host__ __device__ constexpr int select_smem_bytes(int nkb) {
+  // P / keys row (8 B per block) + histograms (weights, counts, one index per
+  // bucket) + scratch
+  return ((nkb + 1) / 2 * 2) * 8 + 256 * 16 + 1024;
+}
+
+// Block-wide exclusive scan of one int per thread (256 threads).
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[wid] = x;
+  __syncthreads();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kSelectThreads / 32; ++w) {
+    const int s = scratch[w];
+    if (w < wid) base += s;
+    tot += s;
+  }
+  __syncthreads();
+  *total = tot;
+  return base + x - v;
+}
+
+// Block-wide maximum / minimum of one 64-bit value per thread (256 threads).
+template <bool MAX>
+__device__ __forceinline__ unsigned long long block_ext64(unsigned long long v, unsigned long long* scratch) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = MAX ? umax64(v, y) : umin64(v, y);
+  }
+  if (lane == 0) scratch[wid] = v;
+  __syncthreads();
+  v = scratch[0];
+#pragma unroll
+  for (int w = 1; w < kSelectThreads / 32; ++w) v = MAX ? umax64(v, scratch[w]) : umin64(v, scratch[w]);
+  __syncthreads();
+  return v;
+}
+
+// Selection with one CTA (256 threads) per row, for rows longer than the
+// warp kernel takes.
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __restrict__ Z, int64_t rows, int nkb,
                                                                  int kc, double topp, int32_t* __restrict__ kv_idx,
                                                                  int32_t* __restrict__ kv_cnt,
@@ -460,7 +510,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(smraw);
   unsigned long long* hsum = reinterpret_cast<unsigned long long*>(smraw + npad * 8);  // [256]
   unsigned int* hcnt = reinterpret_cast<unsigned int*>(hsum + 256);                   // [256]
-  RadixState* shared_st = reinterpret_cast<RadixState*>(hcnt + 256);                  // [1]
+  unsigned int* hidx = hcnt + 256;                                                     // [256]
+  RadixState* shared_st = reinterpret_cast<RadixState*>(hidx + 256);                   // [1]
   double* red = reinterpret_cast<double*>(shared_st + 1);                             // [8]
   unsigned long long* ured = reinterpret_cast<unsigned long long*>(red + 8);          // [8]
   int* scratch = reinterpret_cast<int*>(ured + 8);                                    // [8]
@@ -497,13 +548,14 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
   double rsum = 0.0;
 #pragma unroll
   for (int w = 0; w < kSelectThreads / 32; ++w) rsum = __dadd_rn(rsum, red[w]);
-  unsigned long long tot = 0ull;  // total weight (exact integer sum)
+  unsigned long long tot = 0ull, kmax = 0ull;  // total weight (exact integer sum), largest key
   for (int j = tid; j < nkb; j += kSelectThreads) {
     const double pj = __ddiv_rn(ev[j], rsum);
     if (probs) probs[row * (int64_t)nkb + j] = (float)pj;
     const unsigned long long k = (unsigned long long)__double_as_longlong(pj);
     keys[j] = k;
     tot += p_fixed62(k);
+    kmax = umax64(kmax, k);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
@@ -512,10 +564,43 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
   tot = 0ull;
 #pragma unroll
   for (int w = 0; w < kSelectThreads / 32; ++w) tot += ured[w];
+  __syncthreads();
+  kmax = block_ext64<true>(kmax, ured);
+  const int e_top = (int)((kmax >> 52) & 0x7FFull);
 
-  auto pass = [&](int shift, bool by_weight, unsigned long long target, RadixState st) {
-    return radix_pass_cta(keys, nkb, shift, by_weight, target, st, hcnt, hsum, shared_st);
+  auto pass = [&](int shift, int etop, bool by_weight, unsigned long long target, RadixState st) {
+    hcnt[tid] = 0u;
+    hsum[tid] = 0ull;
+    __syncthreads();
+    for (int j = tid; j < nkb; j += kSelectThreads) {
+      const unsigned long long k = keys[j];
+      unsigned int d;
+      if (key_bucket(k, shift, etop, st, &d)) {
+        atomicAdd(&hcnt[d], 1u);
+        if (by_weight) atomicAdd(&hsum[d], p_fixed62(k));
+        hidx[d] = (unsigned int)j;
+      }
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const RadixState s2 = radix_scan_warp(hcnt, hsum, hidx, by_weight, target, shift, st);
+      if (tid == 0) *shared_st = s2;
+    }
+    __syncthreads();
+    st = *shared_st;
+    __syncthreads();
+    return st;
   };
+  auto class_min = [&](const RadixState& st) {
+    unsigned long long v = ~0ull;
+    for (int j = tid; j < nkb; j += kSelectThreads) {
+      const unsigned long long k = keys[j];
+      if ((k & st.mask) == st.prefix) v = umin64(v, k);
+    }
+    return block_ext64<false>(v, ured);
+  };
+  auto key_at = [&](int j) { return keys[j]; };
+
   // 1. Top-p count.
   int pc = 0;
   bool have_p = false;
@@ -525,31 +610,29 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
     if (tot < target) {
       pc = nkb;  // never reached
     } else {
-      thr = select_by_weight(pass, target, &pc);
+      thr = radix_select(pass, class_min, key_at, e_top, true, target);
+      pc = thr.count;
       have_p = true;
     }
   }
   const int m = min(nkb, max(max(kc, pc), 1));
   // 2. Threshold of the m-th largest block.
-  if (!(have_p && m == pc)) thr = select_by_count(pass, m);
+  if (!(have_p && m == pc)) thr = radix_select(pass, class_min, key_at, e_top, false, (unsigned long long)m);
 
   // 3. Compaction in block order: each thread owns a contiguous chunk.
   const int per = (nkb + kSelectThreads - 1) / kSelectThreads;
   const int j0 = min(nkb, tid * per), j1 = min(nkb, j0 + per);
   int nt = 0;
-  for (int j = j0; j < j1; ++j) nt += at_threshold(keys[j], thr);
+  for (int j = j0; j < j1; ++j) nt += keys[j] == thr.key;
   int tie_tot;
   const int tie_rank = block_excl_scan(nt, scratch, &tie_tot);
   int nk = 0;
-  unsigned long long kmin = ~0ull;
   {
     int tr = tie_rank;
     for (int j = j0; j < j1; ++j) {
       const unsigned long long k = keys[j];
-      if (above_threshold(k, thr) || (at_threshold(k, thr) && tr++ < thr.ties_kept)) {
-        ++nk;
-        kmin = umin64(kmin, k);
-      }
+      nk += keep_key(k, thr, tr);
+      tr += k == thr.key;
     }
   }
   int kept_tot;
@@ -559,20 +642,14 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
     int tr = tie_rank;
     for (int j = j0; j < j1; ++j) {
       const unsigned long long k = keys[j];
-      if (above_threshold(k, thr) || (at_threshold(k, thr) && tr++ < thr.ties_kept)) out[pos++] = j;
+      if (keep_key(k, thr, tr)) out[pos++] = j;
+      tr += k == thr.key;
     }
   }
-  if (row_thresh) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kmin = umin64(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    if (lane == 0) ured[wid] = kmin;
-    __syncthreads();
-    if (tid == 0) {
-      for (int w = 1; w < kSelectThreads / 32; ++w) kmin = umin64(kmin, ured[w]);
-      row_thresh[row] = (float)__longlong_as_double((long long)kmin);
-    }
+  if (tid == 0) {
+    kv_cnt[row] = m;
+    if (row_thresh) row_thresh[row] = (float)__longlong_as_double((long long)thr.key);
   }
-  if (tid == 0) kv_cnt[row] = m;
 }
 
 // ----------------------------------------------------------------------------
@@ -585,7 +662,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
 constexpr int kSelWarpRows = 8;
 constexpr int kSelWarpMaxNkb = 2048;
 
-__host__ __device__ constexpr int select_warp_bytes(int nkb) { return (nkb + 1) / 2 * 16 + 256 * 12 + 16; }
+__host__ __device__ constexpr int select_warp_bytes(int nkb) { return (nkb + 1) / 2 * 16 + 256 * 16; }
 __host__ __device__ constexpr int select_warp_smem_bytes(int nkb) { return kSelWarpRows * select_warp_bytes(nkb); }
 
 __global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(const double* __restrict__ Z, int64_t rows,
@@ -603,6 +680,7 @@ __global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(const do
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(mine);
   unsigned long long* hsum = reinterpret_cast<unsigned long long*>(mine + (nkb + 1) / 2 * 16);  // [256]
   unsigned int* hcnt = reinterpret_cast<unsigned int*>(hsum + 256);                           // [256]
+  unsigned int* hidx = hcnt + 256;                                                             // [256]
   const double* zrow = Z + row * (int64_t)nkb;
 
   // 0. Row softmax.
@@ -623,21 +701,56 @@ __global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(const do
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
   const double rsum = part;
-  unsigned long long tot = 0ull;  // total weight (exact integer sum)
+  unsigned long long tot = 0ull, kmax = 0ull;  // total weight (exact integer sum), largest key
   for (int j = lane; j < nkb; j += 32) {
     const double pj = __ddiv_rn(ev[j], rsum);
     if (probs) probs[row * (int64_t)nkb + j] = (float)pj;
     const unsigned long long k = (unsigned long long)__double_as_longlong(pj);
     keys[j] = k;
     tot += p_fixed62(k);
+    kmax = umax64(kmax, k);
   }
   __syncwarp();
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  for (int o = 16; o > 0; o >>= 1) {
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    kmax = umax64(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  const int e_top = (int)((kmax >> 52) & 0x7FFull);
 
-  auto pass = [&](int shift, bool by_weight, unsigned long long target, RadixState st) {
-    return radix_pass_warp(keys, nkb, shift, by_weight, target, st, hcnt, hsum);
+  auto pass = [&](int shift, int etop, bool by_weight, unsigned long long target, RadixState st) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      hcnt[lane * 8 + i] = 0u;
+      hsum[lane * 8 + i] = 0ull;
+    }
+    __syncwarp();
+    for (int j = lane; j < nkb; j += 32) {
+      const unsigned long long k = keys[j];
+      unsigned int d;
+      if (key_bucket(k, shift, etop, st, &d)) {
+        atomicAdd(&hcnt[d], 1u);
+        if (by_weight) atomicAdd(&hsum[d], p_fixed62(k));
+        hidx[d] = (unsigned int)j;
+      }
+    }
+    __syncwarp();
+    st = radix_scan_warp(hcnt, hsum, hidx, by_weight, target, shift, st);
+    __syncwarp();
+    return st;
   };
+  auto class_min = [&](const RadixState& st) {
+    unsigned long long v = ~0ull;
+    for (int j = lane; j < nkb; j += 32) {
+      const unsigned long long k = keys[j];
+      if ((k & st.mask) == st.prefix) v = umin64(v, k);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = umin64(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+  };
+  auto key_at = [&](int j) { return keys[j]; };
+
   // 1. Top-p count.
   int pc = 0;
   bool have_p = false;
@@ -647,41 +760,34 @@ __global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(const do
     if (tot < target) {
       pc = nkb;
     } else {
-      thr = select_by_weight(pass, target, &pc);
+      thr = radix_select(pass, class_min, key_at, e_top, true, target);
+      pc = thr.count;
       have_p = true;
     }
   }
   const int m = min(nkb, max(max(kc, pc), 1));
   // 2. Threshold of the m-th largest block.
-  if (!(have_p && m == pc)) thr = select_by_count(pass, m);
+  if (!(have_p && m == pc)) thr = radix_select(pass, class_min, key_at, e_top, false, (unsigned long long)m);
 
   // 3. Compaction in block order, 32 blocks per round: ties at the threshold
   //    are kept lowest index first.
   int32_t* out = kv_idx + row * (int64_t)nkb;
   const unsigned int lt = (1u << lane) - 1u;
   int ties_before = 0, kept_before = 0;
-  unsigned long long kmin = ~0ull;
   for (int j0 = 0; j0 < nkb; j0 += 32) {
     const int j = j0 + lane;
     const unsigned long long k = j < nkb ? keys[j] : 0ull;
-    const bool tie = j < nkb && at_threshold(k, thr);
+    const bool tie = j < nkb && k == thr.key;
     const unsigned int tb = __ballot_sync(0xffffffffu, tie);
-    const bool keep = j < nkb && (above_threshold(k, thr) || (tie && ties_before + __popc(tb & lt) < thr.ties_kept));
+    const bool keep = j < nkb && keep_key(k, thr, ties_before + __popc(tb & lt));
     const unsigned int kb = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      out[kept_before + __popc(kb & lt)] = j;
-      kmin = umin64(kmin, k);
-    }
+    if (keep) out[kept_before + __popc(kb & lt)] = j;
     ties_before += __popc(tb);
     kept_before += __popc(kb);
   }
-  if (row_thresh) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kmin = umin64(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-  }
   if (lane == 0) {
     kv_cnt[row] = m;
-    if (row_thresh) row_thresh[row] = (float)__longlong_as_double((long long)kmin);
+    if (row_thresh) row_thresh[row] = (float)__longlong_as_double((long long)thr.key);
   }
 }
 

@@ -385,19 +385,19 @@ int oracle_attention_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* 
 //     x * s in float. S = q8 . k8 is an exact integer.
 //   * V: fp8 e4m3, one scale per (batch, head, channel) over all keys: the
 //     channel's max |v| maps to 448; v8 = e4m3(v * s_v), the product in float.
-//   * P: e4m3 relative to a running integer log2 maximum, in the order the
-//     kept key tiles (64 keys, ascending blocks) are visited:
-//       x_j   = float(S_j) * c, c = float(log2(e)/sqrt(d)) / (s_q * s_k) in float;
-//       m     = ceil(max_j x_j) of the first tile; afterwards it moves up to
-//               a tile's ceil(max_j x_j) only when that exceeds m + 8, the
-//               accumulators then scaled by 2^(m_old - m_new) (exact), so
-//               every e_j <= 2^8 stays inside e4m3's range;
-//       e_j   = 2^(x_j - m), x_j - m in float; p_j = e4m3(e_j);
-//       l += e_j (the normaliser is not quantised: only the operands of the
-//       two products are); acc += p_j v8_j;
+//   * P: e4m3 relative to the row's integer log2 maximum, in two passes over
+//     the keys of the row's kept blocks (in any order):
+//       x_j   = float(S_j) * c, c = float(log2(e)/sqrt(d)) / (s_q * s_k) in float
+//               (s_k the scale of key j's block);
+//       m     = ceil(max_j x_j) over every kept key of the row (first pass),
+//               so every e_j below is at most 1;
+//       e_j   = 2^(x_j - m), x_j - m in float; p_j = e4m3(e_j) (second pass);
+//       l     = sum_j e_j (the normaliser is not quantised: only the operands
+//               of the two products are); acc = sum_j p_j v8_j;
 //     O = acc / (l * s_v). Because m is an integer and e4m3 rounding commutes
-//     with powers of two (above its subnormal range), the result does not
-//     depend on where in the walk m settled.
+//     with powers of two above its subnormal range, any other integer
+//     reference at or above the max changes the result only through keys
+//     whose e_j falls below 2^-6.
 // e4m3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; largest finite 448,
 // subnormals down to 2^-9; rounding to nearest, ties to even; magnitudes
 // above 448 saturate to 448.
@@ -486,8 +486,7 @@ int oracle_e4m3(const double* x, int64_t n, double* out) {
 int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t BH, int64_t N,
                              int d, int bq, int bk, const int32_t* kv_idx, const int32_t* kv_cnt,
                              const int64_t* rows, int64_t nrows, double* O) {
-  if (!Q || !K || !V || !rows || !O || !kv_idx || !kv_cnt || !shape_ok(BH, N, d, bq) || bk <= 0 || bk % 64 != 0)
-    return ERR_ARG;
+  if (!Q || !K || !V || !rows || !O || !kv_idx || !kv_cnt || !shape_ok(BH, N, d, bq) || bk <= 0) return ERR_ARG;
   const int64_t Nqb = ceil_div(N, bq), Nkb = ceil_div(N, bk);
   std::vector<int8_t> q8(static_cast<size_t>(BH * N * d)), k8(static_cast<size_t>(BH * N * d));
   std::vector<float> sq(static_cast<size_t>(BH * Nqb)), sk(static_cast<size_t>(BH * Nkb)), sv(static_cast<size_t>(BH * d));
@@ -497,7 +496,8 @@ int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_
   if (rc != OK) return rc;
   const float c0 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   std::vector<double> acc(d);
-  std::vector<float> x(64);
+  std::vector<float> x;        // x_j of the row's kept keys
+  std::vector<int64_t> keys;   // their key indices
   for (int64_t t = 0; t < nrows; ++t) {
     const int64_t r = rows[t];
     if (r < 0 || r >= BH * N) return ERR_ARG;
@@ -505,40 +505,32 @@ int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_
     const int64_t cnt = kv_cnt[bh * Nqb + I];
     if (cnt < 0 || cnt > Nkb) return ERR_ARG;
     const int8_t* qi = &q8[static_cast<size_t>((bh * N + i) * d)];
-    float m = -std::numeric_limits<float>::infinity();
-    double l = 0.0;
-    std::fill(acc.begin(), acc.end(), 0.0);
+    // Pass 1: scaled integer scores of every kept key, and their maximum.
+    x.clear();
+    keys.clear();
+    float mx = -std::numeric_limits<float>::infinity();
     for (int64_t e = 0; e < cnt; ++e) {
       const int64_t J = kv_idx[(bh * Nqb + I) * Nkb + e];
       if (J < 0 || J >= Nkb) return ERR_ARG;
       const float c = c0 / (sq[bh * Nqb + I] * sk[bh * Nkb + J]);
-      for (int64_t key0 = J * bk; key0 < std::min<int64_t>(N, (J + 1) * bk); key0 += 64) {
-        const int64_t key1 = std::min<int64_t>(N, key0 + 64);
-        float mt = -std::numeric_limits<float>::infinity();
-        for (int64_t j = key0; j < key1; ++j) {
-          const int8_t* kj = &k8[static_cast<size_t>((bh * N + j) * d)];
-          int64_t S = 0;
-          for (int cc = 0; cc < d; ++cc) S += static_cast<int64_t>(qi[cc]) * kj[cc];
-          x[j - key0] = static_cast<float>(S) * c;
-          mt = std::max(mt, x[j - key0]);
-        }
-        const float cm = std::ceil(mt);
-        if (m == -std::numeric_limits<float>::infinity()) {
-          m = cm;
-        } else if (cm > m + 8.0f) {
-          const double f = std::exp2(static_cast<double>(m - cm));
-          l *= f;
-          for (int cc = 0; cc < d; ++cc) acc[cc] *= f;
-          m = cm;
-        }
-        for (int64_t j = key0; j < key1; ++j) {
-          const float y = x[j - key0] - m;
-          const double ej = std::exp2(static_cast<double>(y));
-          const double pj = e4m3_rne(ej);
-          l += ej;
-          for (int cc = 0; cc < d; ++cc) acc[cc] += pj * v8[static_cast<size_t>((bh * N + j) * d + cc)];
-        }
+      for (int64_t j = J * bk; j < std::min<int64_t>(N, (J + 1) * bk); ++j) {
+        const int8_t* kj = &k8[static_cast<size_t>((bh * N + j) * d)];
+        int64_t S = 0;
+        for (int cc = 0; cc < d; ++cc) S += static_cast<int64_t>(qi[cc]) * kj[cc];
+        x.push_back(static_cast<float>(S) * c);
+        keys.push_back(j);
+        mx = std::max(mx, x.back());
       }
+    }
+    // Pass 2: codes of 2^(x - m) against the integer reference m.
+    const float m = std::ceil(mx);
+    double l = 0.0;
+    std::fill(acc.begin(), acc.end(), 0.0);
+    for (size_t u = 0; u < x.size(); ++u) {
+      const double ej = std::exp2(static_cast<double>(x[u] - m));
+      const double pj = e4m3_rne(ej);
+      l += ej;
+      for (int cc = 0; cc < d; ++cc) acc[cc] += pj * v8[static_cast<size_t>((bh * N + keys[u]) * d + cc)];
     }
     for (int cc = 0; cc < d; ++cc)
       O[t * d + cc] = l > 0.0 ? acc[cc] / (l * static_cast<double>(sv[bh * d + cc])) : 0.0;

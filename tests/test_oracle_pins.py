@@ -439,6 +439,53 @@ def test_q8_close_to_exact_sparse_attention(oracle_mod):
     assert rel > 1e-4  # the quantisation is really applied
 
 
+def test_q8_dominant_late_block_keeps_the_codes_in_range(oracle_mod):
+    # The row's largest scores sit in the LAST kept block, about 2^12 above
+    # those of the first kept block. The integer reference must be the max
+    # over every kept key: a reference taken from the first block alone would
+    # put 2^(x - m) of the late keys far above e4m3's largest value (448),
+    # saturate them and collapse the output. Against exact sparse attention
+    # the result must stay within the 8-bit error budget.
+    N, d, bq, bk = 256, 64, 64, 64
+    g = torch.Generator().manual_seed(43)
+    q = torch.randn(1, 1, N, d, generator=g)
+    k = torch.randn(1, 1, N, d, generator=g) * 0.3
+    v = torch.randn(1, 1, N, d, generator=g)
+    # keys of block 3 point along their query block's mean direction
+    u = q[0, 0, :bq].mean(0)
+    u = u / u.norm()
+    k[0, 0, 3 * bk:] = u * 16.0 + 0.05 * torch.randn(bk, d, generator=g)
+    q[0, 0, :bq] = q[0, 0, :bq] + 8.0 * u
+    q, k, v = _bf16(q), _bf16(k), _bf16(v)
+    kv_idx = np.zeros((1, 1, 4, 4), np.int32)
+    kv_idx[0, 0, 0, :2] = [0, 3]  # first block weak, last block dominant
+    kv_cnt = np.array([[[2, 0, 0, 0]]], np.int32)
+    rows = np.arange(bq)
+    a = oracle_mod.attention_q8_rows(q, k, v, bq, bk, kv_idx, kv_cnt, rows)
+    e, lse = oracle_mod.attention_rows(q, k, v, bq, bk, kv_idx, kv_cnt, mode="sparse", rows=rows)
+    # the late block really dominates: its keys carry almost all the weight
+    s = (q[0, 0, :bq].double() @ k[0, 0].double().T / math.sqrt(d)).numpy()
+    late = np.exp(s[:, 3 * bk:] - lse[:, None]).sum(1)
+    assert late.min() > 0.999
+    assert (s[:, 3 * bk:].max(1) - s[:, :bk].max(1)).min() * math.log2(math.e) > 12
+    rel = np.abs(a - e).sum() / np.abs(e).sum()
+    assert rel < 0.06, rel
+
+
+def test_q8_output_does_not_depend_on_the_kept_list_order(oracle_mod):
+    # The definition has no walk order: a reversed kept list gives the same
+    # output up to the order of the double sums.
+    q, k, v = _rand_qkv(1, 1, 512, 32, 44, scale=2.0)
+    kv_idx, kv_cnt = (np.asarray(x) for x in synth.random_mask(1, 1, 8, 8, 5, seed=14))
+    rev = kv_idx.copy()
+    for I in range(8):
+        c = kv_cnt[0, 0, I]
+        rev[0, 0, I, :c] = kv_idx[0, 0, I, :c][::-1]
+    a = oracle_mod.attention_q8_rows(q, k, v, 64, 64, kv_idx, kv_cnt)
+    b = oracle_mod.attention_q8_rows(q, k, v, 64, 64, rev, kv_cnt)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
 # ----------------------------------------------------------------------------- learnt router
 def _router_inputs(seed, H=2, N=2048, d=64, s=1.5):
     Q, K, V = synth.make_qkv(1, H, N, d, grid=(2, 32, 32), s=s, seed=seed)
