@@ -50,6 +50,9 @@ def parse():
                     help="score the mask through a learnt router of this width (seeded stand-in projections)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--report", choices=["regimes"], default=None,
+                    help="regimes: kept fraction and error against dense attention of Top-k alone, Top-p alone "
+                         "and the hybrid on the flat and peaked sweep workloads (one GPU; prints a table)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other headline shapes (720p sparse and SLA2, sla2_480p) timed after the 480p line")
     return ap.parse_args()
@@ -496,6 +499,86 @@ def time_other_workloads(args, dev, stream, flush):
     return out
 
 
+# ----------------------------------------------------------------------------- mask regimes
+def regime_settings():
+    """(rule, top-k, top-p) of the mask-regime sweep: Top-k alone, Top-p alone
+    and the hybrid over the sweep grid."""
+    out = [("top-k", k, 0.0) for k in synth.SWEEP_TOPK]
+    out += [("top-p", 0.0, p) for p in synth.SWEEP_TOPP]
+    out += [("hybrid", k, p) for k in synth.SWEEP_TOPK for p in synth.SWEEP_TOPP]
+    return out
+
+
+def regime_rows(w, Q, K, V, settings, dev, check_rows=64):
+    """For each (rule, k, p): the kept fraction of the mask sparge_mask builds
+    and the error of sparge_attn_fwd on it against dense attention (the same
+    kernel with every block kept). The dense reference is first checked
+    against the oracle's dense attention on sampled rows. Returns (rows,
+    dense_check)."""
+    import oracle
+    from block_sparse_attention_pooled_b200 import sparge
+
+    B, H, N, d = Q.shape
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    shape = sparge.make_shape(Qd, w.bq, w.bk)
+    ws_mask = torch.empty(sparge.workspace_bytes(sparge.OP_MASK, shape), dtype=torch.uint8, device=dev)
+    ws_attn = torch.empty(sparge.workspace_bytes(sparge.OP_ATTN, shape), dtype=torch.uint8, device=dev)
+    all_idx = torch.arange(w.nkb, dtype=torch.int32, device=dev).expand(B, H, w.nqb, w.nkb).contiguous()
+    all_cnt = torch.full((B, H, w.nqb), w.nkb, dtype=torch.int32, device=dev)
+    Od = sparge.sparge_attn_fwd(Qd, Kd, Vd, all_idx, all_cnt, w.bq, w.bk, workspace=ws_attn)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(w.seed)
+    rows = np.sort(rng.choice(B * H * N, size=check_rows, replace=False)).astype(np.int64)
+    ref, _ = oracle.attention_rows(Q, K, V, w.bq, w.bk, mode="dense", rows=rows)
+    got = Od.float().cpu().numpy().reshape(-1, d)[rows].astype(np.float64)
+    err = np.abs(got - ref)
+    dense_check = {"rows": int(len(rows)), "max_abs": float(err.max()),
+                   "mean_rel_l1": float(err.sum() / np.abs(ref).sum())}
+    Odf = Od.double()
+    den_l1, den_l2 = float(Odf.abs().sum()), float(Odf.norm())
+    dense_flops = 4.0 * B * H * N * N * d
+    out = []
+    for rule, k, p in settings:
+        kv_idx, kv_cnt = sparge.sparge_mask(Qd, Kd, w.bq, w.bk, k, p, workspace=ws_mask)
+        O = sparge.sparge_attn_fwd(Qd, Kd, Vd, kv_idx, kv_cnt, w.bq, w.bk, workspace=ws_attn)
+        diff = O.double() - Odf
+        out.append({"rule": rule, "topk": k, "topp": p,
+                    "kept_fraction": kept_flops(kv_idx, kv_cnt, N, d, w.bq, w.bk) / dense_flops,
+                    "mean_kept_blocks": float(kv_cnt.double().mean()),
+                    "rel_l1_vs_dense": float(diff.abs().sum()) / den_l1,
+                    "rel_l2_vs_dense": float(diff.norm()) / den_l2,
+                    "max_abs_vs_dense": float(diff.abs().max()),
+                    "cos_sim_vs_dense": float((O.double() * Odf).sum()) / (float(O.double().norm()) * den_l2)})
+    assert sparge.device_status() == 0, "a kernel gave up a bounded wait"
+    return out, dense_check
+
+
+def run_regime_report(args):
+    """The mask-regime report: for the flat and the peaked sweep workloads,
+    the kept fraction and the error against dense attention of Top-k alone,
+    Top-p alone and their union. Prints a markdown table and one JSON line."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    report = {"report": "mask regimes", "workloads": {}}
+    lines = ["| distribution | rule | top-k | top-p | kept fraction | mean kept blocks | rel. L1 error | "
+             "rel. L2 error | max abs error | cosine similarity |", "|---|---|---|---|---|---|---|---|---|---|"]
+    for name in ("sweep_flat", "sweep_peaked"):
+        w = synth.WORKLOADS[name]
+        Q, K, V, _ = synth.make_workload(w)
+        rows, check = regime_rows(w, Q, K, V, regime_settings(), dev)
+        report["workloads"][name] = {"dense_check_vs_oracle": check, "rows": rows,
+                                     "config": {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk,
+                                                "s": w.s}}
+        for r in rows:
+            lines.append(f"| {name.split('_')[1]} (s = {w.s}) | {r['rule']} | {r['topk']:.2f} | {r['topp']:.2f} | "
+                         f"{r['kept_fraction']:.4f} | {r['mean_kept_blocks']:.1f} | {r['rel_l1_vs_dense']:.4f} | "
+                         f"{r['rel_l2_vs_dense']:.4f} | {r['max_abs_vs_dense']:.3f} | {r['cos_sim_vs_dense']:.4f} |")
+        del Q, K, V
+        torch.cuda.empty_cache()
+    print("\n".join(lines), flush=True)
+    print(json.dumps(report), flush=True)
+
+
 # ----------------------------------------------------------------------------- runs
 def run_reference(args, w, rank, world):
     if rank != 0:
@@ -748,6 +831,9 @@ def main():
         if backend == "nccl":
             torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if args.report == "regimes":
+        run_regime_report(args)
+        return
     try:
         if args.impl == "reference":
             run_reference(args, w, rank, world)

@@ -9,15 +9,17 @@
 //   S_j = q8_i . k8_j                     exact int32, tcgen05 kind::i8
 //   x_j = float(S_j) * c_IJ,              c_IJ = c0 / (s_q[I] * s_k[J]) in fp32,
 //                                         c0 = log2(e) / sqrt(d)
-//   m   = ceil(max_j x_j) of the first     an integer; later it moves up to a
-//         tile                            tile's ceil(max_j x_j) only when that
-//                                         exceeds m + 8 (so e_j <= 2^8 < 448),
-//                                         O and l then scaled by 2^(m_old - m_new)
-//   e_j = 2^(x_j - m),  l += e_j,  p_j = e4m3(e_j)
+//   m   = an integer reference: ceil(max_j x_j) of the first tile, moved up
+//         to a tile's ceil(max_j x_j) only when that exceeds m + 2 (O and l
+//         then scaled by the exact 2^(m_old - m_new)), so max_j x_j <= m + 2
+//   e_j = 2^(x_j - (m - 6)),  l += e_j,  p_j = e4m3(e_j)   (e_j <= 2^8 < 448)
 //   O  += p_j v8_j                        fp32 in TMEM, tcgen05 kind::f8f6f4
-// and O_i = O / (l * s_v) per channel. Because m only takes integer values
-// and e4m3 rounding commutes with powers of two (above its subnormals), the
-// codes do not depend on where in the walk m settled.
+// and O_i = O / (l * s_v) per channel. P is thereby scaled into e4m3's range:
+// the row's largest code lies in (2^5, 2^8]. The library's definition puts
+// it in (2^7, 2^8] (reference ceil of the max over every kept key, minus 8);
+// since the references are integers and e4m3 rounding commutes with powers
+// of two above its subnormals, the two differ only in the codes of keys more
+// than 12 binades below the row's max.
 //
 // Same warp roles and pipeline as the bf16 kernel (attn.cuh): warp 0 TMA
 // producer, warp 1 MMA issuer (whole warp, one elected lane issues), warps
@@ -314,9 +316,10 @@ __global__ void __launch_bounds__(kQ8Threads, 2)
       // A tile wholly past N (the second tile of a ragged 128-key block) has
       // no valid key: it leaves m as it is and contributes nothing.
       const float cm = nvalid > 0 ? ceilf(__fmul_rn(i2f_small(smax), c)) : m_run;
-      // Each row moves its reference only past a margin of 2^8 (its own
-      // decision, so the result does not depend on the other rows of the warp).
-      const float m_new = (t == 0 || cm > m_run + 8.0f) ? cm : m_run;
+      // Each row moves its reference only past a margin of 2 binades (its
+      // own decision, so the result does not depend on the other rows of the
+      // warp).
+      const float m_new = (t == 0 || cm > m_run + 2.0f) ? cm : m_run;
       if (t == 0) {
         m_run = m_new;
       } else if (__any_sync(0xffffffffu, m_new > m_run)) {
@@ -331,8 +334,9 @@ __global__ void __launch_bounds__(kQ8Threads, 2)
         l_run *= f;
         m_run = m_new;
       }
-      // e = 2^(x - m), x = float(S) * c; codes e4m3(e); l += e.
-      const uint64_t c2 = f2(c, c), negm2 = f2(-m_run, -m_run), magic2 = f2(12582912.0f, 12582912.0f);
+      // e = 2^(x - (m - 6)), x = float(S) * c; codes e4m3(e); l += e.
+      const float negref = 6.0f - m_run;
+      const uint64_t c2 = f2(c, c), negm2 = f2(negref, negref), magic2 = f2(12582912.0f, 12582912.0f);
       uint64_t acc[2] = {0ull, 0ull};
       uint32_t pw[kTileK / 4];
 #pragma unroll

@@ -78,11 +78,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 
 // Waits until the phase with the given parity has completed. Returns false
 // (after recording `site`) if that takes longer than kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int site) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       record_error(site);
       return false;
     }
@@ -253,12 +254,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Waits on an mbarrier unless another role already gave up; gives up itself
 // (and tells the others through *abort) after the global time limit.
 __device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, unsigned int site,
-                                          volatile int* abort) {
+                                          volatile int* abort, unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       record_error(site);
       *abort = 1;
       return false;

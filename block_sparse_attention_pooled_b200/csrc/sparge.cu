@@ -19,6 +19,7 @@
 #include "quant.cuh"
 #include "attn_q8.cuh"
 #include "attn_bwd.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -890,6 +891,14 @@ sparge_status sla2_attn_bwd(const void* Q, const void* K, const void* V, const s
     return SPARGE_ERR_WORKSPACE;
   return launch_sla2_bwd(Q, K, V, shape, dm, kv_idx, kv_cnt, alpha, dO, dQ, dK, dV, dalpha,
                          static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+sparge_status sparge_selftest_wait(int32_t limit_us, int32_t* gave_up, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return SPARGE_ERR_INVALID_ARG;
+  if (gave_up != nullptr && (reinterpret_cast<uintptr_t>(gave_up) & 3u)) return SPARGE_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 128, 0, static_cast<cudaStream_t>(stream)>>>((unsigned long long)limit_us * 1000ull,
+                                                                         gave_up);
+  return cuda_status(cudaGetLastError());
 }
 
 sparge_status sparge_device_status(void* stream, int32_t* code) {

@@ -32,7 +32,7 @@ SLA2_BWD_LAUNCHES = 12
 # Every symbol the header declares.
 EXPORTS = ("sparge_workspace_bytes", "sparge_mask", "sparge_attn_fwd", "sla2_attn_fwd",
            "sparge_device_status", "sparge_status_string", "sparge_mask_noalloc", "sparge_attn_fwd_q8",
-           "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd")
+           "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd", "sparge_selftest_wait")
 
 
 def order_launches(shape) -> int:
@@ -61,9 +61,11 @@ _lib.sparge_attn_bwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp,
 _lib.sla2_attn_bwd.argtypes = [_vp, _vp, _vp, ctypes.POINTER(Shape), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                _vp]
 _lib.sparge_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
+_lib.sparge_selftest_wait.argtypes = [ctypes.c_int32, _vp, _vp]
 _lib.sparge_status_string.argtypes = [ctypes.c_int]
 _lib.sparge_status_string.restype = ctypes.c_char_p
-for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8"):
+for _f in ("sparge_mask", "sparge_mask_router", "sparge_attn_bwd", "sla2_attn_bwd", "sparge_attn_fwd", "sla2_attn_fwd", "sparge_device_status", "sparge_attn_fwd_q8",
+           "sparge_selftest_wait"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -271,6 +273,15 @@ def sla2_attn_fwd(Q, K, V, kv_idx, kv_cnt, alpha, bq: int, bk: int, O=None, work
     _check(_lib.sla2_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(kv_idx), _ptr(kv_cnt),
                               _ptr(alpha), _ptr(O), _ptr(workspace), nws, _stream(stream)), "sla2_attn_fwd")
     return O
+
+
+SITE_SELFTEST = 0xF00
+
+
+def selftest_wait(limit_us: int, gave_up=None, stream=None) -> None:
+    """Launches the bounded-wait self-test kernel (it waits on a barrier that
+    nothing arrives on and gives up after limit_us microseconds)."""
+    _check(_lib.sparge_selftest_wait(int(limit_us), _ptr(gave_up), _stream(stream)), "sparge_selftest_wait")
 
 
 def device_status(stream=None) -> int:

@@ -242,8 +242,13 @@ sparge_status sla2_attn_bwd(const void* Q, const void* K, const void* V, const s
  *   V     fp8 e4m3 codes, one scale per (batch, head, channel): s = 448 / max|v|.
  *   S     exact int32 products of the codes; x = float(S) * c with
  *         c = (log2(e)/sqrt(d)) / (s_q * s_k) in fp32.
- *   P     e4m3 codes of e = 2^(x - m), m a running integer maximum of x over
- *         the kept key tiles (64 keys, ascending); the normaliser sums e.
+ *   P     e4m3 codes of e = 2^(x - (m - 8)), m = ceil of the row's max of x
+ *         over its kept keys, so the row's largest code lies in (2^7, 2^8];
+ *         the normaliser sums e. The kernel tracks the reference while it
+ *         walks the key tiles (codes 2^(x - (m_run - 6)), m_run moved by an
+ *         exact power-of-two rescale when the max passes it by more than 2),
+ *         which changes only the codes of keys more than 12 binades below
+ *         the row's max.
  *   O     = sum(P * v_codes) / (sum(e) * s_v), stored as bf16.
  * Workspace: sparge_workspace_bytes(SPARGE_OP_ATTN_Q8, shape) (codes and
  * scales, the tiles' launch order). Three or four launches: Q/K codes with V channel maxima,
@@ -274,6 +279,18 @@ sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const s
  * site code of the first one. Returns SPARGE_ERR_DEVICE_TIMEOUT in that
  * case, SPARGE_ERR_CUDA if the synchronisation or the read fails. */
 sparge_status sparge_device_status(void* stream, int32_t* code);
+
+/* Self-test of the bounded device waits (the articles have no counterpart:
+ * this checks the library's failure handling). Launches one small kernel that
+ * allocates tensor memory, waits on a barrier that nothing arrives on through
+ * the same bounded wait every kernel of the library uses, gives up after
+ * limit_us microseconds (1 .. 1e6), frees its tensor memory and returns.
+ * Afterwards sparge_device_status returns SPARGE_ERR_DEVICE_TIMEOUT with the
+ * code SPARGE_SITE_SELFTEST, and the context stays usable.
+ *   gave_up     optional device int32: 1 if every thread of the kernel gave
+ *               up its wait, else 0 (NULL to skip). */
+#define SPARGE_SITE_SELFTEST 0xF00
+sparge_status sparge_selftest_wait(int32_t limit_us, int32_t* gave_up, void* stream);
 
 /* Static, human-readable name of a status. */
 const char* sparge_status_string(sparge_status status);

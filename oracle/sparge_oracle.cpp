@@ -385,19 +385,19 @@ int oracle_attention_rows(const uint16_t* Q, const uint16_t* K, const uint16_t* 
 //     x * s in float. S = q8 . k8 is an exact integer.
 //   * V: fp8 e4m3, one scale per (batch, head, channel) over all keys: the
 //     channel's max |v| maps to 448; v8 = e4m3(v * s_v), the product in float.
-//   * P: e4m3 relative to the row's integer log2 maximum, in two passes over
-//     the keys of the row's kept blocks (in any order):
+//   * P: e4m3, scaled into the format's range by a power of two: the row's
+//     largest value lands in (2^7, 2^8], the top binade below e4m3's largest
+//     finite value 448. In two passes over the keys of the row's kept blocks
+//     (in any order):
 //       x_j   = float(S_j) * c, c = float(log2(e)/sqrt(d)) / (s_q * s_k) in float
 //               (s_k the scale of key j's block);
-//       m     = ceil(max_j x_j) over every kept key of the row (first pass),
-//               so every e_j below is at most 1;
-//       e_j   = 2^(x_j - m), x_j - m in float; p_j = e4m3(e_j) (second pass);
+//       m     = ceil(max_j x_j) over every kept key of the row (first pass);
+//       e_j   = 2^(x_j - (m - 8)), x_j - (m - 8) in float, so e_j <= 2^8;
+//       p_j   = e4m3(e_j) (second pass);
 //       l     = sum_j e_j (the normaliser is not quantised: only the operands
 //               of the two products are); acc = sum_j p_j v8_j;
-//     O = acc / (l * s_v). Because m is an integer and e4m3 rounding commutes
-//     with powers of two above its subnormal range, any other integer
-//     reference at or above the max changes the result only through keys
-//     whose e_j falls below 2^-6.
+//     O = acc / (l * s_v). Keys more than 14 binades below the row's max fall
+//     into e4m3's subnormal range (below 2^-6).
 // e4m3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; largest finite 448,
 // subnormals down to 2^-9; rounding to nearest, ties to even; magnitudes
 // above 448 saturate to 448.
@@ -522,12 +522,12 @@ int oracle_attention_q8_rows(const uint16_t* Q, const uint16_t* K, const uint16_
         mx = std::max(mx, x.back());
       }
     }
-    // Pass 2: codes of 2^(x - m) against the integer reference m.
-    const float m = std::ceil(mx);
+    // Pass 2: codes of 2^(x - (m - 8)) for the integer reference m.
+    const float ref = std::ceil(mx) - 8.0f;
     double l = 0.0;
     std::fill(acc.begin(), acc.end(), 0.0);
     for (size_t u = 0; u < x.size(); ++u) {
-      const double ej = std::exp2(static_cast<double>(x[u] - m));
+      const double ej = std::exp2(static_cast<double>(x[u] - ref));
       const double pj = e4m3_rne(ej);
       l += ej;
       for (int cc = 0; cc < d; ++cc) acc[cc] += pj * v8[static_cast<size_t>((bh * N + keys[u]) * d + cc)];

@@ -51,7 +51,8 @@ def test_workspace_bytes_host_arithmetic(lib):
     s = lib.Shape(1, 40, 75600, 128, 128, 64)
     nqb, nkb = 591, 1182
     need = lib.workspace_bytes(lib.OP_MASK, s)
-    assert need >= 40 * (nqb + nkb) * 128 * 4 + 40 * nqb * nkb * 4
+    # pooled Q and K and the score rows, all in double
+    assert need >= 40 * (nqb + nkb) * 128 * 8 + 40 * nqb * nkb * 8
     assert lib.workspace_bytes(lib.OP_ATTN, s) >= 40 * nqb * 4  # the tiles' launch order
     bad = lib.Shape(1, 1, 100, 96, 64, 64)  # unsupported head dim
     assert lib.workspace_bytes(lib.OP_MASK, bad) == 0
@@ -61,8 +62,15 @@ def test_workspace_bytes_host_arithmetic(lib):
     assert lib.workspace_bytes(lib.OP_ATTN_Q8, lib.Shape(1, 1, 4096, 64, 64, 64)) == 0  # d = 128 only
     # Learnt router: the mask's scratch plus the projected blocks at the widest router width.
     need_r = lib.workspace_bytes(lib.OP_MASK_ROUTER, s)
-    assert need_r >= need + 40 * (nqb + nkb) * 128 * 4
+    assert need_r >= need + 40 * (nqb + nkb) * 128 * 8
     assert lib.workspace_bytes(lib.OP_MASK_ROUTER, bad) == 0
+
+
+def test_selftest_wait_rejects_limits_before_any_launch(lib):
+    raw = lib.raw()
+    for bad in (0, -5, 1000001):
+        assert raw.sparge_selftest_wait(bad, None, None) == lib.ERR_INVALID_ARG
+    assert raw.sparge_selftest_wait(100, ctypes.c_void_p(2), None) == lib.ERR_INVALID_ARG  # misaligned flag
 
 
 def test_invalid_arguments_rejected_before_any_launch(lib):
