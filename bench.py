@@ -48,8 +48,13 @@ def parse():
                          "workloads, whose backward recomputes its forward pieces)")
     ap.add_argument("--router", type=int, default=0, choices=[0, 64, 128],
                     help="score the mask through a learnt router of this width (seeded stand-in projections)")
+    ap.add_argument("--sparse-only", action="store_true",
+                    help="on an SLA2 workload, run the sparse branch alone (sparge_attn_fwd)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first H heads of batch 0 of the workload (a smaller case of the same "
+                         "shape, for profiler captures); 0 = all")
     ap.add_argument("--report", choices=["regimes"], default=None,
                     help="regimes: kept fraction and error against dense attention of Top-k alone, Top-p alone "
                          "and the hybrid on the flat and peaked sweep workloads (one GPU; prints a table)")
@@ -482,6 +487,7 @@ def time_other_workloads(args, dev, stream, flush):
         achieved = flops / (span * 1e-3) / 1e12
         peak, fracs, desc = roofline_peak(achieved, clocks)
         kernel = f"attn_fwd_kernel<{d}, {1 if call == 'sla2_attn_fwd' else 0}>"
+        capture_key = name + ("_sparse" if call == "sparge_attn_fwd" and w.sla2 else "")
         out[f"{name}:{call}"] = {
             "config": {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "bq": w.bq, "bk": w.bk, "topk": w.topk,
                        "topp": w.topp, "alpha": "U[0.6,1] per head" if call == "sla2_attn_fwd" else 1.0},
@@ -490,7 +496,8 @@ def time_other_workloads(args, dev, stream, flush):
             "mask_ms": ms - span, "attn_ms": span,
             "roofline": {"kernel": kernel, "timed_span": call, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "peak_kind": desc, **fracs,
-                         "ncu_tensor_pipe_active_pct": tensor_pipe_pct(name, kernel)},
+                         "ncu_tensor_pipe_active_pct": tensor_pipe_pct(capture_key, kernel),
+                         "traffic": dram_traffic(capture_key, kernel)},
             "clocks": clocks,
         }
         del ws_mask, ws, kv_idx, kv_cnt, O
@@ -769,8 +776,13 @@ def run_ours(args, w, rank, world, local_rank):
             "sparge_attn_fwd_q8 (codes, V codes, tile order when used, attention)" if q8 else
             "sla2_attn_fwd (4-5 launches)" if sla2 else "sparge_attn_fwd (tile order when used, attention)")
     # Counters were captured with the plain mask; a router mask keeps other tiles.
-    traffic = None if (args.router or bwd) else dram_traffic(w.name + ("_q8" if q8 else ""), kernel_name)
-    tensor_pct = None if (args.router or bwd) else tensor_pipe_pct(w.name + ("_q8" if q8 else ""), kernel_name)
+    # Captures are stored per workload and path: "<name>", "<name>_q8", and
+    # "<name>_sparse" for the sparse branch alone on a sparse + linear workload.
+    named = synth.WORKLOADS.get(w.name)
+    key = w.name + ("_q8" if q8 else "_sparse" if named is not None and named.sla2 and not sla2 else "")
+    partial = args.router or bwd or getattr(args, "heads", 0)  # captures were taken on the full plain path
+    traffic = None if partial else dram_traffic(key, kernel_name)
+    tensor_pct = None if partial else tensor_pipe_pct(key, kernel_name)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v, desc, cores = cpu_sample(w, Qh, Kh, Vh, alpha_h, variant=args.variant, router=router_h,
@@ -821,6 +833,12 @@ def run_ours(args, w, rank, world, local_rank):
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        # The first heads of batch 0: the generator seeds every (batch, head)
+        # on its own, so these are the same tensors as in the full workload.
+        w = synth.Workload(**{**w.__dict__, "B": 1, "H": min(args.heads, w.H)})
+    if args.sparse_only:
+        w = synth.Workload(**{**w.__dict__, "sla2": False})
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
