@@ -20,21 +20,23 @@
 // 192 threads:
 //   warp 0      TMA producer (whole warp, one elected lane issues): phi(K)
 //               and V tiles of the kept blocks into a three-slot ring, then
-//               the Q tile once the ring is idle;
+//               the Q tile into the slot the next tile would take, as soon
+//               as that slot is free;
 //   warp 1      MMA issuer (whole warp, one elected lane issues) and TMEM
 //               owner: D[feature, 0..127] += phi(K_t)^T V_t (M 128, N 128,
-//               K 64 per tile, both operands MN-major) on top of D = -S_all,
-//               which leaves D = -S_c; then phi(Q) S_c into the same columns;
-//   warps 2..5  first D = -S_all (thread r writes feature row r), then, while
-//               the MMAs run, z_kept (thread r adds z_tile[t][r] over the kept
-//               tiles); then the epilogue: TMEM lane r is feature r for S_c
+//               K 64 per tile, both operands MN-major), starting from zero,
+//               which leaves D = S_kept; then phi(Q) S_c into the same columns;
+//   warps 2..5  while the MMAs run, z_kept (thread r adds z_tile[t][r] over
+//               the kept tiles) and the loads of row r of S_all; then the
+//               epilogue: TMEM lane r is feature r for S_c = S_all - S_kept
 //               (bf16, staged in shared memory as the MN-major B operand) and
 //               query row r for the output, whose denominator phi(q_r) . z_c
 //               they take in fp32.
-// Shared memory: ring slot s = [phi(K) 16 KB | V 16 KB]; after the last MMA
-// of the ring the same bytes hold S_c (two 128-row boxes, 32 KB) and the Q
-// tile (32 KB), which becomes phi(Q) and then the output. Three slots keep two
-// CTAs per SM, six tiles in flight per SM.
+// Shared memory: ring slot s = [phi(K) 16 KB | V 16 KB]. With T kept tiles the
+// Q tile (32 KB) goes to slot T % 3 (free once tile T - 3's product is done)
+// and becomes phi(Q) and then the output; S_c (two 128-row boxes, 32 KB) goes
+// to slot (T + 1) % 3 after the last product. Three slots keep two CTAs per
+// SM, six tiles in flight per SM.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -48,7 +50,7 @@ namespace sparge {
 constexpr int kLoThreads = 192;
 
 enum : unsigned int {
-  kErrLoFull = 0x300, kErrLoEmpty, kErrLoKept, kErrLoQ, kErrLoStage, kErrLoOut, kErrLoDrain, kErrLoInit
+  kErrLoFull = 0x300, kErrLoEmpty, kErrLoKept, kErrLoQ, kErrLoStage, kErrLoOut, kErrLoDrain
 };
 
 #ifndef SPARGE_LO_SLOTS
@@ -59,16 +61,15 @@ struct LoSmem {
   static constexpr int NS = SPARGE_LO_SLOTS;
   static constexpr int kTile = 64 * 128 * 2;         // phi(K) or V tile: two 64-column boxes of 64 keys
   static constexpr int kSlot = 2 * kTile;            // 32 KB
-  static constexpr int kOffStage = 0;                // epilogue: S_c, two boxes of 128 rows
-  static constexpr int kOffQ = 2 * 128 * 128;        // epilogue: Q tile -> phi(Q) -> output
   static constexpr int kOffX = NS * kSlot;           // zc[128] (fp32)
   static constexpr int kOffBar = kOffX + 128 * 4;
   static constexpr int kBarFull = 0, kBarEmpty = NS, kBarKept = 2 * NS, kBarQ = 2 * NS + 1,
-                       kBarStage = 2 * NS + 2, kBarOut = 2 * NS + 3, kBarDrain = 2 * NS + 4, kBarInit = 2 * NS + 5;
-  static constexpr int kNumBars = 2 * NS + 6;
+                       kBarStage = 2 * NS + 2, kBarOut = 2 * NS + 3, kBarDrain = 2 * NS + 4;
+  static constexpr int kNumBars = 2 * NS + 5;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;  // + alignment slack: two CTAs per SM
-  static_assert(kOffQ + 2 * 128 * 128 <= kOffX, "epilogue tiles must fit in the ring");
+  static_assert(kSlot == 2 * 128 * 128, "the Q tile and S_c each fill one ring slot");
+  static_assert(NS >= 2, "Q and S_c take two different slots");
 };
 
 struct LoParams {
@@ -102,7 +103,12 @@ __global__ void __launch_bounds__(kLoThreads, 2)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw);
-  const uint32_t sStage = sbase + L::kOffStage, sQ = sbase + L::kOffQ;
+  const int tile_ = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;
+  const int cnt_ = min(max(__ldg(p.kv_cnt + tile_), 0), p.nkb);
+  const int T_ = cnt_ * (p.bk / 64);
+  // Q in the slot the next tile would take, S_c in the one after.
+  const uint32_t sQ = sbase + (T_ % NS) * L::kSlot, sStage = sbase + ((T_ + 1) % NS) * L::kSlot;
+  const int q_off = (T_ % NS) * L::kSlot;
   float* zc = reinterpret_cast<float*>(sgen + L::kOffX);  // [128] z_c
   const uint32_t bar0 = sbase + L::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -110,13 +116,13 @@ __global__ void __launch_bounds__(kLoThreads, 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int tile = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;  // (bh, query block)
+  const int tile = tile_;  // (bh, query block)
   const int bh = tile / p.nqb;
   const int qb = tile % p.nqb;
   const int q0 = qb * p.bq;
   const int tiles_per_block = p.bk / 64;
-  const int cnt = min(max(__ldg(p.kv_cnt + tile), 0), p.nkb);
-  const int T = cnt * tiles_per_block;
+  const int cnt = cnt_;
+  const int T = T_;
   const int32_t* lst = p.kv_idx + (int64_t)tile * p.nkb;
 
   if (threadIdx.x == 0) {
@@ -129,7 +135,6 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     mbar_init(bar(L::kBarStage), 128);
     mbar_init(bar(L::kBarOut), 1);
     mbar_init(bar(L::kBarDrain), 1);
-    mbar_init(bar(L::kBarInit), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -181,9 +186,10 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       __syncwarp();
       ++issued;
     }
-    // Q goes where the ring was, once every MMA that reads the ring is done.
+    // Q goes to slot T % NS, as a tile T would: once tile T - NS's product
+    // (if any) has read that slot.
     bool q_issued = false;
-    if (ok && warp_wait(L::kBarKept, 0, kErrLoKept)) {
+    if (ok && (T < NS || warp_wait(L::kBarEmpty + T % NS, (T / NS - 1) & 1, kErrLoEmpty))) {
       if (leader) {
         mbar_arrive_expect_tx(bar(L::kBarQ), 2 * 128 * 128);
         for (int b = 0; b < 2; ++b) tma_load_3d(sQ + b * (128 * 128), &tmQ, bar(L::kBarQ), b * 64, q0, bh);
@@ -204,7 +210,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     const uint64_t dRing = sdesc_sw128(sbase, 64 * 128, 1024);     // MN-major, 64-row boxes
     const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);                 // K-major, 128-row boxes
     const uint64_t dStage = sdesc_sw128(sStage, 128 * 128, 1024);  // MN-major, 128-row boxes
-    bool ok = warp_wait(L::kBarInit, 0, kErrLoInit);  // D = -S_all
+    bool ok = true;
     for (int t = 0; ok && t < T; ++t) {
       const int slot = t % NS;
       if (!warp_wait(L::kBarFull + slot, (t / NS) & 1, kErrLoFull)) {
@@ -217,7 +223,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
         const uint64_t dV = dP + (uint64_t)(L::kTile >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // 16 keys = 2048 bytes of each operand
-          mma_ss(tmem, dP + kk * 128, dV + kk * 128, idKept, 1u);
+          mma_ss(tmem, dP + kk * 128, dV + kk * 128, idKept, (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(L::kBarEmpty + slot));
       }
       __syncwarp();
@@ -244,29 +250,6 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     const int q = warp & 3;            // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;       // feature (S_c, z_c) / query row (output)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    // D = -S_all, row r (feature r): all 32 loads in flight at once, so
-    // the MMAs wait for one round trip only.
-    {
-      const float4* srow = reinterpret_cast<const float4*>(p.s_all + ((int64_t)bh * 128 + r) * 128);
-      float4 v4[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) v4[k] = __ldg(srow + k);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        uint32_t v[16];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[4 * j] = __float_as_uint(-v4[4 * k + j].x);
-          v[4 * j + 1] = __float_as_uint(-v4[4 * k + j].y);
-          v[4 * j + 2] = __float_as_uint(-v4[4 * k + j].z);
-          v[4 * j + 3] = __float_as_uint(-v4[4 * k + j].w);
-        }
-        tmem_st16(tmem + lane_off + 16 * k, v);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarInit));
-    }
     // z_kept[r] over the kept tiles, four loads in flight at a time. A last
     // 128-key block may hold a single 64-key tile: its second tile lies past
     // N, has no z_tile entry and adds nothing.
@@ -286,23 +269,38 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       }
       for (; t < T; ++t) zk += ztile(t);
     }
+    // Row r (feature r) of S_all: all 32 loads in flight at once, issued
+    // while the products still run.
+    float4 sa[32];
+    {
+      const float4* srow = reinterpret_cast<const float4*>(p.s_all + ((int64_t)bh * 128 + r) * 128);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) sa[k] = __ldg(srow + k);
+    }
     bool ok = warp_wait(L::kBarKept, 0, kErrLoKept);
     tc_fence_after();
-    // 1. S_c row a = r (= -D) as bf16, MN-major for the last MMA (two
-    //    64-column boxes of 128 rows, 128-byte swizzle).
-#pragma unroll 1
+    // 1. S_c row a = r (S_all - D; D = 0 when nothing is kept) as bf16,
+    //    MN-major for the last MMA (two 64-column boxes of 128 rows,
+    //    128-byte swizzle).
+#pragma unroll
     for (int c = 0; c < 128; c += 16) {
       uint32_t v[16];
-      if (ok) {
+      if (ok && T > 0) {
         tmem_ld16(tmem + lane_off + c, v);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(v);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0u;
       }
       float sc[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) sc[j] = -__uint_as_float(v[j]);
+      for (int j = 0; j < 4; ++j) {
+        const float4 a = sa[c / 4 + j];
+        sc[4 * j] = a.x - __uint_as_float(v[4 * j]);
+        sc[4 * j + 1] = a.y - __uint_as_float(v[4 * j + 1]);
+        sc[4 * j + 2] = a.z - __uint_as_float(v[4 * j + 2]);
+        sc[4 * j + 3] = a.w - __uint_as_float(v[4 * j + 3]);
+      }
       stage_row16(sStage, r, c, sc);
     }
     // 2. z_c, then phi(Q) in place. phi is elementwise, so the tile is
@@ -311,7 +309,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     zc[r] = __ldg(p.z_all + (int64_t)bh * 128 + r) - zk;
     if (ok) ok = warp_wait(L::kBarQ, 0, kErrLoQ);
     if (ok) {
-      uint4* qt = reinterpret_cast<uint4*>(sgen + L::kOffQ);
+      uint4* qt = reinterpret_cast<uint4*>(sgen + q_off);
 #pragma unroll 4
       for (int k = 0; k < (2 * 128 * 128) / 16 / 128; ++k) {
         uint4 x = qt[r + 128 * k];
