@@ -111,3 +111,14 @@ def test_mask_exact_ties_take_lower_indices(topk, topp):
     for r, c in enumerate(g_cnt.reshape(-1)):
         np.testing.assert_array_equal(g_idx.reshape(-1, g_idx.shape[-1])[r, :c], np.arange(c))
         np.testing.assert_array_equal(o_idx.reshape(-1, o_idx.shape[-1])[r, :c], np.arange(c))
+
+
+@pytest.mark.parametrize("s", [20.0, 60.0])
+@pytest.mark.parametrize("topk,topp", [(0.5, 0.0), (0.9, 0.0), (1.0, 0.0), (0.0, 1.0), (0.3, 0.99)])
+def test_mask_with_underflowing_probabilities(s, topk, topp):
+    # Very wide score ranges: most of a row's probabilities are exactly 0 in
+    # double or lie more than 255 binades below its largest, so the
+    # selection's threshold falls among keys of mixed binades (and among
+    # exact zeros, which tie and go to the lower indices).
+    Q, K, _ = synth.make_qkv(1, 2, 4096, 64, grid=None, s=s, seed=123)
+    _check(Q, K, 64, 64, topk, topp, what=f"s={s} k={topk} p={topp}")
