@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (warp == 2 && lane == 0) {
       for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmO, sQ + b * (kTileQ * 128), b * 64, q0, bh);
       tma_store_commit();
-      tma_store_wait0();
+      tma_store_wait_read0();  // the staging tile has been read: the CTA may end
     }
   }
   tc_fence_before();

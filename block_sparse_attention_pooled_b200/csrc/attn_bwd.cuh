@@ -658,7 +658,7 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
     if (warp == 2 && lane == 0) {
       for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmDQ, sQ + b * (kTileQ * 128), b * 64, q0, bh);
       tma_store_commit();
-      tma_store_wait0();
+      tma_store_wait_read0();  // the staging tile has been read: the CTA may end
     }
   }
   tc_fence_before();
@@ -1087,7 +1087,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_store_3d(&tmDK, sOutK + b * (kTileK * 128), b * 64, key0, bh);
         }
         tma_store_commit();
-        tma_store_wait0();
+        tma_store_wait_read0();  // the staging tile has been read: the CTA may end
       }
     }
   }

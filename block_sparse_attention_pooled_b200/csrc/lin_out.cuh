@@ -90,7 +90,6 @@ struct LoParams {
   int bk;
 };
 
-__device__ __forceinline__ float phi_lin(float x) { return x > 0.0f ? x + 1.0f : __expf(x); }
 
 
 __global__ void __launch_bounds__(kLoThreads, 2)
@@ -309,18 +308,24 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     zc[r] = __ldg(p.z_all + (int64_t)bh * 128 + r) - zk;
     if (ok) ok = warp_wait(L::kBarQ, 0, kErrLoQ);
     if (ok) {
+      // Sixteen 16-byte units per thread: every load in flight before the
+      // first conversion, every store after the last.
+      constexpr int kUnits = (2 * 128 * 128) / 16 / 128;
       uint4* qt = reinterpret_cast<uint4*>(sgen + q_off);
-#pragma unroll 4
-      for (int k = 0; k < (2 * 128 * 128) / 16 / 128; ++k) {
-        uint4 x = qt[r + 128 * k];
-        __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&x);
+      uint4 x[kUnits];
+#pragma unroll
+      for (int k = 0; k < kUnits; ++k) x[k] = qt[r + 128 * k];
+#pragma unroll
+      for (int k = 0; k < kUnits; ++k) {
+        __nv_bfloat162* hx = reinterpret_cast<__nv_bfloat162*>(&x[k]);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = __bfloat1622float2(hx[j]);
-          hx[j] = __floats2bfloat162_rn(phi_lin(f.x), phi_lin(f.y));
+          hx[j] = __floats2bfloat162_rn(phi_elu1(f.x), phi_elu1(f.y));
         }
-        qt[r + 128 * k] = x;
       }
+#pragma unroll
+      for (int k = 0; k < kUnits; ++k) qt[r + 128 * k] = x[k];
     }
     fence_async_smem();
     tc_fence_before();
@@ -363,7 +368,7 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     if (warp == 2 && lane == 0) {
       for (int b = 0; b < 2; ++b) tma_store_3d(&tmO, sQ + b * (128 * 128), b * 64, q0, bh);
       tma_store_commit();
-      tma_store_wait0();
+      tma_store_wait_read0();  // the staging tile has been read: the CTA may end
     }
   }
   tc_fence_before();

@@ -63,7 +63,6 @@ struct LinParams {
   int ctas_per_head;
 };
 
-__device__ __forceinline__ float phi_f(float x) { return x > 0.0f ? x + 1.0f : __expf(x); }
 
 // Applies phi to 8 packed bf16 values.
 __device__ __forceinline__ uint4 phi8(uint4 v) {
@@ -71,7 +70,7 @@ __device__ __forceinline__ uint4 phi8(uint4 v) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     float2 f = __bfloat1622float2(h[j]);
-    h[j] = __floats2bfloat162_rn(phi_f(f.x), phi_f(f.y));
+    h[j] = __floats2bfloat162_rn(phi_elu1(f.x), phi_elu1(f.y));
   }
   return v;
 }
@@ -216,7 +215,7 @@ __global__ void __launch_bounds__(kLinThreads)
   if (tid == 0) {
     mma_commit(bar_drain);
     mbar_wait(bar_drain, 0, kErrLinDrain);
-    tma_store_wait0();
+    tma_store_wait_read0();  // the phi(K) tiles have been read from shared memory: the CTA may end
   }
   tc_fence_before();
   __syncthreads();

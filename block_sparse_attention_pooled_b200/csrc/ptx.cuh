@@ -121,7 +121,6 @@ __device__ __forceinline__ void tma_store_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
-__device__ __forceinline__ void tma_store_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_async_smem() {
@@ -329,6 +328,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// phi(x) = elu(x) + 1, the linear branch's feature map, without a branch:
+// the exponential of min(x, 0) (which cannot overflow) is taken for every x
+// and a select keeps x + 1 for x > 0.
+__device__ __forceinline__ float phi_elu1(float x) {
+  const float e = ex2_approx(fminf(x, 0.0f) * 1.4426950408889634f);
+  return x > 0.0f ? x + 1.0f : e;
 }
 
 }  // namespace sparge
