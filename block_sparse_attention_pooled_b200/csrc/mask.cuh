@@ -8,7 +8,7 @@
 //   pool : exact double sums of a block's valid bf16 rows, divided by the
 //          number of valid rows;
 //   score: double fused multiply-adds over the channels, times 1/sqrt(d);
-//   prob : exp(z - rowmax) / rowsum in double;
+//   prob : exp(z - rowmax) times the reciprocal of the row sum, in double;
 //   order: probability descending, block index ascending for ties, on the
 //          64-bit patterns of the double probabilities;
 //   Top-p: running sums of the ordered probabilities in 2^-62 fixed point
@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
 // truncated to a multiple of 2^-62 below, so running sums are exact integers
 // whatever the summation order (the truncation moves a row's total by less
 // than Nkb * 2^-62).
-//   0. P = exp(z - rowmax) / rowsum (double).
+//   0. P = exp(z - rowmax) * (1 / rowsum) (double; within a rounding unit of
+//      the quotient, and equal scores still give equal probabilities).
 //   1. Top-p: a radix select of the key at which the descending running
 //      weight first reaches p. The first pass buckets the keys by binade
 //      below the row's largest (bucket 255 - (e_top - e)); the next passes
@@ -549,8 +550,9 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
 #pragma unroll
   for (int w = 0; w < kSelectThreads / 32; ++w) rsum = __dadd_rn(rsum, red[w]);
   unsigned long long tot = 0ull, kmax = 0ull;  // total weight (exact integer sum), largest key
+  const double rinv = __drcp_rn(rsum);
   for (int j = tid; j < nkb; j += kSelectThreads) {
-    const double pj = __ddiv_rn(ev[j], rsum);
+    const double pj = __dmul_rn(ev[j], rinv);
     if (probs) probs[row * (int64_t)nkb + j] = (float)pj;
     const unsigned long long k = (unsigned long long)__double_as_longlong(pj);
     keys[j] = k;
@@ -702,8 +704,9 @@ __global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(const do
   for (int o = 16; o > 0; o >>= 1) part = __dadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
   const double rsum = part;
   unsigned long long tot = 0ull, kmax = 0ull;  // total weight (exact integer sum), largest key
+  const double rinv = __drcp_rn(rsum);
   for (int j = lane; j < nkb; j += 32) {
-    const double pj = __ddiv_rn(ev[j], rsum);
+    const double pj = __dmul_rn(ev[j], rinv);
     if (probs) probs[row * (int64_t)nkb + j] = (float)pj;
     const unsigned long long k = (unsigned long long)__double_as_longlong(pj);
     keys[j] = k;
