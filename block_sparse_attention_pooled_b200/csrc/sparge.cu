@@ -455,7 +455,7 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
 sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape* s, const Dims& dm,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, const void* phik, const float* s_all,
                                 const float* z_all, const float* z_tile, const float* alpha, void* O,
-                                cudaStream_t st, float* den_out = nullptr, const int32_t* order = nullptr) {
+                                cudaStream_t st, float* den_out = nullptr) {
   CUtensorMap mq, mv, mp, mo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, 128, 128) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
@@ -463,7 +463,6 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   LoParams p;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
-  p.order = order;
   p.s_all = s_all;
   p.z_all = z_all;
   p.z_tile = z_tile;
@@ -478,7 +477,8 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   p.bk = s->bk;
   cudaError_t e = ensure_smem(linear_out_kernel, LoSmem::kBytes, 7);
   if (e != cudaSuccess) return cuda_status(e);
-  linear_out_kernel<<<(unsigned)(dm.BH * dm.nqb), kLoThreads, LoSmem::kBytes, st>>>(mq, mv, mp, mo, p);
+  const int64_t pairs = dm.BH * ceil_div(dm.nqb, 2);  // two neighbouring query blocks per CTA
+  linear_out_kernel<<<(unsigned)pairs, kLoThreads, LoSmem::kBytes, st>>>(mq, mv, mp, mo, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -573,7 +573,7 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   e = launch_tile_order(kv_cnt, s, dm, &order, st);
   if (e != cudaSuccess) return cuda_status(e);
   r = launch_linear_out(Q, V, s, dm, kv_idx, kv_cnt, at(w.f.phik), fat(w.f.s_all), fat(w.f.z_all), fat(w.f.z_tile),
-                        fat(w.alpha0), at(w.ol), st, fat(w.den), order);
+                        fat(w.alpha0), at(w.ol), st, fat(w.den));
   if (r != SPARGE_OK) return r;
   r = launch_attn<D, false>(Q, K, V, s, dm, kv_idx, kv_cnt, at(w.os), fat(w.lse), nullptr, st, order);
   if (r != SPARGE_OK) return r;
@@ -847,7 +847,7 @@ sparge_status sla2_attn_fwd(const void* Q, const void* K, const void* V, const s
   if (e != cudaSuccess) return cuda_status(e);
   st = launch_summaries(K, V, shape, dm, phik, partial, s_all, z_all, z_tile, s);
   if (st != SPARGE_OK) return st;
-  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, z_tile, alpha, O, s, nullptr, order);
+  st = launch_linear_out(Q, V, shape, dm, kv_idx, kv_cnt, phik, s_all, z_all, z_tile, alpha, O, s);
   if (st != SPARGE_OK) return st;
   return launch_attn<128, true>(Q, K, V, shape, dm, kv_idx, kv_cnt, O, nullptr, alpha, s, order);
 }

@@ -76,6 +76,63 @@ def test_sla2_empty_and_full_rows():
     _check(Q, K, V, idx, cnt, np.array([0.7], np.float32), bq, bk)
 
 
+def _neighbour_masks(H, nqb, nkb, seed):
+    """Kept lists for query blocks 2c and 2c + 1 with every relation two
+    ascending lists can have: identical, nested either way, interleaved with a
+    shared part, disjoint, one or both empty, one complete."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 7])))
+    idx = np.zeros((1, H, nqb, nkb), np.int32)
+    cnt = np.zeros((1, H, nqb), np.int32)
+
+    def pick(pool, k):
+        return np.sort(rng.choice(pool, size=min(k, len(pool)), replace=False))
+
+    kinds = 9
+    for h in range(H):
+        for c in range((nqb + 1) // 2):
+            kind = (c + h) % kinds
+            base = pick(np.arange(nkb), int(rng.integers(1, nkb + 1)))
+            if kind == 0:
+                a, b = base, base
+            elif kind == 1:
+                a, b = pick(base, max(1, len(base) // 2)), base
+            elif kind == 2:
+                a, b = base, pick(base, max(1, len(base) // 2))
+            elif kind == 3:
+                rest = np.setdiff1d(np.arange(nkb), base)
+                a = np.union1d(pick(base, len(base) // 2 + 1), pick(rest, 3))
+                b = np.union1d(pick(base, len(base) // 2 + 1), pick(rest, 3))
+            elif kind == 4:
+                perm = rng.permutation(nkb)
+                a, b = np.sort(perm[: nkb // 3]), np.sort(perm[nkb // 3: nkb // 3 + nkb // 4])
+            elif kind == 5:
+                a, b = np.array([], np.int64), base
+            elif kind == 6:
+                a, b = base, np.array([], np.int64)
+            elif kind == 7:
+                a, b = np.arange(nkb), base
+            else:
+                a, b = np.array([], np.int64), np.array([], np.int64)
+            for I, lst in ((2 * c, a), (2 * c + 1, b)):
+                if I < nqb:
+                    idx[0, h, I, :len(lst)] = lst
+                    cnt[0, h, I] = len(lst)
+    return idx, cnt
+
+
+@pytest.mark.parametrize("N,bq,bk", [(1100, 128, 64), (1300, 64, 64), (2200, 128, 128), (900, 64, 128)])
+def test_sla2_neighbouring_blocks_share_key_blocks(N, bq, bk):
+    # One CTA takes query blocks 2c and 2c + 1 and walks the union of their
+    # lists; every relation between the two lists, odd block counts and a
+    # ragged last key block.
+    H = 9
+    Q, K, V = synth.make_qkv(1, H, N, 128, grid=None, s=1.5, seed=N + bk)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    idx, cnt = _neighbour_masks(H, nqb, nkb, seed=N)
+    alpha = np.linspace(0.55, 0.95, H).astype(np.float32)
+    _check(Q, K, V, idx, cnt, alpha, bq, bk)
+
+
 def test_sla2_long_rows_at_the_block_limit():
     # 4096 key blocks per row (the library's maximum), ragged last block: the
     # first query block keeps every block (empty complement, O_l = 0), the
