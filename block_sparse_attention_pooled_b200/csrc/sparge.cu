@@ -409,8 +409,6 @@ struct Sla2Ws {
   size_t phik, s_all, z_all, z_tile, partial, order, total;
 };
 
-inline int lin_ctas_per_head(int N) { return (int)ceil_div(ceil_div(N, 64), kLinTilesPerCta); }
-
 Sla2Ws sla2_ws(const sparge_shape* s, const Dims& d) {
   Sla2Ws w;
   w.phik = 0;
@@ -418,7 +416,7 @@ Sla2Ws sla2_ws(const sparge_shape* s, const Dims& d) {
   w.z_all = w.s_all + align256((size_t)d.BH * s->d * s->d * 4);
   w.z_tile = w.z_all + align256((size_t)d.BH * s->d * 4);
   w.partial = w.z_tile + align256((size_t)d.BH * ceil_div(s->N, 64) * s->d * 4);
-  w.order = w.partial + align256((size_t)d.BH * lin_ctas_per_head(s->N) * kLinPartial * 4);
+  w.order = w.partial + align256((size_t)(lin_grid(d.BH, s->N) + d.BH) * kLinPartial * 4);
   w.total = w.order + order_bytes(d);
   return w;
 }
@@ -497,20 +495,21 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
   p.row_w = row_w;
   p.N = s->N;
   p.ntiles = (int)ceil_div(s->N, 64);
-  p.ctas_per_head = lin_ctas_per_head(s->N);
-  const unsigned grid = (unsigned)(dm.BH * p.ctas_per_head);
+  p.total = dm.BH * p.ntiles;
+  const int64_t grid = lin_grid(dm.BH, s->N);
+  p.per_cta = ceil_div(p.total, grid);
   cudaError_t e;
   if (row_scale != nullptr) {  // the backward's G_all / g_all (K -> Q, V -> dO)
     e = ensure_smem(linear_summary_kernel<true>, LinSmem::kBytes, 13);
     if (e != cudaSuccess) return cuda_status(e);
-    linear_summary_kernel<true><<<grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+    linear_summary_kernel<true><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
   } else {
     e = ensure_smem(linear_summary_kernel<false>, LinSmem::kBytes, 6);
     if (e != cudaSuccess) return cuda_status(e);
-    linear_summary_kernel<false><<<grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+    linear_summary_kernel<false><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
   }
   dim3 rgrid((unsigned)ceil_div(kLinPartial, 256), (unsigned)dm.BH);
-  linear_reduce_kernel<<<rgrid, 256, 0, st>>>(partial, p.ctas_per_head, s_all, z_all, s_bf16);
+  linear_reduce_kernel<<<rgrid, 256, 0, st>>>(partial, p.ntiles, p.per_cta, s_all, z_all, s_bf16);
   return cuda_status(cudaGetLastError());
 }
 
