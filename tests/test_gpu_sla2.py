@@ -133,6 +133,18 @@ def test_sla2_neighbouring_blocks_share_key_blocks(N, bq, bk):
     _check(Q, K, V, idx, cnt, alpha, bq, bk)
 
 
+@pytest.mark.parametrize("B,H,N,bq,bk", [(2, 350, 100, 64, 64), (1, 900, 64, 64, 64), (3, 200, 200, 128, 128)])
+def test_sla2_many_short_heads(B, H, N, bq, bk):
+    # The summary kernel splits all heads' 64-key tiles evenly over its
+    # persistent grid: with short heads one CTA's run crosses three or more
+    # heads, so its two TMEM accumulators are each reused after release.
+    Q, K, V = synth.make_qkv(B, H, N, 128, grid=None, s=1.5, seed=N + H)
+    nqb, nkb = -(-N // bq), -(-N // bk)
+    idx, cnt = synth.random_mask(B, H, nqb, nkb, nkb, seed=H)
+    alpha = np.linspace(0.6, 1.0, H).astype(np.float32)
+    _check(Q, K, V, idx.numpy(), cnt.numpy(), alpha, bq, bk)
+
+
 def test_sla2_long_rows_at_the_block_limit():
     # 4096 key blocks per row (the library's maximum), ragged last block: the
     # first query block keeps every block (empty complement, O_l = 0), the

@@ -41,6 +41,25 @@ def test_sla2_bwd_matches_oracle(N, bq, bk, kind):
     np.testing.assert_allclose(got, ra, rtol=1e-2, atol=1e-2 * np.abs(ra).max())
 
 
+def test_sla2_bwd_many_short_heads():
+    # Short heads: the summary kernel's runs (forward summaries and the
+    # gradient summaries G_all, g_all) cross three or more heads per CTA.
+    B, H, N, bq, bk = 1, 750, 100, 64, 64
+    Q, K, V = synth.make_qkv(B, H, N, 128, grid=None, s=1.5, seed=31)
+    dO = synth.make_dout(B, H, N, 128, seed=32)
+    alpha = torch.linspace(0.6, 0.95, H, dtype=torch.float32)
+    kv_idx, kv_cnt = synth.random_mask(B, H, -(-N // bq), -(-N // bk), 2, seed=33)
+    kv_idx, kv_cnt = kv_idx.numpy(), kv_cnt.numpy()
+    dQ, dK, dV, da = _run(Q, K, V, dO, kv_idx, kv_cnt, alpha, bq, bk)
+    rQ, rK, rV, ra = oracle.attention_bwd(Q, K, V, dO, bq, bk, kv_idx, kv_cnt, alpha=alpha, mode="sla2",
+                                          want_dalpha=True)
+    _assert_grad("dQ", dQ.float().cpu().numpy().reshape(-1, 128), rQ)
+    _assert_grad("dK", _kblocks_layout(dK, bk), rK)
+    _assert_grad("dV", _kblocks_layout(dV, bk), rV)
+    got = da.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(got, ra, rtol=1e-2, atol=1e-2 * np.abs(ra).max())
+
+
 def test_sla2_bwd_alpha_one_is_the_sparse_backward():
     # alpha = 1: the linear branch carries no weight, so every linear term is an
     # exact zero and the gradients equal the sparse backward's bit for bit.
