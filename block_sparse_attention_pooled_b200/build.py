@@ -9,7 +9,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "sparge.cu")
-HEADERS = [os.path.join(PKG, "csrc", f) for f in ("ptx.cuh", "mask.cuh", "attn.cuh", "linear.cuh", "lin_out.cuh", "quant.cuh", "attn_q8.cuh", "attn_bwd.cuh", "selftest.cuh")] + [
+HEADERS = [os.path.join(PKG, "csrc", f) for f in ("ptx.cuh", "mask.cuh", "attn.cuh", "linear.cuh", "lin_out.cuh", "lin_bwd.cuh", "quant.cuh", "attn_q8.cuh", "attn_bwd.cuh", "selftest.cuh")] + [
     os.path.join(ROOT, "include", "sparge.h")
 ]
 LIB = os.path.join(PKG, "libsparge.so")

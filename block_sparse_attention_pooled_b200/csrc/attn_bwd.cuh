@@ -682,20 +682,8 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
 // MODE 0: the sparse branch alone; bf16 dK, dV.
 // MODE 1: the sparse part of the SLA2 backward: dV stages alpha_h P, dS uses
 //         alpha_h dP (D_i already carries alpha_h); fp32 partials out.
-// MODE 2: the linear part of the SLA2 backward (SLA2 article, sections 1 and
-//         2), over the same kept pairs, with phi(Q), phi(K) in place of Q, K
-//         and W = phi(Q_u) phi(K)^T in place of S. For key j and the query
-//         rows i whose block does NOT keep j's (c_i, f_i as in the dQ kernel):
-//           dphi(k_j) = sum_i c_i (dP_ij - f_i) phi(q_i)
-//                     = G_all v_j - g_all + sum_{i kept} c_i (f_i - dP_ij) phi(q_i)
-//           dv_j      = G_all^T phi(k_j) - sum_{i kept} c_i W_ij dO_i
-//         (G_all = sum_i phi(q_i) (c_i dO_i)^T, g_all = sum_i c_i f_i phi(q_i)
-//         over every row of the head). The accumulators start as
-//         dphiK^T = G_all V^T and dV^T = G_all^T phi(K)^T (two MMAs with the
-//         bf16 G_all tile in the staging area), gain the kept-pair terms with
-//         the staged -c W and c (f - dP), and the epilogue adds the MODE 1
-//         partials: dK = dK_sparse + (dphiK - g_all) * phi'(k), phi'(k) =
-//         min(phi(k), 1); dV = dV_sparse + dV_linear.
+// (linear_dkdv_kernel then adds the linear branch's dK, dV to the MODE 1
+// partials.)
 // ---------------------------------------------------------------------------
 template <int D>
 struct BwdKVSmem {
@@ -714,13 +702,11 @@ struct BwdKVSmem {
   // dK(u), so the next loads into the slot start as early as possible.
   static constexpr int kBarKV = 0, kBarQFull = 1, kBarDOFull = 1 + NS, kBarQEmpty = 1 + 2 * NS,
                        kBarDOEmpty = 1 + 3 * NS, kBarSFull = 1 + 4 * NS, kBarPReady = 3 + 4 * NS,
-                       kBarStage = 4 + 4 * NS, kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS,
-                       kBarPart = 7 + 4 * NS;
-  static constexpr int kNumBars = 8 + 4 * NS;
+                       kBarStage = 4 + 4 * NS, kBarFinal = 5 + 4 * NS, kBarDrain = 6 + 4 * NS;
+  static constexpr int kNumBars = 7 + 4 * NS;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffTmem + 16 + 1024;
   static constexpr int kTmemCols = 512;
-  static constexpr int kPartBytes = kTileK * D * 4;  // one fp32 partial tile, four 32-column boxes
 };
 
 // 64 bf16 (pairs in pk) as row r of a [128 rows][64 columns] tile with the
@@ -755,12 +741,11 @@ __device__ __forceinline__ float tile_at(const uint8_t* tile, int j, int c) {
       tile + (c / 64) * (kTileK * 128) + j * 128 + ((cc ^ (j & 7)) * 16) + (c % 8) * 2));
 }
 
-// Inputs and outputs of the SLA2 modes of the dK/dV kernel.
+// Inputs and outputs of the SLA2 mode of the dK/dV kernel.
 struct BwdKVLin {
   const float* alpha;   // [H] (MODE 1)
-  float* dk_part;       // [BH, N, d] fp32: MODE 1 writes scale * dK_sparse, MODE 2 reads it
-  float* dv_part;       // [BH, N, d] fp32: MODE 1 writes dV_sparse, MODE 2 reads it
-  const float* g_all;   // [BH, d] (MODE 2)
+  float* dk_part;       // [BH, N, d] fp32: MODE 1 writes scale * dK_sparse
+  float* dv_part;       // [BH, N, d] fp32: MODE 1 writes dV_sparse
   int H;
 };
 
@@ -769,8 +754,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-                         const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmKp,
-                         const __grid_constant__ CUtensorMap tmVp, const BwdParams p, const BwdKVLin lk) {
+                         const BwdParams p, const BwdKVLin lk) {
   using L = BwdKVSmem<D>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -792,10 +776,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int64_t jrow = (int64_t)bh * p.nkb + key0 / p.bk;  // (bh, key block)
   const int T = min(max(__ldg(p.cnt + jrow), 0), p.nqb);
   const int32_t* lst = p.lst + jrow * p.nqb;
-  const bool work = T > 0 || MODE == 2;  // the linear part has the G_all terms even when nothing is kept
-  // The staging tiles are free for tile t once phase t - 1 (MODE 2: t, the
-  // first phase being the G_all MMAs) of the stage barrier has completed.
-  constexpr int kStageShift = MODE == 2 ? 0 : 1;
+  const bool work = T > 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarKV), 1);
@@ -810,7 +791,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar(L::kBarStage), 1);
     mbar_init(bar(L::kBarFinal), 1);
     mbar_init(bar(L::kBarDrain), 1);
-    mbar_init(bar(L::kBarPart), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -833,11 +813,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmDO);
-        mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes + (MODE == 2 ? 2 * L::kStBytes : 0));
+        mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKBytes);
         for (int b = 0; b < D / 64; ++b) {
           tma_load_3d(sK + b * (kTileK * 128), &tmK, bar(L::kBarKV), b * 64, key0, bh);
           tma_load_3d(sV + b * (kTileK * 128), &tmV, bar(L::kBarKV), b * 64, key0, bh);
-          if (MODE == 2) tma_load_3d(sP + b * (kTileQ * 128), &tmG, bar(L::kBarKV), b * 64, 0, bh);
         }
       }
       ListChunks lc(lst, T, lane);
@@ -878,15 +857,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16_f32(kTileQ, kTileK, false, false);
       constexpr uint32_t idT = idesc_bf16_f32(D, kTileK, true, true);
-      constexpr uint32_t idGK = idesc_bf16_f32(D, kTileK, false, false);  // G_all V^T
       const uint64_t dRingK = sdesc_sw128(sRing, 16, 1024);               // Q_u, dO_u as K-major A
       const uint64_t dRingM = sdesc_sw128(sRing, kTileQ * 128, 1024);     // Q_u, dO_u as MN-major A
       const uint64_t dK = sdesc_sw128(sK, 16, 1024);
       const uint64_t dV = sdesc_sw128(sV, 16, 1024);
       const uint64_t dPst = sdesc_sw128(sP, kTileQ * 128, 1024);          // MN-major B, one 64-wide atom
       const uint64_t dDSst = sdesc_sw128(sDS, kTileQ * 128, 1024);
-      const uint64_t dGk = sdesc_sw128(sP, 16, 1024);                     // G_all as K-major A
-      const uint64_t dGm = sdesc_sw128(sP, kTileQ * 128, 1024);           // G_all^T as MN-major A
       auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
         return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
       };
@@ -922,25 +898,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       bool ok = warp_wait(L::kBarKV, 0, kErrBwdKV);
       tc_fence_after();
-      if (MODE == 2 && ok) {
-        // dphiK^T = G_all V^T and dV^T = G_all^T phi(K)^T (K = the d features).
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t go = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
-            const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
-            mma_ss(tDK, dGk + go, dV + ko, idGK, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ko = ((kk >> 2) * (kTileK * 128) + (kk & 3) * 32) >> 4;
-            mma_ss(tDV, dGm + kk * 128, dK + ko, idGK | (1u << 15), kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(L::kBarStage));  // the staging area (G_all) is free again
-          if (T == 0) mma_commit(bar(L::kBarFinal));
-        }
-        __syncwarp();
-      }
       // S and dP run two tiles ahead; dV(u) and dK(u) are issued as soon as
       // P(u) and dS(u) are staged, before the loads of tile u + 2 are awaited.
       for (int t = 0; ok && t < T && t < 2; ++t) ok = issue_sdp(t);
@@ -953,11 +910,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t doo = (uint32_t)((slot * L::kSlot + L::kQBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTileQ / 16; ++kk)  // 16 query rows = 2048 bytes of each operand
-            mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (MODE == 2 || u > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tDV, dRingM + doo + kk * 128, dPst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::kBarDOEmpty + slot));
 #pragma unroll
           for (int kk = 0; kk < kTileQ / 16; ++kk)
-            mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (MODE == 2 || u > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tDK, dRingM + so + kk * 128, dDSst + kk * 128, idT, (u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::kBarQEmpty + slot));
           mma_commit(bar(L::kBarStage));
           if (u == T - 1) mma_commit(bar(L::kBarFinal));
@@ -982,7 +939,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int q0 = lc.get(lst, T, t, lane) * p.bq;
       const bool row_ok = r < p.bq && q0 + r < p.N;
       const int64_t grow = (int64_t)bh * p.N + q0 + r;
-      // MODE 0/1: lse and D of the row; MODE 2: c_i and f_i.
+      // lse and D of the row.
       const float x0 = row_ok ? __ldg(p.lse + grow) : 0.0f;
       const float x1 = row_ok ? __ldg(p.dsum + grow) : 0.0f;
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t >> 1) & 1, kErrBwdSFull, abort_flag));
@@ -992,21 +949,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       load_row64(tS + lane_off + b * 64, s);
       load_row64(tP + lane_off + b * 64, dp);
       uint32_t pp[kTileK / 2], pds[kTileK / 2];
-      if (MODE == 2) {
-        // -c W for dV, c (f - dP) for dphi(K); zero on rows outside the block.
-        const float ci = row_ok ? x0 : 0.0f;
-#pragma unroll
-        for (int k = 0; k < kTileK / 2; ++k) {
-          pp[k] = pack_bf16x2(-ci * s[2 * k], -ci * s[2 * k + 1]);
-          pds[k] = pack_bf16x2(ci * (x1 - dp[2 * k]), ci * (x1 - dp[2 * k + 1]));
-        }
-      } else {
-        p_and_ds(s, dp, p.scale_log2, x0 * 1.4426950408889634f, x1, a_h, key0, p.N, row_ok, pp, pds);
-      }
-      // The staging tiles are free once the MMAs of the previous tile (MODE 2
-      // at t = 0: the G_all MMAs) have read them.
-      if (t + 1 - kStageShift > 0) {
-        ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarStage), (t - kStageShift) & 1, kErrBwdStage, abort_flag));
+      p_and_ds(s, dp, p.scale_log2, x0 * 1.4426950408889634f, x1, a_h, key0, p.N, row_ok, pp, pds);
+      // The staging tiles are free once the MMAs of the previous tile have
+      // read them.
+      if (t > 0) {
+        ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarStage), (t - 1) & 1, kErrBwdStage, abort_flag));
         if (!ok) break;
       }
       stage_row64(sP, r, pp);
@@ -1020,25 +967,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
     }
     // Epilogue: lane r holds channel r of dV^T and dK^T (keys along the columns).
-    // MODE 2 brings the fp32 sparse partials of the tile into the (now idle)
-    // ring by TMA and stages its outputs in the staging area instead.
-    const uint32_t sOutV = MODE == 2 ? sP : sRing, sOutK = MODE == 2 ? sDS : sRing + L::kKBytes;
-    const uint8_t* partK = sgen + L::kOffRing;
-    const uint8_t* partV = sgen + L::kOffRing + L::kPartBytes;
-    if (MODE == 2) {
-      if (warp == 2 && lane == 0 && ok) {
-        mbar_arrive_expect_tx(bar(L::kBarPart), 2 * L::kPartBytes);
-        for (int b = 0; b < D / 32; ++b) {
-          tma_load_3d(sRing + b * (kTileK * 128), &tmKp, bar(L::kBarPart), b * 32, key0, bh);
-          tma_load_3d(sRing + L::kPartBytes + b * (kTileK * 128), &tmVp, bar(L::kBarPart), b * 32, key0, bh);
-        }
-      }
-      if (ok) ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarPart), 0, kErrBwdIn, abort_flag));
-    }
-    // Element (key j, channel r) of a loaded partial tile: 32-column boxes of 64 rows.
-    auto part_at = [&](const uint8_t* t, int j) {
-      return *reinterpret_cast<const float*>(t + (r / 32) * (kTileK * 128) + j * 128 + (r % 32) * 4);
-    };
+    const uint32_t sOutV = sRing, sOutK = sRing + L::kKBytes;
     float v[kTileK];
     if (work && ok) {
       load_row64(tDV + lane_off, v);
@@ -1053,10 +982,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int j = 0; j < kTileK; ++j)
         if (j < nvalid) lk.dv_part[obase + (int64_t)j * D] = v[j];
     } else {
-      if (MODE == 2) {
-#pragma unroll
-        for (int j = 0; j < kTileK; ++j) v[j] += part_at(partV, j);
-      }
       stage_col64<D>(sOutV, r, v, 1.0f);
     }
     if (work && ok) {
@@ -1070,15 +995,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int j = 0; j < kTileK; ++j)
         if (j < nvalid) lk.dk_part[obase + (int64_t)j * D] = v[j] * p.scale;
     } else {
-      if (MODE == 2) {
-        const float g = __ldg(lk.g_all + (int64_t)bh * D + r);
-#pragma unroll
-        for (int j = 0; j < kTileK; ++j)
-          v[j] = part_at(partK, j) + (v[j] - g) * fminf(tile_at(sgen + L::kOffK, j, r), 1.0f);
-      }
-      stage_col64<D>(sOutK, r, v, MODE == 0 ? p.scale : 1.0f);
+      stage_col64<D>(sOutK, r, v, p.scale);
     }
-    if (MODE != 1) {
+    if (MODE == 0) {
       fence_async_smem();
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (warp == 2 && lane == 0) {

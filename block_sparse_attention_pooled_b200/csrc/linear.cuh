@@ -15,10 +15,11 @@
 // linear branch needs (rows are query rows then, with per-row weights c_i and
 // e_i from the backward's row pass):
 //   phiQ  = phi(Q)                         bf16 [N, d]
+//   cdO   = c_i dO_i                       bf16 [N, d]
 //   G_all = sum_i phi(q_i) (c_i dO_i)^T     fp32 [d, d]
 //   g_all = sum_i e_i phi(q_i)              fp32 [d]
-// (K -> Q, V -> dO with row i scaled by c_i, the column sums weighted by e_i;
-// no z_tile).
+//   g_tile[t] = sum of e_i phi(q_i) over the 64 rows of tile t
+// (K -> Q, V -> dO with row i scaled by c_i, the column sums weighted by e_i).
 //
 // The flattened (head, 64-key tile) range is split evenly over a persistent
 // grid of kLinCtas CTAs (two per SM on 148 SMs); CTA c takes the tiles
@@ -28,7 +29,7 @@
 //               ring (32 KB a slot);
 //   warp 1      TMEM owner and issuer (one elected lane): for each tile, once
 //               the compute warps have applied phi, a TMA store of the phi(K)
-//               tile and four MMAs D[feature, 0..127] += phi(K)^T V (M 128,
+//               tile (GRAD: and of the scaled V tile) and four MMAs D[feature, 0..127] += phi(K)^T V (M 128,
 //               N 128, K 64, both operands MN-major in shared memory); two
 //               accumulators (TMEM columns 0..127 and 128..255) alternate
 //               between the head segments of the range;
@@ -43,8 +44,10 @@
 // linear_reduce_kernel adds each head's partials in CTA order: the result
 // does not depend on scheduling.
 //
-// GRAD: V rows are scaled by c_i in place before the MMAs, and the column sum
-// of the segment is sum_i e_i phi(q_i) (e_i staged per tile in shared memory).
+// GRAD: V rows are scaled by c_i in place before the MMAs (and the scaled
+// tile is stored too), and the column sums are those of e_i phi(q_i) (e_i
+// staged per tile in shared memory): per 64-row tile into z_tile, per
+// segment into the partial.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -75,7 +78,7 @@ struct LinSmem {
 
 struct LinParams {
   float* partial;  // [grid + BH][128][129]: partial of (CTA c, head h) at slot c + h
-  float* z_tile;   // [BH, ntiles, 128] (null with GRAD)
+  float* z_tile;   // [BH, ntiles, 128] per-tile column sums, or null
   const float* row_scale;  // GRAD: c_i [BH, N]
   const float* row_w;      // GRAD: e_i [BH, N]
   int N;
@@ -116,7 +119,8 @@ __device__ __forceinline__ float box_at(const uint8_t* box, int row, int col) {
 template <bool GRAD>
 __global__ void __launch_bounds__(kLinThreads, 2)
     linear_summary_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                          const __grid_constant__ CUtensorMap tmPhiK, const LinParams p) {
+                          const __grid_constant__ CUtensorMap tmPhiK, const __grid_constant__ CUtensorMap tmVs,
+                          const LinParams p) {
   using L = LinSmem;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -194,7 +198,10 @@ __global__ void __launch_bounds__(kLinThreads, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA and phi(K) store issuer
     const bool leader = elect_one();
-    if (leader) tma_prefetch_desc(&tmPhiK);
+    if (leader) {
+      tma_prefetch_desc(&tmPhiK);
+      if (GRAD) tma_prefetch_desc(&tmVs);
+    }
     constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);
     bool ok = true;
     int seg = 0;          // segment index of tile i
@@ -209,7 +216,10 @@ __global__ void __launch_bounds__(kLinThreads, 2)
       if (leader) {
         const uint32_t sk = sbase + slot * L::kSlot, sv = sk + L::kTile;
         const int key0 = tile_of(i) * 64, bh = head_of(i);
-        for (int b = 0; b < 2; ++b) tma_store_3d(&tmPhiK, sk + b * 8192, b * 64, key0, bh);
+        for (int b = 0; b < 2; ++b) {
+          tma_store_3d(&tmPhiK, sk + b * 8192, b * 64, key0, bh);
+          if (GRAD) tma_store_3d(&tmVs, sv + b * 8192, b * 64, key0, bh);  // c_i dO_i
+        }
         tma_store_commit();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {  // 16 keys = 2048 bytes of each operand
@@ -294,7 +304,7 @@ __global__ void __launch_bounds__(kLinThreads, 2)
         }
         cs = (part[0] + part[1]) + (part[2] + part[3]);
       }
-      if (!GRAD) p.z_tile[((int64_t)bh * p.ntiles + tile_of(i)) * 128 + ct] = cs;
+      if (p.z_tile != nullptr) p.z_tile[((int64_t)bh * p.ntiles + tile_of(i)) * 128 + ct] = cs;
       zacc += cs;
       mbar_arrive(bar(L::kBarEmpty + slot));
       if (seg_last(i)) {

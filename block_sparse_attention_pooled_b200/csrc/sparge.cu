@@ -19,6 +19,7 @@
 #include "quant.cuh"
 #include "attn_q8.cuh"
 #include "attn_bwd.cuh"
+#include "lin_bwd.cuh"
 #include "selftest.cuh"
 
 namespace {
@@ -252,20 +253,6 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t BH, int N, int box_ro
   return r == CUDA_SUCCESS;
 }
 
-// 3-D fp32 map over [BH][N][128] with (32 columns x rows x 1) boxes, no swizzle.
-bool make_map_f32(CUtensorMap* m, const void* base, int64_t BH, int N, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {128 * 4, (cuuint64_t)N * 128 * 4};
-  cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // Workspace of the backward: D_i per row, the transposed mask (query-block
 // lists per key block and their lengths).
 struct BwdWs {
@@ -335,7 +322,7 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   e = ensure_smem(attn_bwd_dkdv_kernel<D, 0>, BwdKVSmem<D>::kBytes, 12);
   if (e != cudaSuccess) return cuda_status(e);
   attn_bwd_dkdv_kernel<D, 0><<<(unsigned)(dm.BH * ceil_div(s->N, kTileK)), kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(
-      mq, mk, mv, mdo, mdk, mdv, mq, mq, mq, p, lk);
+      mq, mk, mv, mdo, mdk, mdv, p, lk);
   return cuda_status(cudaGetLastError());
 }
 
@@ -483,10 +470,11 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
 sparge_status launch_summaries(const void* K, const void* V, const sparge_shape* s, const Dims& dm, void* phik,
                                float* partial, float* s_all, float* z_all, float* z_tile, cudaStream_t st,
                                __nv_bfloat16* s_bf16 = nullptr, const float* row_scale = nullptr,
-                               const float* row_w = nullptr) {
-  CUtensorMap mk, mv, mp;
+                               const float* row_w = nullptr, void* v_scaled = nullptr) {
+  CUtensorMap mk, mv, mp, mvs;
   if (!make_map_bhnd(&mk, K, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
-      !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64))
+      !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) ||
+      !make_map_bhnd(&mvs, v_scaled != nullptr ? v_scaled : phik, dm.BH, s->N, 128, 64))
     return SPARGE_ERR_CUDA;
   LinParams p;
   p.partial = partial;
@@ -502,11 +490,11 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
   if (row_scale != nullptr) {  // the backward's G_all / g_all (K -> Q, V -> dO)
     e = ensure_smem(linear_summary_kernel<true>, LinSmem::kBytes, 13);
     if (e != cudaSuccess) return cuda_status(e);
-    linear_summary_kernel<true><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+    linear_summary_kernel<true><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, mvs, p);
   } else {
     e = ensure_smem(linear_summary_kernel<false>, LinSmem::kBytes, 6);
     if (e != cudaSuccess) return cuda_status(e);
-    linear_summary_kernel<false><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, p);
+    linear_summary_kernel<false><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, mp, p);
   }
   dim3 rgrid((unsigned)ceil_div(kLinPartial, 256), (unsigned)dm.BH);
   linear_reduce_kernel<<<rgrid, 256, 0, st>>>(partial, p.ntiles, p.per_cta, s_all, z_all, s_bf16);
@@ -518,8 +506,8 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
 // transposed mask and the fp32 sparse partials of dK and dV.
 struct Sla2BwdWs {
   Sla2Ws f;  // phi(K), S_all, z_all, z_tile, summary partials
-  size_t s_bf16, os, lse, ol, den, alpha0, dsum, cw, fw, ew, dpart, phiq, g, gall, g_bf16, qidx, qcnt, dkp, dvp,
-      total;
+  size_t s_bf16, os, lse, ol, den, alpha0, dsum, cw, fw, ew, dpart, phiq, cdo, g, gall, gtile, qidx, qcnt, dkp,
+      dvp, total;
 };
 
 inline int sla2_row_chunks(int N) { return (int)ceil_div(N, kRowsPerCta); }
@@ -541,10 +529,11 @@ Sla2BwdWs sla2_bwd_ws(const sparge_shape* s, const Dims& d) {
   w.ew = w.fw + rows;
   w.dpart = w.ew + rows;
   w.phiq = w.dpart + align256((size_t)d.BH * sla2_row_chunks(s->N) * 4);
-  w.g = w.phiq + tens;
+  w.cdo = w.phiq + tens;
+  w.g = w.cdo + tens;
   w.gall = w.g + mat32;
-  w.g_bf16 = w.gall + align256((size_t)d.BH * s->d * 4);
-  w.qidx = w.g_bf16 + mat16;
+  w.gtile = w.gall + align256((size_t)d.BH * s->d * 4);
+  w.qidx = w.gtile + align256((size_t)d.BH * ceil_div(s->N, 64) * s->d * 4);
   w.qcnt = w.qidx + align256((size_t)d.BH * d.nkb * d.nqb * 4);
   w.dkp = w.qcnt + align256((size_t)d.BH * d.nkb * 4);
   w.dvp = w.dkp + align256((size_t)d.BH * s->N * s->d * 4);
@@ -560,7 +549,6 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
   auto fat = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
   __nv_bfloat16* s_bf16 = static_cast<__nv_bfloat16*>(at(w.s_bf16));
-  __nv_bfloat16* g_bf16 = static_cast<__nv_bfloat16*>(at(w.g_bf16));
   // 1. The forward's pieces: summaries (and a bf16 S_all), O_l unscaled with
   //    its denominators (alpha = 0 gives weight 1), the sparse branch with lse.
   sparge_status r = launch_summaries(K, V, s, dm, at(w.f.phik), fat(w.f.partial), fat(w.f.s_all), fat(w.f.z_all),
@@ -583,9 +571,10 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
       static_cast<const __nv_bfloat16*>(dO), fat(w.den), alpha, s->H, s->N, chunks, fat(w.dsum), fat(w.cw),
       fat(w.fw), fat(w.ew), fat(w.dpart));
   sla2_dalpha_kernel<<<1, 128, 0, st>>>(fat(w.dpart), s->B, s->H, chunks, dalpha);
-  // 3. G_all, g_all and phi(Q) (the summary kernel on Q and dO with c_i, e_i).
-  r = launch_summaries(Q, dO, s, dm, at(w.phiq), fat(w.f.partial), fat(w.g), fat(w.gall), nullptr, st, g_bf16,
-                       fat(w.cw), fat(w.ew));
+  // 3. G_all, g_all, g_tile, phi(Q) and c_i dO_i (the summary kernel on Q
+  //    and dO with c_i, e_i).
+  r = launch_summaries(Q, dO, s, dm, at(w.phiq), fat(w.f.partial), fat(w.g), fat(w.gall), fat(w.gtile), st, nullptr,
+                       fat(w.cw), fat(w.ew), at(w.cdo));
   if (r != SPARGE_OK) return r;
   // 4. Transposed mask.
   int32_t* q_idx = reinterpret_cast<int32_t*>(ws + w.qidx);
@@ -597,15 +586,14 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
       kv_idx, kv_cnt, (int)dm.nqb, (int)dm.nkb, q_idx, q_cnt);
   // 5. dQ (sparse + linear), then dK and dV: sparse part into fp32 partials,
   //    linear part and the combination into bf16.
-  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, mpq, msall, mg, mkp, mvp;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, mpq, msall, mpq64, mcdo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mdo, dO, dm.BH, s->N, D, kTileQ) ||
       !make_map_bhnd(&mdq, dQ, dm.BH, s->N, D, s->bq) || !make_map_bhnd(&mdk, dK, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mdv, dV, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mpk, at(w.f.phik), dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mpq, at(w.phiq), dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&msall, s_bf16, dm.BH, D, D, kTileQ) ||
-      !make_map_bhnd(&mg, g_bf16, dm.BH, D, D, kTileQ) || !make_map_f32(&mkp, ws + w.dkp, dm.BH, s->N, kTileK) ||
-      !make_map_f32(&mvp, ws + w.dvp, dm.BH, s->N, kTileK))
+      !make_map_bhnd(&mpq64, at(w.phiq), dm.BH, s->N, D, 64) || !make_map_bhnd(&mcdo, at(w.cdo), dm.BH, s->N, D, 64))
     return SPARGE_ERR_CUDA;
   BwdParams p;
   p.lse = fat(w.lse);
@@ -638,20 +626,31 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   lk.alpha = alpha;
   lk.dk_part = fat(w.dkp);
   lk.dv_part = fat(w.dvp);
-  lk.g_all = fat(w.gall);
   lk.H = s->H;
   const unsigned kgrid = (unsigned)(dm.BH * ceil_div(s->N, kTileK));
   e = ensure_smem(attn_bwd_dkdv_kernel<D, 1>, BwdKVSmem<D>::kBytes, 15);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dkdv_kernel<D, 1><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mq, mk, mv, mdo, mdk, mdv, mg, mkp,
-                                                                              mvp, p, lk);
-  BwdParams pl = p;
-  pl.lse = fat(w.cw);
-  pl.dsum = fat(w.fw);
-  e = ensure_smem(attn_bwd_dkdv_kernel<D, 2>, BwdKVSmem<D>::kBytes, 16);
+  attn_bwd_dkdv_kernel<D, 1><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mq, mk, mv, mdo, mdk, mdv, p, lk);
+  LbParams lb;
+  lb.q_idx = q_idx;
+  lb.q_cnt = q_cnt;
+  lb.g_all = fat(w.g);
+  lb.g_vec = fat(w.gall);
+  lb.g_tile = fat(w.gtile);
+  lb.dk_part = fat(w.dkp);
+  lb.dv_part = fat(w.dvp);
+  lb.dK = static_cast<__nv_bfloat16*>(dK);
+  lb.dV = static_cast<__nv_bfloat16*>(dV);
+  lb.N = s->N;
+  lb.ntiles = (int)ceil_div(s->N, 64);
+  lb.nqb = (int)dm.nqb;
+  lb.nkb = (int)dm.nkb;
+  lb.bq = s->bq;
+  lb.bk = s->bk;
+  e = ensure_smem(linear_dkdv_kernel, LbSmem::kBytes, 18);
   if (e != cudaSuccess) return cuda_status(e);
-  attn_bwd_dkdv_kernel<D, 2><<<kgrid, kAttnThreads, BwdKVSmem<D>::kBytes, st>>>(mpq, mpk, mv, mdo, mdk, mdv, mg,
-                                                                              mkp, mvp, pl, lk);
+  const int64_t kpairs = dm.BH * ceil_div(lb.ntiles, 2);  // two neighbouring key tiles per CTA
+  linear_dkdv_kernel<<<(unsigned)kpairs, kLoThreads, LbSmem::kBytes, st>>>(mpq64, mcdo, mpk, mv, lb);
   return cuda_status(cudaGetLastError());
 }
 
