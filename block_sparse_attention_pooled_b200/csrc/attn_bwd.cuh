@@ -30,8 +30,7 @@
 //                          keep M = 128 for 64-key blocks.
 // Warp roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer and
 // TMEM owner, then one row (TMEM lane) per thread in warpgroups of four
-// warps (three in the sparse dQ kernel, two in the SLA2 dQ kernel, one in the
-// dK/dV kernel). d = 128.
+// warps (three in the dQ kernel, one in the dK/dV kernel). d = 128.
 #pragma once
 #include <cuda.h>
 #include <cstdint>
@@ -265,47 +264,46 @@ struct ListChunks {
 
 // ---------------------------------------------------------------------------
 // dQ: one CTA per (bh, query block), the forward's walk over kept key tiles.
-// TMEM columns: S(b) [64b, 64b+64) and dP(b) [64 NB + 64b, ...) for NB tile
-// buffers b = t % NB, dQ [128 NB, 128 NB + 128); dS(t) (bf16 pairs) over the
-// first 32 columns of S(t)'s buffer. One CTA per SM (512 columns), so two dS
-// warpgroups share the SM: warps 2..5 take the even tiles, warps 6..9 the odd
-// ones, and each writes half of the dQ columns in the epilogue. With three
-// buffers (sparse branch alone) the MMA warp computes S and dP two tiles
-// ahead, so a warpgroup that finishes a tile finds its next one ready.
+// TMEM columns: S(b) [64b, 64b+64) and dP(b) [192 + 64b, ...) for the three
+// tile buffers b = t % 3, dQ [384, 512); dS(t) (bf16 pairs) over the first
+// 32 columns of S(t)'s buffer. One CTA per SM (512 columns) with three dS
+// warpgroups: warpgroup w takes the tiles t = w mod 3 (and buffer w), and a
+// run of the dQ columns in the epilogue. The MMA warp computes S and dP two
+// tiles ahead, so a warpgroup that finishes a tile finds its next one ready.
 //
 // SLA2 = true adds the linear branch's query gradient (SLA2 article,
 // arXiv:2602.12675, sections 1 and 2). With c_i = (1 - alpha_h) / den_i,
 // f_i = dO_i . O_l,i (den_i, O_l from the forward's linear branch) and the
-// complement of i's kept keys:
-//   dphi(q_i) = c_i sum_{j not kept} (dP_ij - f_i) phi(k_j)
-//             = c_i (S_all dO_i - f_i z_all + sum_{j kept} (f_i - dP_ij) phi(k_j))
-// so a second accumulator L [128 NB + 128, +128) starts as dO S_all^T (one MMA
-// from a bf16 copy of S_all) and gains X(t) phi(K_t) per kept tile, X = f - dP
-// written as bf16 over dP(t)'s first 32 columns; the epilogue forms
-//   dq_i = scale * dQ_i + c_i (L_i - f_i z_all) * phi'(q_i).
+// complement of i's kept keys,
+//   dphi(q_i) = c_i sum_{j not kept} (dP_ij - f_i) phi(k_j) = c_i (S_c dO_i - f_i z_c)
+// with S_c, z_c the complement summaries of i's query block, which
+// linear_out_kernel forms anyway (it stores them for the backward: S_c as a
+// bf16 [128][128] tile per block). After the last dQ product the MMA warp
+// adds L = dO S_c^T (one M 128, N 128, K 128 product) into the S columns
+// [0, 128), which every dQ product has read by then, and the epilogue forms
+//   dq_i = scale * dQ_i + c_i (L_i - f_i z_c) * phi'(q_i).
 // The sparse part uses alpha_h dO: dS = P (alpha_h dP - D_i), D_i = alpha_h dO_i . O_s,i.
-// NB = 2 then (TMEM: 4 x 64 + 128 + 128 columns).
 // ---------------------------------------------------------------------------
-// dS warpgroups of the dQ kernel: three for the sparse branch alone (each
-// takes every third tile and owns one of the three S / dP buffers; dS is
-// formed half a tile at a time so 448 threads fit the register file), two
-// with SLA2 (the linear accumulator leaves room for two buffers).
+// dS warpgroups of the dQ kernel: three (each takes every third tile and owns
+// one of the three S / dP buffers; dS is formed half a tile at a time so 448
+// threads fit the register file).
 template <bool SLA2>
-__host__ __device__ constexpr int bwd_q_wgs() { return SLA2 ? 2 : 3; }
+__host__ __device__ constexpr int bwd_q_wgs() { return 3; }
 template <bool SLA2>
 __host__ __device__ constexpr int bwd_q_threads() { return 64 + 128 * bwd_q_wgs<SLA2>(); }
 
-// dS = P (dP - D) for 32 keys (half a tile) of the sparse branch, read from
-// TMEM at the given S and dP columns; 16 bf16 pairs out.
-__device__ __forceinline__ void ds_half(uint32_t ts, uint32_t tp, float scale_log2, float lse2, float Di, int key0,
-                                        int N, bool row_ok, uint32_t (&pds)[16]) {
+// dS = P (a dP - D) for 32 keys (half a tile) of the sparse branch, read
+// from TMEM at the given S and dP columns; 16 bf16 pairs out. a = 1, or
+// alpha_h in the SLA2 backward.
+__device__ __forceinline__ void ds_half(uint32_t ts, uint32_t tp, float scale_log2, float lse2, float Di, float a,
+                                        int key0, int N, bool row_ok, uint32_t (&pds)[16]) {
   uint32_t sv[2][16], pv[2][16];
   tmem_ld16(ts, sv[0]);
   tmem_ld16(ts + 16, sv[1]);
   tmem_ld16(tp, pv[0]);
   tmem_ld16(tp + 16, pv[1]);
   tmem_ld_wait();
-  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di);
+  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di), a2 = f2(a, a);
   const bool tail = key0 + 32 > N;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -314,7 +312,7 @@ __device__ __forceinline__ void ds_half(uint32_t ts, uint32_t tp, float scale_lo
     float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
     if (!row_ok || (tail && key0 + 2 * k >= N)) p0 = 0.0f;
     if (!row_ok || (tail && key0 + 2 * k + 1 >= N)) p1 = 0.0f;
-    const float2 g = f2_split(add2(f2(__uint_as_float(pv[h][c]), __uint_as_float(pv[h][c + 1])), nd2));
+    const float2 g = f2_split(fma2(f2(__uint_as_float(pv[h][c]), __uint_as_float(pv[h][c + 1])), a2, nd2));
     pds[k] = pack_bf16x2(p0 * g.x, p1 * g.y);
   }
 }
@@ -323,17 +321,16 @@ template <int D, bool SLA2>
 struct BwdQSmem {
   // K(t) is held until dQ(t) has read it, one softmax period after S(t): a
   // four-slot K ring keeps its loads two tiles ahead. V(t) frees after dP(t).
-  // SLA2: phi(K_t) rides with K(t); the bf16 S_all tile sits after dO.
-  static constexpr int NB = SLA2 ? 2 : 3;
-  static constexpr int NSK = SLA2 ? 2 : 4, NSV = 2;
+  // SLA2: the query block's bf16 S_c tile sits after dO.
+  static constexpr int NB = 3;
+  static constexpr int NSK = 4, NSV = 2;
   static constexpr int kQBytes = kTileQ * D * 2;
   static constexpr int kKBytes = kTileK * D * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffDO = kOffQ + kQBytes;
-  static constexpr int kOffSall = kOffDO + kQBytes;
-  static constexpr int kOffK = kOffSall + (SLA2 ? kQBytes : 0);
-  static constexpr int kOffPK = kOffK + NSK * kKBytes;
-  static constexpr int kOffV = kOffPK + (SLA2 ? NSK * kKBytes : 0);
+  static constexpr int kOffSc = kOffDO + kQBytes;
+  static constexpr int kOffK = kOffSc + (SLA2 ? kQBytes : 0);
+  static constexpr int kOffV = kOffK + NSK * kKBytes;
   static constexpr int kOffBar = kOffV + NSV * kKBytes;
   static constexpr int kBarIn = 0, kBarKFull = 1, kBarKEmpty = 1 + NSK, kBarVFull = 1 + 2 * NSK,
                        kBarVEmpty = 1 + 2 * NSK + NSV, kBarSFull = 1 + 2 * NSK + 2 * NSV,
@@ -349,35 +346,16 @@ struct BwdLinParams {
   const float* alpha;  // [H]
   const float* cw;     // [BH, N] c_i
   const float* fw;     // [BH, N] f_i
-  const float* z_all;  // [BH, d]
+  const float* zc;     // [BH * nqb, d] z_c of each query block
   int H;
 };
-
-// dS = P (alpha dP - D) (bf16 pairs) and, with SLA2, X = f - dP (bf16 pairs).
-template <bool SLA2>
-__device__ __forceinline__ void ds_and_x(const float (&s)[kTileK], const float (&dp)[kTileK], float scale_log2,
-                                         float lse2, float Di, float a, float f, int key0, int N, bool row_ok,
-                                         uint32_t (&pds)[kTileK / 2], uint32_t (&px)[kTileK / 2]) {
-  const uint64_t sc2 = f2(scale_log2, scale_log2), nl2 = f2(-lse2, -lse2), nd2 = f2(-Di, -Di), a2 = f2(a, a);
-  const bool tail = key0 + kTileK > N;
-#pragma unroll
-  for (int k = 0; k < kTileK / 2; ++k) {
-    const float2 x = f2_split(fma2(f2(s[2 * k], s[2 * k + 1]), sc2, nl2));
-    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-    if (!row_ok || (tail && key0 + 2 * k >= N)) p0 = 0.0f;
-    if (!row_ok || (tail && key0 + 2 * k + 1 >= N)) p1 = 0.0f;
-    const float2 g = f2_split(fma2(f2(dp[2 * k], dp[2 * k + 1]), a2, nd2));
-    pds[k] = pack_bf16x2(p0 * g.x, p1 * g.y);
-    if (SLA2) px[k] = row_ok ? pack_bf16x2(f - dp[2 * k], f - dp[2 * k + 1]) : 0u;
-  }
-}
 
 template <int D, bool SLA2>
 __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                       const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmPK,
-                       const __grid_constant__ CUtensorMap tmSall, const BwdParams p, const BwdLinParams lp) {
+                       const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmSc,
+                       const BwdParams p, const BwdLinParams lp) {
   using L = BwdQSmem<D, SLA2>;
   constexpr int NSK = L::NSK, NSV = L::NSV, NB = L::NB;
   extern __shared__ uint8_t smem_raw[];
@@ -385,7 +363,7 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw);
   const uint32_t sQ = sbase + L::kOffQ, sDO = sbase + L::kOffDO, sK = sbase + L::kOffK, sV = sbase + L::kOffV;
-  const uint32_t sSall = sbase + L::kOffSall, sPK = sbase + L::kOffPK;
+  const uint32_t sSc = sbase + L::kOffSc;
   const uint32_t bar0 = sbase + L::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + L::kOffTmem);
@@ -428,13 +406,12 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 64 * NB, tQ = tmem + 128 * NB, tL = tQ + 128;
+  const uint32_t tS = tmem, tP = tmem + 64 * NB, tQ = tmem + 128 * NB;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // The whole warp walks the list (indices by shuffle); lane 0 waits and issues.
     if (work) {
-      constexpr uint32_t kKTx = (SLA2 ? 2 : 1) * L::kKBytes;
       int nk = 0, nv = 0;
       bool ok = true;
       if (lane == 0) {
@@ -444,7 +421,7 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
         for (int b = 0; b < D / 64; ++b) {
           tma_load_3d(sQ + b * (kTileQ * 128), &tmQ, bar(L::kBarIn), b * 64, q0, bh);
           tma_load_3d(sDO + b * (kTileQ * 128), &tmDO, bar(L::kBarIn), b * 64, q0, bh);
-          if (SLA2) tma_load_3d(sSall + b * (kTileQ * 128), &tmSall, bar(L::kBarIn), b * 64, 0, bh);
+          if (SLA2) tma_load_3d(sSc + b * (kTileQ * 128), &tmSc, bar(L::kBarIn), b * 64, 0, tile);
         }
       }
       ListChunks lc(lst, cnt, lane);
@@ -463,14 +440,10 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
             ok = t < NSK || role_wait(bar(L::kBarKEmpty + ks), (t / NSK - 1) & 1, kErrBwdKEmpty, abort_flag);
           }
           if (ok) {
-            mbar_arrive_expect_tx(bar(L::kBarKFull + ks), kKTx);
-            for (int b = 0; b < D / 64; ++b) {
+            mbar_arrive_expect_tx(bar(L::kBarKFull + ks), L::kKBytes);
+            for (int b = 0; b < D / 64; ++b)
               tma_load_3d(sK + ks * L::kKBytes + b * (kTileK * 128), &tmK, bar(L::kBarKFull + ks), b * 64, key0,
                           bh);
-              if (SLA2)
-                tma_load_3d(sPK + ks * L::kKBytes + b * (kTileK * 128), &tmPK, bar(L::kBarKFull + ks), b * 64,
-                            key0, bh);
-            }
             ++nk;
           }
         }
@@ -494,34 +467,23 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
       constexpr uint32_t idL = idesc_bf16_f32(kTileQ, D, false, false);
       const uint64_t dQd = sdesc_sw128(sQ, 16, 1024);
       const uint64_t dDO = sdesc_sw128(sDO, 16, 1024);
-      const uint64_t dSall = sdesc_sw128(sSall, 16, 1024);           // K-major B (row = feature)
+      const uint64_t dSc = sdesc_sw128(sSc, 16, 1024);               // K-major B (row = feature)
       const uint64_t dK = sdesc_sw128(sK, 16, 1024);                // K-major (S = Q K^T)
       const uint64_t dKmn = sdesc_sw128(sK, kTileK * 128, 1024);    // MN-major (dQ += dS K)
-      const uint64_t dPKmn = sdesc_sw128(sPK, kTileK * 128, 1024);  // MN-major (L += X phi(K))
       const uint64_t dV = sdesc_sw128(sV, 16, 1024);                // K-major (dP = dO V^T)
       auto warp_wait = [&](int b, uint32_t parity, unsigned int site) {
         return __all_sync(0xffffffffu, role_wait(bar(b), parity, site, abort_flag));
       };
       bool ok = warp_wait(L::kBarIn, 0, kErrBwdIn);
       tc_fence_after();
-      if (SLA2 && ok) {
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
-            mma_ss(tL, dDO + qo, dSall + qo, idL, kk > 0 ? 1u : 0u);
-          }
-          if (T == 0) mma_commit(bar(L::kBarFinal));
-        }
-        __syncwarp();
-      }
       // S(t) and dP(t) run NB - 1 tiles ahead of dQ(t): buffer t % NB was last
       // read by dQ(t - NB), issued (and its dS written) before.
       for (int t = 0; ok && t < T + NB - 1; ++t) {
         if (t < T) {
           const int ks = t % NSK, vs = t % NSV, b = t % NB;
-          if (!warp_wait(L::kBarKFull + ks, (t / NSK) & 1, kErrBwdKFull)) break;
-          if (!warp_wait(L::kBarVFull + vs, (t / NSV) & 1, kErrBwdVFull)) break;
+          ok = warp_wait(L::kBarKFull + ks, (t / NSK) & 1, kErrBwdKFull) &&
+               warp_wait(L::kBarVFull + vs, (t / NSV) & 1, kErrBwdVFull);
+          if (!ok) break;
           tc_fence_after();
           if (leader) {
             const uint64_t dKs = dK + (uint64_t)((ks * L::kKBytes) >> 4);
@@ -545,24 +507,32 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
         }
         if (t >= NB - 1) {
           const int u = t - (NB - 1), ks = u % NSK, b = u % NB;
-          if (!warp_wait(L::kBarPFull + b, (u / NB) & 1, kErrBwdPFull)) break;
+          ok = warp_wait(L::kBarPFull + b, (u / NB) & 1, kErrBwdPFull);
+          if (!ok) break;
           tc_fence_after();
           if (leader) {
             const uint64_t dKm = dKmn + (uint64_t)((ks * L::kKBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk)  // 16 keys = 2048 bytes of K = 8 packed dS columns
               mma_ts(tQ, tS + b * 64 + kk * 8, dKm + kk * 128, idQ, (u > 0 || kk > 0) ? 1u : 0u);
-            if (SLA2) {
-              const uint64_t dPKm = dPKmn + (uint64_t)((ks * L::kKBytes) >> 4);
-#pragma unroll
-              for (int kk = 0; kk < kTileK / 16; ++kk)
-                mma_ts(tL, tP + b * 64 + kk * 8, dPKm + kk * 128, idQ, 1u);
-            }
             mma_commit(bar(L::kBarKEmpty + ks));
-            if (u == T - 1) mma_commit(bar(L::kBarFinal));
+            if (!SLA2 && u == T - 1) mma_commit(bar(L::kBarFinal));
           }
           __syncwarp();
         }
+      }
+      if (SLA2 && ok) {
+        // L = dO S_c^T into the S columns [0, 128): every dS there has been
+        // read by a dQ product issued before this one.
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qo = ((kk >> 2) * (kTileQ * 128) + (kk & 3) * 32) >> 4;
+            mma_ss(tS, dDO + qo, dSc + qo, idL, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::kBarFinal));
+        }
+        __syncwarp();
       }
       if (leader) mma_commit(bar(L::kBarDrain));
       __syncwarp();
@@ -590,26 +560,16 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
       ok = __all_sync(0xffffffffu, role_wait(bar(L::kBarSFull + b), (t / NB) & 1, kErrBwdSFull, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      if (SLA2) {
-        float s[kTileK], dp[kTileK];
-        load_row64(tS + lane_off + b * 64, s);
-        load_row64(tP + lane_off + b * 64, dp);
-        uint32_t pds[kTileK / 2], px[kTileK / 2];
-        ds_and_x<SLA2>(s, dp, p.scale_log2, lse2, Di, a_h, fi, key0, p.N, row_ok, pds, px);
-        store_p(tS + lane_off + b * 64, pds);
-        store_p(tP + lane_off + b * 64, px);
-      } else {
-        // Half a tile at a time; the half written back (columns 16h..16h+15 of
-        // S) holds S values already read.
+      // Half a tile at a time; the half written back (columns 16h..16h+15 of
+      // S) holds S values already read.
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pds[16];
-          ds_half(tS + lane_off + b * 64 + 32 * h, tP + lane_off + b * 64 + 32 * h, p.scale_log2, lse2, Di,
-                  key0 + 32 * h, p.N, row_ok, pds);
-          tmem_st16(tS + lane_off + b * 64 + 16 * h, pds);
-        }
-        tmem_st_wait();
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pds[16];
+        ds_half(tS + lane_off + b * 64 + 32 * h, tP + lane_off + b * 64 + 32 * h, p.scale_log2, lse2, Di, a_h,
+                key0 + 32 * h, p.N, row_ok, pds);
+        tmem_st16(tS + lane_off + b * 64 + 16 * h, pds);
       }
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::kBarPFull + b));
     }
@@ -636,7 +596,7 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
       if (SLA2) {
         uint32_t l[16];
         if (ok) {
-          tmem_ld16(tL + lane_off + c, l);
+          tmem_ld16(tS + lane_off + c, l);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -644,7 +604,7 @@ __global__ void __launch_bounds__(bwd_q_threads<SLA2>(), 1)
         }
         float qv[16];
         read_row16(sQ, r, c, qv);
-        const float* z = lp.z_all + (int64_t)bh * D + c;
+        const float* z = lp.zc + (int64_t)tile * D + c;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float dphi = ci * (__uint_as_float(l[j]) - fi * __ldg(z + j));

@@ -101,6 +101,8 @@ struct LoParams {
   const float* z_tile;    // [BH, ntiles, 128] fp32
   const float* alpha;     // [H]
   float* den_out;         // [BH, N] or null: phi(q) . z_c per row (0 where the branch is off)
+  float* zc_out;          // [BH * nqb, 128] or null: z_c per query block
+  int store_sc;           // nonzero: S_c per query block as bf16 [BH * nqb, 128, 128] through tmSc
   int H;
   int N;
   int ntiles;             // ceil(N / 64)
@@ -154,7 +156,7 @@ __device__ __forceinline__ bool union_next(KeptCursor& a, KeptCursor& b, int lan
 __global__ void __launch_bounds__(kLoThreads, 2)
     linear_out_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmPhiK, const __grid_constant__ CUtensorMap tmO,
-                      const LoParams p) {
+                      const __grid_constant__ CUtensorMap tmSc, const LoParams p) {
   using L = LoSmem;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -483,6 +485,15 @@ __global__ void __launch_bounds__(kLoThreads, 2)
     tc_fence_before();
     mbar_arrive(bar(L::kBarStage0));
     asm volatile("bar.sync 1, 128;" ::: "memory");  // z_c and phi(Q_A) complete
+    // For the backward: S_c,A (staged above) and both z_c out.
+    if (p.store_sc && warp == 2 && lane == 0) {
+      for (int b = 0; b < 2; ++b) tma_store_3d(&tmSc, sStage + b * (128 * 128), b * 64, 0, (int)tile_a);
+      tma_store_commit();
+    }
+    if (p.zc_out != nullptr) {
+      p.zc_out[tile_a * 128 + r] = zc[r];
+      if (has_b) p.zc_out[(tile_a + 1) * 128 + r] = zc[128 + r];
+    }
     // Denominator phi(q_r) . z_c in fp32; every block kept: the complement
     // is empty and the linear branch is 0.
     const float a_h = __ldg(p.alpha + (bh % p.H));
@@ -507,9 +518,14 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       asm volatile("bar.sync 1, 128;" ::: "memory");  // phi(Q_B) complete
       wl_b = row_weight(sQb, zc + 128, cnt_b, q0b);
     }
-    // 3. A's product done: the staging slot is free for S_c,B.
+    // 3. A's product done: the staging slot is free for S_c,B (once the
+    //    store of S_c,A, if any, has read it).
     if (ok) ok = warp_wait(L::kBarOut0, 0, kErrLoOut);
     tc_fence_after();
+    if (p.store_sc && has_b) {
+      if (warp == 2 && lane == 0) tma_store_wait_read0();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
     if (has_b) {
 #pragma unroll
       for (int c = 0; c < 128; c += 16) {
@@ -555,6 +571,10 @@ __global__ void __launch_bounds__(kLoThreads, 2)
       }
     };
     store_output(tD0, sQa, wl_a, q0a);
+    if (p.store_sc && has_b && warp == 2 && lane == 0) {  // S_c,B staged before the barrier in store_output
+      for (int b = 0; b < 2; ++b) tma_store_3d(&tmSc, sStage + b * (128 * 128), b * 64, 0, (int)(tile_a + 1));
+      tma_store_commit();
+    }
     if (has_b) {
       if (ok) ok = warp_wait(L::kBarOut1, 0, kErrLoOut);
       tc_fence_after();

@@ -314,7 +314,7 @@ sparge_status launch_bwd(const void* Q, const void* K, const void* V, const spar
   if (e != cudaSuccess) return cuda_status(e);
   attn_bwd_dq_kernel<D, false><<<(unsigned)(dm.BH * dm.nqb), bwd_q_threads<false>(), BwdQSmem<D, false>::kBytes,
                                  st>>>(
-      mq, mk, mv, mdo, mdq, mk, mq, p, lp);
+      mq, mk, mv, mdo, mdq, mq, p, lp);
   p.order = nullptr;
   p.lst = q_idx;
   p.cnt = q_cnt;
@@ -440,10 +440,13 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
 sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape* s, const Dims& dm,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, const void* phik, const float* s_all,
                                 const float* z_all, const float* z_tile, const float* alpha, void* O,
-                                cudaStream_t st, float* den_out = nullptr) {
-  CUtensorMap mq, mv, mp, mo;
+                                cudaStream_t st, float* den_out = nullptr, void* sc_out = nullptr,
+                                float* zc_out = nullptr) {
+  CUtensorMap mq, mv, mp, mo, msc;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, 128, 128) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
-      !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq))
+      !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mo, O, dm.BH, s->N, 128, s->bq) ||
+      !make_map_bhnd(&msc, sc_out != nullptr ? sc_out : O, sc_out != nullptr ? dm.BH * dm.nqb : dm.BH,
+                     sc_out != nullptr ? 128 : s->N, 128, 128))
     return SPARGE_ERR_CUDA;
   LoParams p;
   p.kv_idx = kv_idx;
@@ -453,6 +456,8 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   p.z_tile = z_tile;
   p.alpha = alpha;
   p.den_out = den_out;
+  p.zc_out = zc_out;
+  p.store_sc = sc_out != nullptr;
   p.H = s->H;
   p.N = s->N;
   p.ntiles = (int)ceil_div(s->N, 64);
@@ -463,7 +468,7 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
   cudaError_t e = ensure_smem(linear_out_kernel, LoSmem::kBytes, 7);
   if (e != cudaSuccess) return cuda_status(e);
   const int64_t pairs = dm.BH * ceil_div(dm.nqb, 2);  // two neighbouring query blocks per CTA
-  linear_out_kernel<<<(unsigned)pairs, kLoThreads, LoSmem::kBytes, st>>>(mq, mv, mp, mo, p);
+  linear_out_kernel<<<(unsigned)pairs, kLoThreads, LoSmem::kBytes, st>>>(mq, mv, mp, mo, msc, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -506,7 +511,7 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
 // transposed mask and the fp32 sparse partials of dK and dV.
 struct Sla2BwdWs {
   Sla2Ws f;  // phi(K), S_all, z_all, z_tile, summary partials
-  size_t s_bf16, os, lse, ol, den, alpha0, dsum, cw, fw, ew, dpart, phiq, cdo, g, gall, gtile, qidx, qcnt, dkp,
+  size_t sc, zc, os, lse, ol, den, alpha0, dsum, cw, fw, ew, dpart, phiq, cdo, g, gall, gtile, qidx, qcnt, dkp,
       dvp, total;
 };
 
@@ -516,9 +521,10 @@ Sla2BwdWs sla2_bwd_ws(const sparge_shape* s, const Dims& d) {
   Sla2BwdWs w;
   w.f = sla2_ws(s, d);
   const size_t tens = align256((size_t)d.BH * s->N * s->d * 2), rows = align256((size_t)d.BH * s->N * 4);
-  const size_t mat32 = align256((size_t)d.BH * s->d * s->d * 4), mat16 = align256((size_t)d.BH * s->d * s->d * 2);
-  w.s_bf16 = w.f.total;
-  w.os = w.s_bf16 + mat16;
+  const size_t mat32 = align256((size_t)d.BH * s->d * s->d * 4);
+  w.sc = w.f.total;
+  w.zc = w.sc + align256((size_t)d.BH * d.nqb * s->d * s->d * 2);
+  w.os = w.zc + align256((size_t)d.BH * d.nqb * s->d * 4);
   w.lse = w.os + tens;
   w.ol = w.lse + rows;
   w.den = w.ol + tens;
@@ -548,11 +554,11 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   const Sla2BwdWs w = sla2_bwd_ws(s, dm);
   auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
   auto fat = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
-  __nv_bfloat16* s_bf16 = static_cast<__nv_bfloat16*>(at(w.s_bf16));
-  // 1. The forward's pieces: summaries (and a bf16 S_all), O_l unscaled with
-  //    its denominators (alpha = 0 gives weight 1), the sparse branch with lse.
+  // 1. The forward's pieces: summaries, O_l unscaled with its denominators
+  //    (alpha = 0 gives weight 1) and each query block's S_c (bf16) and z_c,
+  //    the sparse branch with lse.
   sparge_status r = launch_summaries(K, V, s, dm, at(w.f.phik), fat(w.f.partial), fat(w.f.s_all), fat(w.f.z_all),
-                                     fat(w.f.z_tile), st, s_bf16);
+                                     fat(w.f.z_tile), st);
   if (r != SPARGE_OK) return r;
   cudaError_t e = cudaMemsetAsync(at(w.alpha0), 0, (size_t)s->H * 4, st);
   if (e != cudaSuccess) return cuda_status(e);
@@ -560,7 +566,7 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   e = launch_tile_order(kv_cnt, s, dm, &order, st);
   if (e != cudaSuccess) return cuda_status(e);
   r = launch_linear_out(Q, V, s, dm, kv_idx, kv_cnt, at(w.f.phik), fat(w.f.s_all), fat(w.f.z_all), fat(w.f.z_tile),
-                        fat(w.alpha0), at(w.ol), st, fat(w.den));
+                        fat(w.alpha0), at(w.ol), st, fat(w.den), at(w.sc), fat(w.zc));
   if (r != SPARGE_OK) return r;
   r = launch_attn<D, false>(Q, K, V, s, dm, kv_idx, kv_cnt, at(w.os), fat(w.lse), nullptr, st, order);
   if (r != SPARGE_OK) return r;
@@ -586,13 +592,13 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
       kv_idx, kv_cnt, (int)dm.nqb, (int)dm.nkb, q_idx, q_cnt);
   // 5. dQ (sparse + linear), then dK and dV: sparse part into fp32 partials,
   //    linear part and the combination into bf16.
-  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, mpq, msall, mpq64, mcdo;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv, mpk, msc, mpq64, mcdo;
   if (!make_map_bhnd(&mq, Q, dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&mk, K, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mv, V, dm.BH, s->N, D, kTileK) || !make_map_bhnd(&mdo, dO, dm.BH, s->N, D, kTileQ) ||
       !make_map_bhnd(&mdq, dQ, dm.BH, s->N, D, s->bq) || !make_map_bhnd(&mdk, dK, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mdv, dV, dm.BH, s->N, D, kTileK) ||
       !make_map_bhnd(&mpk, at(w.f.phik), dm.BH, s->N, D, kTileK) ||
-      !make_map_bhnd(&mpq, at(w.phiq), dm.BH, s->N, D, kTileQ) || !make_map_bhnd(&msall, s_bf16, dm.BH, D, D, kTileQ) ||
+      !make_map_bhnd(&msc, at(w.sc), dm.BH * dm.nqb, D, D, kTileQ) ||
       !make_map_bhnd(&mpq64, at(w.phiq), dm.BH, s->N, D, 64) || !make_map_bhnd(&mcdo, at(w.cdo), dm.BH, s->N, D, 64))
     return SPARGE_ERR_CUDA;
   BwdParams p;
@@ -612,13 +618,13 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   lp.alpha = alpha;
   lp.cw = fat(w.cw);
   lp.fw = fat(w.fw);
-  lp.z_all = fat(w.f.z_all);
+  lp.zc = fat(w.zc);
   lp.H = s->H;
   e = ensure_smem(attn_bwd_dq_kernel<D, true>, BwdQSmem<D, true>::kBytes, 14);
   if (e != cudaSuccess) return cuda_status(e);
   attn_bwd_dq_kernel<D, true><<<(unsigned)(dm.BH * dm.nqb), bwd_q_threads<true>(), BwdQSmem<D, true>::kBytes,
                                 st>>>(
-      mq, mk, mv, mdo, mdq, mpk, msall, p, lp);
+      mq, mk, mv, mdo, mdq, msc, p, lp);
   p.order = nullptr;
   p.lst = q_idx;
   p.cnt = q_cnt;
