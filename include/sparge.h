@@ -224,9 +224,9 @@ sparge_status sparge_attn_bwd(const void* Q, const void* K, const void* V, const
  * The call recomputes what it needs of the forward (the linear summaries,
  * O_linear and its denominators, the sparse branch and its log-sum-exp), so
  * it takes no forward outputs. Precision: as sparge_attn_bwd for the sparse
- * part; the linear part's products take bf16 operands (S_all, the per-tile
- * complements of G_all, phi(Q), c_i dO_i, phi(K), V) with fp32 accumulation;
- * row scalars in fp32.
+ * part; the linear part's products take bf16 operands (each query block's
+ * complement S_c, each key tile's complement of G_all, phi(Q), c_i dO_i,
+ * phi(K), V) with fp32 accumulation; row scalars in fp32.
  * d must be 128 and Nqb * 32 bytes must not exceed 200 KiB.
  * Workspace: sparge_workspace_bytes(SPARGE_OP_SLA2_BWD, shape). */
 sparge_status sla2_attn_bwd(const void* Q, const void* K, const void* V, const sparge_shape* shape,
