@@ -349,11 +349,9 @@ __global__ void __launch_bounds__(kLinThreads, 2)
 // was covered by the CTAs c = floor(h ntiles / W) .. floor(((h + 1) ntiles - 1) / W),
 // whose partials sit at slots c + h. One thread per element of the
 // [128][129] summary.
-// s_bf16 (optional): a bf16 copy of S_all, [BH, 128, 128] row-major.
 __global__ void __launch_bounds__(256) linear_reduce_kernel(const float* __restrict__ partial, int ntiles,
                                                             int64_t per_cta, float* __restrict__ s_all,
-                                                            float* __restrict__ z_all,
-                                                            __nv_bfloat16* __restrict__ s_bf16) {
+                                                            float* __restrict__ z_all) {
   const int bh = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;
   if (e >= kLinPartial) return;
@@ -361,10 +359,9 @@ __global__ void __launch_bounds__(256) linear_reduce_kernel(const float* __restr
   float acc = 0.0f;
   for (int64_t c = c0; c <= c1; ++c) acc += partial[(c + bh) * kLinPartial + e];
   const int a = e / 129, c = e % 129;
-  if (c < 128) {
+  if (c < 128)
     s_all[((int64_t)bh * 128 + a) * 128 + c] = acc;
-    if (s_bf16 != nullptr) s_bf16[((int64_t)bh * 128 + a) * 128 + c] = __float2bfloat16_rn(acc);
-  } else
+  else
     z_all[(int64_t)bh * 128 + a] = acc;
 }
 

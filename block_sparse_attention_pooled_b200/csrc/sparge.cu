@@ -474,8 +474,8 @@ sparge_status launch_linear_out(const void* Q, const void* V, const sparge_shape
 
 sparge_status launch_summaries(const void* K, const void* V, const sparge_shape* s, const Dims& dm, void* phik,
                                float* partial, float* s_all, float* z_all, float* z_tile, cudaStream_t st,
-                               __nv_bfloat16* s_bf16 = nullptr, const float* row_scale = nullptr,
-                               const float* row_w = nullptr, void* v_scaled = nullptr) {
+                               const float* row_scale = nullptr, const float* row_w = nullptr,
+                               void* v_scaled = nullptr) {
   CUtensorMap mk, mv, mp, mvs;
   if (!make_map_bhnd(&mk, K, dm.BH, s->N, 128, 64) || !make_map_bhnd(&mv, V, dm.BH, s->N, 128, 64) ||
       !make_map_bhnd(&mp, phik, dm.BH, s->N, 128, 64) ||
@@ -502,7 +502,7 @@ sparge_status launch_summaries(const void* K, const void* V, const sparge_shape*
     linear_summary_kernel<false><<<(unsigned)grid, kLinThreads, LinSmem::kBytes, st>>>(mk, mv, mp, mp, p);
   }
   dim3 rgrid((unsigned)ceil_div(kLinPartial, 256), (unsigned)dm.BH);
-  linear_reduce_kernel<<<rgrid, 256, 0, st>>>(partial, p.ntiles, p.per_cta, s_all, z_all, s_bf16);
+  linear_reduce_kernel<<<rgrid, 256, 0, st>>>(partial, p.ntiles, p.per_cta, s_all, z_all);
   return cuda_status(cudaGetLastError());
 }
 
@@ -579,7 +579,7 @@ sparge_status launch_sla2_bwd(const void* Q, const void* K, const void* V, const
   sla2_dalpha_kernel<<<1, 128, 0, st>>>(fat(w.dpart), s->B, s->H, chunks, dalpha);
   // 3. G_all, g_all, g_tile, phi(Q) and c_i dO_i (the summary kernel on Q
   //    and dO with c_i, e_i).
-  r = launch_summaries(Q, dO, s, dm, at(w.phiq), fat(w.f.partial), fat(w.g), fat(w.gall), fat(w.gtile), st, nullptr,
+  r = launch_summaries(Q, dO, s, dm, at(w.phiq), fat(w.f.partial), fat(w.g), fat(w.gall), fat(w.gtile), st,
                        fat(w.cw), fat(w.ew), at(w.cdo));
   if (r != SPARGE_OK) return r;
   // 4. Transposed mask.
