@@ -241,6 +241,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kOffTmem + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tile = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;  // (bh, query block)
+  const int bh = tile / p.nqb;
+  const int qb = tile % p.nqb;
+  const int q0 = qb * p.bq;                    // first query row of the tile
+  const int tiles_per_block = p.bk / kTileK;
+  const int cnt = min(max(__ldg(p.kv_cnt + tile), 0), p.nkb);  // a bad count cannot walk past the list
+  const int T = cnt * tiles_per_block;         // key tiles to visit
+  const int32_t* lst = p.kv_idx + (int64_t)tile * p.nkb;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
@@ -269,18 +277,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // Launched right behind the mask (or the launch order), this CTA has set
-  // up its barriers and TMEM while that kernel finished; its inputs are read
-  // only from here on.
-  griddep_wait();
-  const int tile = p.order ? __ldg(p.order + blockIdx.x) : (int)blockIdx.x;  // (bh, query block)
-  const int bh = tile / p.nqb;
-  const int qb = tile % p.nqb;
-  const int q0 = qb * p.bq;                    // first query row of the tile
-  const int tiles_per_block = p.bk / kTileK;
-  const int cnt = min(max(__ldg(p.kv_cnt + tile), 0), p.nkb);  // a bad count cannot walk past the list
-  const int T = cnt * tiles_per_block;         // key tiles to visit
-  const int32_t* lst = p.kv_idx + (int64_t)tile * p.nkb;
   const uint32_t tS = tmem, tO = tmem + 128;
 
   if (warp == 0) {

@@ -37,7 +37,6 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
                                                    const __nv_bfloat16* __restrict__ K, int64_t BH, int N, int bq,
                                                    int bk, int64_t q_ctas, double* __restrict__ qbar,
                                                    double* __restrict__ kbar) {
-  griddep_launch();  // the next kernel may start launching (it waits for this one to end)
   constexpr int TPB = D / 8;            // threads per block-row
   constexpr int BLOCKS_PER_CTA = 128 / TPB;
   // CTAs [0, q_ctas) pool Q blocks, the rest pool K blocks.
@@ -103,8 +102,6 @@ __host__ __device__ constexpr int project_smem_bytes() {
 template <int D, int DR>
 __global__ void __launch_bounds__(128) project_kernel(const double* __restrict__ in, int64_t nb, int H,
                                                       const float* __restrict__ W, double* __restrict__ out) {
-  griddep_wait();  // the pooled vectors are complete
-  griddep_launch();
   constexpr int G = 128 / DR, RPT = kProjRows / G;  // row groups, rows per thread
   extern __shared__ __align__(16) double sx[];        // [kProjRows][D]
   const int64_t chunks = (nb + kProjRows - 1) / kProjRows;
@@ -177,8 +174,6 @@ __device__ __forceinline__ void dmma_884(double& c0, double& c1, double a, doubl
 template <int D>
 __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                                                     int nqb, int nkb, double scale, double* __restrict__ Z) {
-  griddep_wait();  // the pooled (or projected) vectors are complete
-  griddep_launch();
   extern __shared__ __align__(16) double smd[];
   constexpr int kStage = (kScoreRows + kScoreTileJ) * kScorePitch;  // doubles per stage
   constexpr int kChunks = D / kScoreChunk;
@@ -510,8 +505,6 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const double* __
                                                                  int32_t* __restrict__ kv_cnt,
                                                                  float* __restrict__ row_thresh,
                                                                  float* __restrict__ probs) {
-  griddep_wait();  // the scores are complete
-  griddep_launch();
   extern __shared__ __align__(16) unsigned char smraw[];
   const int npad = (nkb + 1) / 2 * 2;
   double* ev = reinterpret_cast<double*>(smraw);                                       // [npad], then the keys
@@ -680,8 +673,6 @@ __global__ void __launch_bounds__(kSelWarpRows * 32) select_warp_kernel(const do
                                                                         int32_t* __restrict__ kv_cnt,
                                                                         float* __restrict__ row_thresh,
                                                                         float* __restrict__ probs) {
-  griddep_wait();  // the scores are complete
-  griddep_launch();
   extern __shared__ __align__(16) unsigned char smraw[];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t row = (int64_t)blockIdx.x * kSelWarpRows + wid;
@@ -821,8 +812,6 @@ __host__ __device__ constexpr int tile_order_smem_bytes(int nkb) { return (nkb +
 __global__ void __launch_bounds__(kOrderThreads) tile_order_kernel(const int32_t* __restrict__ kv_cnt, int64_t BH,
                                                                    int nqb, int nkb, int G,
                                                                    int32_t* __restrict__ order) {
-  griddep_wait();  // the kept counts are complete
-  griddep_launch();
   extern __shared__ int hist[];  // [nkb + 1] bins (descending kept count), then 32 warp totals
   int* wsum = hist + nkb + 1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

@@ -38,15 +38,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-// Programmatic dependent launch. A kernel launched with programmatic stream
-// serialization may start while the kernel ahead of it in the stream still
-// runs: griddep_wait() blocks until that kernel has completed and its memory
-// operations are visible (a no-op when the launch had no such attribute), and
-// griddep_launch() lets the next kernel in the stream begin launching once
-// every CTA of this one has executed it.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

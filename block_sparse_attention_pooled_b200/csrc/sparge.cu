@@ -5,7 +5,6 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
-#include <utility>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -149,26 +148,6 @@ cudaError_t ensure_smem(K kernel, int bytes, int slot) {
   return e;
 }
 
-// Launches a kernel that may begin while the kernel ahead of it in the stream
-// finishes (programmatic dependent launch): its CTAs set up while the other
-// kernel's last CTAs run, and its griddep_wait() holds every read of that
-// kernel's results until it has completed.
-template <typename... P, typename... A>
-cudaError_t launch_dependent(void (*kernel)(P...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
-                             A&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
-}
-
 // Launch order of the query tiles (tile_order_kernel): heads in groups whose
 // K and V (2 N d bf16 each) fit in 64 MB of L2, heaviest tiles first. When not
 // even two heads fit, the grid stays head-major (sorting inside one head
@@ -182,9 +161,9 @@ cudaError_t launch_tile_order(const int32_t* kv_cnt, const sparge_shape* s, cons
     *order = nullptr;
     return cudaSuccess;
   }
-  return launch_dependent(tile_order_kernel, (unsigned)ceil_div(dm.BH, G), kOrderThreads,
-                          tile_order_smem_bytes((int)dm.nkb), st, kv_cnt, dm.BH, (int)dm.nqb, (int)dm.nkb, (int)G,
-                          *order);
+  tile_order_kernel<<<(unsigned)ceil_div(dm.BH, G), kOrderThreads, tile_order_smem_bytes((int)dm.nkb), st>>>(
+      kv_cnt, dm.BH, (int)dm.nqb, (int)dm.nkb, (int)G, *order);
+  return cudaGetLastError();
 }
 
 inline size_t order_bytes(const Dims& d) { return align256((size_t)d.BH * d.nqb * 4); }
@@ -197,7 +176,8 @@ cudaError_t launch_scores(const double* a, const double* b, const Dims& dm, doub
   cudaError_t e = ensure_smem(score_kernel<DD>, ssm, DD == 64 ? 0 : 1);
   if (e != cudaSuccess) return e;
   const int64_t tiles = dm.BH * ceil_div(dm.nqb, kScoreRows) * ceil_div(dm.nkb, kScoreTileJ);
-  return launch_dependent(score_kernel<DD>, (unsigned)tiles, 128, ssm, st, a, b, (int)dm.nqb, (int)dm.nkb, scale, Z);
+  score_kernel<DD><<<(unsigned)tiles, 128, ssm, st>>>(a, b, (int)dm.nqb, (int)dm.nkb, scale, Z);
+  return cudaGetLastError();
 }
 
 // Router projections of the pooled vectors (DR output columns).
@@ -207,9 +187,9 @@ cudaError_t launch_projection(const double* qbar, const double* kbar, const Dims
   const unsigned gq = (unsigned)(ceil_div(dm.nqb, kProjRows) * dm.BH);
   const unsigned gk = (unsigned)(ceil_div(dm.nkb, kProjRows) * dm.BH);
   constexpr int psm = project_smem_bytes<D>();
-  cudaError_t e = launch_dependent(project_kernel<D, DR>, gq, 128, psm, st, qbar, dm.nqb, H, Wq, qhat);
-  if (e != cudaSuccess) return e;
-  return launch_dependent(project_kernel<D, DR>, gk, 128, psm, st, kbar, dm.nkb, H, Wk, khat);
+  project_kernel<D, DR><<<gq, 128, psm, st>>>(qbar, dm.nqb, H, Wq, qhat);
+  project_kernel<D, DR><<<gk, 128, psm, st>>>(kbar, dm.nkb, H, Wk, khat);
+  return cudaGetLastError();
 }
 
 // Pool, (project,) score, select. Wq / Wk null: no router.
@@ -246,15 +226,16 @@ sparge_status launch_mask(const void* Q, const void* K, const sparge_shape* s, c
     const int sel_sm = select_warp_smem_bytes((int)dm.nkb);
     e = ensure_smem(select_warp_kernel, sel_sm, 17);
     if (e != cudaSuccess) return cuda_status(e);
-    return cuda_status(launch_dependent(select_warp_kernel, (unsigned)ceil_div(dm.BH * dm.nqb, kSelWarpRows),
-                                        kSelWarpRows * 32, sel_sm, st, Z, dm.BH * dm.nqb, (int)dm.nkb, kc, topp,
-                                        kv_idx, kv_cnt, row_thresh, probs));
+    select_warp_kernel<<<(unsigned)ceil_div(dm.BH * dm.nqb, kSelWarpRows), kSelWarpRows * 32, sel_sm, st>>>(
+        Z, dm.BH * dm.nqb, (int)dm.nkb, kc, topp, kv_idx, kv_cnt, row_thresh, probs);
+    return cuda_status(cudaGetLastError());
   }
   const int sel_sm = select_smem_bytes((int)dm.nkb);
   e = ensure_smem(select_kernel, sel_sm, 2);
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(launch_dependent(select_kernel, (unsigned)(dm.BH * dm.nqb), kSelectThreads, sel_sm, st, Z,
-                                      dm.BH * dm.nqb, (int)dm.nkb, kc, topp, kv_idx, kv_cnt, row_thresh, probs));
+  select_kernel<<<(unsigned)(dm.BH * dm.nqb), kSelectThreads, sel_sm, st>>>(Z, dm.BH * dm.nqb, (int)dm.nkb, kc, topp,
+                                                                           kv_idx, kv_cnt, row_thresh, probs);
+  return cuda_status(cudaGetLastError());
 }
 
 // 3-D map over one-byte codes [BH][N][128] with a (128 x rows x 1) box,
@@ -451,8 +432,8 @@ sparge_status launch_attn(const void* Q, const void* K, const void* V, const spa
   const int smem = AttnSmem<D, MIX>::kBytes;
   cudaError_t e = ensure_smem(attn_fwd_kernel<D, MIX>, smem, MIX ? 5 : (D == 64 ? 3 : 4));
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(
-      launch_dependent(attn_fwd_kernel<D, MIX>, (unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st, mq, mk, mv, mo, p));
+  attn_fwd_kernel<D, MIX><<<(unsigned)(dm.BH * dm.nqb), kAttnThreads, smem, st>>>(mq, mk, mv, mo, p);
+  return cuda_status(cudaGetLastError());
 }
 
 // (1 - alpha_h) O_linear into O, one CTA per query block (d = 128).
